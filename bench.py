@@ -1,0 +1,442 @@
+"""Benchmark: segmented chunkwise gated linear attention on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C1] [--schedule auto]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on this host's cores
+
+A step is one pass of the whole path over one batch of the workload: every per-segment chunk
+pass, the cross-segment state scan and the output / correction pass (plus the backward
+passes for a fwd+bwd workload), each through the library's C ABI on the current stream.
+Inputs are resident in HBM and L2 is flushed (256 MiB write, untimed) before every step; each
+step is bracketed by CUDA events and its phases by events in between, on the same stream.
+With N > 1 ranks (torchrun), every rank runs its own replica of the workload on its own GPU:
+the path has no cross-rank exchange, so there is no collective on the data path ("weak"
+scaling); the max over ranks of the device time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+from sequence_linear_attention_chunked_b200.inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+METRIC = "tokens/sec of gated linear attn fwd(+bwd) at 1 B200; % bf16 TC peak / % HBM BW"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def csrc_digest() -> str:
+    d = os.path.join(ROOT, "sequence_linear_attention_chunked_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("csrc_digest") != csrc_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, interval_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.interval = interval_s
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hi = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hi)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    h = hi
+            self.nvml, self.h = pynvml, h
+            if h is not None:
+                self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.nvml, self.h, self.error = None, None, repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample_once()
+            time.sleep(self.interval)
+
+    def sample_once(self):
+        if self.h is None:
+            return
+        try:
+            mhz = self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+            r = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return
+        self.samples.append(mhz)
+        for bit, name in self.REASONS.items():
+            if r & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def __enter__(self):
+        self.sample_once()
+        self._thr = threading.Thread(target=self._run, daemon=True)
+        self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+        self.sample_once()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- our arm
+class Step:
+    """One pass of the whole path through the C ABI's per-step entry points, with CUDA events
+    between the phases on the launching stream."""
+
+    def __init__(self, w: Workload, x, schedule: str, device):
+        from sequence_linear_attention_chunked_b200 import la_seg
+        self.la = la_seg
+        self.w, self.x, self.dev = w, x, device
+        dt = la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16
+        self.NP = la_seg.la_seg_subsegments(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt)
+        self.schedule = schedule
+        B, H, L, dk, dv, NP = w.B, w.H, w.L, w.dk, w.dv, self.NP
+        f32 = dict(dtype=torch.float32, device=device)
+        self.o = torch.empty((B, H, L, dv), dtype=w.torch_dtype, device=device)
+        self.S_loc = torch.empty((B, H, NP, dk, dv), **f32)
+        self.logG = torch.empty((B, H, NP, dk), **f32)
+        self.S_recv = torch.empty((B, H, NP, dk, dv), **f32)
+        self.S_final = torch.empty((B, H, dk, dv), **f32)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.phases = (["state pass", "state scan", "output pass"] if schedule != "three"
+                       else ["local pass", "state scan", "correction pass"])
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
+        self.launches_per_step = len(self.phases)
+
+    def run(self, record=True):
+        la, x, w, NP = self.la, self.x, self.w, self.NP
+        ev = self.events
+        if record:
+            ev[0].record()
+        if self.schedule != "three":
+            la.la_seg_state_pass(x["k"], x["v"], x["log_g"], NP, w.chunk, S_loc=self.S_loc,
+                                 log_gamma=self.logG, status=self.status)
+        else:
+            la.la_seg_local_pass(x["q"], x["k"], x["v"], x["log_g"], NP, w.chunk, o=self.o,
+                                 S_loc=self.S_loc, log_gamma=self.logG, status=self.status)
+        if record:
+            ev[1].record()
+        BH = w.B * w.H
+        la.lib().la_seg_scan(la._ptr(self.S_loc), la._ptr(self.logG), None, BH, NP, w.dk, w.dv, 0,
+                             la._ptr(self.S_recv), la._ptr(self.S_final), la._stream(None))
+        if record:
+            ev[2].record()
+        if self.schedule != "three":
+            la.la_seg_output_pass(x["q"], x["k"], x["v"], x["log_g"], self.S_recv, NP, w.chunk,
+                                  o=self.o, status=self.status)
+        else:
+            la.la_seg_correct_pass(x["q"], x["log_g"], self.S_recv, NP, w.chunk, self.o,
+                                   status=self.status)
+        if record:
+            ev[3].record()
+
+    def phase_ms(self):
+        return [self.events[i].elapsed_time(self.events[i + 1]) for i in range(len(self.phases))]
+
+    def algorithmic_bytes(self):
+        """Bytes each phase must move at minimum (inputs read once, outputs written once)."""
+        w = self.w
+        e = 4 if w.dtype == "f32" else 2
+        th = w.B * w.H * w.L
+        st = w.B * w.H * self.NP * w.dk * w.dv * 4
+        lg = w.B * w.H * self.NP * w.dk * 4
+        if self.schedule != "three":
+            return {"state pass": th * (2 * w.dk + w.dv) * e + st + lg,
+                    "state scan": 2 * st + lg + w.B * w.H * w.dk * w.dv * 4,
+                    "output pass": th * (3 * w.dk + 2 * w.dv) * e + st}
+        return {"local pass": th * (3 * w.dk + 2 * w.dv) * e + st + lg,
+                "state scan": 2 * st + lg + w.B * w.H * w.dk * w.dv * 4,
+                "correction pass": th * (2 * w.dk + 2 * w.dv) * e + st}
+
+    def flops(self):
+        w = self.w
+        th = w.B * w.H * w.L
+        C = w.chunk
+        intra = 2 * C * w.dk + 2 * C * w.dv  # QK^T and PV on full chunk tiles
+        inter = 2 * w.dk * w.dv              # q . S
+        state = 2 * w.dk * w.dv              # K^T V
+        if self.schedule != "three":
+            return {"state pass": th * state, "state scan": 0, "output pass": th * (intra + inter + state)}
+        return {"local pass": th * (intra + inter + state), "state scan": 0, "correction pass": th * inter}
+
+
+def bench_ours(args, rank, world, device):
+    from sequence_linear_attention_chunked_b200 import la_seg
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, device)
+    step = Step(w, x, args.schedule, device)
+
+    # The per-step composition must reproduce the public entry point bit for bit.
+    sched = {"auto": la_seg.SCHED_AUTO, "two": la_seg.SCHED_TWO_PASS,
+             "three": la_seg.SCHED_THREE_PHASE}[args.schedule]
+    ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk,
+                          la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16, False, device)
+    o_api, Sf_api, _ = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, w.P,
+                                             w.chunk, sched, ws=ws)
+    la_seg.la_seg_check_status(ws)
+    step.run(record=False)
+    torch.cuda.synchronize()
+    if not (torch.equal(o_api, step.o) and torch.equal(Sf_api, step.S_final)):
+        raise RuntimeError("per-step composition differs from la_seg_forward")
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} after the check run")
+    del o_api, Sf_api
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.run()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, phase_ms = [], []
+    sampler = ClockSampler(device.index)
+    with sampler:
+        for _ in range(args.steps):
+            flush.zero_()
+            step.run()
+            torch.cuda.synchronize()  # read this step's events before the next one reuses them
+            pm = step.phase_ms()
+            phase_ms.append(pm)
+            step_ms.append(step.events[0].elapsed_time(step.events[-1]))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    tokens_per_step = w.B * w.L
+    value = tokens_per_step * world * args.steps / (total_ms / 1e3)
+
+    # phases and the dominant kernel's roofline
+    mean_phase = [statistics.fmean(p[i] for p in phase_ms) for i in range(len(step.phases))]
+    ab = step.algorithmic_bytes()
+    fl = step.flops()
+    peaks, peak_src = load_peaks()
+    dom = max(range(len(step.phases)), key=lambda i: mean_phase[i])
+    dname = step.phases[dom]
+    achieved = ab[dname] / (mean_phase[dom] / 1e3) / 1e9
+    kernel_key = {"state pass": "state_pass", "output pass": "output_pass", "local pass": "local_pass",
+                  "correction pass": "correct_pass", "state scan": "scan"}[dname]
+    phases = {}
+    for i, name in enumerate(step.phases):
+        sec = mean_phase[i] / 1e3
+        phases[name] = {"ms": round(mean_phase[i], 5), "GB/s": round(ab[name] / sec / 1e9, 1),
+                        "hbm_frac": round(ab[name] / sec / 1e9 / peaks["hbm_gbs"], 4),
+                        "TFLOP/s": round(fl[name] / sec / 1e12, 2),
+                        "tc_frac": round(fl[name] / sec / 1e12 / peaks["bf16_tflops"], 4)}
+    roofline = {"bound": "hbm", "kernel": dname, "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peak_src} hbm_gbs (burst copy)",
+                "algorithmic_bytes_per_launch": ab[dname],
+                "traffic": ncu_traffic(kernel_key, w.name)}
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "ms_per_step_median": round(statistics.median(step_ms), 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.describe(), "B": w.B, "H": w.H, "L": w.L, "d": w.dk, "P": w.P,
+                       "chunk": w.chunk, "subsegments": step.NP, "schedule": args.schedule,
+                       "l2": "flushed before every step (256 MiB write, untimed)",
+                       "parallelism": f"replicas x{world}"},
+            "phases": phases, "roofline": roofline,
+            "gpu_launches": step.launches_per_step * args.steps,
+            "clocks": sampler.summary()}
+    if not args.no_e2e:
+        line["e2e"] = bench_e2e(args, w, x, device, world)
+    return line
+
+
+def bench_e2e(args, w, x, device, world):
+    """Same metric through the public entry point with host buffers: per step, pinned host ->
+    device copies of q, k, v, log_g, la_seg_forward, and the device -> host copy of o."""
+    from sequence_linear_attention_chunked_b200 import la_seg
+    host = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "log_g")}
+    dev = {n: torch.empty_like(x[n]) for n in host}
+    o_host = torch.empty(x["q"].shape[:-1] + (w.dv,), dtype=w.torch_dtype).pin_memory()
+    dt = la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16
+    ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device)
+    o_dev = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype, device=device)
+    Sf = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
+    Sf_host = torch.empty_like(Sf, device="cpu").pin_memory()
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        st = la_seg.lib().la_seg_forward(
+            la_seg._ptr(dev["q"]), la_seg._ptr(dev["k"]), la_seg._ptr(dev["v"]),
+            la_seg._ptr(dev["log_g"]), None, w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt,
+            la_seg._ptr(o_dev), la_seg._ptr(Sf), None, 0, la_seg._ptr(ws), ws.numel(),
+            la_seg._stream(None))
+        la_seg._check(st, "la_seg_forward")
+        o_host.copy_(o_dev, non_blocking=True)
+        Sf_host.copy_(Sf, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o_host.numel() * o_host.element_size() + Sf_host.numel() * 4
+    return {"value": round(w.B * w.L * world * steps / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "api": "la_seg_forward (C ABI) with pinned host buffers"}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def cpu_sample(w: Workload, budget_s: float):
+    """Times the fp64 oracle on a bounded sample of the workload: all B*H heads over the first
+    n tokens (n a power of two <= L), repeated until about budget_s seconds have passed."""
+    import oracle
+    n = min(w.L, 4096)
+    xs = make_inputs(w.with_(L=n), "cpu")
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward(xs["q"], xs["k"], xs["v"], xs["log_g"])
+        if w.backward:
+            oracle.backward(xs["q"], xs["k"], xs["v"], xs["log_g"], xs["dO"])
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    cores = oracle.num_threads()
+    value = w.B * n * reps / el
+    return {"value": round(value, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 token-by-token oracle, all {w.B * w.H} heads x first {n} tokens of "
+                      f"{w.name}, {reps} repetitions, {el:.1f} s; tokens/s = B*n*reps/seconds",
+            "seconds": round(el, 2)}
+
+
+def bench_reference(args, w):
+    cb = cpu_sample(w, args.cpu_seconds)
+    return {"metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.describe(), "B": w.B, "H": w.H, "L": w.L, "d": w.dk, "P": w.P,
+                       "chunk": w.chunk},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="C1", choices=sorted(WORKLOADS))
+    ap.add_argument("--schedule", default="auto", choices=["auto", "two", "three"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(bench_reference(args, w)), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    try:
+        line = bench_ours(args, rank, world, device)
+        if rank == 0 and world == 1 and not args.no_cpu:
+            line["cpu_baseline"] = cpu_sample(w, args.cpu_seconds)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * la_seg.h -- C ABI of libla_seg.so: segmented chunkwise gated linear attention on one GPU.
+ *
+ * The operation (ZeCO review, "key machinery" and "core discovery"; GLA recurrence of the
+ * review's supporting citation Yang et al. 2024), per (b, h) pair, with a_t = exp(log_g_t):
+ *
+ *     S_t = diag(a_t) S_{t-1} + k_t^T v_t,   S_{-1} = S0 (or 0),   o_t = q_t S_t,
+ *     S_final = S_{L-1}.
+ *
+ * The sequence of L tokens is cut into P equal segments (the "devices" of ZeCO's sequence
+ * parallelism, all on this GPU).  Each segment computes its local state from zero and its
+ * intra-chunk outputs; an exclusive decayed scan over segments (the All-Scan update of the
+ * ZeCO review's "key machinery", with the accumulated state forwarded as the referee's
+ * comment on Alg. 2 requires)
+ *
+ *     S_recv_0 = S0,   S_recv_p = Gamma_{p-1} S_recv_{p-1} + S_{p-1},
+ *     Gamma_p = diag(exp(sum_{t in segment p} log_g_t))
+ *
+ * gives the state each segment receives, and each output gets its q . S_recv term.  The
+ * result equals the unsegmented recurrence up to rounding (the review's linear-decomposition
+ * identity), for every P and chunk size.
+ *
+ * Conventions for every entry point below
+ * ---------------------------------------
+ *  Layout     q, k, log_g: [B, H, L, dk]; v, o: [B, H, L, dv]; row-major, d fastest, dense.
+ *             States (S0, S_final, S_recv, dS_final, dS0): fp32 [B, H, dk, dv] (S_recv:
+ *             [B, H, P, dk, dv]).  log_g is the natural log of the per-key-dim gate.
+ *  dtype      la_dtype names the element type of q, k, v, log_g, o and of dO, dq, dk, dv,
+ *             dlog_g.  States are always fp32 and all accumulation is fp32.
+ *  Pointers   All tensor pointers are DEVICE pointers owned by the caller, 16-byte aligned.
+ *             The library allocates and frees nothing: scratch lives in the caller's
+ *             workspace (size from la_seg_workspace_bytes, 256-byte aligned).
+ *  Stream     cuda_stream is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *             asynchronous on it; nothing blocks the host except la_seg_check_status.
+ *  Errors     Argument checks run on the host before any launch and return a negative
+ *             la_status; la_last_error_detail then describes the failure.  Conditions found
+ *             on the device (a gate range the chunk factorisation cannot represent) set a
+ *             status word inside the workspace, read by la_seg_check_status.  No C++
+ *             exception crosses this boundary.
+ *  Sizes      dk == dv in {32, 64, 128}; chunk in {16, 32, 64}; L % P == 0 and (L / P) % chunk
+ *             == 0; B, H, P >= 1.  L == 0 is legal and does nothing but write S_final = S0.
+ *  Determinism Identical inputs give bit-identical outputs (no atomics on data).
+ */
+#ifndef LA_SEG_H
+#define LA_SEG_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_ARG = -1,        /* null pointer where one is required, bad enum value            */
+    LA_ERR_SHAPE = -2,      /* unsupported or inconsistent sizes                              */
+    LA_ERR_ALIGN = -3,      /* a pointer is not 16-byte aligned (workspace: 256-byte)         */
+    LA_ERR_DTYPE = -4,      /* unknown la_dtype                                               */
+    LA_ERR_WORKSPACE = -5,  /* workspace missing or smaller than la_seg_workspace_bytes       */
+    LA_ERR_GATE_RANGE = -6, /* |sum of log_g over one chunk| > 80 in some key dim: outputs of  */
+                            /* that chunk are not reliable (reported by la_seg_check_status)  */
+    LA_ERR_TIMEOUT = -7,    /* a bounded device-side wait gave up                             */
+    LA_ERR_CUDA = -8        /* a CUDA runtime call failed (launch, attribute, memset)         */
+} la_status;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+/* Forward schedules (both compute the same result):
+ *  LA_SCHED_AUTO    the library's choice (currently LA_SCHED_TWO_PASS).
+ *  LA_SCHED_TWO_PASS ZeCO's own order: a state-only pass over k, v, log_g per segment, the
+ *                   exclusive decayed scan, then one output pass per segment that starts from
+ *                   the received state (so the q . S_recv term is folded into the chunk loop).
+ *  LA_SCHED_THREE_PHASE  local pass (intra-chunk outputs + local states from zero), scan, then
+ *                   a separate correction pass o += (q . exp(B_seg)) S_recv. */
+typedef enum { LA_SCHED_AUTO = 0, LA_SCHED_TWO_PASS = 1, LA_SCHED_THREE_PHASE = 2 } la_schedule;
+
+/* Bytes of workspace la_seg_forward (backward = 0) or la_seg_backward (backward = 1) needs for
+ * these sizes.  Returns 0 for sizes the library rejects. */
+LA_API size_t la_seg_workspace_bytes(int B, int H, long long L, int dk, int dv, int P, int chunk,
+                              la_dtype dt, int backward);
+
+/* Forward pass (ZeCO review: Alg. 1 passes, All-Scan state update of "key machinery").
+ *  q, k, v, log_g  inputs (dtype dt).          S0        nullable: zero initial state.
+ *  o               output [B,H,L,dv] (dtype dt), fully overwritten.
+ *  S_final         nullable: the state after the last token, fp32 [B,H,dk,dv].
+ *  S_recv_save     nullable: the state each of the P segments receives, fp32 [B,H,P,dk,dv]
+ *                  (S_recv_save[:, :, 0] = S0); la_seg_backward can reuse it.
+ *  schedule        la_schedule (LA_SCHED_AUTO recommended).
+ * Returns LA_OK once every kernel is queued on cuda_stream. */
+LA_API la_status la_seg_forward(const void *q, const void *k, const void *v, const void *log_g,
+                         const float *S0, int B, int H, long long L, int dk, int dv, int P,
+                         int chunk, la_dtype dt, void *o, float *S_final, float *S_recv_save,
+                         int schedule, void *workspace, size_t ws_bytes, void *cuda_stream);
+
+/* Backward pass for loss = <o, dO> + <S_final, dS_final>.
+ *  S_recv_saved    nullable: the forward's S_recv_save (reused, as the ZeCO review's "forward
+ *                  implications" describe); when NULL the states are recomputed.
+ *  dS_final        nullable: zero.
+ *  dq, dk_, dv_, dlog_g  outputs (dtype dt), fully overwritten.
+ *  dS0             nullable: gradient with respect to S0, fp32 [B,H,dk,dv]. */
+LA_API la_status la_seg_backward(const void *q, const void *k, const void *v, const void *log_g,
+                          const float *S0, const float *S_recv_saved, const void *dO,
+                          const float *dS_final, int B, int H, long long L, int dk, int dv,
+                          int P, int chunk, la_dtype dt, void *dq, void *dk_, void *dv_,
+                          void *dlog_g, float *dS0, void *workspace, size_t ws_bytes,
+                          void *cuda_stream);
+
+/* The exclusive decayed scan alone (the All-Scan recurrence of the ZeCO review's "key
+ * machinery", run on one device over NP segments; the referee's Alg. 2 comment fixes that
+ * the accumulated state is what moves on).  Per (b, h), element-wise over (i, j):
+ *   reverse == 0:  acc = init;  for p = 0 .. NP-1:  out[p] = acc;  acc = exp(log_gamma[p][i]) * acc + S_in[p]
+ *   reverse != 0:  acc = init;  for p = NP-1 .. 0:  out[p] = acc;  acc = exp(log_gamma[p][i]) * acc + S_in[p]
+ *   final = acc.
+ *  S_in, out: fp32 [BH, NP, dk, dv]; log_gamma: fp32 [BH, NP, dk]; init, final: fp32
+ *  [BH, dk, dv], init nullable (zero), final nullable.  dv % 4 == 0.  out may not alias S_in. */
+LA_API la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
+                      int NP, int dk, int dv, int reverse, float *out, float *final_state,
+                      void *cuda_stream);
+
+/* ---- The steps of the path, one entry point each -------------------------------------
+ * la_seg_forward runs these in order; they are exported so that callers can compose their own
+ * schedule (e.g. replace the on-device scan by a cross-device one) and time each step.  Each
+ * cuts every (b, h) sequence into NP equal segments of L/NP tokens (L % NP == 0, (L/NP) %
+ * chunk == 0) and processes every segment independently, chunk by chunk, in one CTA.
+ * status: nullable device int; a kernel that meets a chunk whose |sum of log_g| exceeds the
+ * factorisation range ORs 1 into it (see LA_ERR_GATE_RANGE). */
+
+/* State pass (ZeCO Alg. 1, "local state stored to HBM"; GLA chunk-state update):
+ * S_loc[b,h,p] = state after segment p from a zero start, fp32 [B,H,NP,dk,dv];
+ * log_gamma[b,h,p] = sum over segment p of log_g, fp32 [B,H,NP,dk].  Reads k, v, log_g. */
+LA_API la_status la_seg_state_pass(const void *k, const void *v, const void *log_g, int B, int H,
+                                   long long L, int dk, int dv, int NP, int chunk, la_dtype dt,
+                                   float *S_loc, float *log_gamma, int *status, void *cuda_stream);
+
+/* Local pass (three-phase step 1): the state pass plus the segment-local outputs (intra-chunk
+ * attention and the inter-chunk term from a zero segment start), written to o. */
+LA_API la_status la_seg_local_pass(const void *q, const void *k, const void *v, const void *log_g,
+                                   int B, int H, long long L, int dk, int dv, int NP, int chunk,
+                                   la_dtype dt, void *o, float *S_loc, float *log_gamma,
+                                   int *status, void *cuda_stream);
+
+/* Output pass (two-pass step 3, ZeCO Alg. 1 second pass): o for every segment p, the chunk
+ * recurrence starting from S_recv[b,h,p] (fp32 [B,H,NP,dk,dv]; null = zero states). */
+LA_API la_status la_seg_output_pass(const void *q, const void *k, const void *v,
+                                    const void *log_g, const float *S_recv, int B, int H,
+                                    long long L, int dk, int dv, int NP, int chunk, la_dtype dt,
+                                    void *o, int *status, void *cuda_stream);
+
+/* Correction pass (three-phase step 3): o_t += (q_t . exp(B_t)) S_recv[b,h,p] for every token
+ * t of segment p, B_t the inclusive cumsum of log_g from the segment's first token. */
+LA_API la_status la_seg_correct_pass(const void *q, const void *log_g, const float *S_recv,
+                                     int B, int H, long long L, int dk, int dv, int NP, int chunk,
+                                     la_dtype dt, void *o, int *status, void *cuda_stream);
+
+/* Number of segments (P times the internal split) la_seg_forward uses for these sizes, or 0
+ * for rejected sizes.  la_seg_forward's S_recv_save keeps every (NP/P)-th received state. */
+LA_API int la_seg_subsegments(int B, int H, long long L, int dk, int dv, int P, int chunk,
+                              la_dtype dt);
+
+/* Synchronises cuda_stream and returns the device status word a previous call left in
+ * workspace (LA_OK, LA_ERR_GATE_RANGE or LA_ERR_TIMEOUT), or LA_ERR_CUDA. */
+LA_API la_status la_seg_check_status(void *workspace, void *cuda_stream);
+
+/* Copies a NUL-terminated description of the calling thread's last failure into buf (at most
+ * n bytes).  Returns LA_OK, or LA_ERR_ARG when buf is NULL or n == 0. */
+LA_API la_status la_last_error_detail(char *buf, size_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_SEG_H */

@@ -1,0 +1,56 @@
+// internal.h -- launchers shared between the translation units of libla_seg.so (C++ only,
+// never part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace la {
+
+// What one chunk-pass launch computes for each (b, h, sub-segment j), starting from state
+// S_init[j] (or zero) and walking the sub-segment chunk by chunk:
+enum PassMode : int {
+    kPassState = 0,    // local state S_j (from zero) + log-decay sum only; reads k, v, log_g
+    kPassOutput = 1,   // o from S_init[j]; reads q, k, v, log_g; writes o
+    kPassLocal = 2,    // o_local from zero, local state and log-decay sum; writes o, S, logG
+    kPassCorrect = 3,  // o += (q . exp(B_seg)) S_init[j]; reads q, log_g, o
+};
+
+struct PassArgs {
+    const void *q, *k, *v, *g;
+    void *o;
+    const float *S_init;  // [BH, NP, dk, dv] or null (zero)
+    float *S_out;         // [BH, NP, dk, dv] (kPassState / kPassLocal)
+    float *logG;          // [BH, NP, dk]    (kPassState / kPassLocal)
+    int *status;
+    long long L, T;       // tokens per (b, h), tokens per sub-segment
+    int BH, NP, dk, dv, chunk;
+    la_dtype dt;
+};
+
+// Generic CUDA-core (FFMA) chunk pass: any supported dtype, d and chunk.
+cudaError_t launch_simt_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
+
+// The chunk pass for these arguments: the tensor-core kernels where they apply, else SIMT.
+cudaError_t launch_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
+
+// Exclusive decayed scan over NP sub-segments (see la_seg_scan in la_seg.h).
+cudaError_t launch_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
+                        int NP, int dk, int dv, int reverse, float *out, float *final_state,
+                        cudaStream_t st);
+
+// Copies the per-sub-segment states at API-segment boundaries: dst[bh][p] = src[bh][p*m].
+cudaError_t launch_gather_states(const float *src, int BH, int NP, int m, int dk, int dv,
+                                 float *dst, cudaStream_t st);
+
+// dst[bh][p] = src[bh] (or zeros when src is null) for p < P; dst is [BH, P, dk, dv].
+cudaError_t launch_broadcast_state(const float *src, int BH, int P, int dk, int dv, float *dst,
+                                   cudaStream_t st);
+
+// Copies S0 (or zeros) into dst [BH, dk, dv].
+cudaError_t launch_copy_state(const float *src, int BH, int dk, int dv, float *dst,
+                              cudaStream_t st);
+
+}  // namespace la

@@ -1,0 +1,322 @@
+// la_seg_api.cu -- the C ABI of libla_seg.so: argument checks, workspace layout, the
+// sub-segment split and the launch sequence of each schedule.  No allocation, no host sync
+// (except la_seg_check_status), no C++ exception across the boundary.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <initializer_list>
+#include <utility>
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "la_seg.h"
+
+namespace {
+
+thread_local char g_detail[512] = "no error";
+
+la_status fail(la_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+la_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(LA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Shapes accepted by every entry point.
+la_status check_shape(int B, int H, long long L, int dk, int dv, int P, int chunk, la_dtype dt) {
+    if (dt != LA_F32 && dt != LA_BF16) return fail(LA_ERR_DTYPE, "unknown la_dtype %d", (int)dt);
+    if (B < 1 || H < 1 || P < 1 || L < 0)
+        return fail(LA_ERR_SHAPE, "need B, H, P >= 1 and L >= 0 (got B=%d H=%d P=%d L=%lld)", B, H,
+                    P, L);
+    if (!(dk == 32 || dk == 64 || dk == 128) || dv != dk)
+        return fail(LA_ERR_SHAPE, "need dk == dv in {32, 64, 128} (got dk=%d dv=%d)", dk, dv);
+    if (!(chunk == 16 || chunk == 32 || chunk == 64))
+        return fail(LA_ERR_SHAPE, "chunk must be 16, 32 or 64 (got %d)", chunk);
+    if (L % P != 0) return fail(LA_ERR_SHAPE, "L=%lld is not a multiple of P=%d", L, P);
+    if ((L / P) % chunk != 0)
+        return fail(LA_ERR_SHAPE, "segment length L/P=%lld is not a multiple of chunk=%d", L / P,
+                    chunk);
+    if ((long long)B * H > (1LL << 24) || L > (1LL << 40))
+        return fail(LA_ERR_SHAPE, "sizes out of range");
+    return LA_OK;
+}
+
+// Internal split of every API segment into m equal sub-segments (the linear-decomposition
+// identity makes the result independent of the split).  Chooses the m (a power of two that
+// divides the chunks of a segment) with the fewest estimated CTA-waves x chunks per CTA, so
+// that small B*H*P still fill the 148 SMs while large ones keep whole segments.
+la::Split make_split(int B, int H, long long L, int P, int chunk) {
+    la::Split s;
+    s.BH = B * H;
+    s.P = P;
+    s.L = L;
+    const long long chunks_per_seg = (L / P) / chunk;
+    const long long bhp = (long long)s.BH * P;
+    int best_m = 1;
+    double best_cost = 1e300;
+    for (long long m = 1; chunks_per_seg > 0 && m <= chunks_per_seg; m *= 2) {
+        if (chunks_per_seg % m) break;
+        const long long ctas = bhp * m;
+        const long long waves = (ctas + la::kNumSMs - 1) / la::kNumSMs;
+        const double cost = (double)waves * ((double)(chunks_per_seg / m) + 2.0);
+        if (cost < best_cost * 0.97) {
+            best_cost = cost;
+            best_m = (int)m;
+        }
+    }
+    s.m = best_m;
+    s.NP = P * best_m;
+    s.T = (L / P) / best_m;
+    return s;
+}
+
+struct FwdLayout {
+    size_t status, S_loc, logG, S_recv, total;
+};
+
+FwdLayout fwd_layout(const la::Split &s, int dk, int dv) {
+    FwdLayout w;
+    const size_t states = (size_t)s.BH * s.NP * dk * dv * sizeof(float);
+    const size_t gam = (size_t)s.BH * s.NP * dk * sizeof(float);
+    w.status = 0;
+    w.S_loc = 256;
+    w.logG = align_up(w.S_loc + states, 256);
+    w.S_recv = align_up(w.logG + gam, 256);
+    w.total = align_up(w.S_recv + states, 256);
+    return w;
+}
+
+template <typename Ptr>
+char *at(Ptr base, size_t off) {
+    return static_cast<char *>(const_cast<void *>(static_cast<const void *>(base))) + off;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_seg_workspace_bytes(int B, int H, long long L, int dk, int dv, int P, int chunk,
+                              la_dtype dt, int backward) {
+    if (check_shape(B, H, L, dk, dv, P, chunk, dt) != LA_OK) return 0;
+    const la::Split s = make_split(B, H, L, P, chunk);
+    if (backward) return 0;  // backward workspace: see la_seg_backward
+    return fwd_layout(s, dk, dv).total;
+}
+
+}  // extern "C"
+
+// ---- per-step entry points ---------------------------------------------------------
+namespace {
+
+la_status check_pass(int B, int H, long long L, int dk, int dv, int NP, int chunk, la_dtype dt,
+                     std::initializer_list<std::pair<const void *, const char *>> need,
+                     std::initializer_list<std::pair<const void *, const char *>> opt) {
+    la_status st = check_shape(B, H, L, dk, dv, NP, chunk, dt);
+    if (st != LA_OK) return st;
+    for (auto &p : need) {
+        if (L > 0 && !p.first) return fail(LA_ERR_ARG, "%s must be non-null", p.second);
+        if (p.first && !aligned(p.first, 16))
+            return fail(LA_ERR_ALIGN, "%s is not 16-byte aligned", p.second);
+    }
+    for (auto &p : opt)
+        if (p.first && !aligned(p.first, 16))
+            return fail(LA_ERR_ALIGN, "%s is not 16-byte aligned", p.second);
+    return LA_OK;
+}
+
+la::PassArgs pass_args(const void *q, const void *k, const void *v, const void *g, void *o,
+                       const float *S_init, float *S_out, float *logG, int *status, int B, int H,
+                       long long L, int dk, int dv, int NP, int chunk, la_dtype dt) {
+    la::PassArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.o = o;
+    a.S_init = S_init; a.S_out = S_out; a.logG = logG; a.status = status;
+    a.L = L; a.T = NP > 0 ? L / NP : 0; a.BH = B * H; a.NP = NP;
+    a.dk = dk; a.dv = dv; a.chunk = chunk; a.dt = dt;
+    return a;
+}
+
+la_status run_pass(const la::PassArgs &a, la::PassMode mode, cudaStream_t st, const char *what) {
+    if (a.L == 0) return LA_OK;
+    cudaError_t e = la::launch_pass(a, mode, st);
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status la_seg_state_pass(const void *k, const void *v, const void *log_g, int B, int H,
+                            long long L, int dk, int dv, int NP, int chunk, la_dtype dt,
+                            float *S_loc, float *log_gamma, int *status, void *cuda_stream) {
+    la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
+                              {{k, "k"}, {v, "v"}, {log_g, "log_g"}, {S_loc, "S_loc"}, {log_gamma, "log_gamma"}}, {});
+    if (st != LA_OK) return st;
+    return run_pass(pass_args(nullptr, k, v, log_g, nullptr, nullptr, S_loc, log_gamma, status, B,
+                              H, L, dk, dv, NP, chunk, dt),
+                    la::kPassState, static_cast<cudaStream_t>(cuda_stream), "state pass");
+}
+
+la_status la_seg_local_pass(const void *q, const void *k, const void *v, const void *log_g, int B,
+                            int H, long long L, int dk, int dv, int NP, int chunk, la_dtype dt,
+                            void *o, float *S_loc, float *log_gamma, int *status,
+                            void *cuda_stream) {
+    la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
+                              {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {o, "o"},
+                               {S_loc, "S_loc"}, {log_gamma, "log_gamma"}}, {});
+    if (st != LA_OK) return st;
+    return run_pass(pass_args(q, k, v, log_g, o, nullptr, S_loc, log_gamma, status, B, H, L, dk, dv,
+                              NP, chunk, dt),
+                    la::kPassLocal, static_cast<cudaStream_t>(cuda_stream), "local pass");
+}
+
+la_status la_seg_output_pass(const void *q, const void *k, const void *v, const void *log_g,
+                             const float *S_recv, int B, int H, long long L, int dk, int dv,
+                             int NP, int chunk, la_dtype dt, void *o, int *status,
+                             void *cuda_stream) {
+    la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
+                              {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {o, "o"}},
+                              {{S_recv, "S_recv"}});
+    if (st != LA_OK) return st;
+    return run_pass(pass_args(q, k, v, log_g, o, S_recv, nullptr, nullptr, status, B, H, L, dk, dv,
+                              NP, chunk, dt),
+                    la::kPassOutput, static_cast<cudaStream_t>(cuda_stream), "output pass");
+}
+
+la_status la_seg_correct_pass(const void *q, const void *log_g, const float *S_recv, int B, int H,
+                              long long L, int dk, int dv, int NP, int chunk, la_dtype dt, void *o,
+                              int *status, void *cuda_stream) {
+    la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
+                              {{q, "q"}, {log_g, "log_g"}, {o, "o"}, {S_recv, "S_recv"}}, {});
+    if (st != LA_OK) return st;
+    return run_pass(pass_args(q, nullptr, nullptr, log_g, o, S_recv, nullptr, nullptr, status, B,
+                              H, L, dk, dv, NP, chunk, dt),
+                    la::kPassCorrect, static_cast<cudaStream_t>(cuda_stream), "correction pass");
+}
+
+int la_seg_subsegments(int B, int H, long long L, int dk, int dv, int P, int chunk, la_dtype dt) {
+    if (check_shape(B, H, L, dk, dv, P, chunk, dt) != LA_OK) return 0;
+    return make_split(B, H, L, P, chunk).NP;
+}
+
+la_status la_seg_forward(const void *q, const void *k, const void *v, const void *log_g,
+                         const float *S0, int B, int H, long long L, int dk, int dv, int P,
+                         int chunk, la_dtype dt, void *o, float *S_final, float *S_recv_save,
+                         int schedule, void *workspace, size_t ws_bytes, void *cuda_stream) {
+    la_status st = check_shape(B, H, L, dk, dv, P, chunk, dt);
+    if (st != LA_OK) return st;
+    if (schedule != LA_SCHED_AUTO && schedule != LA_SCHED_TWO_PASS &&
+        schedule != LA_SCHED_THREE_PHASE)
+        return fail(LA_ERR_ARG, "unknown schedule %d", schedule);
+    if (L > 0 && (!q || !k || !v || !log_g || !o))
+        return fail(LA_ERR_ARG, "q, k, v, log_g and o must be non-null");
+    const void *ptrs[] = {q, k, v, log_g, o, S0, S_final, S_recv_save};
+    const char *names[] = {"q", "k", "v", "log_g", "o", "S0", "S_final", "S_recv_save"};
+    for (int i = 0; i < 8; ++i)
+        if (ptrs[i] && !aligned(ptrs[i], 16))
+            return fail(LA_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    const la::Split s = make_split(B, H, L, P, chunk);
+    const FwdLayout w = fwd_layout(s, dk, dv);
+    if (!workspace || ws_bytes < w.total)
+        return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu%s)", w.total,
+                    ws_bytes, workspace ? "" : ", null");
+    if (!aligned(workspace, 256)) return fail(LA_ERR_ALIGN, "workspace is not 256-byte aligned");
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    int *status = reinterpret_cast<int *>(at(workspace, w.status));
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "status reset");
+
+    if (L == 0) {
+        if (S_final && (e = la::launch_copy_state(S0, s.BH, dk, dv, S_final, stream)) != cudaSuccess)
+            return cuda_fail(e, "S_final copy");
+        if (S_recv_save &&
+            (e = la::launch_broadcast_state(S0, s.BH, P, dk, dv, S_recv_save, stream)) != cudaSuccess)
+            return cuda_fail(e, "S_recv_save fill");
+        return LA_OK;
+    }
+
+    float *S_loc = reinterpret_cast<float *>(at(workspace, w.S_loc));
+    float *logG = reinterpret_cast<float *>(at(workspace, w.logG));
+    float *S_recv = reinterpret_cast<float *>(at(workspace, w.S_recv));
+
+    la::PassArgs a = pass_args(q, k, v, log_g, o, nullptr, S_loc, logG, status, B, H, L, dk, dv,
+                               s.NP, chunk, dt);
+    const bool three = schedule == LA_SCHED_THREE_PHASE;
+    // 1. per sub-segment: local state from zero (+ intra-chunk outputs for three-phase)
+    if ((e = la::launch_pass(a, three ? la::kPassLocal : la::kPassState, stream)) != cudaSuccess)
+        return cuda_fail(e, three ? "local pass" : "state pass");
+    // 2. exclusive decayed scan across sub-segments
+    if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_final, stream)) !=
+        cudaSuccess)
+        return cuda_fail(e, "state scan");
+    // 3. outputs from the received states (two-pass) or the q . S_recv correction (three-phase)
+    a.S_init = S_recv;
+    if ((e = la::launch_pass(a, three ? la::kPassCorrect : la::kPassOutput, stream)) != cudaSuccess)
+        return cuda_fail(e, three ? "correction pass" : "output pass");
+    if (S_recv_save &&
+        (e = la::launch_gather_states(S_recv, s.BH, s.NP, s.m, dk, dv, S_recv_save, stream)) !=
+            cudaSuccess)
+        return cuda_fail(e, "S_recv_save gather");
+    return LA_OK;
+}
+
+la_status la_seg_backward(const void *, const void *, const void *, const void *, const float *,
+                          const float *, const void *, const float *, int, int, long long, int,
+                          int, int, int, la_dtype, void *, void *, void *, void *, float *, void *,
+                          size_t, void *) {
+    return fail(LA_ERR_SHAPE, "la_seg_backward: not built in this version");
+}
+
+la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
+                      int NP, int dk, int dv, int reverse, float *out, float *final_state,
+                      void *cuda_stream) {
+    if (BH < 0 || NP < 0 || dk < 1 || dv < 4 || dv % 4)
+        return fail(LA_ERR_SHAPE, "need BH, NP >= 0, dk >= 1, dv a positive multiple of 4");
+    if ((long long)BH * NP > 0 && (!S_in || !log_gamma || !out))
+        return fail(LA_ERR_ARG, "S_in, log_gamma and out must be non-null");
+    const void *ptrs[] = {S_in, init, out, final_state};
+    const char *names[] = {"S_in", "init", "out", "final_state"};
+    for (int i = 0; i < 4; ++i)
+        if (ptrs[i] && !aligned(ptrs[i], 16))
+            return fail(LA_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    if (log_gamma && !aligned(log_gamma, 4)) return fail(LA_ERR_ALIGN, "log_gamma misaligned");
+    if (S_in && out == S_in) return fail(LA_ERR_ARG, "out may not alias S_in");
+    cudaError_t e = la::launch_scan(S_in, log_gamma, init, BH, NP, dk, dv, reverse, out,
+                                    final_state, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, "scan");
+}
+
+la_status la_seg_check_status(void *workspace, void *cuda_stream) {
+    if (!workspace) return fail(LA_ERR_ARG, "workspace is null");
+    int h = 0;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (h & la::kStatusTimeout) return fail(LA_ERR_TIMEOUT, "a device-side wait gave up");
+    if (h & la::kStatusGateRange)
+        return fail(LA_ERR_GATE_RANGE,
+                    "some chunk has |sum of log_g| > %.0f in a key dimension; use a smaller chunk",
+                    (double)la::kGateRangeLimit);
+    return LA_OK;
+}
+
+la_status la_last_error_detail(char *buf, size_t n) {
+    if (!buf || n == 0) return LA_ERR_ARG;
+    strncpy(buf, g_detail, n - 1);
+    buf[n - 1] = '\0';
+    return LA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+// scan.cu -- exclusive decayed scan of fp32 dk x dv states across segments.
+//
+// The All-Scan state update of the ZeCO review ("key machinery", Alg. 2 as the referee
+// corrects it: the accumulated state moves on, not the local one), run on one device:
+//
+//   acc = init;  for p in order:  out[p] = acc;  acc = exp(log_gamma[p][i]) * acc + S_in[p]
+//
+// Rows i (and columns j) are independent, so the scan is element-parallel over
+// (bh, i, j/4) and sequential over p.  It is HBM-bound: every thread streams float4 states,
+// with the loads of UNROLL segments issued before the dependent FMA chain consumes them.
+// Splitting d_k into blocks (the review's K blocks of All-Scan) changes nothing here: each
+// element's chain is the same whatever the block split.
+#include "common.cuh"
+#include "internal.h"
+
+namespace la {
+namespace {
+
+constexpr int kScanThreads = 256;
+constexpr int kUnroll = 8;
+
+__global__ void __launch_bounds__(kScanThreads)
+scan_kernel(const float4 *__restrict__ S_in, const float *__restrict__ log_gamma,
+            const float4 *__restrict__ init, int BH, int NP, int dk, int dv4, int reverse,
+            float4 *__restrict__ out, float4 *__restrict__ final_state) {
+    const long long e = (long long)blockIdx.x * kScanThreads + threadIdx.x;  // (bh, i, j4)
+    const long long per_bh = (long long)dk * dv4;
+    if (e >= (long long)BH * per_bh) return;
+    const long long bh = e / per_bh;
+    const long long ij = e % per_bh;
+    const int i = (int)(ij / dv4);
+    const float4 *src = S_in + bh * NP * per_bh + ij;
+    float4 *dst = out + bh * NP * per_bh + ij;
+    const float *lg = log_gamma + bh * (long long)NP * dk + i;
+
+    float4 acc = init ? init[bh * per_bh + ij] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < NP; p0 += kUnroll) {
+        float4 x[kUnroll];
+        float gm[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int p = p0 + u;
+            if (p < NP) {
+                const int pp = reverse ? NP - 1 - p : p;
+                x[u] = __ldcs(src + (long long)pp * per_bh);
+                gm[u] = __expf(lg[(long long)pp * dk]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int p = p0 + u;
+            if (p < NP) {
+                const int pp = reverse ? NP - 1 - p : p;
+                __stcs(dst + (long long)pp * per_bh, acc);
+                acc.x = fmaf(gm[u], acc.x, x[u].x);
+                acc.y = fmaf(gm[u], acc.y, x[u].y);
+                acc.z = fmaf(gm[u], acc.z, x[u].z);
+                acc.w = fmaf(gm[u], acc.w, x[u].w);
+            }
+        }
+    }
+    if (final_state) final_state[bh * per_bh + ij] = acc;
+}
+
+__global__ void gather_states_kernel(const float4 *__restrict__ src, int BH, int NP, int m,
+                                     long long per_state4, float4 *__restrict__ dst) {
+    const int P = NP / m;
+    const long long n = (long long)BH * P * per_state4;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long bhp = e / per_state4, r = e % per_state4;
+        const long long bh = bhp / P, p = bhp % P;
+        dst[e] = src[(bh * NP + p * m) * per_state4 + r];
+    }
+}
+
+__global__ void copy_state_kernel(const float4 *__restrict__ src, long long n4,
+                                  float4 *__restrict__ dst) {
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n4;
+         e += (long long)gridDim.x * blockDim.x)
+        dst[e] = src ? src[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+}  // namespace
+
+cudaError_t launch_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
+                        int NP, int dk, int dv, int reverse, float *out, float *final_state,
+                        cudaStream_t st) {
+    const int dv4 = dv / 4;
+    const long long n = (long long)BH * dk * dv4;
+    if (n == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)((n + kScanThreads - 1) / kScanThreads);
+    scan_kernel<<<blocks, kScanThreads, 0, st>>>(
+        reinterpret_cast<const float4 *>(S_in), log_gamma, reinterpret_cast<const float4 *>(init),
+        BH, NP, dk, dv4, reverse, reinterpret_cast<float4 *>(out),
+        reinterpret_cast<float4 *>(final_state));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_states(const float *src, int BH, int NP, int m, int dk, int dv,
+                                 float *dst, cudaStream_t st) {
+    const long long per4 = (long long)dk * dv / 4;
+    const long long n = (long long)BH * (NP / m) * per4;
+    if (n == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    gather_states_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(src), BH, NP, m,
+                                                 per4, reinterpret_cast<float4 *>(dst));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_state(const float *src, int BH, int dk, int dv, float *dst,
+                              cudaStream_t st) {
+    const long long n4 = (long long)BH * dk * dv / 4;
+    if (n4 == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
+    copy_state_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(src), n4,
+                                              reinterpret_cast<float4 *>(dst));
+    return cudaGetLastError();
+}
+
+}  // namespace la
+
+namespace la {
+namespace {
+__global__ void broadcast_state_kernel(const float4 *__restrict__ src, int BH, int P,
+                                       long long per4, float4 *__restrict__ dst) {
+    const long long n = (long long)BH * P * per4;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long bhp = e / per4, r = e % per4;
+        const long long bh = bhp / P;
+        dst[e] = src ? src[bh * per4 + r] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+}  // namespace
+
+cudaError_t launch_broadcast_state(const float *src, int BH, int P, int dk, int dv, float *dst,
+                                   cudaStream_t st) {
+    const long long per4 = (long long)dk * dv / 4;
+    const long long n = (long long)BH * P * per4;
+    if (n == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    broadcast_state_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(src), BH, P,
+                                                   per4, reinterpret_cast<float4 *>(dst));
+    return cudaGetLastError();
+}
+}  // namespace la

@@ -1,0 +1,263 @@
+"""ctypes binding of libla_seg.so -- argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module checks tensor
+placement and dtypes, allocates outputs and the workspace through PyTorch (plumbing), passes
+raw device pointers and the current CUDA stream, and raises ``LaSegError`` on any non-OK
+status.  There is no CPU or PyTorch fallback: if the library is missing, importing the
+functions fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libla_seg.so")
+
+LA_OK = 0
+STATUS_NAMES = {0: "LA_OK", -1: "LA_ERR_ARG", -2: "LA_ERR_SHAPE", -3: "LA_ERR_ALIGN",
+                -4: "LA_ERR_DTYPE", -5: "LA_ERR_WORKSPACE", -6: "LA_ERR_GATE_RANGE",
+                -7: "LA_ERR_TIMEOUT", -8: "LA_ERR_CUDA"}
+LA_F32, LA_BF16 = 0, 1
+SCHED_AUTO, SCHED_TWO_PASS, SCHED_THREE_PHASE = 0, 1, 2
+EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_seg_scan",
+            "la_seg_state_pass", "la_seg_local_pass", "la_seg_output_pass", "la_seg_correct_pass",
+            "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail")
+
+_lib = None
+
+
+class LaSegError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
+
+
+def lib():
+    """The loaded library (ctypes.CDLL) with argument types declared."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m sequence_linear_attention_chunked_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+        L.la_seg_workspace_bytes.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32, i32]
+        L.la_seg_workspace_bytes.restype = sz
+        L.la_seg_forward.argtypes = [P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32,
+                                     P, P, P, i32, P, sz, P]
+        L.la_seg_forward.restype = i32
+        L.la_seg_backward.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
+                                      i32, P, P, P, P, P, P, sz, P]
+        L.la_seg_backward.restype = i32
+        L.la_seg_scan.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P]
+        L.la_seg_scan.restype = i32
+        L.la_seg_state_pass.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P, P, P]
+        L.la_seg_state_pass.restype = i32
+        L.la_seg_local_pass.argtypes = [P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P, P,
+                                        P, P]
+        L.la_seg_local_pass.restype = i32
+        L.la_seg_output_pass.argtypes = [P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P,
+                                         P, P]
+        L.la_seg_output_pass.restype = i32
+        L.la_seg_correct_pass.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P, P]
+        L.la_seg_correct_pass.restype = i32
+        L.la_seg_subsegments.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32]
+        L.la_seg_subsegments.restype = i32
+        L.la_seg_check_status.argtypes = [P, P]
+        L.la_seg_check_status.restype = i32
+        L.la_last_error_detail.argtypes = [ctypes.c_char_p, sz]
+        L.la_last_error_detail.restype = i32
+        _lib = L
+    return _lib
+
+
+def la_last_error_detail() -> str:
+    buf = ctypes.create_string_buffer(512)
+    lib().la_last_error_detail(buf, 512)
+    return buf.value.decode(errors="replace")
+
+
+def _check(status: int, where: str):
+    if status != LA_OK:
+        raise LaSegError(status, where, la_last_error_detail())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LA_F32
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, shape=None, device=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def la_seg_workspace_bytes(B, H, L, dk, dv, P, chunk, dt=LA_BF16, backward=False) -> int:
+    return int(lib().la_seg_workspace_bytes(B, H, L, dk, dv, P, chunk, dt, int(bool(backward))))
+
+
+def workspace(B, H, L, dk, dv, P, chunk, dt, backward=False, device="cuda"):
+    """A caller-owned workspace of the size the library asks for (256-byte aligned)."""
+    n = la_seg_workspace_bytes(B, H, L, dk, dv, P, chunk, dt, backward)
+    if n == 0:
+        raise LaSegError(-2, "la_seg_workspace_bytes", "sizes rejected by the library")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def la_seg_forward(q, k, v, log_g, S0=None, P=1, chunk=64, schedule=SCHED_AUTO, *, o=None,
+                   want_S_final=True, want_S_recv=False, ws=None, stream=None):
+    """o, S_final, S_recv = la_seg_forward(q, k, v, log_g, S0, P, chunk).
+
+    q, k, log_g [B,H,L,dk], v [B,H,L,dv]: float32 or bfloat16 CUDA tensors of one dtype.
+    S0: fp32 [B,H,dk,dv] or None.  S_final / S_recv (fp32 [B,H,dk,dv] / [B,H,P,dk,dv]) are
+    None unless asked for.
+    """
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    for t, n, shp in ((q, "q", (B, H, L, dk)), (k, "k", (B, H, L, dk)), (v, "v", (B, H, L, dv)),
+                      (log_g, "log_g", (B, H, L, dk))):
+        _need(t, n, q.dtype, shp, dev)
+    _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    dt = _dt(q)
+    if o is None:
+        o = torch.empty((B, H, L, dv), dtype=q.dtype, device=dev)
+    _need(o, "o", q.dtype, (B, H, L, dv), dev)
+    S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_S_final else None
+    S_recv = torch.empty((B, H, P, dk, dv), dtype=torch.float32, device=dev) if want_S_recv else None
+    if ws is None:
+        ws = workspace(B, H, L, dk, dv, P, chunk, dt, False, dev)
+    st = lib().la_seg_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(S0), B, H, L, dk, dv,
+                              P, chunk, dt, _ptr(o), _ptr(S_final), _ptr(S_recv), int(schedule),
+                              _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "la_seg_forward")
+    return o, S_final, S_recv
+
+
+def la_seg_backward(q, k, v, log_g, dO, S0=None, S_recv_saved=None, dS_final=None, P=1,
+                    chunk=64, *, want_dS0=False, ws=None, stream=None):
+    """dq, dk, dv, dlog_g, dS0 for loss = <o, dO> + <S_final, dS_final>."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    for t, n, shp in ((q, "q", (B, H, L, dk)), (k, "k", (B, H, L, dk)), (v, "v", (B, H, L, dv)),
+                      (log_g, "log_g", (B, H, L, dk)), (dO, "dO", (B, H, L, dv))):
+        _need(t, n, q.dtype, shp, dev)
+    _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    _need(S_recv_saved, "S_recv_saved", torch.float32, (B, H, P, dk, dv), dev)
+    _need(dS_final, "dS_final", torch.float32, (B, H, dk, dv), dev)
+    dt = _dt(q)
+    dq = torch.empty_like(q)
+    dk_ = torch.empty_like(k)
+    dv_ = torch.empty_like(v)
+    dg = torch.empty_like(log_g)
+    dS0 = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_dS0 else None
+    if ws is None:
+        ws = workspace(B, H, L, dk, dv, P, chunk, dt, True, dev)
+    st = lib().la_seg_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(S0),
+                               _ptr(S_recv_saved), _ptr(dO), _ptr(dS_final), B, H, L, dk, dv, P,
+                               chunk, dt, _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dS0),
+                               _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "la_seg_backward")
+    return dq, dk_, dv_, dg, dS0
+
+
+def la_seg_scan(S_in, log_gamma, init=None, reverse=False, *, want_final=True, stream=None):
+    """out, final = exclusive decayed scan over dim 1 of S_in [BH, NP, dk, dv] (fp32)."""
+    BH, NP, dk, dv = S_in.shape
+    dev = S_in.device
+    _need(S_in, "S_in", torch.float32, None, dev)
+    _need(log_gamma, "log_gamma", torch.float32, (BH, NP, dk), dev)
+    _need(init, "init", torch.float32, (BH, dk, dv), dev)
+    out = torch.empty_like(S_in)
+    final = torch.empty((BH, dk, dv), dtype=torch.float32, device=dev) if want_final else None
+    st = lib().la_seg_scan(_ptr(S_in), _ptr(log_gamma), _ptr(init), BH, NP, dk, dv,
+                           int(bool(reverse)), _ptr(out), _ptr(final), _stream(stream))
+    _check(st, "la_seg_scan")
+    return out, final
+
+
+def la_seg_check_status(ws, stream=None):
+    """Synchronise and raise LaSegError if a kernel flagged a device-side condition."""
+    _check(lib().la_seg_check_status(_ptr(ws), _stream(stream)), "la_seg_check_status")
+
+
+# ---- the steps of the path (see la_seg.h) ----------------------------------------------
+def la_seg_subsegments(B, H, L, dk, dv, P, chunk, dt=LA_BF16) -> int:
+    """Segments per (b, h) that la_seg_forward runs its passes over (P times the split)."""
+    return int(lib().la_seg_subsegments(B, H, L, dk, dv, P, chunk, dt))
+
+
+def _seq_shapes(q_or_k, v=None):
+    B, H, L, dk = q_or_k.shape
+    dv = v.shape[-1] if v is not None else dk
+    return B, H, L, dk, dv
+
+
+def la_seg_state_pass(k, v, log_g, NP, chunk, *, S_loc=None, log_gamma=None, status=None,
+                      stream=None):
+    B, H, L, dk, dv = _seq_shapes(k, v)
+    dev = k.device
+    S_loc = torch.empty((B, H, NP, dk, dv), dtype=torch.float32, device=dev) if S_loc is None else S_loc
+    log_gamma = (torch.empty((B, H, NP, dk), dtype=torch.float32, device=dev)
+                 if log_gamma is None else log_gamma)
+    _check(lib().la_seg_state_pass(_ptr(k), _ptr(v), _ptr(log_g), B, H, L, dk, dv, NP, chunk,
+                                   _dt(k), _ptr(S_loc), _ptr(log_gamma), _ptr(status),
+                                   _stream(stream)), "la_seg_state_pass")
+    return S_loc, log_gamma
+
+
+def la_seg_local_pass(q, k, v, log_g, NP, chunk, *, o=None, S_loc=None, log_gamma=None,
+                      status=None, stream=None):
+    B, H, L, dk, dv = _seq_shapes(q, v)
+    dev = q.device
+    o = torch.empty((B, H, L, dv), dtype=q.dtype, device=dev) if o is None else o
+    S_loc = torch.empty((B, H, NP, dk, dv), dtype=torch.float32, device=dev) if S_loc is None else S_loc
+    log_gamma = (torch.empty((B, H, NP, dk), dtype=torch.float32, device=dev)
+                 if log_gamma is None else log_gamma)
+    _check(lib().la_seg_local_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), B, H, L, dk, dv, NP,
+                                   chunk, _dt(q), _ptr(o), _ptr(S_loc), _ptr(log_gamma),
+                                   _ptr(status), _stream(stream)), "la_seg_local_pass")
+    return o, S_loc, log_gamma
+
+
+def la_seg_output_pass(q, k, v, log_g, S_recv, NP, chunk, *, o=None, status=None, stream=None):
+    B, H, L, dk, dv = _seq_shapes(q, v)
+    o = torch.empty((B, H, L, dv), dtype=q.dtype, device=q.device) if o is None else o
+    _check(lib().la_seg_output_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(S_recv), B, H, L,
+                                    dk, dv, NP, chunk, _dt(q), _ptr(o), _ptr(status),
+                                    _stream(stream)), "la_seg_output_pass")
+    return o
+
+
+def la_seg_correct_pass(q, log_g, S_recv, NP, chunk, o, *, status=None, stream=None):
+    B, H, L, dk, dv = _seq_shapes(q, o)
+    _check(lib().la_seg_correct_pass(_ptr(q), _ptr(log_g), _ptr(S_recv), B, H, L, dk, dv, NP,
+                                     chunk, _dt(q), _ptr(o), _ptr(status), _stream(stream)),
+           "la_seg_correct_pass")
+    return o

@@ -1,0 +1,112 @@
+"""The C ABI library on the host: it loads, exports what include/la_seg.h declares, sizes its
+workspace, and rejects bad arguments before touching a GPU (CPU only, no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sequence_linear_attention_chunked_b200 import build as la_build
+from sequence_linear_attention_chunked_b200 import la_seg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "la_seg.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    la_build.build()
+    return la_seg.lib()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(", src)))
+
+
+def test_header_declares_binding_symbols():
+    assert declared_symbols() == sorted(la_seg.EXPORTED)
+
+
+def test_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {la_seg.LIB_PATH}").read()
+    exported = set(re.findall(r" T (la_\w+)", out))
+    assert set(declared_symbols()) <= exported
+
+
+def test_workspace_sizes(lib):
+    w = la_seg.la_seg_workspace_bytes
+    assert w(1, 16, 16384, 128, 128, 1, 64) > 0
+    assert w(1, 16, 4194304, 128, 128, 256, 64) > 0
+    assert w(1, 2, 256, 32, 32, 4, 16, la_seg.LA_F32) > 0
+    assert w(1, 1, 0, 32, 32, 1, 16) > 0  # empty sequence is legal
+    # rejected sizes report 0
+    assert w(1, 1, 100, 32, 32, 3, 16) == 0     # L % P
+    assert w(1, 1, 96, 32, 32, 1, 64) == 0      # segment not a multiple of chunk
+    assert w(1, 1, 64, 48, 48, 1, 16) == 0      # d not supported
+    assert w(1, 1, 64, 32, 64, 1, 16) == 0      # dk != dv
+    assert w(1, 1, 64, 32, 32, 1, 8) == 0       # chunk not supported
+    assert w(1, 1, 64, 32, 32, 1, 16, 7) == 0   # dtype
+
+
+def _fwd(lib, **kw):
+    """Calls la_seg_forward with fake (but aligned) pointers: only argument checks may run."""
+    args = dict(q=0x1000, k=0x2000, v=0x3000, g=0x4000, S0=None, B=1, H=1, L=64, dk=32, dv=32,
+                P=1, chunk=16, dt=0, o=0x5000, Sf=None, Sr=None, sched=0, ws=0x10000,
+                ws_bytes=1 << 30, stream=None)
+    args.update(kw)
+    V = ctypes.c_void_p
+    return lib.la_seg_forward(V(args["q"]), V(args["k"]), V(args["v"]), V(args["g"]),
+                              V(args["S0"]), args["B"], args["H"], args["L"], args["dk"],
+                              args["dv"], args["P"], args["chunk"], args["dt"], V(args["o"]),
+                              V(args["Sf"]), V(args["Sr"]), args["sched"], V(args["ws"]),
+                              args["ws_bytes"], V(args["stream"]))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(L=100, P=3), -2),
+    (dict(L=96, chunk=64), -2),
+    (dict(dk=48, dv=48), -2),
+    (dict(dk=32, dv=64), -2),
+    (dict(chunk=8), -2),
+    (dict(B=0), -2),
+    (dict(P=0), -2),
+    (dict(L=-64), -2),
+    (dict(dt=5), -4),
+    (dict(q=None), -1),
+    (dict(o=None), -1),
+    (dict(sched=9), -1),
+    (dict(q=0x1008), -3),
+    (dict(S0=0x7004), -3),
+    (dict(ws=None), -5),
+    (dict(ws_bytes=16), -5),
+    (dict(ws=0x10010), -3),
+])
+def test_forward_rejects_bad_arguments(lib, kw, status):
+    assert _fwd(lib, **kw) == status
+    assert len(la_seg.la_last_error_detail()) > 0
+
+
+def test_scan_rejects_bad_arguments(lib):
+    V = ctypes.c_void_p
+    assert lib.la_seg_scan(V(0x1000), V(0x2000), None, 1, 2, 32, 30, 0, V(0x3000), None, None) == -2
+    assert lib.la_seg_scan(None, V(0x2000), None, 1, 2, 32, 32, 0, V(0x3000), None, None) == -1
+    assert lib.la_seg_scan(V(0x1004), V(0x2000), None, 1, 2, 32, 32, 0, V(0x3000), None, None) == -3
+    assert lib.la_seg_scan(V(0x1000), V(0x2000), None, 1, 2, 32, 32, 0, V(0x1000), None, None) == -1
+
+
+def test_error_detail_handles_small_buffers(lib):
+    assert _fwd(lib, chunk=8) == -2
+    buf = ctypes.create_string_buffer(8)
+    assert lib.la_last_error_detail(buf, 8) == 0
+    assert len(buf.value) == 7
+    assert lib.la_last_error_detail(None, 8) == -1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(la_seg, "_lib", None)
+    monkeypatch.setattr(la_seg, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        la_seg.lib()

@@ -1,0 +1,150 @@
+"""Forward parity of the CUDA path (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sequence_linear_attention_chunked_b200 import la_seg
+from sequence_linear_attention_chunked_b200.inputs import WORKLOADS, Workload, make_inputs
+from tests.parity import TOL, oracle_window, rel_err
+
+pytestmark = pytest.mark.gpu
+
+SCHEDULES = [la_seg.SCHED_TWO_PASS, la_seg.SCHED_THREE_PHASE]
+
+
+def run(x, w, schedule=la_seg.SCHED_AUTO, want_recv=True):
+    ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk,
+                          la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16, False, x["q"].device)
+    o, Sf, Sr = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], x.get("S0"), w.P, w.chunk,
+                                      schedule, want_S_recv=want_recv, ws=ws)
+    la_seg.la_seg_check_status(ws)
+    return o, Sf, Sr
+
+
+def full_check(w, device, with_s0=False, schedule=la_seg.SCHED_AUTO):
+    x = make_inputs(w, device, with_s0=with_s0)
+    o, Sf, Sr = run(x, w, schedule)
+    o_ref, Sf_ref, Sr_ref = oracle.forward(x["q"], x["k"], x["v"], x["log_g"], x.get("S0"),
+                                           seg_len=w.L // w.P)
+    tol = TOL[w.torch_dtype]
+    errs = (rel_err(o, o_ref), rel_err(Sf, Sf_ref), rel_err(Sr, Sr_ref))
+    assert errs[0] <= tol and errs[1] <= tol and errs[2] <= tol, (w.describe(), errs)
+    return errs
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_c0_fp32(cuda_device, schedule):
+    full_check(WORKLOADS["C0"], cuda_device, schedule=schedule)
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_c0_fp32_with_s0(cuda_device, schedule):
+    full_check(WORKLOADS["C0"], cuda_device, with_s0=True, schedule=schedule)
+
+
+SMALL = [  # (B, H, L, d, P, chunk, dtype, dist)
+    (1, 2, 512, 128, 2, 64, "bf16", "gla"),
+    (2, 3, 768, 64, 3, 32, "bf16", "gla"),
+    (1, 1, 64, 32, 4, 16, "bf16", "toy"),
+    (1, 2, 1024, 128, 1, 64, "f32", "gla"),
+    (1, 4, 2048, 128, 8, 64, "bf16", "weak"),
+    (3, 1, 192, 32, 1, 64, "f32", "toy"),
+    (1, 1, 128, 128, 2, 64, "bf16", "gla"),   # one chunk per segment... x2
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_small_shapes(cuda_device, shape, schedule):
+    B, H, L, d, P, C, dt, dist = shape
+    w = Workload("small", B, H, L, d, d, P, C, dt, dist, seed=L + d)
+    full_check(w, cuda_device, with_s0=(L % 3 == 0), schedule=schedule)
+
+
+def test_weak_decay_scan_matters(cuda_device):
+    """Weak decay: the received state carries real signal into every segment."""
+    w = WORKLOADS["WEAK"].with_(H=2, L=8192, P=4)
+    x = make_inputs(w, cuda_device, with_s0=True)
+    o, Sf, Sr = run(x, w)
+    o_ref, Sf_ref, Sr_ref = oracle.forward(x["q"], x["k"], x["v"], x["log_g"], x["S0"],
+                                           seg_len=w.L // w.P)
+    assert np.abs(Sr_ref[:, :, 1:]).max() > 0.1  # the scan is not trivially zero here
+    for got, ref in ((o, o_ref), (Sf, Sf_ref), (Sr, Sr_ref)):
+        assert rel_err(got, ref) <= 2e-2
+
+
+def test_empty_sequence(cuda_device):
+    w = Workload("empty", 1, 2, 0, 32, 32, 3, 16, "f32", "toy")
+    x = make_inputs(w, cuda_device, with_s0=True)
+    o, Sf, Sr = run(x, w)
+    assert o.numel() == 0
+    assert torch.equal(Sf, x["S0"])
+    assert torch.equal(Sr, x["S0"][:, :, None].expand(-1, -1, 3, -1, -1))
+
+
+def test_deterministic(cuda_device):
+    w = WORKLOADS["C1"].with_(H=4, L=4096)
+    x = make_inputs(w, cuda_device)
+    o1, s1, _ = run(x, w)
+    o2, s2, _ = run(x, w)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_schedules_agree(cuda_device):
+    w = WORKLOADS["C1"].with_(H=2, L=4096, P=4)
+    x = make_inputs(w, cuda_device, with_s0=True)
+    a = run(x, w, la_seg.SCHED_TWO_PASS)
+    b = run(x, w, la_seg.SCHED_THREE_PHASE)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])  # same state path
+    assert rel_err(a[0], b[0].double().cpu().numpy()) <= 2e-2
+
+
+def test_gate_range_flagged(cuda_device):
+    """A chunk whose log-gate sum leaves the factorisation's range is reported, not hidden."""
+    w = Workload("strong", 1, 1, 128, 32, 32, 1, 64, "f32", "toy")
+    x = make_inputs(w, cuda_device)
+    x["log_g"].fill_(-2.0)  # chunk sum -128 < -80
+    ws = la_seg.workspace(1, 1, 128, 32, 32, 1, 64, la_seg.LA_F32, False, cuda_device)
+    la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, 1, 64, ws=ws)
+    with pytest.raises(la_seg.LaSegError) as ei:
+        la_seg.la_seg_check_status(ws)
+    assert ei.value.status == -6
+    # the same data in chunks of 16 (sum -32) is fine and matches the oracle
+    w16 = w.with_(chunk=16)
+    ws16 = la_seg.workspace(1, 1, 128, 32, 32, 1, 16, la_seg.LA_F32, False, cuda_device)
+    o, _, _ = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, 1, 16, ws=ws16)
+    la_seg.la_seg_check_status(ws16)
+    o_ref, _, _ = oracle.forward(x["q"], x["k"], x["v"], x["log_g"])
+    assert rel_err(o, o_ref) <= 1e-4
+
+
+# --------------------------------------------------------------------------- full sizes
+def test_c1_full(cuda_device):
+    """The bench workload at full size; the oracle checks 4 whole heads."""
+    w = WORKLOADS["C1"]
+    x = make_inputs(w, cuda_device)
+    o, Sf, _ = run(x, w, want_recv=False)
+    heads = [0, 5, 10, 15]
+    sub = {n: x[n][:, heads] for n in ("q", "k", "v", "log_g")}
+    o_ref, Sf_ref, _ = oracle.forward(sub["q"], sub["k"], sub["v"], sub["log_g"])
+    assert rel_err(o[:, heads], o_ref) <= 2e-2
+    assert rel_err(Sf[:, heads], Sf_ref) <= 2e-2
+
+
+@pytest.mark.parametrize("name", ["C2", "C3"])
+def test_large_sampled(cuda_device, name):
+    """C2 / C3 at full size: sampled windows (including segment starts) against the oracle."""
+    w = WORKLOADS[name]
+    x = make_inputs(w, cuda_device)
+    o, Sf, _ = run(x, w, want_recv=False)
+    T = w.L // w.P
+    rng = np.random.default_rng(7)
+    for h in (0, w.H - 1):
+        for p in (0, 1, w.P - 1, int(rng.integers(1, w.P))):
+            for t0 in (p * T, p * T + int(rng.integers(0, T - 512)) // 64 * 64):
+                ref = oracle_window(x, 0, h, t0, t0 + 512)
+                got = o[0, h, t0:t0 + 512]
+                assert rel_err(got, ref) <= 2e-2, (name, h, p, t0)
+    del x, o
+    torch.cuda.empty_cache()
