@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kThreads) simt_pass_kernel(PassArgs a) {
         for (int idx = tid; idx < DK * DV; idx += kThreads) Sout[idx] = sS[idx];
         if (tid < DK) a.logG[((long long)bh * a.NP + j) * DK + tid] = logG;
     }
-    if (range_bad) atomicOr(a.status, kStatusGateRange);
+    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
 }
 
 template <typename T, int DK, int DV, int C, int MODE>
