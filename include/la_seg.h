@@ -163,6 +163,33 @@ LA_API la_status la_seg_correct_pass(const void *q, const void *log_g, const flo
 LA_API int la_seg_subsegments(int B, int H, long long L, int dk, int dv, int P, int chunk,
                               la_dtype dt);
 
+/* ---- Forward for callers that cannot allocate device memory --------------------------
+ * The ZeCO pages have no counterpart to this entry point; it exists for deployments, not for
+ * the method.  Some callers cannot call cudaMalloc: plug-ins hosted by an engine that owns
+ * every byte of device memory through its own pool, runtimes that forbid any allocation
+ * after start-up (fixed memory budgets, certified real-time loops), or foreign-language
+ * hosts that reach this library but not the CUDA allocator.  They still own q, k, v, log_g,
+ * S0 and the outputs; the scratch comes from a static device array of
+ * LA_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU which loads this library holds until the
+ * process exits.
+ *
+ * Same arguments and result as la_seg_forward, without the workspace.  Sizes whose
+ * workspace (la_seg_workspace_bytes) exceeds LA_NOALLOC_SCRATCH_BYTES are rejected with
+ * LA_ERR_WORKSPACE before anything runs.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  Every call on a device shares the one array, which keeps
+ * the last call's contents (the status word is cleared at the start of each call): calls
+ * that overlap on the GPU -- on different streams, or from different host threads -- race
+ * on it and must be serialised by the caller.  Device-side conditions (LA_ERR_GATE_RANGE)
+ * are not reported by this entry point. */
+#define LA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+LA_API la_status la_seg_forward_noalloc(const void *q, const void *k, const void *v,
+                                        const void *log_g, const float *S0, int B, int H,
+                                        long long L, int dk, int dv, int P, int chunk,
+                                        la_dtype dt, void *o, float *S_final, float *S_recv_save,
+                                        int schedule, void *cuda_stream);
+
 /* Synchronises cuda_stream and returns the device status word a previous call left in
  * workspace (LA_OK, LA_ERR_GATE_RANGE or LA_ERR_TIMEOUT), or LA_ERR_CUDA. */
 LA_API la_status la_seg_check_status(void *workspace, void *cuda_stream);

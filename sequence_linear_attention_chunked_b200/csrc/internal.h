@@ -49,6 +49,10 @@ cudaError_t launch_gather_states(const float *src, int BH, int NP, int m, int dk
 cudaError_t launch_broadcast_state(const float *src, int BH, int P, int dk, int dv, float *dst,
                                    cudaStream_t st);
 
+// Record the calling thread's error detail (printf-style) and return s / LA_ERR_CUDA.
+la_status set_error(la_status s, const char *fmt, ...);
+la_status set_cuda_error(cudaError_t e, const char *what);
+
 // Copies S0 (or zeros) into dst [BH, dk, dv].
 cudaError_t launch_copy_state(const float *src, int BH, int dk, int dv, float *dst,
                               cudaStream_t st);

@@ -105,6 +105,20 @@ char *at(Ptr base, size_t off) {
 
 }  // namespace
 
+namespace la {
+
+la_status set_error(la_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+la_status set_cuda_error(cudaError_t e, const char *what) { return cuda_fail(e, what); }
+
+}  // namespace la
+
 extern "C" {
 
 size_t la_seg_workspace_bytes(int B, int H, long long L, int dk, int dv, int P, int chunk,

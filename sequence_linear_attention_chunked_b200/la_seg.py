@@ -24,7 +24,8 @@ LA_F32, LA_BF16 = 0, 1
 SCHED_AUTO, SCHED_TWO_PASS, SCHED_THREE_PHASE = 0, 1, 2
 EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_seg_scan",
             "la_seg_state_pass", "la_seg_local_pass", "la_seg_output_pass", "la_seg_correct_pass",
-            "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail")
+            "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail",
+            "la_seg_forward_noalloc")
 
 _lib = None
 
@@ -66,6 +67,9 @@ def lib():
         L.la_seg_correct_pass.restype = i32
         L.la_seg_subsegments.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32]
         L.la_seg_subsegments.restype = i32
+        L.la_seg_forward_noalloc.argtypes = [P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
+                                             i32, P, P, P, i32, P]
+        L.la_seg_forward_noalloc.restype = i32
         L.la_seg_check_status.argtypes = [P, P]
         L.la_seg_check_status.restype = i32
         L.la_last_error_detail.argtypes = [ctypes.c_char_p, sz]
