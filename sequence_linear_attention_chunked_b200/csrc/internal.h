@@ -33,6 +33,10 @@ struct PassArgs {
 // Generic CUDA-core (FFMA) chunk pass: any supported dtype, d and chunk.
 cudaError_t launch_simt_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
 
+// tcgen05 / TMEM chunk pass (bf16, d_k = d_v = 128, chunk 64).
+bool tc_pass_supported(const PassArgs &a);
+cudaError_t launch_tc_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
+
 // The chunk pass for these arguments: the tensor-core kernels where they apply, else SIMT.
 cudaError_t launch_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
 

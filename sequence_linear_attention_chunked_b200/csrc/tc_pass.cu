@@ -1,0 +1,515 @@
+// tc_pass.cu -- chunkwise GLA passes on the 5th-generation tensor cores (tcgen05 + TMEM),
+// bf16 inputs, d_k = d_v = 128, chunk = 64.
+//
+// One CTA walks one (b, h, segment) chunk by chunk; all matrices of the chunk form live in
+// shared memory (TMA-loaded, 128-byte swizzle) or tensor memory.  Per chunk, with b_t the
+// inclusive in-chunk cumsum of log_g and b_C its total (GLA chunkwise form; the decayed state
+// update is the one of the ZeCO review's "key machinery"):
+//
+//   Qbar'[t,i] = q[t,i] e^{b_t,i - b_C,i}     Ktil[s,i] = k[s,i] e^{b_C,i - b_s,i}
+//   P   = mask_{s<=t}(Qbar' Ktil^T)                       M=64  (t)  N=64  (s)  K=128 (i)
+//   O^T = V^T P^T + S'^T Qbar'^T,  S' = diag(e^{b_C}) S    M=128 (dv) N=64  (t)  K=64 / 128
+//   dS^T = V^T Ktil,  S <- S' + dS                         M=128 (dv) N=128 (i)  K=64  (s)
+//
+// The outputs and the state are kept transposed (d_v on the TMEM lanes) so that each pair of
+// the 256 epilogue threads owns one d_v column: each keeps half of that column of the fp32
+// state in registers, scales it by the decay (per-row factors from shared memory), and writes its bf16
+// copy straight into tensor memory as the A operand of the inter-chunk MMA -- the state never
+// goes through shared memory.  q and k tiles are rescaled in place by the gate warps (one
+// thread per key dimension runs the sequential cumsum), so every MMA operand has the layout
+// TMA wrote.
+//
+// Warp roles (448 threads): 0-7 epilogue (TMEM lane quarter = warp % 4; warps 0-3 own key
+// dims 0-63 of the state column, warps 4-7 key dims 64-127), 8-11 gates, 12 TMA producer,
+// 13 MMA issuer / TMEM owner.  Every wait is bounded (about a second of clock), after
+// which the CTA stops, drains what it issued, frees its TMEM and reports kStatusTimeout.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace la {
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;                 // d_k = d_v
+constexpr int CH = 64;                 // tokens per chunk
+constexpr int kHalfBytes = CH * 64 * 2;  // one 64-column swizzle half of a tile: 8 KB
+constexpr int kTileBytes = 2 * kHalfBytes;
+constexpr int kEpiWarps = 8, kGateWarps = 4;
+constexpr int kTmaWarp = 12, kMmaWarp = 13;
+constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Tensor-memory columns (fp32 accumulators; SA holds bf16 pairs).
+constexpr uint32_t kColDS = 0;    // dS^T         128 lanes x 128 cols
+constexpr uint32_t kColO = 128;   // O^T          128 lanes x 64 cols
+constexpr uint32_t kColSA = 192;  // bf16 S'^T    128 lanes x 64 cols (128 values)
+constexpr uint32_t kColQK = 256;  // Qbar' Ktil^T M=64 layout, 64 cols
+constexpr uint32_t kTmemCols = 512;
+
+template <int MODE>
+struct Cfg {
+    static constexpr bool q = MODE != kPassState;
+    static constexpr bool kv = MODE != kPassCorrect;
+    static constexpr bool qk = MODE == kPassOutput || MODE == kPassLocal;
+    static constexpr bool out = MODE != kPassState;
+    static constexpr bool write_state = MODE == kPassState || MODE == kPassLocal;
+    static constexpr bool init_state = MODE == kPassOutput || MODE == kPassCorrect;
+    static constexpr int stages = (MODE == kPassOutput || MODE == kPassLocal) ? 3 : 4;
+    static constexpr int off_q = 0;
+    static constexpr int off_k = off_q + (q ? kTileBytes : 0);
+    static constexpr int off_v = off_k + (kv ? kTileBytes : 0);
+    static constexpr int off_g = off_v + (kv ? kTileBytes : 0);
+    static constexpr int stage_bytes = off_g + kTileBytes;
+    static constexpr int off_p = stages * stage_bytes;
+    static constexpr int off_ec = off_p + (qk ? CH * CH * 2 : 0);
+    static constexpr int off_bar = off_ec + stages * D * 4;
+    static constexpr int n_bars = 3 * stages + 10;
+    static constexpr int off_misc = off_bar + n_bars * 8;
+    static constexpr int smem_bytes = off_misc + 16 + 1024;  // + slack to align the base to 1 KB
+    static_assert(smem_bytes <= 232448, "shared memory budget");
+};
+
+struct Bars {
+    uint64_t *full, *gated, *empty;
+    uint64_t *qk_full, *qk_free, *p_full, *ds_full, *ds_free, *sa_full, *sa_free, *o_full,
+        *o_free, *fin;
+};
+
+// Byte offset of element (t, i) of a [64 x 128] bf16 tile TMA-loaded as two 64-column halves
+// with the 128-byte swizzle (16-byte chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t tile_off(int t, int i) {
+    const int half = i >> 6, ii = i & 63;
+    return (uint32_t)(half * kHalfBytes + t * 128 + (((ii >> 3) ^ (t & 7)) << 4) + ((ii & 7) << 1));
+}
+
+// Descriptor of a K-major operand (rows x 128 K-elements, two swizzle halves) at K-step kk.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk) {
+    return smem_desc_sw128(base + (uint32_t)((kk >> 2) * kHalfBytes + (kk & 3) * 32), 16, 1024);
+}
+// Descriptor of an MN-major operand ([64 K-rows] x 128 MN-elements, two halves) at K-step kk.
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int kk) {
+    return smem_desc_sw128(base + (uint32_t)(kk * 2048), kHalfBytes, 1024);
+}
+
+__device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity) {
+    int dummy = 0;
+    return mbar_wait(bar, parity, &dummy);
+}
+
+// ------------------------------------------------------------------ TMA producer (1 thread)
+template <int MODE>
+__device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tq,
+                         const CUtensorMap *tk, const CUtensorMap *tv, const CUtensorMap *tg,
+                         long long row0, int nchunks) {
+    using C = Cfg<MODE>;
+    int issued = 0;
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % C::stages;
+        if (c >= C::stages && !mbar_wait(&b.empty[s], ((c / C::stages) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&b.full[s], C::stage_bytes);
+        uint8_t *st = smem + s * C::stage_bytes;
+        const int y = (int)(row0 + (long long)c * CH);
+        if (C::q) {
+            tma_load_2d(st + C::off_q, tq, 0, y, &b.full[s]);
+            tma_load_2d(st + C::off_q + kHalfBytes, tq, 64, y, &b.full[s]);
+        }
+        if (C::kv) {
+            tma_load_2d(st + C::off_k, tk, 0, y, &b.full[s]);
+            tma_load_2d(st + C::off_k + kHalfBytes, tk, 64, y, &b.full[s]);
+            tma_load_2d(st + C::off_v, tv, 0, y, &b.full[s]);
+            tma_load_2d(st + C::off_v + kHalfBytes, tv, 64, y, &b.full[s]);
+        }
+        tma_load_2d(st + C::off_g, tg, 0, y, &b.full[s]);
+        tma_load_2d(st + C::off_g + kHalfBytes, tg, 64, y, &b.full[s]);
+        issued = c + 1;
+    }
+    if (*abort)  // let every copy this CTA started land before it exits
+        for (int c = issued > C::stages ? issued - C::stages : 0; c < issued; ++c)
+            wait_drain(&b.full[c % C::stages], (c / C::stages) & 1);
+}
+
+// ------------------------------------------------------------------ MMA issuer (1 thread)
+template <int MODE>
+__device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
+                           int nchunks) {
+    using C = Cfg<MODE>;
+    constexpr uint32_t i_qk = idesc_bf16_f32(64, 64, 0, 0);
+    constexpr uint32_t i_pv = idesc_bf16_f32(128, 64, 1, 0);
+    constexpr uint32_t i_qs = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t i_ds = idesc_bf16_f32(128, 128, 1, 1);
+    const uint32_t p_addr = smem_u32(smem + C::off_p);
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % C::stages;
+        const uint32_t ph = (c / C::stages) & 1;
+        if (!mbar_wait(&b.gated[s], ph, abort)) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * C::stage_bytes);
+        const uint32_t qa = st + C::off_q, ka = st + C::off_k, va = st + C::off_v;
+        if (C::qk) {  // intra-chunk scores
+            if (c > 0 && !mbar_wait(b.qk_free, (c - 1) & 1, abort)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + kColQK, desc_kmajor(qa, kk), desc_kmajor(ka, kk), i_qk, kk > 0);
+            mma_commit(b.qk_full);
+        }
+        if (C::kv) {  // chunk state increment dS^T = V^T Ktil
+            if (c > 0 && !mbar_wait(b.ds_free, (c - 1) & 1, abort)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(ka, kk), i_ds, kk > 0);
+            mma_commit(b.ds_full);
+        }
+        if (C::out) {
+            if (c > 0 && !mbar_wait(b.o_free, (c - 1) & 1, abort)) break;
+            if (C::qk) {  // O^T = V^T P^T
+                if (!mbar_wait(b.p_full, c & 1, abort)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem + kColO, desc_mnmajor(va, kk),
+                           smem_desc_sw128(p_addr + kk * 32, 16, 1024), i_pv, kk > 0);
+            }
+            if (!mbar_wait(b.sa_full, c & 1, abort)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // O^T += S'^T Qbar'^T, A from tensor memory
+                mma_ts(tmem + kColO, tmem + kColSA + kk * 8, desc_kmajor(qa, kk), i_qs,
+                       (C::qk || kk > 0) ? 1u : 0u);
+            mma_commit(b.o_full);
+            mma_commit(b.sa_free);
+        }
+        mma_commit(&b.empty[s]);
+    }
+    mma_commit(b.fin);  // nothing of this CTA may still run on the tensor cores at dealloc
+    wait_drain(b.fin, 0);
+}
+
+// ------------------------------------------------------------------ gate warps (128 threads)
+// Thread i owns key dimension i: it sums its column of log_g for b_C, then walks the column
+// again with the running cumsum b_t and rescales its column of the q and k tiles in place
+// (Qbar', Ktil), and publishes e^{b_C,i} for the state decay.
+template <int MODE>
+__device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
+                          int bh, int j, int nchunks) {
+    using C = Cfg<MODE>;
+    const int i = threadIdx.x - 32 * kEpiWarps;
+    const int lane = threadIdx.x & 31;
+    float *ec = reinterpret_cast<float *>(smem + C::off_ec);
+    float logG = 0.f;
+    bool range_bad = false;
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % C::stages;
+        if (!mbar_wait(&b.full[s], (c / C::stages) & 1, abort)) break;
+        uint8_t *st = smem + s * C::stage_bytes;
+        const __nv_bfloat16 *gcol = reinterpret_cast<const __nv_bfloat16 *>(st + C::off_g);
+        float bC = 0.f;
+#pragma unroll 16
+        for (int t = 0; t < CH; ++t) bC += __bfloat162float(gcol[tile_off(t, i) >> 1]);
+        range_bad |= !(fabsf(bC) <= kGateRangeLimit);
+        logG += bC;
+        ec[s * D + i] = exp2f(bC * kLog2e);
+        float bt = 0.f;
+#pragma unroll 8
+        for (int t = 0; t < CH; ++t) {
+            const uint32_t off = tile_off(t, i);
+            bt += __bfloat162float(gcol[off >> 1]);
+            if (C::q) {
+                __nv_bfloat16 *qp = reinterpret_cast<__nv_bfloat16 *>(st + C::off_q + off);
+                *qp = __float2bfloat16_rn(__bfloat162float(*qp) * exp2f((bt - bC) * kLog2e));
+            }
+            if (C::kv) {
+                __nv_bfloat16 *kp = reinterpret_cast<__nv_bfloat16 *>(st + C::off_k + off);
+                *kp = __float2bfloat16_rn(__bfloat162float(*kp) * exp2f((bC - bt) * kLog2e));
+            }
+        }
+        fence_proxy_async_smem();  // the tensor cores read these tiles through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.gated[s]);
+    }
+    if (C::write_state && !*abort) a.logG[((long long)bh * a.NP + j) * D + i] = logG;
+    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// ------------------------------------------------------------------ epilogue warps (256 threads)
+// Warp w reads TMEM lane quarter q = w % 4, so thread (w, lane) owns d_v column dv = 32q+lane;
+// half h = w / 4 selects which 64 key dims of that state column it keeps (fp32, registers),
+// which 32 of the 64 P / O columns it handles.
+template <int MODE>
+__device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
+                              const PassArgs &a, uint32_t tmem, int bh, int j, long long row0,
+                              int nchunks) {
+    using C = Cfg<MODE>;
+    constexpr int HD = D / 2;  // key dims per thread
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3, h = warp >> 2;
+    const int dv = quarter * 32 + lane;
+    const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+    const float *ec = reinterpret_cast<const float *>(smem + C::off_ec) + h * HD;
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
+
+    float S[HD];  // S^T[dv][h*64 + e] = S[h*64 + e][dv]
+    if (C::init_state && a.S_init) {
+        const float *Si = a.S_init + ((long long)bh * a.NP + j) * D * D + (long long)h * HD * D + dv;
+#pragma unroll
+        for (int e = 0; e < HD; ++e) S[e] = Si[e * D];
+    } else {
+#pragma unroll
+        for (int e = 0; e < HD; ++e) S[e] = 0.f;
+    }
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % C::stages;
+        const uint32_t ph = (c / C::stages) & 1;
+        uint32_t r[32];
+        if (C::qk) {  // (a) scores -> causal mask -> bf16 P tile (K-major, swizzled rows)
+            if (!mbar_wait(b.qk_full, c & 1, abort)) break;
+            tc_fence_after();
+            tmem_ld32(tmem + lrow + kColQK + h * 32, r);  // columns s = 32h .. 32h+31
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.qk_free);
+            if (lane < 16) {  // M=64 accumulator: lanes 0-15 of each quarter hold rows 16q+l
+                const int t = quarter * 16 + lane;
+                uint8_t *prow = smem + C::off_p + t * 128;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int sl = jj * 8 + 2 * e;  // local column; key index 32h + sl
+                        const int s0 = h * 32 + sl;
+                        const float x0 = s0 <= t ? __uint_as_float(r[sl]) : 0.f;
+                        const float x1 = s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f;
+                        w4[e] = pack_bf16(x0, x1);
+                    }
+                    const int chunk16 = h * 4 + jj;
+                    *reinterpret_cast<uint4 *>(prow + ((chunk16 ^ (t & 7)) << 4)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.p_full);
+        }
+        // (b) state decayed to the chunk end: S' = diag(e^{b_C}) S
+        if (!mbar_wait(&b.gated[s], ph, abort)) break;
+        {
+            const float4 *e4 = reinterpret_cast<const float4 *>(ec + s * D);
+#pragma unroll
+            for (int i4 = 0; i4 < HD / 4; ++i4) {
+                const float4 e = e4[i4];
+                S[4 * i4 + 0] *= e.x;
+                S[4 * i4 + 1] *= e.y;
+                S[4 * i4 + 2] *= e.z;
+                S[4 * i4 + 3] *= e.w;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.empty[s]);
+        if (C::out) {  // bf16 S'^T into tensor memory: A operand of the inter-chunk MMA
+            if (c > 0 && !mbar_wait(b.sa_free, (c - 1) & 1, abort)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = pack_bf16(S[2 * e], S[2 * e + 1]);
+            tmem_st32(tmem + lrow + kColSA + h * 32, r);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.sa_full);
+        }
+        if (C::kv) {  // (c) S = S' + dS
+            if (!mbar_wait(b.ds_full, c & 1, abort)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[p * 32 + e] += __uint_as_float(r[e]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.ds_free);
+        }
+        if (C::out) {  // (d) outputs: rows t = 32h .. 32h+31 of column dv
+            if (!mbar_wait(b.o_full, c & 1, abort)) break;
+            tc_fence_after();
+            tmem_ld32(tmem + lrow + kColO + h * 32, r);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.o_free);
+            __nv_bfloat16 *orow = o + (row0 + (long long)c * CH + h * 32) * D + dv;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                float x = __uint_as_float(r[t]);
+                if (MODE == kPassCorrect) x += __bfloat162float(orow[t * D]);
+                orow[t * D] = __float2bfloat16_rn(x);
+            }
+        }
+    }
+    if (C::write_state && !*abort) {
+        float *So = a.S_out + ((long long)bh * a.NP + j) * D * D + (long long)h * HD * D + dv;
+#pragma unroll
+        for (int e = 0; e < HD; ++e) So[e * D] = S[e];
+    }
+}
+
+// ------------------------------------------------------------------ the kernel
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+               const PassArgs a) {
+    using C = Cfg<MODE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + C::off_bar);
+    Bars b;
+    b.full = bar;
+    b.gated = bar + C::stages;
+    b.empty = bar + 2 * C::stages;
+    uint64_t *x = bar + 3 * C::stages;
+    b.qk_full = x + 0; b.qk_free = x + 1; b.p_full = x + 2; b.ds_full = x + 3; b.ds_free = x + 4;
+    b.sa_full = x + 5; b.sa_free = x + 6; b.o_full = x + 7; b.o_free = x + 8; b.fin = x + 9;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::off_misc);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::off_misc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x / a.NP, j = blockIdx.x % a.NP;
+    const long long row0 = (long long)bh * a.L + (long long)j * a.T;
+    const int nchunks = (int)(a.T / CH);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::stages; ++s) {
+            mbar_init(&b.full[s], 1);
+            mbar_init(&b.gated[s], kGateWarps);
+            mbar_init(&b.empty[s], 1 + kEpiWarps);
+        }
+        mbar_init(b.qk_full, 1);
+        mbar_init(b.qk_free, kEpiWarps);
+        mbar_init(b.p_full, kEpiWarps);
+        mbar_init(b.ds_full, 1);
+        mbar_init(b.ds_free, kEpiWarps);
+        mbar_init(b.sa_full, kEpiWarps);
+        mbar_init(b.sa_free, 1);
+        mbar_init(b.o_full, 1);
+        mbar_init(b.o_free, kEpiWarps);
+        mbar_init(b.fin, 1);
+        *abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        if (C::q) prefetch_tmap(&tm_q);
+        if (C::kv) {
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+        }
+        prefetch_tmap(&tm_g);
+    }
+    if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) producer<MODE>(smem, b, abort, &tm_q, &tm_k, &tm_v, &tm_g, row0, nchunks);
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) mma_issuer<MODE>(smem, b, abort, tmem, nchunks);
+    } else if (warp >= kEpiWarps) {
+        gate_role<MODE>(smem, b, abort, a, bh, j, nchunks);
+    } else {
+        epilogue_role<MODE>(smem, b, abort, a, tmem, bh, j, row0, nchunks);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort && a.status) atomicOr(a.status, kStatusTimeout);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// [rows, 128] bf16 view, 64 x 64 boxes, 128-byte swizzle.
+cudaError_t make_map(CUtensorMap *m, const void *base, long long rows) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)CH};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const PassArgs &a, cudaStream_t st) {
+    using C = Cfg<MODE>;
+    const long long rows = (long long)a.BH * a.L;
+    if (rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
+    CUtensorMap mq, mk, mv, mg;
+    cudaError_t e;
+    const void *qp = C::q ? a.q : a.g, *kp = C::kv ? a.k : a.g, *vp = C::kv ? a.v : a.g;
+    if ((e = make_map(&mq, qp, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mk, kp, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, vp, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
+    auto kern = tc_pass_kernel<MODE>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem_bytes);
+    if (e != cudaSuccess) return e;
+    const long long nblk = (long long)a.BH * a.NP;
+    if (nblk == 0) return cudaSuccess;
+    kern<<<(unsigned)nblk, kThreads, C::smem_bytes, st>>>(mq, mk, mv, mg, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_pass_supported(const PassArgs &a) {
+    return a.dt == LA_BF16 && a.dk == D && a.dv == D && a.chunk == CH && a.T % CH == 0;
+}
+
+cudaError_t launch_tc_pass(const PassArgs &a, PassMode mode, cudaStream_t st) {
+    switch (mode) {
+        case kPassState: return launch_mode<kPassState>(a, st);
+        case kPassOutput: return launch_mode<kPassOutput>(a, st);
+        case kPassLocal: return launch_mode<kPassLocal>(a, st);
+        case kPassCorrect: return launch_mode<kPassCorrect>(a, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace la
