@@ -193,54 +193,142 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
 }
 
 // ------------------------------------------------------------------ gate warps (128 threads)
-// Thread i owns key dimension i: it sums its column of log_g for b_C, then walks the column
-// again with the running cumsum b_t and rescales its column of the q and k tiles in place
-// (Qbar', Ktil), and publishes e^{b_C,i} for the state decay.
+// Warp gw owns key dims 32gw .. 32gw+31.  Lane = 4*tg + ig: token group tg (rows 8tg .. 8tg+7)
+// and 16-byte key chunk ig (key dims 32gw + 8ig .. +7), so every shared-memory access moves one
+// swizzled 16-byte chunk.  The in-chunk cumsum of log_g runs down each thread's 8 rows, then
+// a 3-step shuffle scan across the 8 token groups adds the earlier groups' totals; the last
+// group's inclusive value is b_C.  Then q and k are rescaled in place in batches of 4 rows.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        f[2 * e] = __uint_as_float(w[e] << 16);
+        f[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
 template <int MODE>
 __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
                           int bh, int j, int nchunks) {
     using C = Cfg<MODE>;
-    const int i = threadIdx.x - 32 * kEpiWarps;
+    const int gw = (threadIdx.x >> 5) - kEpiWarps;
     const int lane = threadIdx.x & 31;
+    const int tg = lane >> 2, ig = lane & 3;
+    const int i0 = gw * 32 + ig * 8;  // first key dim of this thread's chunk
     float *ec = reinterpret_cast<float *>(smem + C::off_ec);
-    float logG = 0.f;
+    float logG[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) logG[e] = 0.f;
     bool range_bad = false;
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % C::stages;
         if (!mbar_wait(&b.full[s], (c / C::stages) & 1, abort)) break;
         uint8_t *st = smem + s * C::stage_bytes;
-        const __nv_bfloat16 *gcol = reinterpret_cast<const __nv_bfloat16 *>(st + C::off_g);
-        float bC = 0.f;
-#pragma unroll 16
-        for (int t = 0; t < CH; ++t) bC += __bfloat162float(gcol[tile_off(t, i) >> 1]);
-        range_bad |= !(fabsf(bC) <= kGateRangeLimit);
-        logG += bC;
-        ec[s * D + i] = exp2f(bC * kLog2e);
-        float bt = 0.f;
-#pragma unroll 8
-        for (int t = 0; t < CH; ++t) {
-            const uint32_t off = tile_off(t, i);
-            bt += __bfloat162float(gcol[off >> 1]);
-            if (C::q) {
-                __nv_bfloat16 *qp = reinterpret_cast<__nv_bfloat16 *>(st + C::off_q + off);
-                *qp = __float2bfloat16_rn(__bfloat162float(*qp) * exp2f((bt - bC) * kLog2e));
+        // local inclusive cumsum down rows 8tg .. 8tg+7
+        float bt[8][8];
+        {
+            uint4 graw[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+                graw[r] = *reinterpret_cast<const uint4 *>(st + C::off_g + tile_off(tg * 8 + r, i0));
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                float f[8];
+                unpack8(graw[r], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) bt[r][e] = (r ? bt[r - 1][e] : 0.f) + f[e];
             }
-            if (C::kv) {
-                __nv_bfloat16 *kp = reinterpret_cast<__nv_bfloat16 *>(st + C::off_k + off);
-                *kp = __float2bfloat16_rn(__bfloat162float(*kp) * exp2f((bC - bt) * kLog2e));
+        }
+        // inclusive scan of the group totals across tg (lanes ig, ig+4, ..., ig+28)
+        float incl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) incl[e] = bt[7][e];
+#pragma unroll
+        for (int d = 1; d < 8; d <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float up = __shfl_up_sync(0xFFFFFFFFu, incl[e], 4 * d);
+                if (tg >= d) incl[e] += up;
+            }
+        }
+        float bC[8], nbCl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            bC[e] = __shfl_sync(0xFFFFFFFFu, incl[e], 28 + ig);
+            const float off = incl[e] - bt[7][e];  // exclusive prefix of this token group
+#pragma unroll
+            for (int r = 0; r < 8; ++r) bt[r][e] += off;
+            nbCl[e] = -bC[e] * kLog2e;
+            range_bad |= !(fabsf(bC[e]) <= kGateRangeLimit);
+        }
+        if (tg == 0) {
+            float4 *e4 = reinterpret_cast<float4 *>(ec + s * D + i0);
+            e4[0] = make_float4(ex2_approx(-nbCl[0]), ex2_approx(-nbCl[1]), ex2_approx(-nbCl[2]),
+                                ex2_approx(-nbCl[3]));
+            e4[1] = make_float4(ex2_approx(-nbCl[4]), ex2_approx(-nbCl[5]), ex2_approx(-nbCl[6]),
+                                ex2_approx(-nbCl[7]));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) logG[e] += bC[e];
+        }
+        // rescale q (by e^{b_t - b_C}) and k (by e^{b_C - b_t}) in place, 4 rows per batch
+#pragma unroll
+        for (int r0 = 0; r0 < 8; r0 += 4) {
+            uint4 qr[4], kr[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+                if (C::q) qr[r] = *reinterpret_cast<const uint4 *>(st + C::off_q + off);
+                if (C::kv) kr[r] = *reinterpret_cast<const uint4 *>(st + C::off_k + off);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = fmaf(bt[r0 + r][e], kLog2e, nbCl[e]);
+                if (C::q) {
+                    float f[8];
+                    unpack8(qr[r], f);
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w[e] = pack_bf16(f[2 * e] * ex2_approx(x[2 * e]),
+                                         f[2 * e + 1] * ex2_approx(x[2 * e + 1]));
+                    *reinterpret_cast<uint4 *>(st + C::off_q + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                if (C::kv) {
+                    float f[8];
+                    unpack8(kr[r], f);
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w[e] = pack_bf16(f[2 * e] * ex2_approx(-x[2 * e]),
+                                         f[2 * e + 1] * ex2_approx(-x[2 * e + 1]));
+                    *reinterpret_cast<uint4 *>(st + C::off_k + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
             }
         }
         fence_proxy_async_smem();  // the tensor cores read these tiles through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.gated[s]);
     }
-    if (C::write_state && !*abort) a.logG[((long long)bh * a.NP + j) * D + i] = logG;
+    if (C::write_state && !*abort && tg == 0) {
+        float4 *lg = reinterpret_cast<float4 *>(a.logG + ((long long)bh * a.NP + j) * D + i0);
+        lg[0] = make_float4(logG[0], logG[1], logG[2], logG[3]);
+        lg[1] = make_float4(logG[4], logG[5], logG[6], logG[7]);
+    }
     if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
 }
 
 // ------------------------------------------------------------------ epilogue warps (256 threads)
