@@ -10,4 +10,8 @@ cudaError_t launch_pass(const PassArgs &a, PassMode mode, cudaStream_t st) {
     return launch_simt_pass(a, mode, st);
 }
 
+cudaError_t launch_bwd_dstate(const BwdArgs &a, cudaStream_t st) { return launch_simt_dstate(a, st); }
+
+cudaError_t launch_bwd_grad(const BwdArgs &a, cudaStream_t st) { return launch_simt_grad(a, st); }
+
 }  // namespace la

@@ -30,6 +30,31 @@ struct PassArgs {
     la_dtype dt;
 };
 
+// Arguments of the backward chunk passes (one CTA per (b, h, segment j)).
+struct BwdArgs {
+    const void *q, *k, *v, *g, *dO;
+    void *dq_out, *dk_out, *dv_out, *dg_out;
+    const float *S_recv;      // [BH, NP, dk, dv] state each segment receives (null: zero)
+    const float *S_end_next;  // same array as S_recv: S_end_j = S_recv[j+1] for j < NP-1 (null: no carry)
+    const float *S_fin;       // [BH, dk, dv] state after the last token (null: no carry there)
+    const float *dX;          // [BH, NP, dk, dv] gradient of each segment's end state
+    float *dq_ws;             // [BH, L, dk] fp32 dq between the two sweeps
+    float *dSloc;             // [BH, NP, dk, dv] per-segment gradient states (dstate pass)
+    float *logG;              // [BH, NP, dk] per-segment log-decay sums (dstate pass)
+    int *status;
+    long long L, T;
+    int BH, NP, dk, dv, chunk;
+    la_dtype dt;
+};
+
+// Backward passes for these arguments (tensor-core kernels where they apply, else SIMT).
+cudaError_t launch_bwd_dstate(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_grad(const BwdArgs &a, cudaStream_t st);
+
+// Generic CUDA-core backward passes.
+cudaError_t launch_simt_dstate(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_simt_grad(const BwdArgs &a, cudaStream_t st);
+
 // Generic CUDA-core (FFMA) chunk pass: any supported dtype, d and chunk.
 cudaError_t launch_simt_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
 

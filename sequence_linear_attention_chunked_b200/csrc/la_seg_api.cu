@@ -98,6 +98,26 @@ FwdLayout fwd_layout(const la::Split &s, int dk, int dv) {
     return w;
 }
 
+struct BwdLayout {
+    size_t status, S_loc, logG, S_recv, S_fin, dSloc, dX, dq_ws, total;
+};
+
+BwdLayout bwd_layout(const la::Split &s, int dk, int dv) {
+    BwdLayout w;
+    const size_t states = (size_t)s.BH * s.NP * dk * dv * sizeof(float);
+    const size_t gam = (size_t)s.BH * s.NP * dk * sizeof(float);
+    w.status = 0;
+    w.S_loc = 256;
+    w.logG = align_up(w.S_loc + states, 256);
+    w.S_recv = align_up(w.logG + gam, 256);
+    w.S_fin = align_up(w.S_recv + states, 256);
+    w.dSloc = align_up(w.S_fin + (size_t)s.BH * dk * dv * sizeof(float), 256);
+    w.dX = align_up(w.dSloc + states, 256);
+    w.dq_ws = align_up(w.dX + states, 256);
+    w.total = align_up(w.dq_ws + (size_t)s.BH * s.L * dk * sizeof(float), 256);
+    return w;
+}
+
 template <typename Ptr>
 char *at(Ptr base, size_t off) {
     return static_cast<char *>(const_cast<void *>(static_cast<const void *>(base))) + off;
@@ -125,8 +145,13 @@ size_t la_seg_workspace_bytes(int B, int H, long long L, int dk, int dv, int P, 
                               la_dtype dt, int backward) {
     if (check_shape(B, H, L, dk, dv, P, chunk, dt) != LA_OK) return 0;
     const la::Split s = make_split(B, H, L, P, chunk);
-    if (backward) return 0;  // backward workspace: see la_seg_backward
-    return fwd_layout(s, dk, dv).total;
+    if (!backward) return fwd_layout(s, dk, dv).total;
+    la::Split whole = s;  // la_seg_backward keeps whole segments when it reuses saved states
+    whole.m = 1;
+    whole.NP = P;
+    whole.T = L / P;
+    const size_t a = bwd_layout(s, dk, dv).total, b = bwd_layout(whole, dk, dv).total;
+    return a > b ? a : b;
 }
 
 }  // extern "C"
@@ -285,11 +310,80 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     return LA_OK;
 }
 
-la_status la_seg_backward(const void *, const void *, const void *, const void *, const float *,
-                          const float *, const void *, const float *, int, int, long long, int,
-                          int, int, int, la_dtype, void *, void *, void *, void *, float *, void *,
-                          size_t, void *) {
-    return fail(LA_ERR_SHAPE, "la_seg_backward: not built in this version");
+la_status la_seg_backward(const void *q, const void *k, const void *v, const void *log_g,
+                          const float *S0, const float *S_recv_saved, const void *dO,
+                          const float *dS_final, int B, int H, long long L, int dk, int dv, int P,
+                          int chunk, la_dtype dt, void *dq, void *dk_, void *dv_, void *dlog_g,
+                          float *dS0, void *workspace, size_t ws_bytes, void *cuda_stream) {
+    la_status st = check_shape(B, H, L, dk, dv, P, chunk, dt);
+    if (st != LA_OK) return st;
+    if (L > 0 && (!q || !k || !v || !log_g || !dO || !dq || !dk_ || !dv_ || !dlog_g))
+        return fail(LA_ERR_ARG, "q, k, v, log_g, dO, dq, dk, dv and dlog_g must be non-null");
+    const void *ptrs[] = {q, k, v, log_g, dO, dq, dk_, dv_, dlog_g, S0, S_recv_saved, dS_final, dS0};
+    const char *names[] = {"q", "k", "v", "log_g", "dO", "dq", "dk", "dv", "dlog_g", "S0",
+                           "S_recv_saved", "dS_final", "dS0"};
+    for (int i = 0; i < 13; ++i)
+        if (ptrs[i] && !aligned(ptrs[i], 16))
+            return fail(LA_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    // Saved states are per API segment: when they can be reused (S_final not needed), keep
+    // whole segments so that every segment's received state is one the forward saved.
+    la::Split s = make_split(B, H, L, P, chunk);
+    const bool reuse = S_recv_saved && !dS_final;
+    if (reuse) {
+        s.m = 1;
+        s.NP = P;
+        s.T = L / P;
+    }
+    const BwdLayout w = bwd_layout(s, dk, dv);
+    const size_t need = la_seg_workspace_bytes(B, H, L, dk, dv, P, chunk, dt, 1);
+    if (!workspace || ws_bytes < need)
+        return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu%s)", need,
+                    ws_bytes, workspace ? "" : ", null");
+    if (!aligned(workspace, 256)) return fail(LA_ERR_ALIGN, "workspace is not 256-byte aligned");
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    int *status = reinterpret_cast<int *>(at(workspace, w.status));
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "status reset");
+    if (L == 0) {  // no tokens: S_final = S0, so dS0 = dS_final
+        if (dS0 && (e = la::launch_copy_state(dS_final, s.BH, dk, dv, dS0, stream)) != cudaSuccess)
+            return cuda_fail(e, "dS0 copy");
+        return LA_OK;
+    }
+    float *S_loc = reinterpret_cast<float *>(at(workspace, w.S_loc));
+    float *logG = reinterpret_cast<float *>(at(workspace, w.logG));
+    float *S_recv = reinterpret_cast<float *>(at(workspace, w.S_recv));
+    float *S_fin = reinterpret_cast<float *>(at(workspace, w.S_fin));
+    float *dSloc = reinterpret_cast<float *>(at(workspace, w.dSloc));
+    float *dX = reinterpret_cast<float *>(at(workspace, w.dX));
+    float *dq_ws = reinterpret_cast<float *>(at(workspace, w.dq_ws));
+
+    // 1. the states each segment receives: the forward's when given and S_final is not needed
+    //    (dS_final = 0); otherwise recomputed (state pass + scan)
+    const float *recv = reuse ? S_recv_saved : S_recv;
+    if (!reuse) {
+        la::PassArgs a = pass_args(nullptr, k, v, log_g, nullptr, nullptr, S_loc, logG, status, B,
+                                   H, L, dk, dv, s.NP, chunk, dt);
+        if ((e = la::launch_pass(a, la::kPassState, stream)) != cudaSuccess)
+            return cuda_fail(e, "backward state pass");
+        if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_fin, stream)) !=
+            cudaSuccess)
+            return cuda_fail(e, "backward state scan");
+    }
+    la::BwdArgs b;
+    b.q = q; b.k = k; b.v = v; b.g = log_g; b.dO = dO;
+    b.dq_out = dq; b.dk_out = dk_; b.dv_out = dv_; b.dg_out = dlog_g;
+    b.S_recv = recv; b.S_end_next = recv; b.S_fin = reuse ? nullptr : S_fin; b.dX = dX;
+    b.dq_ws = dq_ws; b.dSloc = dSloc; b.logG = logG; b.status = status;
+    b.L = L; b.T = s.T; b.BH = s.BH; b.NP = s.NP; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
+    // 2. per-segment gradient states and log-decay sums
+    if ((e = la::launch_bwd_dstate(b, stream)) != cudaSuccess) return cuda_fail(e, "gradient-state pass");
+    // 3. reverse exclusive decayed scan: gradient of every segment's end state, and dS0
+    if ((e = la::launch_scan(dSloc, logG, dS_final, s.BH, s.NP, dk, dv, 1, dX, dS0, stream)) !=
+        cudaSuccess)
+        return cuda_fail(e, "reverse state scan");
+    // 4. dq, dk, dv, dlog_g per segment
+    if ((e = la::launch_bwd_grad(b, stream)) != cudaSuccess) return cuda_fail(e, "gradient pass");
+    return LA_OK;
 }
 
 la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *init, int BH,

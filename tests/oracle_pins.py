@@ -17,6 +17,10 @@ the ZeCO pages, never against a retyped copy of its own loop:
 * ``propagation``   -- P >= 3: the state segment 2 receives carries Gamma_1 Gamma_0 S0 +
                        Gamma_1 S_0 + S_1 (the accumulated state is forwarded, not only the
                        local one; the ZeCO review's referee flags Alg. 2 for exactly this).
+* ``seg_backward``  -- a chunked, segmented restatement of the backward (per-segment gradient
+                       states, a reverse exclusive decayed scan, forward and reverse chunk
+                       sweeps, dlog_g from a chunk-local suffix sum plus the carry
+                       rowsum(S_end . dX)) reproduces the oracle's gradients.
 * ``finite_diff``   -- the backward equals central finite differences of the forward.
 * ``dg_identity``   -- dlog_g_t = sum_{s>=t} (q_s . dq_s - k_s . dk_s) + rowsum(dS_final . S_final).
 """
@@ -105,6 +109,77 @@ def segmented(q, k, v, g, S0, P, C):
     return o, Sf, S_recv_all
 
 
+def segmented_backward(q, k, v, g, dO, S0, dSf, P, C):
+    """Gradients of loss = <o, dO> + <S_final, dSf> by segments and chunks (fp64)."""
+    Bn, H, L, dk = q.shape
+    dv = v.shape[-1]
+    T = L // P
+    out = [np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(g)]
+    dS0 = np.zeros((Bn, H, dk, dv))
+    for b in range(Bn):
+        for h in range(H):
+            qq, kk, vv, gg, dd = q[b, h], k[b, h], v[b, h], g[b, h], dO[b, h]
+            # forward: local states, decays, received states, final state
+            S_loc, logG = [], []
+            for p in range(P):
+                sl = slice(p * T, (p + 1) * T)
+                _, Sl, lg = chunked_segment_local(qq[sl], kk[sl], vv[sl], gg[sl], C)
+                S_loc.append(Sl)
+                logG.append(lg)
+            S_recv = [np.zeros((dk, dv)) if S0 is None else S0[b, h].copy()]
+            for p in range(P):
+                S_recv.append(np.exp(logG[p])[:, None] * S_recv[p] + S_loc[p])
+            # per-segment gradient states dSloc_p = sum_t diag(e^{B_t}) q_t^T dO_t
+            dSloc = []
+            for p in range(P):
+                sl = slice(p * T, (p + 1) * T)
+                Bseg = np.cumsum(gg[sl], axis=0)
+                dSloc.append((qq[sl] * np.exp(Bseg)).T @ dd[sl])
+            # reverse exclusive scan: dX_p = d loss / d S_end_p
+            dX = [None] * P
+            acc = np.zeros((dk, dv)) if dSf is None else dSf[b, h].copy()
+            for p in range(P - 1, -1, -1):
+                dX[p] = acc
+                acc = np.exp(logG[p])[:, None] * acc + dSloc[p]
+            dS0[b, h] = acc
+            for p in range(P):
+                sl = slice(p * T, (p + 1) * T)
+                qs, ks, vs, gs, ds = qq[sl], kk[sl], vv[sl], gg[sl], dd[sl]
+                dq = np.zeros_like(qs)
+                S = S_recv[p].copy()
+                for c0 in range(0, T, C):  # forward sweep: dq
+                    cs = slice(c0, c0 + C)
+                    bt = np.cumsum(gs[cs], axis=0)
+                    bC = bt[-1]
+                    Sp = np.exp(bC)[:, None] * S
+                    Kt = ks[cs] * np.exp(bC - bt)
+                    M = np.tril(ds[cs] @ vs[cs].T)
+                    dq[cs] = np.exp(bt - bC) * (ds[cs] @ Sp.T + M @ Kt)
+                    S = Sp + Kt.T @ vs[cs]
+                dk_ = np.zeros_like(ks)
+                dv_ = np.zeros_like(vs)
+                dgs = np.zeros_like(gs)
+                dS = dX[p].copy()
+                acc_g = np.sum(S_recv[p + 1] * dX[p], axis=1)  # carry: rowsum(S_end . dX)
+                for c0 in reversed(range(0, T, C)):  # reverse sweep: dk, dv, dlog_g
+                    cs = slice(c0, c0 + C)
+                    bt = np.cumsum(gs[cs], axis=0)
+                    bC = bt[-1]
+                    Qb = qs[cs] * np.exp(bt - bC)
+                    Kt = ks[cs] * np.exp(bC - bt)
+                    M = np.tril(ds[cs] @ vs[cs].T)
+                    A = np.tril(Qb @ Kt.T)
+                    dk_[cs] = np.exp(bC - bt) * (M.T @ Qb + vs[cs] @ dS.T)
+                    dv_[cs] = A.T @ ds[cs] + Kt @ dS
+                    contrib = qs[cs] * dq[cs] - ks[cs] * dk_[cs]
+                    suffix = np.flip(np.cumsum(np.flip(contrib, 0), 0), 0)
+                    dgs[cs] = suffix + acc_g
+                    acc_g = acc_g + contrib.sum(axis=0)
+                    dS = np.exp(bC)[:, None] * (dS + Qb.T @ ds[cs])
+                out[0][b, h, sl], out[1][b, h, sl], out[2][b, h, sl], out[3][b, h, sl] = dq, dk_, dv_, dgs
+    return out[0], out[1], out[2], out[3], dS0
+
+
 # --------------------------------------------------------------------------- pins
 def pin_brute_force(orc, tol=1e-12):
     worst = 0.0
@@ -177,6 +252,20 @@ def pin_propagation(orc, tol=1e-12):
     return (err <= tol and distinct), err
 
 
+def pin_seg_backward(orc, tol=1e-11):
+    worst = 0.0
+    for seed, (L, P, C, s0, dsf) in enumerate([(64, 4, 8, True, True), (96, 3, 16, False, False),
+                                               (48, 1, 16, True, False), (128, 8, 4, False, True)]):
+        q, k, v, g, S0 = rand_case(300 + seed, L=L, dk=5, dv=4, s0=s0)
+        rng = np.random.default_rng(400 + seed)
+        dO = rng.standard_normal(v.shape)
+        dSf = rng.standard_normal((q.shape[0], q.shape[1], 5, 4)) if dsf else None
+        ref = orc.backward(q, k, v, g, dO, S0, dSf)
+        got = segmented_backward(q, k, v, g, dO, S0, dSf, P, C)
+        worst = max(worst, *(rel_err(a, b) for a, b in zip(got, ref)))
+    return worst <= tol, worst
+
+
 def _loss(orc, q, k, v, g, S0, dO, dSf):
     o, Sf, _ = orc.forward(q, k, v, g, S0)
     return float(np.sum(o * dO) + np.sum(Sf * dSf))
@@ -228,6 +317,7 @@ ALL_PINS = {
     "closed_form": pin_closed_form,
     "segmented": pin_segmented,
     "propagation": pin_propagation,
+    "seg_backward": pin_seg_backward,
     "finite_diff": pin_finite_diff,
     "dg_identity": pin_dg_identity,
 }

@@ -110,3 +110,33 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(la_seg, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         la_seg.lib()
+
+
+def _bwd(lib, **kw):
+    """Calls la_seg_backward with fake (but aligned) pointers: only argument checks may run."""
+    a = dict(q=0x1000, k=0x2000, v=0x3000, g=0x4000, S0=None, Sr=None, dO=0x5000, dSf=None, B=1,
+             H=1, L=64, d=32, P=1, chunk=16, dt=0, dq=0x6000, dk=0x7000, dv=0x8000, dg=0x9000,
+             dS0=None, ws=0x10000, ws_bytes=1 << 30)
+    a.update(kw)
+    V = ctypes.c_void_p
+    return lib.la_seg_backward(V(a["q"]), V(a["k"]), V(a["v"]), V(a["g"]), V(a["S0"]), V(a["Sr"]),
+                               V(a["dO"]), V(a["dSf"]), a["B"], a["H"], a["L"], a["d"], a["d"],
+                               a["P"], a["chunk"], a["dt"], V(a["dq"]), V(a["dk"]), V(a["dv"]),
+                               V(a["dg"]), V(a["dS0"]), V(a["ws"]), a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(L=100, P=3), -2), (dict(d=48), -2), (dict(chunk=128), -2), (dict(dt=2), -4),
+    (dict(dO=None), -1), (dict(dg=None), -1), (dict(dq=0x6004), -3), (dict(Sr=0x1234), -3),
+    (dict(ws=None), -5), (dict(ws_bytes=1024), -5),
+])
+def test_backward_rejects_bad_arguments(lib, kw, status):
+    assert _bwd(lib, **kw) == status
+
+
+def test_backward_workspace_covers_both_splits(lib):
+    w = la_seg.la_seg_workspace_bytes
+    # C4: the fwd+bwd workload; the backward needs the fp32 dq staging buffer
+    need = w(2, 16, 131072, 128, 128, 8, 64, la_seg.LA_BF16, True)
+    assert need >= 2 * 16 * 131072 * 128 * 4
+    assert w(2, 16, 131072, 128, 128, 8, 64, la_seg.LA_BF16, False) < need

@@ -1,0 +1,147 @@
+"""Backward parity of the CUDA path (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sequence_linear_attention_chunked_b200 import la_seg
+from sequence_linear_attention_chunked_b200.inputs import WORKLOADS, Workload, make_inputs
+from tests.parity import TOL, forgetting_bound, rel_err
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("dq", "dk", "dv", "dlog_g", "dS0")
+
+
+def run_bwd(x, w, S_recv=None, dS_final=None):
+    dt = la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16
+    ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, x["q"].device)
+    out = la_seg.la_seg_backward(x["q"], x["k"], x["v"], x["log_g"], x["dO"], x.get("S0"), S_recv,
+                                 dS_final, w.P, w.chunk, want_dS0=True, ws=ws)
+    la_seg.la_seg_check_status(ws)
+    return out
+
+
+def check(w, device, with_s0=False, with_dsf=False, reuse=False):
+    x = make_inputs(w, device, with_s0=with_s0)
+    dSf = None
+    if with_dsf:
+        dSf = torch.randn((w.B, w.H, w.dk, w.dv), generator=torch.Generator(device=device).manual_seed(9),
+                          device=device)
+    Sr = None
+    if reuse:
+        _, _, Sr = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], x.get("S0"), w.P, w.chunk,
+                                         want_S_recv=True)
+    got = run_bwd(x, w, Sr, dSf)
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["log_g"], x["dO"], x.get("S0"), dSf)
+    tol = TOL[w.torch_dtype]
+    errs = {n: rel_err(g, r) for n, g, r in zip(NAMES, got, ref)}
+    assert all(e <= tol for e in errs.values()), (w.describe(), errs)
+    return errs
+
+
+@pytest.mark.parametrize("with_s0,with_dsf,reuse", [(False, False, False), (True, True, False),
+                                                    (True, False, True), (False, True, True)])
+def test_c0_fp32_backward(cuda_device, with_s0, with_dsf, reuse):
+    check(WORKLOADS["C0"].with_(backward=True), cuda_device, with_s0, with_dsf, reuse)
+
+
+SMALL = [  # (B, H, L, d, P, chunk, dtype, dist)
+    (1, 2, 512, 128, 2, 64, "bf16", "gla"),
+    (2, 2, 384, 64, 3, 32, "bf16", "gla"),
+    (1, 1, 128, 32, 4, 16, "f32", "toy"),
+    (1, 2, 512, 128, 1, 64, "f32", "gla"),
+    (1, 2, 2048, 128, 4, 64, "bf16", "weak"),
+    (1, 1, 128, 128, 2, 64, "bf16", "gla"),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("reuse", [False, True])
+def test_small_backward(cuda_device, shape, reuse):
+    B, H, L, d, P, C, dt, dist = shape
+    w = Workload("small-bwd", B, H, L, d, d, P, C, dt, dist, backward=True, seed=L + d + 1)
+    check(w, cuda_device, with_s0=(L % 3 == 0), with_dsf=(L % 256 == 0), reuse=reuse)
+
+
+def test_reuse_matches_recompute(cuda_device):
+    """Reusing the forward's received states (ZeCO review, "forward implications") gives the
+    same gradients as recomputing them."""
+    w = WORKLOADS["C1"].with_(H=2, L=4096, P=4, backward=True)
+    x = make_inputs(w, cuda_device, with_s0=True)
+    _, _, Sr = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], x["S0"], w.P, w.chunk,
+                                     want_S_recv=True)
+    a = run_bwd(x, w, None)
+    b = run_bwd(x, w, Sr)
+    for n, ga, gb in zip(NAMES, a, b):
+        assert rel_err(ga, gb.double().cpu().numpy()) <= 1e-2, n
+
+
+def test_backward_empty(cuda_device):
+    w = Workload("empty", 1, 2, 0, 32, 32, 2, 16, "f32", "toy", backward=True)
+    x = make_inputs(w, cuda_device, with_s0=True)
+    dSf = torch.randn((1, 2, 32, 32), device=cuda_device)
+    out = run_bwd(x, w, None, dSf)
+    assert out[0].numel() == 0 and torch.equal(out[4], dSf)
+
+
+def test_backward_deterministic(cuda_device):
+    w = WORKLOADS["C1"].with_(H=2, L=2048, P=2, backward=True)
+    x = make_inputs(w, cuda_device)
+    a = run_bwd(x, w)
+    b = run_bwd(x, w)
+    assert all(torch.equal(ga, gb) for ga, gb in zip(a, b))
+
+
+def oracle_bwd_windows(x, wins, warm=8192, min_forget=-200.0):
+    """Oracle gradients on token windows of a long sequence.  Each window is replayed from
+    `warm` tokens before it (zero state) to `warm` tokens after it (zero upstream state
+    gradient beyond): both truncated pieces reach the window only through a decay factor of at
+    most exp(sum of log_g over the warm-up), asserted <= exp(min_forget)."""
+    L = x["q"].shape[2]
+    lo_hi = []
+    for b, h, t0, t1 in wins:
+        lo, hi = max(0, t0 - warm), min(L, t1 + warm)
+        if lo > 0:
+            assert forgetting_bound(x["log_g"][b:b + 1, h:h + 1, lo:t0]) <= min_forget
+        if hi < L:
+            assert forgetting_bound(x["log_g"][b:b + 1, h:h + 1, t1:hi]) <= min_forget
+        lo_hi.append((lo, hi))
+    n = max(hi - lo for lo, hi in lo_hi)
+    stack = {k: [] for k in ("q", "k", "v", "log_g", "dO")}
+    for (b, h, t0, t1), (lo, hi) in zip(wins, lo_hi):
+        for k in stack:  # left-align; pad the tail with zeros (zero dO and k add nothing)
+            t = x[k][b, h, lo:hi].double().cpu()
+            pad = torch.zeros((n - (hi - lo), t.shape[1]), dtype=torch.float64)
+            stack[k].append(torch.cat([t, pad]))
+    S = {k: torch.stack(v)[None] for k, v in stack.items()}
+    grads = oracle.backward(S["q"], S["k"], S["v"], S["log_g"], S["dO"])
+    res = []
+    for i, ((b, h, t0, t1), (lo, hi)) in enumerate(zip(wins, lo_hi)):
+        res.append([g[0, i, t0 - lo:t1 - lo] for g in grads[:4]])
+    return res
+
+
+def test_c4_full_sampled(cuda_device):
+    """The fwd+bwd workload at full size: sampled windows (segment starts included)."""
+    w = WORKLOADS["C4"]
+    x = make_inputs(w, cuda_device)
+    _, _, Sr = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, w.P, w.chunk,
+                                     want_S_recv=True)
+    grads = run_bwd(x, w, Sr)
+    T = w.L // w.P
+    rng = np.random.default_rng(11)
+    wins = []
+    for b in (0, 1):
+        for h in (0, w.H - 1):
+            p = int(rng.integers(1, w.P))
+            wins.append((b, h, p * T, p * T + 256))
+            t0 = int(rng.integers(0, w.L - 256)) // 64 * 64
+            wins.append((b, h, t0, t0 + 256))
+    wins.append((0, 3, 0, 256))
+    wins.append((1, 7, w.L - 256, w.L))
+    refs = oracle_bwd_windows(x, wins)
+    for (b, h, t0, t1), ref in zip(wins, refs):
+        for n, g, r in zip(NAMES, grads, ref):
+            e = rel_err(g[b, h, t0:t1], r)
+            assert e <= 2e-2, (n, b, h, t0, e)
