@@ -137,7 +137,14 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- our arm
 class Step:
     """One pass of the whole path through the C ABI's per-step entry points, with CUDA events
-    between the phases on the launching stream."""
+    between the phases on the launching stream.  Forward: state pass, state scan, output pass
+    (or local pass, scan, correction pass); backward (fwd+bwd workloads): gradient-state pass,
+    reverse scan, gradient pass, reusing the forward's received states."""
+
+    KERNEL_KEYS = {"state pass": "state_pass", "output pass": "output_pass",
+                   "local pass": "local_pass", "correction pass": "correct_pass",
+                   "state scan": "scan", "dstate pass": "dstate_pass", "reverse scan": "scan",
+                   "grad pass": "grad_pass"}
 
     def __init__(self, w: Workload, x, schedule: str, device):
         from sequence_linear_attention_chunked_b200 import la_seg
@@ -156,35 +163,54 @@ class Step:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.phases = (["state pass", "state scan", "output pass"] if schedule != "three"
                        else ["local pass", "state scan", "correction pass"])
+        if w.backward:
+            self.phases += ["dstate pass", "reverse scan", "grad pass"]
+            self.dSloc = torch.empty_like(self.S_loc)
+            self.logG_b = torch.empty_like(self.logG)
+            self.dX = torch.empty_like(self.S_loc)
+            self.dS0 = torch.empty_like(self.S_final)
+            self.grads = (torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
+                          torch.empty_like(x["log_g"]))
+            self.dq_ws = torch.empty((B, H, L, dk), **f32)
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
         self.launches_per_step = len(self.phases)
 
     def run(self, record=True):
         la, x, w, NP = self.la, self.x, self.w, self.NP
         ev = self.events
-        if record:
-            ev[0].record()
+        rec = (lambda i: ev[i].record()) if record else (lambda i: None)
+        BH = w.B * w.H
+        rec(0)
         if self.schedule != "three":
             la.la_seg_state_pass(x["k"], x["v"], x["log_g"], NP, w.chunk, S_loc=self.S_loc,
                                  log_gamma=self.logG, status=self.status)
         else:
             la.la_seg_local_pass(x["q"], x["k"], x["v"], x["log_g"], NP, w.chunk, o=self.o,
                                  S_loc=self.S_loc, log_gamma=self.logG, status=self.status)
-        if record:
-            ev[1].record()
-        BH = w.B * w.H
-        la.lib().la_seg_scan(la._ptr(self.S_loc), la._ptr(self.logG), None, BH, NP, w.dk, w.dv, 0,
-                             la._ptr(self.S_recv), la._ptr(self.S_final), la._stream(None))
-        if record:
-            ev[2].record()
+        rec(1)
+        la._check(la.lib().la_seg_scan(la._ptr(self.S_loc), la._ptr(self.logG), None, BH, NP, w.dk,
+                                       w.dv, 0, la._ptr(self.S_recv), la._ptr(self.S_final),
+                                       la._stream(None)), "la_seg_scan")
+        rec(2)
         if self.schedule != "three":
             la.la_seg_output_pass(x["q"], x["k"], x["v"], x["log_g"], self.S_recv, NP, w.chunk,
                                   o=self.o, status=self.status)
         else:
             la.la_seg_correct_pass(x["q"], x["log_g"], self.S_recv, NP, w.chunk, self.o,
                                    status=self.status)
-        if record:
-            ev[3].record()
+        rec(3)
+        if not w.backward:
+            return
+        la.la_seg_dstate_pass(x["q"], x["dO"], x["log_g"], NP, w.chunk, dSloc=self.dSloc,
+                              log_gamma=self.logG_b, status=self.status)
+        rec(4)
+        la._check(la.lib().la_seg_scan(la._ptr(self.dSloc), la._ptr(self.logG_b), None, BH, NP,
+                                       w.dk, w.dv, 1, la._ptr(self.dX), la._ptr(self.dS0),
+                                       la._stream(None)), "la_seg_scan")
+        rec(5)
+        la.la_seg_grad_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_recv, None, self.dX,
+                            NP, w.chunk, out=self.grads, dq_ws=self.dq_ws, status=self.status)
+        rec(6)
 
     def phase_ms(self):
         return [self.events[i].elapsed_time(self.events[i + 1]) for i in range(len(self.phases))]
@@ -196,24 +222,35 @@ class Step:
         th = w.B * w.H * w.L
         st = w.B * w.H * self.NP * w.dk * w.dv * 4
         lg = w.B * w.H * self.NP * w.dk * 4
+        fin = w.B * w.H * w.dk * w.dv * 4
+        scan = 2 * st + lg + fin
         if self.schedule != "three":
-            return {"state pass": th * (2 * w.dk + w.dv) * e + st + lg,
-                    "state scan": 2 * st + lg + w.B * w.H * w.dk * w.dv * 4,
-                    "output pass": th * (3 * w.dk + 2 * w.dv) * e + st}
-        return {"local pass": th * (3 * w.dk + 2 * w.dv) * e + st + lg,
-                "state scan": 2 * st + lg + w.B * w.H * w.dk * w.dv * 4,
-                "correction pass": th * (2 * w.dk + 2 * w.dv) * e + st}
+            ab = {"state pass": th * (2 * w.dk + w.dv) * e + st + lg, "state scan": scan,
+                  "output pass": th * (3 * w.dk + 2 * w.dv) * e + st}
+        else:
+            ab = {"local pass": th * (3 * w.dk + 2 * w.dv) * e + st + lg, "state scan": scan,
+                  "correction pass": th * (2 * w.dk + 2 * w.dv) * e + st}
+        if w.backward:
+            ab["dstate pass"] = th * (2 * w.dk + w.dv) * e + st + lg
+            ab["reverse scan"] = scan
+            ab["grad pass"] = th * (3 * w.dk + 2 * w.dv + 3 * w.dk + w.dv) * e + 2 * st
+        return ab
 
     def flops(self):
         w = self.w
         th = w.B * w.H * w.L
-        C = w.chunk
-        intra = 2 * C * w.dk + 2 * C * w.dv  # QK^T and PV on full chunk tiles
-        inter = 2 * w.dk * w.dv              # q . S
-        state = 2 * w.dk * w.dv              # K^T V
+        C, dk, dv = w.chunk, w.dk, w.dv
+        intra = 2 * C * dk + 2 * C * dv  # QK^T and PV on full chunk tiles
+        dd = 2 * dk * dv                 # one state-sized contraction per token
         if self.schedule != "three":
-            return {"state pass": th * state, "state scan": 0, "output pass": th * (intra + inter + state)}
-        return {"local pass": th * (intra + inter + state), "state scan": 0, "correction pass": th * inter}
+            fl = {"state pass": th * dd, "state scan": 0, "output pass": th * (intra + 2 * dd)}
+        else:
+            fl = {"local pass": th * (intra + 2 * dd), "state scan": 0, "correction pass": th * dd}
+        if w.backward:
+            fl["dstate pass"] = th * dd
+            fl["reverse scan"] = 0
+            fl["grad pass"] = th * (5 * dd + 2 * C * (3 * dk + 3 * dv))
+        return fl
 
 
 def bench_ours(args, rank, world, device):
@@ -234,9 +271,20 @@ def bench_ours(args, rank, world, device):
     torch.cuda.synchronize()
     if not (torch.equal(o_api, step.o) and torch.equal(Sf_api, step.S_final)):
         raise RuntimeError("per-step composition differs from la_seg_forward")
+    del o_api, Sf_api
+    if w.backward:
+        wsb = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk,
+                               la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16, True, device)
+        g_api = la_seg.la_seg_backward(x["q"], x["k"], x["v"], x["log_g"], x["dO"], None, None, None,
+                                       w.P, w.chunk, want_dS0=True, ws=wsb)
+        la_seg.la_seg_check_status(wsb)
+        if not (all(torch.equal(a, b) for a, b in zip(g_api[:4], step.grads))
+                and torch.equal(g_api[4], step.dS0)):
+            raise RuntimeError("per-step composition differs from la_seg_backward")
+        del g_api, wsb
+    torch.cuda.synchronize()
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} after the check run")
-    del o_api, Sf_api
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     for _ in range(args.warmup):
@@ -275,8 +323,7 @@ def bench_ours(args, rank, world, device):
     dom = max(range(len(step.phases)), key=lambda i: mean_phase[i])
     dname = step.phases[dom]
     achieved = ab[dname] / (mean_phase[dom] / 1e3) / 1e9
-    kernel_key = {"state pass": "state_pass", "output pass": "output_pass", "local pass": "local_pass",
-                  "correction pass": "correct_pass", "state scan": "scan"}[dname]
+    kernel_key = Step.KERNEL_KEYS[dname]
     phases = {}
     for i, name in enumerate(step.phases):
         sec = mean_phase[i] / 1e3
@@ -308,30 +355,45 @@ def bench_ours(args, rank, world, device):
 
 
 def bench_e2e(args, w, x, device, world):
-    """Same metric through the public entry point with host buffers: per step, pinned host ->
-    device copies of q, k, v, log_g, la_seg_forward, and the device -> host copy of o."""
+    """Same metric through the public entry points with host buffers: per step, pinned host ->
+    device copies of the inputs (q, k, v, log_g, and dO for fwd+bwd), la_seg_forward (saving
+    the received states), la_seg_backward reusing them, and device -> host copies of the
+    results (o and S_final; dq, dk, dv, dlog_g and dS0 for fwd+bwd)."""
     from sequence_linear_attention_chunked_b200 import la_seg
-    host = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "log_g")}
-    dev = {n: torch.empty_like(x[n]) for n in host}
-    o_host = torch.empty(x["q"].shape[:-1] + (w.dv,), dtype=w.torch_dtype).pin_memory()
+    names = ("q", "k", "v", "log_g") + (("dO",) if w.backward else ())
+    host = {n: x[n].cpu().pin_memory() for n in names}
+    dev = {n: torch.empty_like(x[n]) for n in names}
     dt = la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16
     ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device)
+    wsb = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, device) if w.backward else None
+    f32 = dict(dtype=torch.float32, device=device)
     o_dev = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype, device=device)
-    Sf = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
-    Sf_host = torch.empty_like(Sf, device="cpu").pin_memory()
+    Sf = torch.empty((w.B, w.H, w.dk, w.dv), **f32)
+    Sr = torch.empty((w.B, w.H, w.P, w.dk, w.dv), **f32) if w.backward else None
+    outs = [o_dev, Sf]
+    if w.backward:
+        grads = [torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
+                 torch.empty_like(x["log_g"]), torch.empty_like(Sf)]
+        outs += grads
+    outs_host = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
     steps = max(3, min(args.steps, 20))
+    P = la_seg._ptr
 
     def one():
-        for n in host:
+        for n in names:
             dev[n].copy_(host[n], non_blocking=True)
-        st = la_seg.lib().la_seg_forward(
-            la_seg._ptr(dev["q"]), la_seg._ptr(dev["k"]), la_seg._ptr(dev["v"]),
-            la_seg._ptr(dev["log_g"]), None, w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt,
-            la_seg._ptr(o_dev), la_seg._ptr(Sf), None, 0, la_seg._ptr(ws), ws.numel(),
-            la_seg._stream(None))
-        la_seg._check(st, "la_seg_forward")
-        o_host.copy_(o_dev, non_blocking=True)
-        Sf_host.copy_(Sf, non_blocking=True)
+        la_seg._check(la_seg.lib().la_seg_forward(
+            P(dev["q"]), P(dev["k"]), P(dev["v"]), P(dev["log_g"]), None, w.B, w.H, w.L, w.dk, w.dv,
+            w.P, w.chunk, dt, P(o_dev), P(Sf), P(Sr), 0, P(ws), ws.numel(), la_seg._stream(None)),
+            "la_seg_forward")
+        if w.backward:
+            la_seg._check(la_seg.lib().la_seg_backward(
+                P(dev["q"]), P(dev["k"]), P(dev["v"]), P(dev["log_g"]), None, P(Sr), P(dev["dO"]),
+                None, w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, P(grads[0]), P(grads[1]),
+                P(grads[2]), P(grads[3]), P(grads[4]), P(wsb), wsb.numel(), la_seg._stream(None)),
+                "la_seg_backward")
+        for d, h in zip(outs, outs_host):
+            h.copy_(d, non_blocking=True)
 
     for _ in range(3):
         one()
@@ -350,40 +412,59 @@ def bench_e2e(args, w, x, device, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = o_host.numel() * o_host.element_size() + Sf_host.numel() * 4
+    d2h = sum(v.numel() * v.element_size() for v in outs_host)
+    api = "la_seg_forward" + (" + la_seg_backward" if w.backward else "")
     return {"value": round(w.B * w.L * world * steps / (ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": "la_seg_forward (C ABI) with pinned host buffers"}
+            "api": f"{api} (C ABI) with pinned host buffers"}
 
 
 # ----------------------------------------------------------------------------- oracle arm
-def cpu_sample(w: Workload, budget_s: float):
-    """Times the fp64 oracle on a bounded sample of the workload: all B*H heads over the first
-    n tokens (n a power of two <= L), repeated until about budget_s seconds have passed."""
+def cpu_sample(w: Workload, budget_s: float, steps: int = 0, warmup: int = 0):
+    """Times the fp64 oracle on bounded samples of the workload: all B*H heads over the first
+    n tokens, n a power of two <= L chosen from a calibration run.  With steps = 0 one sample
+    is repeated for about budget_s seconds; otherwise `warmup` untimed and `steps` timed
+    samples are run, n sized so that they take about budget_s in total."""
     import oracle
-    n = min(w.L, 4096)
-    xs = make_inputs(w.with_(L=n), "cpu")
-    reps, t0 = 0, time.perf_counter()
-    while True:
+
+    def run(n):
+        xs = make_inputs(w.with_(L=n), "cpu")
+        t0 = time.perf_counter()
         oracle.forward(xs["q"], xs["k"], xs["v"], xs["log_g"])
         if w.backward:
             oracle.backward(xs["q"], xs["k"], xs["v"], xs["log_g"], xs["dO"])
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s:
-            break
+        return time.perf_counter() - t0
+
+    cal_n = min(w.L, 256)
+    per_token = run(cal_n) / cal_n
+    per_sample = budget_s / max(1, steps + warmup) if steps else min(budget_s, 4.0)
+    n = cal_n
+    while n * 2 <= w.L and per_token * n * 2 <= per_sample:
+        n *= 2
     cores = oracle.num_threads()
+    if steps:
+        for _ in range(warmup):
+            run(n)
+        el = sum(run(n) for _ in range(steps))
+        reps = steps
+    else:
+        reps, el = 0, 0.0
+        while el < budget_s:
+            el += run(n)
+            reps += 1
     value = w.B * n * reps / el
     return {"value": round(value, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"fp64 token-by-token oracle, all {w.B * w.H} heads x first {n} tokens of "
-                      f"{w.name}, {reps} repetitions, {el:.1f} s; tokens/s = B*n*reps/seconds",
+            "sample": f"fp64 token-by-token oracle{' fwd+bwd' if w.backward else ''}, all "
+                      f"{w.B * w.H} heads x first {n} tokens of {w.name}, {reps} timed samples, "
+                      f"{el:.1f} s; tokens/s = B*n*samples/seconds",
             "seconds": round(el, 2)}
 
 
 def bench_reference(args, w):
-    cb = cpu_sample(w, args.cpu_seconds)
+    cb = cpu_sample(w, args.cpu_seconds * 6, steps=args.steps, warmup=args.warmup)
     return {"metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "ms_per_step": round(cb["seconds"] * 1e3 / args.steps, 3),
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": w.describe(), "B": w.B, "H": w.H, "L": w.L, "d": w.dk, "P": w.P,
@@ -400,7 +481,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="C1", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="C4", choices=sorted(WORKLOADS),
+                    help="C4 (fwd+bwd, every step of the path) by default; C0-C3 forward only")
     ap.add_argument("--schedule", default="auto", choices=["auto", "two", "three"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")

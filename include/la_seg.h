@@ -158,6 +158,24 @@ LA_API la_status la_seg_correct_pass(const void *q, const void *log_g, const flo
                                      int B, int H, long long L, int dk, int dv, int NP, int chunk,
                                      la_dtype dt, void *o, int *status, void *cuda_stream);
 
+/* Gradient-state pass (backward step 2): dSloc[b,h,p] = sum over segment p of
+ * diag(exp(B_t)) q_t^T dO_t, B_t the inclusive cumsum of log_g from the segment's first token,
+ * fp32 [B,H,NP,dk,dv]; log_gamma[b,h,p] = sum of log_g over segment p, fp32 [B,H,NP,dk]. */
+LA_API la_status la_seg_dstate_pass(const void *q, const void *dO, const void *log_g, int B,
+                                    int H, long long L, int dk, int dv, int NP, int chunk,
+                                    la_dtype dt, float *dSloc, float *log_gamma, int *status,
+                                    void *cuda_stream);
+
+/* Gradient pass (backward step 4): dq, dk, dv, dlog_g of every segment p, given the state it
+ * received S_recv[b,h,p] (fp32 [B,H,NP,dk,dv]; null = zero), the gradient dX[b,h,p] of its end
+ * state (from la_seg_scan with reverse = 1 over dSloc, initialised with dS_final), and S_final
+ * (fp32 [B,H,dk,dv]; null when dS_final is zero).  dq_ws: caller scratch, fp32 [B,H,L,dk]. */
+LA_API la_status la_seg_grad_pass(const void *q, const void *k, const void *v, const void *log_g,
+                                  const void *dO, const float *S_recv, const float *S_final,
+                                  const float *dX, int B, int H, long long L, int dk, int dv,
+                                  int NP, int chunk, la_dtype dt, void *dq, void *dk_, void *dv_,
+                                  void *dlog_g, float *dq_ws, int *status, void *cuda_stream);
+
 /* Number of segments (P times the internal split) la_seg_forward uses for these sizes, or 0
  * for rejected sizes.  la_seg_forward's S_recv_save keeps every (NP/P)-th received state. */
 LA_API int la_seg_subsegments(int B, int H, long long L, int dk, int dv, int P, int chunk,

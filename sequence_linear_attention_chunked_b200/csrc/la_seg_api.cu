@@ -244,6 +244,43 @@ la_status la_seg_correct_pass(const void *q, const void *log_g, const float *S_r
                     la::kPassCorrect, static_cast<cudaStream_t>(cuda_stream), "correction pass");
 }
 
+la_status la_seg_dstate_pass(const void *q, const void *dO, const void *log_g, int B, int H,
+                             long long L, int dk, int dv, int NP, int chunk, la_dtype dt,
+                             float *dSloc, float *log_gamma, int *status, void *cuda_stream) {
+    la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
+                              {{q, "q"}, {dO, "dO"}, {log_g, "log_g"}, {dSloc, "dSloc"},
+                               {log_gamma, "log_gamma"}}, {});
+    if (st != LA_OK) return st;
+    if (L == 0) return LA_OK;
+    la::BwdArgs b = {};
+    b.q = q; b.g = log_g; b.dO = dO; b.dSloc = dSloc; b.logG = log_gamma; b.status = status;
+    b.L = L; b.T = L / NP; b.BH = B * H; b.NP = NP; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
+    cudaError_t e = la::launch_bwd_dstate(b, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, "gradient-state pass");
+}
+
+la_status la_seg_grad_pass(const void *q, const void *k, const void *v, const void *log_g,
+                           const void *dO, const float *S_recv, const float *S_final,
+                           const float *dX, int B, int H, long long L, int dk, int dv, int NP,
+                           int chunk, la_dtype dt, void *dq, void *dk_, void *dv_, void *dlog_g,
+                           float *dq_ws, int *status, void *cuda_stream) {
+    la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
+                              {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {dO, "dO"},
+                               {dX, "dX"}, {dq, "dq"}, {dk_, "dk"}, {dv_, "dv"},
+                               {dlog_g, "dlog_g"}, {dq_ws, "dq_ws"}},
+                              {{S_recv, "S_recv"}, {S_final, "S_final"}});
+    if (st != LA_OK) return st;
+    if (L == 0) return LA_OK;
+    la::BwdArgs b = {};
+    b.q = q; b.k = k; b.v = v; b.g = log_g; b.dO = dO;
+    b.dq_out = dq; b.dk_out = dk_; b.dv_out = dv_; b.dg_out = dlog_g;
+    b.S_recv = S_recv; b.S_end_next = S_recv; b.S_fin = S_final; b.dX = dX; b.dq_ws = dq_ws;
+    b.status = status;
+    b.L = L; b.T = L / NP; b.BH = B * H; b.NP = NP; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
+    cudaError_t e = la::launch_bwd_grad(b, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, "gradient pass");
+}
+
 int la_seg_subsegments(int B, int H, long long L, int dk, int dv, int P, int chunk, la_dtype dt) {
     if (check_shape(B, H, L, dk, dv, P, chunk, dt) != LA_OK) return 0;
     return make_split(B, H, L, P, chunk).NP;

@@ -25,7 +25,7 @@ SCHED_AUTO, SCHED_TWO_PASS, SCHED_THREE_PHASE = 0, 1, 2
 EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_seg_scan",
             "la_seg_state_pass", "la_seg_local_pass", "la_seg_output_pass", "la_seg_correct_pass",
             "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail",
-            "la_seg_forward_noalloc")
+            "la_seg_forward_noalloc", "la_seg_dstate_pass", "la_seg_grad_pass")
 
 _lib = None
 
@@ -70,6 +70,12 @@ def lib():
         L.la_seg_forward_noalloc.argtypes = [P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
                                              i32, P, P, P, i32, P]
         L.la_seg_forward_noalloc.restype = i32
+        L.la_seg_dstate_pass.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P,
+                                         P, P]
+        L.la_seg_dstate_pass.restype = i32
+        L.la_seg_grad_pass.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
+                                       i32, P, P, P, P, P, P, P]
+        L.la_seg_grad_pass.restype = i32
         L.la_seg_check_status.argtypes = [P, P]
         L.la_seg_check_status.restype = i32
         L.la_last_error_detail.argtypes = [ctypes.c_char_p, sz]
@@ -265,3 +271,31 @@ def la_seg_correct_pass(q, log_g, S_recv, NP, chunk, o, *, status=None, stream=N
                                      chunk, _dt(q), _ptr(o), _ptr(status), _stream(stream)),
            "la_seg_correct_pass")
     return o
+
+
+def la_seg_dstate_pass(q, dO, log_g, NP, chunk, *, dSloc=None, log_gamma=None, status=None,
+                       stream=None):
+    B, H, L, dk, dv = _seq_shapes(q, dO)
+    dev = q.device
+    dSloc = torch.empty((B, H, NP, dk, dv), dtype=torch.float32, device=dev) if dSloc is None else dSloc
+    log_gamma = (torch.empty((B, H, NP, dk), dtype=torch.float32, device=dev)
+                 if log_gamma is None else log_gamma)
+    _check(lib().la_seg_dstate_pass(_ptr(q), _ptr(dO), _ptr(log_g), B, H, L, dk, dv, NP, chunk,
+                                    _dt(q), _ptr(dSloc), _ptr(log_gamma), _ptr(status),
+                                    _stream(stream)), "la_seg_dstate_pass")
+    return dSloc, log_gamma
+
+
+def la_seg_grad_pass(q, k, v, log_g, dO, S_recv, S_final, dX, NP, chunk, *, out=None, dq_ws=None,
+                     status=None, stream=None):
+    B, H, L, dk, dv = _seq_shapes(q, v)
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_g))
+    if dq_ws is None:
+        dq_ws = torch.empty((B, H, L, dk), dtype=torch.float32, device=q.device)
+    dq, dk_, dv_, dg = out
+    _check(lib().la_seg_grad_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(dO), _ptr(S_recv),
+                                  _ptr(S_final), _ptr(dX), B, H, L, dk, dv, NP, chunk, _dt(q),
+                                  _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dq_ws),
+                                  _ptr(status), _stream(stream)), "la_seg_grad_pass")
+    return out
