@@ -143,8 +143,8 @@ class Step:
 
     KERNEL_KEYS = {"state pass": "state_pass", "output pass": "output_pass",
                    "local pass": "local_pass", "correction pass": "correct_pass",
-                   "state scan": "scan", "dstate pass": "dstate_pass", "reverse scan": "scan",
-                   "grad pass": "grad_pass"}
+                   "state scan": "scan", "dq pass": "dq_pass", "dstate pass": "dstate_pass",
+                   "reverse scan": "scan", "dkv pass": "dkv_pass"}
 
     def __init__(self, w: Workload, x, schedule: str, device):
         from sequence_linear_attention_chunked_b200 import la_seg
@@ -164,14 +164,20 @@ class Step:
         self.phases = (["state pass", "state scan", "output pass"] if schedule != "three"
                        else ["local pass", "state scan", "correction pass"])
         if w.backward:
-            self.phases += ["dstate pass", "reverse scan", "grad pass"]
-            self.dSloc = torch.empty_like(self.S_loc)
-            self.logG_b = torch.empty_like(self.logG)
-            self.dX = torch.empty_like(self.S_loc)
+            # the backward's fine split (parts of <= 1024 tokens) under the forward's segments
+            self.NPF = la_seg.la_seg_backward_parts(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt,
+                                                    False)
+            self.fine = self.NPF // NP
+            self.phases += ["dq pass", "dstate pass", "reverse scan", "dkv pass"]
+            NPF = self.NPF
+            self.S_fine = torch.empty((B, H, NPF, dk, dv), **f32)
+            self.dSloc = torch.empty((B, H, NPF, dk, dv), **f32)
+            self.logG_b = torch.empty((B, H, NPF, dk), **f32)
+            self.dX = torch.empty((B, H, NPF, dk, dv), **f32)
             self.dS0 = torch.empty_like(self.S_final)
             self.grads = (torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
                           torch.empty_like(x["log_g"]))
-            self.dq_ws = torch.empty((B, H, L, dk), **f32)
+            self.qdq = torch.empty((B, H, L, dk), **f32)
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
         self.launches_per_step = len(self.phases)
 
@@ -201,16 +207,21 @@ class Step:
         rec(3)
         if not w.backward:
             return
-        la.la_seg_dstate_pass(x["q"], x["dO"], x["log_g"], NP, w.chunk, dSloc=self.dSloc,
-                              log_gamma=self.logG_b, status=self.status)
+        la.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_recv, NP, self.fine,
+                          w.chunk, dq=self.grads[0], qdq=self.qdq, S_fine=self.S_fine,
+                          status=self.status)
         rec(4)
-        la._check(la.lib().la_seg_scan(la._ptr(self.dSloc), la._ptr(self.logG_b), None, BH, NP,
+        NPF = self.NPF
+        la.la_seg_dstate_pass(x["q"], x["dO"], x["log_g"], NPF, w.chunk, dSloc=self.dSloc,
+                              log_gamma=self.logG_b, status=self.status)
+        rec(5)
+        la._check(la.lib().la_seg_scan(la._ptr(self.dSloc), la._ptr(self.logG_b), None, BH, NPF,
                                        w.dk, w.dv, 1, la._ptr(self.dX), la._ptr(self.dS0),
                                        la._stream(None)), "la_seg_scan")
-        rec(5)
-        la.la_seg_grad_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_recv, None, self.dX,
-                            NP, w.chunk, out=self.grads, dq_ws=self.dq_ws, status=self.status)
         rec(6)
+        la.la_seg_dkv_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_fine, None, self.dX,
+                           self.qdq, NPF, w.chunk, out=self.grads[1:], status=self.status)
+        rec(7)
 
     def phase_ms(self):
         return [self.events[i].elapsed_time(self.events[i + 1]) for i in range(len(self.phases))]
@@ -231,9 +242,12 @@ class Step:
             ab = {"local pass": th * (3 * w.dk + 2 * w.dv) * e + st + lg, "state scan": scan,
                   "correction pass": th * (2 * w.dk + 2 * w.dv) * e + st}
         if w.backward:
-            ab["dstate pass"] = th * (2 * w.dk + w.dv) * e + st + lg
-            ab["reverse scan"] = scan
-            ab["grad pass"] = th * (3 * w.dk + 2 * w.dv + 3 * w.dk + w.dv) * e + 2 * st
+            stf = w.B * w.H * self.NPF * w.dk * w.dv * 4
+            lgf = w.B * w.H * self.NPF * w.dk * 4
+            ab["dq pass"] = th * (3 * w.dk + 2 * w.dv + w.dk) * e + st + stf
+            ab["dstate pass"] = th * (2 * w.dk + w.dv) * e + stf + lgf
+            ab["reverse scan"] = 2 * stf + lgf + fin
+            ab["dkv pass"] = th * (3 * w.dk + 2 * w.dv + 2 * w.dk + w.dv) * e + 2 * stf
         return ab
 
     def flops(self):
@@ -247,9 +261,10 @@ class Step:
         else:
             fl = {"local pass": th * (intra + 2 * dd), "state scan": 0, "correction pass": th * dd}
         if w.backward:
+            fl["dq pass"] = th * (2 * C * dv + 2 * C * dk + 2 * dd)
             fl["dstate pass"] = th * dd
             fl["reverse scan"] = 0
-            fl["grad pass"] = th * (5 * dd + 2 * C * (3 * dk + 3 * dv))
+            fl["dkv pass"] = th * (3 * dd + 2 * C * (3 * dk + 2 * dv))
         return fl
 
 

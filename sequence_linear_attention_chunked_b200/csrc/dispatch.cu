@@ -10,8 +10,22 @@ cudaError_t launch_pass(const PassArgs &a, PassMode mode, cudaStream_t st) {
     return launch_simt_pass(a, mode, st);
 }
 
-cudaError_t launch_bwd_dstate(const BwdArgs &a, cudaStream_t st) { return launch_simt_dstate(a, st); }
+cudaError_t launch_bwd_dstate(const BwdArgs &a, cudaStream_t st) {
+    PassArgs p = {};
+    p.q = a.q; p.v = a.dO; p.g = a.g;  // the gradient-state pass reads dO through the v slot
+    p.S_out = a.dSloc; p.logG = a.logG; p.status = a.status;
+    p.L = a.L; p.T = a.T; p.BH = a.BH; p.NP = a.NP; p.dk = a.dk; p.dv = a.dv; p.chunk = a.chunk;
+    p.dt = a.dt;
+    if (tc_pass_supported(p)) return launch_tc_pass(p, kPassDState, st);
+    return launch_simt_dstate(a, st);
+}
 
-cudaError_t launch_bwd_grad(const BwdArgs &a, cudaStream_t st) { return launch_simt_grad(a, st); }
+cudaError_t launch_bwd_dq(const BwdArgs &a, cudaStream_t st) {
+    return tc_bwd_supported(a) ? launch_tc_dq(a, st) : launch_simt_dq(a, st);
+}
+
+cudaError_t launch_bwd_dkv(const BwdArgs &a, cudaStream_t st) {
+    return tc_bwd_supported(a) ? launch_tc_dkv(a, st) : launch_simt_dkv(a, st);
+}
 
 }  // namespace la

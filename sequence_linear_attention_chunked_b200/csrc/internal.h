@@ -16,6 +16,7 @@ enum PassMode : int {
     kPassOutput = 1,   // o from S_init[j]; reads q, k, v, log_g; writes o
     kPassLocal = 2,    // o_local from zero, local state and log-decay sum; writes o, S, logG
     kPassCorrect = 3,  // o += (q . exp(B_seg)) S_init[j]; reads q, log_g, o
+    kPassDState = 4,   // backward gradient state sum_t diag(e^{B_t}) q_t^T dO_t (dO passed as v)
 };
 
 struct PassArgs {
@@ -30,30 +31,42 @@ struct PassArgs {
     la_dtype dt;
 };
 
-// Arguments of the backward chunk passes (one CTA per (b, h, segment j)).
+// Arguments of the backward chunk passes (one CTA per (b, h, segment j)).  The dq sweep runs
+// over NP segments of T tokens and records the state entering every one of its `fine` equal
+// parts in S_fine; the gradient-state pass and the reverse sweep run over those fine parts
+// (NP and T then describe the fine split), so that the exact dlog_g carry
+// rowsum(S_end . dX) is re-anchored every T tokens.
 struct BwdArgs {
     const void *q, *k, *v, *g, *dO;
     void *dq_out, *dk_out, *dv_out, *dg_out;
-    const float *S_recv;      // [BH, NP, dk, dv] state each segment receives (null: zero)
-    const float *S_end_next;  // same array as S_recv: S_end_j = S_recv[j+1] for j < NP-1 (null: no carry)
+    const float *S_recv;      // dq sweep: [BH, NP, dk, dv] state each segment receives (null: zero)
+    float *S_fine;            // dq sweep output: [BH, NP * fine, dk, dv] (null: not recorded)
+    const float *S_end_next;  // reverse sweep: S_end_j = S_end_next[j+1] for j < NP-1 (null: no carry)
     const float *S_fin;       // [BH, dk, dv] state after the last token (null: no carry there)
     const float *dX;          // [BH, NP, dk, dv] gradient of each segment's end state
-    float *dq_ws;             // [BH, L, dk] fp32 dq between the two sweeps
+    float *dq_ws;             // [BH, L, dk] fp32 q . dq, from the dq sweep to the reverse sweep
     float *dSloc;             // [BH, NP, dk, dv] per-segment gradient states (dstate pass)
     float *logG;              // [BH, NP, dk] per-segment log-decay sums (dstate pass)
     int *status;
     long long L, T;
-    int BH, NP, dk, dv, chunk;
+    int BH, NP, dk, dv, chunk, fine;
     la_dtype dt;
 };
 
 // Backward passes for these arguments (tensor-core kernels where they apply, else SIMT).
 cudaError_t launch_bwd_dstate(const BwdArgs &a, cudaStream_t st);
-cudaError_t launch_bwd_grad(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_dq(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_dkv(const BwdArgs &a, cudaStream_t st);
+
+// tcgen05 backward passes (bf16, d = 128, chunk 64).
+bool tc_bwd_supported(const BwdArgs &a);
+cudaError_t launch_tc_dq(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_tc_dkv(const BwdArgs &a, cudaStream_t st);
 
 // Generic CUDA-core backward passes.
 cudaError_t launch_simt_dstate(const BwdArgs &a, cudaStream_t st);
-cudaError_t launch_simt_grad(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_simt_dq(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_simt_dkv(const BwdArgs &a, cudaStream_t st);
 
 // Generic CUDA-core (FFMA) chunk pass: any supported dtype, d and chunk.
 cudaError_t launch_simt_pass(const PassArgs &a, PassMode mode, cudaStream_t st);

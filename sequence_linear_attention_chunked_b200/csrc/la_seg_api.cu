@@ -98,23 +98,44 @@ FwdLayout fwd_layout(const la::Split &s, int dk, int dv) {
     return w;
 }
 
+// Fine parts per segment for the backward's reverse sweep: the largest power-of-two split
+// into parts of at most 1024 tokens (whole chunks).  dlog_g is re-anchored on the exact carry
+// rowsum(S_end . dX) at every part boundary, which keeps the bf16 rounding of the per-token
+// terms it sums from accumulating over long segments.
+int fine_factor(long long T, int chunk) {
+    int r = 1;
+    while (T / r > 1024 && T % (2LL * r) == 0 && (T / (2LL * r)) % chunk == 0) r *= 2;
+    return r;
+}
+
 struct BwdLayout {
-    size_t status, S_loc, logG, S_recv, S_fin, dSloc, dX, dq_ws, total;
+    size_t status, S_loc, logG, S_recv, S_fin, S_fine, dSloc, logG_f, dX, qdq, total;
 };
 
-BwdLayout bwd_layout(const la::Split &s, int dk, int dv) {
+BwdLayout bwd_layout(const la::Split &s, int r, int dk, int dv) {
     BwdLayout w;
     const size_t states = (size_t)s.BH * s.NP * dk * dv * sizeof(float);
+    const size_t fine_states = states * r;
     const size_t gam = (size_t)s.BH * s.NP * dk * sizeof(float);
     w.status = 0;
     w.S_loc = 256;
     w.logG = align_up(w.S_loc + states, 256);
     w.S_recv = align_up(w.logG + gam, 256);
     w.S_fin = align_up(w.S_recv + states, 256);
-    w.dSloc = align_up(w.S_fin + (size_t)s.BH * dk * dv * sizeof(float), 256);
-    w.dX = align_up(w.dSloc + states, 256);
-    w.dq_ws = align_up(w.dX + states, 256);
-    w.total = align_up(w.dq_ws + (size_t)s.BH * s.L * dk * sizeof(float), 256);
+    w.S_fine = align_up(w.S_fin + (size_t)s.BH * dk * dv * sizeof(float), 256);
+    w.dSloc = align_up(w.S_fine + fine_states, 256);
+    w.logG_f = align_up(w.dSloc + fine_states, 256);
+    w.dX = align_up(w.logG_f + gam * r, 256);
+    w.qdq = align_up(w.dX + fine_states, 256);
+    w.total = align_up(w.qdq + (size_t)s.BH * s.L * dk * sizeof(float), 256);
+    return w;
+}
+
+la::Split whole_segments(const la::Split &s) {
+    la::Split w = s;
+    w.m = 1;
+    w.NP = s.P;
+    w.T = s.L / s.P;
     return w;
 }
 
@@ -146,11 +167,10 @@ size_t la_seg_workspace_bytes(int B, int H, long long L, int dk, int dv, int P, 
     if (check_shape(B, H, L, dk, dv, P, chunk, dt) != LA_OK) return 0;
     const la::Split s = make_split(B, H, L, P, chunk);
     if (!backward) return fwd_layout(s, dk, dv).total;
-    la::Split whole = s;  // la_seg_backward keeps whole segments when it reuses saved states
-    whole.m = 1;
-    whole.NP = P;
-    whole.T = L / P;
-    const size_t a = bwd_layout(s, dk, dv).total, b = bwd_layout(whole, dk, dv).total;
+    // la_seg_backward keeps whole segments when it reuses saved states
+    const la::Split whole = whole_segments(s);
+    const size_t a = bwd_layout(s, fine_factor(s.T, chunk), dk, dv).total;
+    const size_t b = bwd_layout(whole, fine_factor(whole.T, chunk), dk, dv).total;
     return a > b ? a : b;
 }
 
@@ -254,31 +274,62 @@ la_status la_seg_dstate_pass(const void *q, const void *dO, const void *log_g, i
     if (L == 0) return LA_OK;
     la::BwdArgs b = {};
     b.q = q; b.g = log_g; b.dO = dO; b.dSloc = dSloc; b.logG = log_gamma; b.status = status;
+    b.fine = 1;
     b.L = L; b.T = L / NP; b.BH = B * H; b.NP = NP; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
     cudaError_t e = la::launch_bwd_dstate(b, static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? LA_OK : cuda_fail(e, "gradient-state pass");
 }
 
-la_status la_seg_grad_pass(const void *q, const void *k, const void *v, const void *log_g,
-                           const void *dO, const float *S_recv, const float *S_final,
-                           const float *dX, int B, int H, long long L, int dk, int dv, int NP,
-                           int chunk, la_dtype dt, void *dq, void *dk_, void *dv_, void *dlog_g,
-                           float *dq_ws, int *status, void *cuda_stream) {
+la_status la_seg_dq_pass(const void *q, const void *k, const void *v, const void *log_g,
+                         const void *dO, const float *S_recv, int B, int H, long long L, int dk,
+                         int dv, int NP, int fine, int chunk, la_dtype dt, void *dq, float *qdq,
+                         float *S_fine, int *status, void *cuda_stream) {
     la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
                               {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {dO, "dO"},
-                               {dX, "dX"}, {dq, "dq"}, {dk_, "dk"}, {dv_, "dv"},
-                               {dlog_g, "dlog_g"}, {dq_ws, "dq_ws"}},
+                               {dq, "dq"}, {qdq, "qdq"}},
+                              {{S_recv, "S_recv"}, {S_fine, "S_fine"}});
+    if (st != LA_OK) return st;
+    if (fine < 1 || (L > 0 && ((L / NP) % fine != 0 || ((L / NP) / fine) % chunk != 0)))
+        return fail(LA_ERR_SHAPE, "fine=%d must cut each segment into whole chunks", fine);
+    if (L == 0) return LA_OK;
+    la::BwdArgs b = {};
+    b.q = q; b.k = k; b.v = v; b.g = log_g; b.dO = dO; b.dq_out = dq; b.dq_ws = qdq;
+    b.S_recv = S_recv; b.S_fine = S_fine; b.status = status;
+    b.L = L; b.T = L / NP; b.BH = B * H; b.NP = NP; b.dk = dk; b.dv = dv; b.chunk = chunk;
+    b.fine = fine; b.dt = dt;
+    cudaError_t e = la::launch_bwd_dq(b, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, "dq pass");
+}
+
+la_status la_seg_dkv_pass(const void *q, const void *k, const void *v, const void *log_g,
+                          const void *dO, const float *S_recv, const float *S_final,
+                          const float *dX, const float *qdq, int B, int H, long long L, int dk,
+                          int dv, int NP, int chunk, la_dtype dt, void *dk_, void *dv_,
+                          void *dlog_g, int *status, void *cuda_stream) {
+    la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
+                              {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {dO, "dO"},
+                               {dX, "dX"}, {qdq, "qdq"}, {dk_, "dk"}, {dv_, "dv"},
+                               {dlog_g, "dlog_g"}},
                               {{S_recv, "S_recv"}, {S_final, "S_final"}});
     if (st != LA_OK) return st;
     if (L == 0) return LA_OK;
     la::BwdArgs b = {};
     b.q = q; b.k = k; b.v = v; b.g = log_g; b.dO = dO;
-    b.dq_out = dq; b.dk_out = dk_; b.dv_out = dv_; b.dg_out = dlog_g;
-    b.S_recv = S_recv; b.S_end_next = S_recv; b.S_fin = S_final; b.dX = dX; b.dq_ws = dq_ws;
+    b.dk_out = dk_; b.dv_out = dv_; b.dg_out = dlog_g;
+    b.S_end_next = S_recv; b.S_fin = S_final; b.dX = dX; b.dq_ws = const_cast<float *>(qdq);
     b.status = status;
-    b.L = L; b.T = L / NP; b.BH = B * H; b.NP = NP; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
-    cudaError_t e = la::launch_bwd_grad(b, static_cast<cudaStream_t>(cuda_stream));
-    return e == cudaSuccess ? LA_OK : cuda_fail(e, "gradient pass");
+    b.L = L; b.T = L / NP; b.BH = B * H; b.NP = NP; b.dk = dk; b.dv = dv; b.chunk = chunk;
+    b.fine = 1; b.dt = dt;
+    cudaError_t e = la::launch_bwd_dkv(b, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, "dkv pass");
+}
+
+int la_seg_backward_parts(int B, int H, long long L, int dk, int dv, int P, int chunk,
+                          la_dtype dt, int reuse) {
+    if (check_shape(B, H, L, dk, dv, P, chunk, dt) != LA_OK) return 0;
+    const la::Split base = make_split(B, H, L, P, chunk);
+    const la::Split s = reuse ? whole_segments(base) : base;
+    return s.NP * fine_factor(s.T, chunk);
 }
 
 int la_seg_subsegments(int B, int H, long long L, int dk, int dv, int P, int chunk, la_dtype dt) {
@@ -362,16 +413,13 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     for (int i = 0; i < 13; ++i)
         if (ptrs[i] && !aligned(ptrs[i], 16))
             return fail(LA_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
-    // Saved states are per API segment: when they can be reused (S_final not needed), keep
-    // whole segments so that every segment's received state is one the forward saved.
-    la::Split s = make_split(B, H, L, P, chunk);
+    // Saved states are per API segment: when they can be reused (S_final not needed), the dq
+    // sweep keeps whole segments so that every segment's received state is one the forward saved.
     const bool reuse = S_recv_saved && !dS_final;
-    if (reuse) {
-        s.m = 1;
-        s.NP = P;
-        s.T = L / P;
-    }
-    const BwdLayout w = bwd_layout(s, dk, dv);
+    const la::Split base = make_split(B, H, L, P, chunk);
+    const la::Split s = reuse ? whole_segments(base) : base;
+    const int r = fine_factor(s.T, chunk);
+    const BwdLayout w = bwd_layout(s, r, dk, dv);
     const size_t need = la_seg_workspace_bytes(B, H, L, dk, dv, P, chunk, dt, 1);
     if (!workspace || ws_bytes < need)
         return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu%s)", need,
@@ -390,9 +438,11 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     float *logG = reinterpret_cast<float *>(at(workspace, w.logG));
     float *S_recv = reinterpret_cast<float *>(at(workspace, w.S_recv));
     float *S_fin = reinterpret_cast<float *>(at(workspace, w.S_fin));
+    float *S_fine = reinterpret_cast<float *>(at(workspace, w.S_fine));
     float *dSloc = reinterpret_cast<float *>(at(workspace, w.dSloc));
+    float *logG_f = reinterpret_cast<float *>(at(workspace, w.logG_f));
     float *dX = reinterpret_cast<float *>(at(workspace, w.dX));
-    float *dq_ws = reinterpret_cast<float *>(at(workspace, w.dq_ws));
+    float *qdq = reinterpret_cast<float *>(at(workspace, w.qdq));
 
     // 1. the states each segment receives: the forward's when given and S_final is not needed
     //    (dS_final = 0); otherwise recomputed (state pass + scan)
@@ -406,20 +456,25 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
             cudaSuccess)
             return cuda_fail(e, "backward state scan");
     }
-    la::BwdArgs b;
+    la::BwdArgs b = {};
     b.q = q; b.k = k; b.v = v; b.g = log_g; b.dO = dO;
     b.dq_out = dq; b.dk_out = dk_; b.dv_out = dv_; b.dg_out = dlog_g;
-    b.S_recv = recv; b.S_end_next = recv; b.S_fin = reuse ? nullptr : S_fin; b.dX = dX;
-    b.dq_ws = dq_ws; b.dSloc = dSloc; b.logG = logG; b.status = status;
-    b.L = L; b.T = s.T; b.BH = s.BH; b.NP = s.NP; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
-    // 2. per-segment gradient states and log-decay sums
+    b.S_recv = recv; b.S_fine = S_fine; b.S_end_next = S_fine; b.S_fin = reuse ? nullptr : S_fin;
+    b.dX = dX; b.dq_ws = qdq; b.dSloc = dSloc; b.logG = logG_f; b.status = status;
+    b.L = L; b.BH = s.BH; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
+    // 2. dq sweep over the segments; records the state entering each of their r fine parts
+    b.NP = s.NP; b.T = s.T; b.fine = r;
+    if ((e = la::launch_bwd_dq(b, stream)) != cudaSuccess) return cuda_fail(e, "dq pass");
+    // 3-5 run over the fine parts
+    b.NP = s.NP * r; b.T = s.T / r; b.fine = 1;
+    // 3. per-part gradient states and log-decay sums
     if ((e = la::launch_bwd_dstate(b, stream)) != cudaSuccess) return cuda_fail(e, "gradient-state pass");
-    // 3. reverse exclusive decayed scan: gradient of every segment's end state, and dS0
-    if ((e = la::launch_scan(dSloc, logG, dS_final, s.BH, s.NP, dk, dv, 1, dX, dS0, stream)) !=
+    // 4. reverse exclusive decayed scan: gradient of every part's end state, and dS0
+    if ((e = la::launch_scan(dSloc, logG_f, dS_final, s.BH, b.NP, dk, dv, 1, dX, dS0, stream)) !=
         cudaSuccess)
         return cuda_fail(e, "reverse state scan");
-    // 4. dq, dk, dv, dlog_g per segment
-    if ((e = la::launch_bwd_grad(b, stream)) != cudaSuccess) return cuda_fail(e, "gradient pass");
+    // 5. dk, dv, dlog_g per part
+    if ((e = la::launch_bwd_dkv(b, stream)) != cudaSuccess) return cuda_fail(e, "dkv pass");
     return LA_OK;
 }
 

@@ -7,7 +7,9 @@
 // A_ts = [s<=t] Qbar'_t . Ktil_s:
 //
 //   forward sweep   dq_t  = e^{b_t - b_C} (dO_t S'^T + sum_s M_ts Ktil_s);  S = S' + Ktil^T V
-//   reverse sweep   dk_s  = e^{b_C - b_s} (sum_t M_ts Qbar'_t + v_s dS^T)
+//                   (one kernel; it also stores q_t . dq_t in fp32 for the reverse sweep)
+//   reverse sweep   (a second kernel)
+//                   dk_s  = e^{b_C - b_s} (sum_t M_ts Qbar'_t + v_s dS^T)
 //                   dv_s  = sum_t A_ts dO_t + Ktil_s dS
 //                   dS   <- diag(e^{b_C}) (dS + Qbar'^T dO)           (dS starts at dX_j)
 //                   dlog_g_t = sum_{u>=t in segment} (q_u dq_u - k_u dk_u) + rowsum(S_end_j . dX_j)
@@ -117,7 +119,95 @@ struct GradSmem {
 };
 
 template <typename T, int DK, int DV, int C>
-__global__ void __launch_bounds__(kThreads) simt_grad_kernel(BwdArgs a) {
+__global__ void __launch_bounds__(kThreads) simt_dq_kernel(BwdArgs a) {
+    using L = GradSmem<DK, DV, C>;
+    constexpr int DKP = L::DKP, CP = L::CP;
+    extern __shared__ float smem[];
+    float *sq = smem + L::q, *sk = smem + L::k, *sv = smem + L::v, *sb = smem + L::b,
+          *sd = smem + L::dO, *sM = smem + L::M, *sA = smem + L::A, *sS = smem + L::S,
+          *scg = smem + L::cg, *seC = smem + L::eC, *sbC = smem + L::bC, *saccg = smem + L::accg;
+    const int tid = threadIdx.x;
+    const int bh = blockIdx.x / a.NP, j = blockIdx.x % a.NP;
+    const long long base = (long long)bh * a.L + (long long)j * a.T;
+    const T *q = static_cast<const T *>(a.q) + base * DK;
+    const T *k = static_cast<const T *>(a.k) + base * DK;
+    const T *g = static_cast<const T *>(a.g) + base * DK;
+    const T *v = static_cast<const T *>(a.v) + base * DV;
+    const T *dO = static_cast<const T *>(a.dO) + base * DV;
+    float *dqw = a.dq_ws + base * DK;
+    T *dqo = static_cast<T *>(a.dq_out) + base * DK;
+    const long long sidx = ((long long)bh * a.NP + j) * DK * DV;
+
+    // cumsum of the chunk's log-gates (threads < DK), then e^{b_C}; returns after a barrier
+    auto gates = [&](long long r0) {
+        if (tid < DK) {
+            float acc = 0.f;
+            for (int t = 0; t < C; ++t) {
+                acc += sb[t * DKP + tid];
+                sb[t * DKP + tid] = acc;
+            }
+            sbC[tid] = acc;
+            seC[tid] = __expf(acc);
+        }
+        __syncthreads();
+    };
+
+    // ---- forward sweep: dq, and q . dq (fp32) for the reverse sweep's dlog_g
+    for (int idx = tid; idx < DK * DV; idx += kThreads) sS[idx] = a.S_recv ? a.S_recv[sidx + idx] : 0.f;
+    const long long Tf = a.T / a.fine;
+    for (long long r0 = 0; r0 < a.T; r0 += C) {
+        __syncthreads();
+        if (a.S_fine && r0 % Tf == 0) {  // the state entering fine part r0 / Tf of this segment
+            float *Sf = a.S_fine + (((long long)bh * a.NP + j) * a.fine + r0 / Tf) * DK * DV;
+            for (int idx = tid; idx < DK * DV; idx += kThreads) Sf[idx] = sS[idx];
+        }
+        for (int idx = tid; idx < C * DK; idx += kThreads) {
+            const int t = idx / DK, i = idx % DK;
+            sk[t * DKP + i] = to_f32(k[(r0 + t) * DK + i]);
+            sb[t * DKP + i] = to_f32(g[(r0 + t) * DK + i]);
+        }
+        for (int idx = tid; idx < C * DV; idx += kThreads) {
+            sv[idx] = to_f32(v[(r0 + idx / DV) * DV + idx % DV]);
+            sd[idx] = to_f32(dO[(r0 + idx / DV) * DV + idx % DV]);
+        }
+        __syncthreads();
+        gates(r0);
+        for (int idx = tid; idx < C * DK; idx += kThreads) {
+            const int t = idx / DK, i = idx % DK;
+            sk[t * DKP + i] *= __expf(sbC[i] - sb[t * DKP + i]);
+        }
+        for (int idx = tid; idx < DK * DV; idx += kThreads) sS[idx] *= seC[idx / DV];
+        for (int idx = tid; idx < C * C; idx += kThreads) {
+            const int t = idx / C, s = idx % C;
+            float acc = 0.f;
+            if (s <= t)
+                for (int jj = 0; jj < DV; ++jj) acc += sd[t * DV + jj] * sv[s * DV + jj];
+            sM[t * CP + s] = acc;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < C * DK; idx += kThreads) {
+            const int t = idx / DK, i = idx % DK;
+            float acc = 0.f;
+            for (int jj = 0; jj < DV; ++jj) acc += sd[t * DV + jj] * sS[i * DV + jj];
+            for (int s = 0; s <= t; ++s) acc += sM[t * CP + s] * sk[s * DKP + i];
+            const float dqv = acc * __expf(sb[t * DKP + i] - sbC[i]);
+            dqo[(r0 + t) * DK + i] = from_f32<T>(dqv);
+            dqw[(r0 + t) * DK + i] = to_f32(q[(r0 + t) * DK + i]) * dqv;  // q . dq for dlog_g
+        }
+        __syncthreads();
+        for (int idx = tid; idx < DK * DV; idx += kThreads) {
+            const int i = idx / DV, jj = idx % DV;
+            float acc = sS[idx];
+            for (int s = 0; s < C; ++s) acc += sk[s * DKP + i] * sv[s * DV + jj];
+            sS[idx] = acc;
+        }
+    }
+    __syncthreads();
+
+}
+
+template <typename T, int DK, int DV, int C>
+__global__ void __launch_bounds__(kThreads) simt_dkv_kernel(BwdArgs a) {
     using L = GradSmem<DK, DV, C>;
     constexpr int DKP = L::DKP, CP = L::CP;
     extern __shared__ float smem[];
@@ -149,52 +239,8 @@ __global__ void __launch_bounds__(kThreads) simt_grad_kernel(BwdArgs a) {
         __syncthreads();
     };
 
-    // ---- forward sweep: dq (fp32, to the workspace)
-    for (int idx = tid; idx < DK * DV; idx += kThreads) sS[idx] = a.S_recv ? a.S_recv[sidx + idx] : 0.f;
-    for (long long r0 = 0; r0 < a.T; r0 += C) {
-        __syncthreads();
-        for (int idx = tid; idx < C * DK; idx += kThreads) {
-            const int t = idx / DK, i = idx % DK;
-            sk[t * DKP + i] = to_f32(k[(r0 + t) * DK + i]);
-            sb[t * DKP + i] = to_f32(g[(r0 + t) * DK + i]);
-        }
-        for (int idx = tid; idx < C * DV; idx += kThreads) {
-            sv[idx] = to_f32(v[(r0 + idx / DV) * DV + idx % DV]);
-            sd[idx] = to_f32(dO[(r0 + idx / DV) * DV + idx % DV]);
-        }
-        __syncthreads();
-        gates(r0);
-        for (int idx = tid; idx < C * DK; idx += kThreads) {
-            const int t = idx / DK, i = idx % DK;
-            sk[t * DKP + i] *= __expf(sbC[i] - sb[t * DKP + i]);
-        }
-        for (int idx = tid; idx < DK * DV; idx += kThreads) sS[idx] *= seC[idx / DV];
-        for (int idx = tid; idx < C * C; idx += kThreads) {
-            const int t = idx / C, s = idx % C;
-            float acc = 0.f;
-            if (s <= t)
-                for (int jj = 0; jj < DV; ++jj) acc += sd[t * DV + jj] * sv[s * DV + jj];
-            sM[t * CP + s] = acc;
-        }
-        __syncthreads();
-        for (int idx = tid; idx < C * DK; idx += kThreads) {
-            const int t = idx / DK, i = idx % DK;
-            float acc = 0.f;
-            for (int jj = 0; jj < DV; ++jj) acc += sd[t * DV + jj] * sS[i * DV + jj];
-            for (int s = 0; s <= t; ++s) acc += sM[t * CP + s] * sk[s * DKP + i];
-            dqw[(r0 + t) * DK + i] = acc * __expf(sb[t * DKP + i] - sbC[i]);
-        }
-        __syncthreads();
-        for (int idx = tid; idx < DK * DV; idx += kThreads) {
-            const int i = idx / DV, jj = idx % DV;
-            float acc = sS[idx];
-            for (int s = 0; s < C; ++s) acc += sk[s * DKP + i] * sv[s * DV + jj];
-            sS[idx] = acc;
-        }
-    }
+    // ---- reverse sweep: dk, dv, dlog_g
     __syncthreads();
-
-    // ---- reverse sweep: dk, dv, dlog_g (and dq converted from the workspace)
     const float *dX = a.dX + sidx;
     for (int idx = tid; idx < DK * DV; idx += kThreads) sS[idx] = dX[idx];
     if (tid < DK) {
@@ -209,7 +255,6 @@ __global__ void __launch_bounds__(kThreads) simt_grad_kernel(BwdArgs a) {
             for (int jj = 0; jj < DV; ++jj) acc += Se[tid * DV + jj] * dX[tid * DV + jj];
         saccg[tid] = acc;
     }
-    T *dq = static_cast<T *>(a.dq_out) + base * DK;
     T *dk = static_cast<T *>(a.dk_out) + base * DK;
     T *dv = static_cast<T *>(a.dv_out) + base * DV;
     T *dg = static_cast<T *>(a.dg_out) + base * DK;
@@ -252,9 +297,7 @@ __global__ void __launch_bounds__(kThreads) simt_grad_kernel(BwdArgs a) {
             for (int jj = 0; jj < DV; ++jj) acc += sS[i * DV + jj] * sv[s * DV + jj];
             const float dks = acc * __expf(sbC[i] - sb[s * DKP + i]);
             dk[(r0 + s) * DK + i] = from_f32<T>(dks);
-            const float dqs = dqw[(r0 + s) * DK + i];
-            dq[(r0 + s) * DK + i] = from_f32<T>(dqs);
-            scg[s * DKP + i] = to_f32(q[(r0 + s) * DK + i]) * dqs - to_f32(k[(r0 + s) * DK + i]) * dks;
+            scg[s * DKP + i] = dqw[(r0 + s) * DK + i] - to_f32(k[(r0 + s) * DK + i]) * dks;
         }
         for (int idx = tid; idx < C * DV; idx += kThreads) {  // dv
             const int s = idx / DV, jj = idx % DV;
@@ -295,7 +338,8 @@ template <typename T, int D, int C>
 cudaError_t launch_c(const BwdArgs &a, int which, cudaStream_t st) {
     if (which == 0) return launch_k(simt_dstate_kernel<T, D, D, C>, DstSmem<D, D, C>::bytes, a, st);
     constexpr int CG = (D == 128 && C > 32) ? 32 : C;  // d = 128: 32-token blocks fit shared memory
-    return launch_k(simt_grad_kernel<T, D, D, CG>, GradSmem<D, D, CG>::bytes, a, st);
+    if (which == 1) return launch_k(simt_dq_kernel<T, D, D, CG>, GradSmem<D, D, CG>::bytes, a, st);
+    return launch_k(simt_dkv_kernel<T, D, D, CG>, GradSmem<D, D, CG>::bytes, a, st);
 }
 
 template <typename T, int D>
@@ -324,8 +368,12 @@ cudaError_t launch_simt_dstate(const BwdArgs &a, cudaStream_t st) {
     return a.dt == LA_F32 ? launch_t<float>(a, 0, st) : launch_t<__nv_bfloat16>(a, 0, st);
 }
 
-cudaError_t launch_simt_grad(const BwdArgs &a, cudaStream_t st) {
+cudaError_t launch_simt_dq(const BwdArgs &a, cudaStream_t st) {
     return a.dt == LA_F32 ? launch_t<float>(a, 1, st) : launch_t<__nv_bfloat16>(a, 1, st);
+}
+
+cudaError_t launch_simt_dkv(const BwdArgs &a, cudaStream_t st) {
+    return a.dt == LA_F32 ? launch_t<float>(a, 2, st) : launch_t<__nv_bfloat16>(a, 2, st);
 }
 
 }  // namespace la

@@ -1,0 +1,957 @@
+// tc_bwd.cu -- backward chunk passes on the 5th-generation tensor cores (bf16, d = 128,
+// chunk = 64): the dq sweep (forward over chunks) and the reverse sweep (dk, dv, dlog_g).
+//
+// dq sweep, per chunk with in-chunk cumsum b_t, total b_C, Ktil_s = k_s e^{b_C - b_s},
+// S' = diag(e^{b_C}) S (S the state entering the chunk, rows = key dims on TMEM lanes):
+//
+//   M    = dO V^T                       M=64  (t)  N=64  (s)  K=128 (j)   -> masked s <= t, bf16
+//   dS   = Ktil^T V                     M=128 (i)  N=128 (j)  K=64  (s)
+//   dq^T = S' dO^T + Ktil^T M^T         M=128 (i)  N=64  (t)  K=128 (j) / 64 (s)
+//   dq[t,i] = e^{b_t,i - b_C,i} dq^T[i,t];   S <- S' + dS
+//
+// The gate warps write e^{b_t - b_C} over the log_g tile (bf16, same swizzled layout) for the
+// epilogue's output scaling.  The epilogue also stores q . dq in fp32, which the reverse sweep
+// needs for dlog_g.  Role layout, bounded waits and the abort path follow tc_pass.cu.
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "tc_common.cuh"
+
+namespace la {
+namespace {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int kEpiWarps = 8, kGateWarps = 4;
+constexpr int kTmaWarp = 12, kMmaWarp = 13;
+constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
+
+// ------------------------------------------------------------------ dq sweep
+namespace dqs {
+
+constexpr uint32_t kColDS = 0, kColDQ = 128, kColSA = 192, kColM = 256;
+constexpr int kStages = 3;
+constexpr int off_k = 0, off_v = kTileBytes, off_do = 2 * kTileBytes, off_g = 3 * kTileBytes;
+constexpr int kStageBytes = 4 * kTileBytes;
+constexpr int off_m = kStages * kStageBytes;
+constexpr int off_ec = off_m + CH * CH * 2;
+constexpr int off_bar = off_ec + kStages * D * 4;
+constexpr int kBars = 3 * kStages + 12;
+constexpr int off_misc = off_bar + kBars * 8;
+constexpr int kSmemBytes = off_misc + 16 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct Bars {
+    uint64_t *full, *gated, *empty;
+    uint64_t *m_full, *m_free, *p_full, *ds_full, *ds_free, *sa_full, *sa_free, *dq_full,
+        *dq_free, *fin;
+};
+
+__device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tk,
+                         const CUtensorMap *tv, const CUtensorMap *tdo, const CUtensorMap *tg,
+                         long long row0, int nchunks) {
+    int issued = 0;
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % kStages;
+        if (c >= kStages && !mbar_wait(&b.empty[s], ((c / kStages) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&b.full[s], kStageBytes);
+        uint8_t *st = smem + s * kStageBytes;
+        const int y = (int)(row0 + (long long)c * CH);
+        tma_load_2d(st + off_k, tk, 0, y, &b.full[s]);
+        tma_load_2d(st + off_k + kHalfBytes, tk, 64, y, &b.full[s]);
+        tma_load_2d(st + off_v, tv, 0, y, &b.full[s]);
+        tma_load_2d(st + off_v + kHalfBytes, tv, 64, y, &b.full[s]);
+        tma_load_2d(st + off_do, tdo, 0, y, &b.full[s]);
+        tma_load_2d(st + off_do + kHalfBytes, tdo, 64, y, &b.full[s]);
+        tma_load_2d(st + off_g, tg, 0, y, &b.full[s]);
+        tma_load_2d(st + off_g + kHalfBytes, tg, 64, y, &b.full[s]);
+        issued = c + 1;
+    }
+    if (*abort)
+        for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
+            wait_drain(&b.full[c % kStages], (c / kStages) & 1);
+}
+
+__device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
+                           int nchunks) {
+    constexpr uint32_t i_m = idesc_bf16_f32(64, 64, 0, 0);
+    constexpr uint32_t i_ds = idesc_bf16_f32(128, 128, 1, 1);
+    constexpr uint32_t i_dqb = idesc_bf16_f32(128, 64, 1, 0);
+    constexpr uint32_t i_dqa = idesc_bf16_f32(128, 64, 0, 0);
+    const uint32_t m_addr = smem_u32(smem + off_m);
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % kStages;
+        if (!mbar_wait(&b.gated[s], (c / kStages) & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * kStageBytes);
+        const uint32_t ka = st + off_k, va = st + off_v, da = st + off_do;
+        if (c > 0 && !mbar_wait(b.m_free, (c - 1) & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // M = dO V^T
+            mma_ss(tmem + kColM, desc_kmajor(da, kk), desc_kmajor(va, kk), i_m, kk > 0);
+        mma_commit(b.m_full);
+        if (c > 0 && !mbar_wait(b.ds_free, (c - 1) & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dS = Ktil^T V
+            mma_ss(tmem + kColDS, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), i_ds, kk > 0);
+        mma_commit(b.ds_full);
+        if (c > 0 && !mbar_wait(b.dq_free, (c - 1) & 1, abort)) break;
+        if (!mbar_wait(b.p_full, c & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dq^T = Ktil^T M^T
+            mma_ss(tmem + kColDQ, desc_mnmajor(ka, kk), smem_desc_sw128(m_addr + kk * 32, 16, 1024),
+                   i_dqb, kk > 0);
+        if (!mbar_wait(b.sa_full, c & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dq^T += S' dO^T, A from tensor memory
+            mma_ts(tmem + kColDQ, tmem + kColSA + kk * 8, desc_kmajor(da, kk), i_dqa, 1u);
+        mma_commit(b.dq_full);
+        mma_commit(b.sa_free);
+        mma_commit(&b.empty[s]);
+    }
+    mma_commit(b.fin);
+    wait_drain(b.fin, 0);
+}
+
+// Gate warps: cumsum as in the forward pass, Ktil in place of k, e^{b_t - b_C} in place of
+// log_g, e^{b_C} per key dim for the state decay.
+__device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
+                          int nchunks) {
+    const int gw = (threadIdx.x >> 5) - kEpiWarps;
+    const int lane = threadIdx.x & 31;
+    const int tg = lane >> 2, ig = lane & 3;
+    const int i0 = gw * 32 + ig * 8;
+    float *ec = reinterpret_cast<float *>(smem + off_ec);
+    bool range_bad = false;
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % kStages;
+        if (!mbar_wait(&b.full[s], (c / kStages) & 1, abort)) break;
+        uint8_t *st = smem + s * kStageBytes;
+        float bt[8][8];
+        {
+            uint4 graw[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+                graw[r] = *reinterpret_cast<const uint4 *>(st + off_g + tile_off(tg * 8 + r, i0));
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                float f[8];
+                unpack8(graw[r], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) bt[r][e] = (r ? bt[r - 1][e] : 0.f) + f[e];
+            }
+        }
+        float incl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) incl[e] = bt[7][e];
+#pragma unroll
+        for (int d = 1; d < 8; d <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float up = __shfl_up_sync(0xFFFFFFFFu, incl[e], 4 * d);
+                if (tg >= d) incl[e] += up;
+            }
+        }
+        float nbCl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float bC = __shfl_sync(0xFFFFFFFFu, incl[e], 28 + ig);
+            const float off = incl[e] - bt[7][e];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) bt[r][e] += off;
+            nbCl[e] = -bC * kLog2e;
+            range_bad |= !(fabsf(bC) <= kGateRangeLimit);
+        }
+        if (tg == 0) {
+            float4 *e4 = reinterpret_cast<float4 *>(ec + s * D + i0);
+            e4[0] = make_float4(ex2_approx(-nbCl[0]), ex2_approx(-nbCl[1]), ex2_approx(-nbCl[2]),
+                                ex2_approx(-nbCl[3]));
+            e4[1] = make_float4(ex2_approx(-nbCl[4]), ex2_approx(-nbCl[5]), ex2_approx(-nbCl[6]),
+                                ex2_approx(-nbCl[7]));
+        }
+#pragma unroll
+        for (int r0 = 0; r0 < 8; r0 += 4) {
+            uint4 kr[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                kr[r] = *reinterpret_cast<const uint4 *>(st + off_k + tile_off(tg * 8 + r0 + r, i0));
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+                float x[8], f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = fmaf(bt[r0 + r][e], kLog2e, nbCl[e]);
+                unpack8(kr[r], f);
+                uint32_t wk[4], wf[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    wk[e] = pack_bf16(f[2 * e] * ex2_approx(-x[2 * e]), f[2 * e + 1] * ex2_approx(-x[2 * e + 1]));
+                    wf[e] = pack_bf16(ex2_approx(x[2 * e]), ex2_approx(x[2 * e + 1]));
+                }
+                *reinterpret_cast<uint4 *>(st + off_k + off) = make_uint4(wk[0], wk[1], wk[2], wk[3]);
+                *reinterpret_cast<uint4 *>(st + off_g + off) = make_uint4(wf[0], wf[1], wf[2], wf[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.gated[s]);
+    }
+    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
+}
+
+// Epilogue warps: thread (w, lane) owns key dim i = 32 (w % 4) + lane (its TMEM lane) and the
+// half h = w / 4 of the state row (value dims 64h .. 64h+63) and of each chunk's 64 tokens.
+__device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
+                              uint32_t tmem, int bh, int j, long long row0, int nchunks) {
+    constexpr int HD = D / 2;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3, h = warp >> 2;
+    const int i = quarter * 32 + lane;
+    const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+    const float *ec = reinterpret_cast<const float *>(smem + off_ec);
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
+    __nv_bfloat16 *dq = static_cast<__nv_bfloat16 *>(a.dq_out);
+
+    float S[HD];  // S[i][64h + e]
+    if (a.S_recv) {
+        const float4 *Si = reinterpret_cast<const float4 *>(
+            a.S_recv + ((long long)bh * a.NP + j) * D * D + (long long)i * D + h * HD);
+#pragma unroll
+        for (int e4 = 0; e4 < HD / 4; ++e4) {
+            const float4 v = Si[e4];
+            S[4 * e4] = v.x; S[4 * e4 + 1] = v.y; S[4 * e4 + 2] = v.z; S[4 * e4 + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < HD; ++e) S[e] = 0.f;
+    }
+    const int cpf = nchunks / a.fine;  // chunks per fine part
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % kStages;
+        uint8_t *st = smem + s * kStageBytes;
+        uint32_t r[32];
+        if (a.S_fine && c % cpf == 0) {  // the state entering fine part c / cpf
+            float4 *Sf = reinterpret_cast<float4 *>(
+                a.S_fine + (((long long)bh * a.NP + j) * a.fine + c / cpf) * D * D + (long long)i * D + h * HD);
+#pragma unroll
+            for (int e4 = 0; e4 < HD / 4; ++e4)
+                Sf[e4] = make_float4(S[4 * e4], S[4 * e4 + 1], S[4 * e4 + 2], S[4 * e4 + 3]);
+        }
+        {  // (a) M -> causal mask -> bf16 tile (K-major rows t)
+            if (!mbar_wait(b.m_full, c & 1, abort)) break;
+            tc_fence_after();
+            tmem_ld32(tmem + lrow + kColM + h * 32, r);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.m_free);
+            if (lane < 16) {
+                const int t = quarter * 16 + lane;
+                uint8_t *mrow = smem + off_m + t * 128;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int sl = jj * 8 + 2 * e, s0 = h * 32 + sl;
+                        w4[e] = pack_bf16(s0 <= t ? __uint_as_float(r[sl]) : 0.f,
+                                          s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f);
+                    }
+                    *reinterpret_cast<uint4 *>(mrow + (((h * 4 + jj) ^ (t & 7)) << 4)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.p_full);
+        }
+        // (b) S' = diag(e^{b_C}) S; bf16 copy into tensor memory (A of dq^T += S' dO^T)
+        if (!mbar_wait(&b.gated[s], (c / kStages) & 1, abort)) break;
+        const float e_i = ec[s * D + i];
+#pragma unroll
+        for (int e = 0; e < HD; ++e) S[e] *= e_i;
+        if (c > 0 && !mbar_wait(b.sa_free, (c - 1) & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = pack_bf16(S[2 * e], S[2 * e + 1]);
+        tmem_st32(tmem + lrow + kColSA + h * 32, r);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.sa_full);
+        // (c) S = S' + dS
+        if (!mbar_wait(b.ds_full, c & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) S[p * 32 + e] += __uint_as_float(r[e]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.ds_free);
+        // (d) dq rows t = 32h .. 32h+31, column i; q . dq for the reverse sweep
+        if (!mbar_wait(b.dq_full, c & 1, abort)) break;
+        tc_fence_after();
+        tmem_ld32(tmem + lrow + kColDQ + h * 32, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.dq_free);
+        const long long t0 = row0 + (long long)c * CH + h * 32;
+        const __nv_bfloat16 *fcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_g);
+#pragma unroll
+        for (int t8 = 0; t8 < 32; t8 += 8) {
+            float qv[8];  // a batch's loads before its stores: none waits behind a possible alias
+#pragma unroll
+            for (int t = 0; t < 8; ++t) qv[t] = __bfloat162float(q[(t0 + t8 + t) * D + i]);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const float f = __bfloat162float(fcol[tile_off(h * 32 + t8 + t, i) >> 1]);
+                const float v = __uint_as_float(r[t8 + t]) * f;
+                const long long idx = (t0 + t8 + t) * D + i;
+                dq[idx] = __float2bfloat16_rn(v);
+                a.dq_ws[idx] = qv[t] * v;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.empty[s]);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+             const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_g,
+             const BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + off_bar);
+    Bars b;
+    b.full = bar;
+    b.gated = bar + kStages;
+    b.empty = bar + 2 * kStages;
+    uint64_t *x = bar + 3 * kStages;
+    b.m_full = x + 0; b.m_free = x + 1; b.p_full = x + 2; b.ds_full = x + 3; b.ds_free = x + 4;
+    b.sa_full = x + 5; b.sa_free = x + 6; b.dq_full = x + 7; b.dq_free = x + 8; b.fin = x + 9;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x / a.NP, j = blockIdx.x % a.NP;
+    const long long row0 = (long long)bh * a.L + (long long)j * a.T;
+    const int nchunks = (int)(a.T / CH);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&b.full[s], 1);
+            mbar_init(&b.gated[s], kGateWarps);
+            mbar_init(&b.empty[s], 1 + kEpiWarps);
+        }
+        mbar_init(b.m_full, 1);
+        mbar_init(b.m_free, kEpiWarps);
+        mbar_init(b.p_full, kEpiWarps);
+        mbar_init(b.ds_full, 1);
+        mbar_init(b.ds_free, kEpiWarps);
+        mbar_init(b.sa_full, kEpiWarps);
+        mbar_init(b.sa_free, 1);
+        mbar_init(b.dq_full, 1);
+        mbar_init(b.dq_free, kEpiWarps);
+        mbar_init(b.fin, 1);
+        *abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+        prefetch_tmap(&tm_g);
+    }
+    if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (warp == kTmaWarp) {
+        if (lane == 0) producer(smem, b, abort, &tm_k, &tm_v, &tm_do, &tm_g, row0, nchunks);
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) mma_issuer(smem, b, abort, tmem, nchunks);
+    } else if (warp >= kEpiWarps) {
+        gate_role(smem, b, abort, a, nchunks);
+    } else {
+        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort && a.status) atomicOr(a.status, kStatusTimeout);
+}
+
+}  // namespace dqs
+
+// ------------------------------------------------------------------ reverse sweep
+// Per chunk, last to first, with dS the gradient of the state at the chunk's end (rows = key
+// dims; starts at dX of the part), Qbar'_t = q_t e^{b_t - b_C}, Ktil_s = k_s e^{b_C - b_s}:
+//
+//   M     = dO V^T,  A = Qbar' Ktil^T   M=64 (t) N=64 (s) K=128          -> masked s <= t, bf16
+//   dk^T  = Qbar'^T M + dS V^T          M=128 (i) N=64 (s) K=64 (t) / 128 (j)
+//   dv    = A^T dO + Ktil dS            M=64 (s) N=128 (j) K=64 (t) / 128 (i)
+//   dS   += Qbar'^T dO                  M=128 (i) N=128 (j) K=64 (t), accumulated in TMEM
+//   dk[s,i] = e^{b_C,i - b_s,i} dk^T[i,s];   dS <- diag(e^{b_C}) dS
+//   dlog_g_s = rowsum(S_end . dX) + sum_{u >= s in the part} (q_u dq_u - k_u dk_u)
+//
+// The fp32 dS lives in tensor memory (the MMA accumulates Qbar'^T dO onto it; the epilogue
+// applies the decay); its bf16 copy lives in one shared tile ([i][j] rows, 128-byte swizzle)
+// read as the K-major A operand of dS V^T and as the MN-major B operand of Ktil dS.
+namespace dkv {
+
+constexpr uint32_t kColM = 0, kColA = 64, kColDK = 128, kColDV = 192, kColDS = 320;
+constexpr int kStages = 2;
+constexpr int off_q = 0, off_k = kTileBytes, off_v = 2 * kTileBytes, off_do = 3 * kTileBytes,
+              off_g = 4 * kTileBytes;
+constexpr int kStageBytes = 5 * kTileBytes;
+constexpr int kDsHalf = 128 * 128;  // one 64-column half of the [128 x 128] bf16 dS tile
+constexpr int off_m = kStages * kStageBytes;
+constexpr int off_a = off_m + CH * CH * 2;
+constexpr int off_ds = off_a + CH * CH * 2;
+constexpr int off_ec = off_ds + 2 * kDsHalf;
+constexpr int off_x = off_ec + kStages * D * 4;  // half-row exchange between the two epilogue halves
+constexpr int off_bar = off_x + 4 * D * 4;
+constexpr int kBars = 3 * kStages + 16;
+constexpr int off_misc = off_bar + kBars * 8;
+constexpr int kSmemBytes = off_misc + 16 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct Bars {
+    uint64_t *full, *gated, *empty;
+    uint64_t *mm_full, *mm_free, *aa_full, *aa_free, *p_full, *dst_full, *dk_full, *dk_free,
+        *dv_full, *dv_free, *dsn_full, *dsn_free, *xchg, *fin;
+};
+
+// [128 rows][128 cols] bf16 tile as two 64-column halves of 16 KiB, 128-byte swizzle.
+__device__ __forceinline__ uint32_t ds_off(int row, int col) {
+    const int half = col >> 6, cc = col & 63;
+    return (uint32_t)(half * kDsHalf + row * 128 + (((cc >> 3) ^ (row & 7)) << 4) + ((cc & 7) << 1));
+}
+
+__device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tq,
+                         const CUtensorMap *tk, const CUtensorMap *tv, const CUtensorMap *tdo,
+                         const CUtensorMap *tg, long long row0, int nchunks) {
+    int issued = 0;
+    for (int it = 0; it < nchunks; ++it) {
+        const int s = it % kStages;
+        const int c = nchunks - 1 - it;  // last chunk first
+        if (it >= kStages && !mbar_wait(&b.empty[s], ((it / kStages) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&b.full[s], kStageBytes);
+        uint8_t *st = smem + s * kStageBytes;
+        const int y = (int)(row0 + (long long)c * CH);
+        tma_load_2d(st + off_q, tq, 0, y, &b.full[s]);
+        tma_load_2d(st + off_q + kHalfBytes, tq, 64, y, &b.full[s]);
+        tma_load_2d(st + off_k, tk, 0, y, &b.full[s]);
+        tma_load_2d(st + off_k + kHalfBytes, tk, 64, y, &b.full[s]);
+        tma_load_2d(st + off_v, tv, 0, y, &b.full[s]);
+        tma_load_2d(st + off_v + kHalfBytes, tv, 64, y, &b.full[s]);
+        tma_load_2d(st + off_do, tdo, 0, y, &b.full[s]);
+        tma_load_2d(st + off_do + kHalfBytes, tdo, 64, y, &b.full[s]);
+        tma_load_2d(st + off_g, tg, 0, y, &b.full[s]);
+        tma_load_2d(st + off_g + kHalfBytes, tg, 64, y, &b.full[s]);
+        issued = it + 1;
+    }
+    if (*abort)
+        for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it)
+            wait_drain(&b.full[it % kStages], (it / kStages) & 1);
+}
+
+__device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
+                           int nchunks) {
+    constexpr uint32_t i_sq = idesc_bf16_f32(64, 64, 0, 0);      // M, A
+    constexpr uint32_t i_dsn = idesc_bf16_f32(128, 128, 1, 1);   // Qbar'^T dO
+    constexpr uint32_t i_dka = idesc_bf16_f32(128, 64, 1, 1);    // Qbar'^T M
+    constexpr uint32_t i_dkb = idesc_bf16_f32(128, 64, 0, 0);    // dS V^T
+    constexpr uint32_t i_dva = idesc_bf16_f32(64, 128, 1, 1);    // A^T dO
+    constexpr uint32_t i_dvb = idesc_bf16_f32(64, 128, 0, 1);    // Ktil dS
+    const uint32_t m_addr = smem_u32(smem + off_m), a_addr = smem_u32(smem + off_a);
+    const uint32_t ds_addr = smem_u32(smem + off_ds);
+    for (int it = 0; it < nchunks; ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(&b.gated[s], (it / kStages) & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * kStageBytes);
+        const uint32_t qa = st + off_q, ka = st + off_k, va = st + off_v, da = st + off_do;
+        const uint32_t pf = (it - 1) & 1;  // phase of the previous chunk's "free" barriers
+        if (it > 0 && !mbar_wait(b.mm_free, pf, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // M = dO V^T
+            mma_ss(tmem + kColM, desc_kmajor(da, kk), desc_kmajor(va, kk), i_sq, kk > 0);
+        mma_commit(b.mm_full);
+        if (it > 0 && !mbar_wait(b.aa_free, pf, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // A = Qbar' Ktil^T
+            mma_ss(tmem + kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), i_sq, kk > 0);
+        mma_commit(b.aa_full);
+        if (!mbar_wait(b.p_full, it & 1, abort)) break;
+        if (!mbar_wait(b.dst_full, it & 1, abort)) break;
+        if (it > 0 && !mbar_wait(b.dk_free, pf, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dk^T = Qbar'^T M   (B: M tile read MN-major)
+            mma_ss(tmem + kColDK, desc_mnmajor(qa, kk), smem_desc_sw128(m_addr + kk * 2048, kHalfBytes, 1024),
+                   i_dka, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dk^T += dS V^T   (A: dS tile K-major, 128 rows)
+            mma_ss(tmem + kColDK,
+                   smem_desc_sw128(ds_addr + (kk >> 2) * kDsHalf + (kk & 3) * 32, 16, 1024),
+                   desc_kmajor(va, kk), i_dkb, 1u);
+        mma_commit(b.dk_full);
+        if (it > 0 && !mbar_wait(b.dv_free, pf, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dv = A^T dO   (A: A tile read MN-major)
+            mma_ss(tmem + kColDV, smem_desc_sw128(a_addr + kk * 2048, kHalfBytes, 1024),
+                   desc_mnmajor(da, kk), i_dva, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dv += Ktil dS   (B: dS tile MN-major)
+            mma_ss(tmem + kColDV, desc_kmajor(ka, kk),
+                   smem_desc_sw128(ds_addr + kk * 2048, kDsHalf, 1024), i_dvb, 1u);
+        mma_commit(b.dv_full);
+        if (it > 0 && !mbar_wait(b.dsn_free, pf, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dS += Qbar'^T dO  (after dk and dv read the old dS)
+            mma_ss(tmem + kColDS, desc_mnmajor(qa, kk), desc_mnmajor(da, kk), i_dsn, 1u);
+        mma_commit(b.dsn_full);
+        mma_commit(&b.empty[s]);
+    }
+    mma_commit(b.fin);
+    wait_drain(b.fin, 0);
+}
+
+// Gate warps: Qbar' and Ktil in place of q and k, e^{b_C - b_t} in place of log_g (the dk
+// output factor), e^{b_C} per key dim.
+__device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
+                          int nchunks) {
+    const int gw = (threadIdx.x >> 5) - kEpiWarps;
+    const int lane = threadIdx.x & 31;
+    const int tg = lane >> 2, ig = lane & 3;
+    const int i0 = gw * 32 + ig * 8;
+    float *ec = reinterpret_cast<float *>(smem + off_ec);
+    bool range_bad = false;
+    for (int it = 0; it < nchunks; ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(&b.full[s], (it / kStages) & 1, abort)) break;
+        uint8_t *st = smem + s * kStageBytes;
+        float bt[8][8];
+        {
+            uint4 graw[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+                graw[r] = *reinterpret_cast<const uint4 *>(st + off_g + tile_off(tg * 8 + r, i0));
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                float f[8];
+                unpack8(graw[r], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) bt[r][e] = (r ? bt[r - 1][e] : 0.f) + f[e];
+            }
+        }
+        float incl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) incl[e] = bt[7][e];
+#pragma unroll
+        for (int d = 1; d < 8; d <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float up = __shfl_up_sync(0xFFFFFFFFu, incl[e], 4 * d);
+                if (tg >= d) incl[e] += up;
+            }
+        }
+        float nbCl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float bC = __shfl_sync(0xFFFFFFFFu, incl[e], 28 + ig);
+            const float off = incl[e] - bt[7][e];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) bt[r][e] += off;
+            nbCl[e] = -bC * kLog2e;
+            range_bad |= !(fabsf(bC) <= kGateRangeLimit);
+        }
+        if (tg == 0) {
+            float4 *e4 = reinterpret_cast<float4 *>(ec + s * D + i0);
+            e4[0] = make_float4(ex2_approx(-nbCl[0]), ex2_approx(-nbCl[1]), ex2_approx(-nbCl[2]),
+                                ex2_approx(-nbCl[3]));
+            e4[1] = make_float4(ex2_approx(-nbCl[4]), ex2_approx(-nbCl[5]), ex2_approx(-nbCl[6]),
+                                ex2_approx(-nbCl[7]));
+        }
+#pragma unroll
+        for (int r0 = 0; r0 < 8; r0 += 2) {
+            uint4 qr[2], kr[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+                qr[r] = *reinterpret_cast<const uint4 *>(st + off_q + off);
+                kr[r] = *reinterpret_cast<const uint4 *>(st + off_k + off);
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+                float x[8], fq[8], fk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = fmaf(bt[r0 + r][e], kLog2e, nbCl[e]);
+                unpack8(qr[r], fq);
+                unpack8(kr[r], fk);
+                uint32_t wq[4], wk[4], wf[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float u0 = ex2_approx(x[2 * e]), u1 = ex2_approx(x[2 * e + 1]);
+                    const float d0 = ex2_approx(-x[2 * e]), d1 = ex2_approx(-x[2 * e + 1]);
+                    wq[e] = pack_bf16(fq[2 * e] * u0, fq[2 * e + 1] * u1);
+                    wk[e] = pack_bf16(fk[2 * e] * d0, fk[2 * e + 1] * d1);
+                    wf[e] = pack_bf16(d0, d1);
+                }
+                *reinterpret_cast<uint4 *>(st + off_q + off) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                *reinterpret_cast<uint4 *>(st + off_k + off) = make_uint4(wk[0], wk[1], wk[2], wk[3]);
+                *reinterpret_cast<uint4 *>(st + off_g + off) = make_uint4(wf[0], wf[1], wf[2], wf[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.gated[s]);
+    }
+    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
+}
+
+// Writes a masked (s <= t) bf16 copy of a M=64 TMEM accumulator half into a 64x64 tile.
+__device__ __forceinline__ void masked_tile(uint8_t *tile, const uint32_t (&r)[32], int quarter,
+                                            int h, int lane) {
+    if (lane < 16) {
+        const int t = quarter * 16 + lane;
+        uint8_t *row = tile + t * 128;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int sl = jj * 8 + 2 * e, s0 = h * 32 + sl;
+                w4[e] = pack_bf16(s0 <= t ? __uint_as_float(r[sl]) : 0.f,
+                                  s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f);
+            }
+            *reinterpret_cast<uint4 *>(row + (((h * 4 + jj) ^ (t & 7)) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+    }
+}
+
+// Exchange point of the 8 epilogue warps (bounded like every other wait): returns false when
+// the CTA is aborting.
+__device__ __forceinline__ bool epi_exchange(const Bars &b, volatile int *abort, int k, int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b.xchg);
+    return mbar_wait(b.xchg, k & 1, abort);
+}
+
+// Epilogue warps: thread (w, lane) owns key dim i = 32 (w % 4) + lane and value dims
+// 64h .. 64h+63 (h = w / 4) of the running state gradient dS, and tokens 32h .. 32h+31 of
+// each chunk for dk and dlog_g; for dv (M=64 accumulator) lanes 0-15 own token 16 (w % 4) + lane.
+__device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
+                              uint32_t tmem, int bh, int j, long long row0, int nchunks) {
+    constexpr int HD = D / 2;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3, h = warp >> 2;
+    const int i = quarter * 32 + lane;
+    const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+    const float *ec = reinterpret_cast<const float *>(smem + off_ec);
+    float *xb = reinterpret_cast<float *>(smem + off_x);  // [2 sets][2 halves][128]
+    const __nv_bfloat16 *kin = static_cast<const __nv_bfloat16 *>(a.k);
+    __nv_bfloat16 *dk = static_cast<__nv_bfloat16 *>(a.dk_out);
+    __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv_out);
+    __nv_bfloat16 *dg = static_cast<__nv_bfloat16 *>(a.dg_out);
+    const long long sidx = ((long long)bh * a.NP + j) * D * D;
+
+    // dS (gradient of the state at the current chunk's end) lives in TMEM: row i, columns
+    // 64h .. 64h+63 of this thread.  Start: dX of the part; carry: rowsum(S_end . dX).
+    float carry;
+    {
+        const float *Se = nullptr;
+        if (j < a.NP - 1) {
+            if (a.S_end_next) Se = a.S_end_next + sidx + (long long)D * D;
+        } else if (a.S_fin) {
+            Se = a.S_fin + (long long)bh * D * D;
+        }
+        float part = 0.f;
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            uint32_t w[32];
+            const float4 *x4 = reinterpret_cast<const float4 *>(a.dX + sidx + (long long)i * D + h * HD + p * 32);
+            const float4 *s4 = Se ? reinterpret_cast<const float4 *>(Se + (long long)i * D + h * HD + p * 32) : nullptr;
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 v = x4[e4];
+                w[4 * e4] = __float_as_uint(v.x); w[4 * e4 + 1] = __float_as_uint(v.y);
+                w[4 * e4 + 2] = __float_as_uint(v.z); w[4 * e4 + 3] = __float_as_uint(v.w);
+                if (s4) {
+                    const float4 u = s4[e4];
+                    part += u.x * v.x + u.y * v.y + u.z * v.z + u.w * v.w;
+                }
+            }
+            tmem_st32(tmem + lrow + kColDS + h * HD + p * 32, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        xb[h * D + i] = part;
+        carry = epi_exchange(b, abort, 0, lane) ? xb[i] + xb[D + i] : 0.f;
+    }
+    for (int it = 0; it < nchunks; ++it) {
+        const int s = it % kStages;
+        const int c = nchunks - 1 - it;
+        uint8_t *st = smem + s * kStageBytes;
+        uint32_t r[32];
+        // (a) masked M and A tiles
+        if (!mbar_wait(b.mm_full, it & 1, abort)) break;
+        tc_fence_after();
+        tmem_ld32(tmem + lrow + kColM + h * 32, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.mm_free);
+        masked_tile(smem + off_m, r, quarter, h, lane);
+        if (!mbar_wait(b.aa_full, it & 1, abort)) break;
+        tc_fence_after();
+        tmem_ld32(tmem + lrow + kColA + h * 32, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.aa_free);
+        masked_tile(smem + off_a, r, quarter, h, lane);
+        // (b) bf16 dS into the shared tile (row i, columns 64h .. 64h+63)
+        tc_fence_after();
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint32_t *x = r + jj * 8;
+                *reinterpret_cast<uint4 *>(smem + off_ds + ds_off(i, h * HD + p * 32 + jj * 8)) =
+                    make_uint4(pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                               pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
+                               pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
+                               pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
+            }
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(b.p_full);
+            mbar_arrive(b.dst_full);
+        }
+        // (c) dk for tokens 32h .. 32h+31 of the chunk; dlog_g suffix sums
+        if (!mbar_wait(b.dk_full, it & 1, abort)) break;
+        tc_fence_after();
+        tmem_ld32(tmem + lrow + kColDK + h * 32, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.dk_free);
+        const long long t0 = row0 + (long long)c * CH + h * 32;
+        const __nv_bfloat16 *fcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_g);
+        float tot = 0.f;
+#pragma unroll
+        for (int t8 = 0; t8 < 32; t8 += 8) {
+            float qdq[8], kr[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const long long idx = (t0 + t8 + t) * D + i;
+                qdq[t] = a.dq_ws[idx];
+                kr[t] = __bfloat162float(kin[idx]);
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const float f = __bfloat162float(fcol[tile_off(h * 32 + t8 + t, i) >> 1]);
+                const float dkv = __uint_as_float(r[t8 + t]) * f;
+                dk[(t0 + t8 + t) * D + i] = __float2bfloat16_rn(dkv);
+                const float cg = qdq[t] - kr[t] * dkv;
+                r[t8 + t] = __float_as_uint(cg);  // contribution, kept for the suffix sums
+                tot += cg;
+            }
+        }
+        float *xs = xb + ((it + 1) & 1) * 2 * D;
+        xs[h * D + i] = tot;
+        if (!epi_exchange(b, abort, it + 1, lane)) break;
+        const float later = h == 0 ? xs[D + i] : 0.f;  // the second half's tokens come later
+        float acc = carry + later;
+#pragma unroll
+        for (int t = 31; t >= 0; --t) {
+            acc += __uint_as_float(r[t]);
+            dg[(t0 + t) * D + i] = __float2bfloat16_rn(acc);
+        }
+        carry += xs[i] + xs[D + i];
+        // (d) dv rows 16q + lane (lanes 0-15), value dims 64h .. 64h+63
+        if (!mbar_wait(b.dv_full, it & 1, abort)) break;
+        tc_fence_after();
+        {
+            uint4 *drow = reinterpret_cast<uint4 *>(
+                dv + (row0 + (long long)c * CH + quarter * 16 + lane) * D + h * HD);
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                tmem_ld32(tmem + lrow + kColDV + h * HD + p * 32, r);
+                tmem_wait_ld();
+                if (lane < 16) {
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        const uint32_t *src = r + q8 * 8;
+                        drow[p * 4 + q8] =
+                            make_uint4(pack_bf16(__uint_as_float(src[0]), __uint_as_float(src[1])),
+                                       pack_bf16(__uint_as_float(src[2]), __uint_as_float(src[3])),
+                                       pack_bf16(__uint_as_float(src[4]), __uint_as_float(src[5])),
+                                       pack_bf16(__uint_as_float(src[6]), __uint_as_float(src[7])));
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.dv_free);
+        // (e) dS <- diag(e^{b_C}) (dS + Qbar'^T dO), the sum already formed by the MMA
+        if (!mbar_wait(b.dsn_full, it & 1, abort)) break;
+        tc_fence_after();
+        const float e_i = ec[s * D + i];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(e_i * __uint_as_float(r[e]));
+            tmem_st32(tmem + lrow + kColDS + h * HD + p * 32, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(b.dsn_free);
+            mbar_arrive(&b.empty[s]);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const __grid_constant__ CUtensorMap tm_g, const BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + off_bar);
+    Bars b;
+    b.full = bar;
+    b.gated = bar + kStages;
+    b.empty = bar + 2 * kStages;
+    uint64_t *x = bar + 3 * kStages;
+    b.mm_full = x + 0; b.mm_free = x + 1; b.aa_full = x + 2; b.aa_free = x + 3; b.p_full = x + 4;
+    b.dst_full = x + 5; b.dk_full = x + 6; b.dk_free = x + 7; b.dv_full = x + 8; b.dv_free = x + 9;
+    b.dsn_full = x + 10; b.dsn_free = x + 11; b.xchg = x + 12; b.fin = x + 13;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x / a.NP, j = blockIdx.x % a.NP;
+    const long long row0 = (long long)bh * a.L + (long long)j * a.T;
+    const int nchunks = (int)(a.T / CH);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&b.full[s], 1);
+            mbar_init(&b.gated[s], kGateWarps);
+            mbar_init(&b.empty[s], 1 + kEpiWarps);
+        }
+        uint64_t *one[] = {b.mm_full, b.aa_full, b.dk_full, b.dv_full, b.dsn_full, b.fin};
+        uint64_t *epi[] = {b.mm_free, b.aa_free, b.p_full, b.dst_full, b.dk_free, b.dv_free,
+                           b.dsn_free, b.xchg};
+        for (uint64_t *p : one) mbar_init(p, 1);
+        for (uint64_t *p : epi) mbar_init(p, kEpiWarps);
+        *abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+        prefetch_tmap(&tm_g);
+    }
+    if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (warp == kTmaWarp) {
+        if (lane == 0) producer(smem, b, abort, &tm_q, &tm_k, &tm_v, &tm_do, &tm_g, row0, nchunks);
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) mma_issuer(smem, b, abort, tmem, nchunks);
+    } else if (warp >= kEpiWarps) {
+        gate_role(smem, b, abort, a, nchunks);
+    } else {
+        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort && a.status) atomicOr(a.status, kStatusTimeout);
+}
+
+}  // namespace dkv
+
+}  // namespace
+
+bool tc_bwd_supported(const BwdArgs &a) {
+    return a.dt == LA_BF16 && a.dk == D && a.dv == D && a.chunk == CH && a.T % CH == 0 &&
+           (long long)a.BH * a.L <= 0x7FFFFFFFLL;
+}
+
+cudaError_t launch_tc_dq(const BwdArgs &a, cudaStream_t st) {
+    const long long rows = (long long)a.BH * a.L;
+    CUtensorMap mk, mv, mdo, mg;
+    cudaError_t e;
+    if ((e = make_map(&mk, a.k, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mdo, a.dO, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(dqs::tc_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dqs::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const long long nblk = (long long)a.BH * a.NP;
+    if (nblk == 0) return cudaSuccess;
+    dqs::tc_dq_kernel<<<(unsigned)nblk, kThreads, dqs::kSmemBytes, st>>>(mk, mv, mdo, mg, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tc_dkv(const BwdArgs &a, cudaStream_t st) {
+    const long long rows = (long long)a.BH * a.L;
+    CUtensorMap mq, mk, mv, mdo, mg;
+    cudaError_t e;
+    if ((e = make_map(&mq, a.q, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mk, a.k, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mdo, a.dO, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(dkv::tc_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dkv::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const long long nblk = (long long)a.BH * a.NP;
+    if (nblk == 0) return cudaSuccess;
+    dkv::tc_dkv_kernel<<<(unsigned)nblk, kThreads, dkv::kSmemBytes, st>>>(mq, mk, mv, mdo, mg, a);
+    return cudaGetLastError();
+}
+
+}  // namespace la

@@ -30,41 +30,34 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "tc_common.cuh"
 
 namespace la {
 namespace {
 
 using namespace sm100;
+using namespace tc;
 
-constexpr int D = 128;                 // d_k = d_v
-constexpr int CH = 64;                 // tokens per chunk
-constexpr int kHalfBytes = CH * 64 * 2;  // one 64-column swizzle half of a tile: 8 KB
-constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr int kEpiWarps = 8, kGateWarps = 4;
 constexpr int kTmaWarp = 12, kMmaWarp = 13;
 constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
-constexpr float kLog2e = 1.4426950408889634f;
-
-// Tensor-memory columns (fp32 accumulators; SA holds bf16 pairs).
-constexpr uint32_t kColDS = 0;    // dS^T         128 lanes x 128 cols
-constexpr uint32_t kColO = 128;   // O^T          128 lanes x 64 cols
-constexpr uint32_t kColSA = 192;  // bf16 S'^T    128 lanes x 64 cols (128 values)
-constexpr uint32_t kColQK = 256;  // Qbar' Ktil^T M=64 layout, 64 cols
-constexpr uint32_t kTmemCols = 512;
 
 template <int MODE>
 struct Cfg {
+    static constexpr bool dstate = MODE == kPassDState;  // v tile holds dO, q tile becomes Qhat
     static constexpr bool q = MODE != kPassState;
-    static constexpr bool kv = MODE != kPassCorrect;
+    static constexpr bool k = MODE != kPassCorrect && !dstate;
+    static constexpr bool v = MODE != kPassCorrect;
+    static constexpr bool kv = k;  // chunk-state increment from Ktil and V
     static constexpr bool qk = MODE == kPassOutput || MODE == kPassLocal;
-    static constexpr bool out = MODE != kPassState;
-    static constexpr bool write_state = MODE == kPassState || MODE == kPassLocal;
+    static constexpr bool out = MODE != kPassState && !dstate;
+    static constexpr bool write_state = MODE == kPassState || MODE == kPassLocal || dstate;
     static constexpr bool init_state = MODE == kPassOutput || MODE == kPassCorrect;
     static constexpr int stages = (MODE == kPassOutput || MODE == kPassLocal) ? 3 : 4;
     static constexpr int off_q = 0;
     static constexpr int off_k = off_q + (q ? kTileBytes : 0);
-    static constexpr int off_v = off_k + (kv ? kTileBytes : 0);
-    static constexpr int off_g = off_v + (kv ? kTileBytes : 0);
+    static constexpr int off_v = off_k + (k ? kTileBytes : 0);
+    static constexpr int off_g = off_v + (v ? kTileBytes : 0);
     static constexpr int stage_bytes = off_g + kTileBytes;
     static constexpr int off_p = stages * stage_bytes;
     static constexpr int off_ec = off_p + (qk ? CH * CH * 2 : 0);
@@ -80,27 +73,6 @@ struct Bars {
     uint64_t *qk_full, *qk_free, *p_full, *ds_full, *ds_free, *sa_full, *sa_free, *o_full,
         *o_free, *fin;
 };
-
-// Byte offset of element (t, i) of a [64 x 128] bf16 tile TMA-loaded as two 64-column halves
-// with the 128-byte swizzle (16-byte chunk index XOR row % 8).
-__device__ __forceinline__ uint32_t tile_off(int t, int i) {
-    const int half = i >> 6, ii = i & 63;
-    return (uint32_t)(half * kHalfBytes + t * 128 + (((ii >> 3) ^ (t & 7)) << 4) + ((ii & 7) << 1));
-}
-
-// Descriptor of a K-major operand (rows x 128 K-elements, two swizzle halves) at K-step kk.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk) {
-    return smem_desc_sw128(base + (uint32_t)((kk >> 2) * kHalfBytes + (kk & 3) * 32), 16, 1024);
-}
-// Descriptor of an MN-major operand ([64 K-rows] x 128 MN-elements, two halves) at K-step kk.
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int kk) {
-    return smem_desc_sw128(base + (uint32_t)(kk * 2048), kHalfBytes, 1024);
-}
-
-__device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity) {
-    int dummy = 0;
-    return mbar_wait(bar, parity, &dummy);
-}
 
 // ------------------------------------------------------------------ TMA producer (1 thread)
 template <int MODE>
@@ -119,9 +91,11 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
             tma_load_2d(st + C::off_q, tq, 0, y, &b.full[s]);
             tma_load_2d(st + C::off_q + kHalfBytes, tq, 64, y, &b.full[s]);
         }
-        if (C::kv) {
+        if (C::k) {
             tma_load_2d(st + C::off_k, tk, 0, y, &b.full[s]);
             tma_load_2d(st + C::off_k + kHalfBytes, tk, 64, y, &b.full[s]);
+        }
+        if (C::v) {
             tma_load_2d(st + C::off_v, tv, 0, y, &b.full[s]);
             tma_load_2d(st + C::off_v + kHalfBytes, tv, 64, y, &b.full[s]);
         }
@@ -159,6 +133,12 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
                 mma_ss(tmem + kColQK, desc_kmajor(qa, kk), desc_kmajor(ka, kk), i_qk, kk > 0);
             mma_commit(b.qk_full);
         }
+        if (C::dstate) {  // R^T += dO^T Qhat, accumulated over the whole segment
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(qa, kk), i_ds,
+                       (c > 0 || kk > 0) ? 1u : 0u);
+        }
         if (C::kv) {  // chunk state increment dS^T = V^T Ktil
             if (c > 0 && !mbar_wait(b.ds_free, (c - 1) & 1, abort)) break;
             tc_fence_after();
@@ -188,6 +168,7 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
         }
         mma_commit(&b.empty[s]);
     }
+    if (C::dstate) mma_commit(b.ds_full);
     mma_commit(b.fin);  // nothing of this CTA may still run on the tensor cores at dealloc
     wait_drain(b.fin, 0);
 }
@@ -198,26 +179,6 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
 // swizzled 16-byte chunk.  The in-chunk cumsum of log_g runs down each thread's 8 rows, then
 // a 3-step shuffle scan across the 8 token groups adds the earlier groups' totals; the last
 // group's inclusive value is b_C.  Then q and k are rescaled in place in batches of 4 rows.
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        f[2 * e] = __uint_as_float(w[e] << 16);
-        f[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-    }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
 template <int MODE>
 __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
                           int bh, int j, int nchunks) {
@@ -227,7 +188,7 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
     const int tg = lane >> 2, ig = lane & 3;
     const int i0 = gw * 32 + ig * 8;  // first key dim of this thread's chunk
     float *ec = reinterpret_cast<float *>(smem + C::off_ec);
-    float logG[8];
+    float logG[8];  // running sum of the chunk totals: log-decay from the segment start
 #pragma unroll
     for (int e = 0; e < 8; ++e) logG[e] = 0.f;
     bool range_bad = false;
@@ -269,18 +230,19 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
             const float off = incl[e] - bt[7][e];  // exclusive prefix of this token group
 #pragma unroll
             for (int r = 0; r < 8; ++r) bt[r][e] += off;
-            nbCl[e] = -bC[e] * kLog2e;
+            // exponent offset of q's factor: e^{b_t - b_C}, or e^{B_start + b_t} for Qhat
+            nbCl[e] = (C::dstate ? logG[e] : -bC[e]) * kLog2e;
             range_bad |= !(fabsf(bC[e]) <= kGateRangeLimit);
         }
         if (tg == 0) {
             float4 *e4 = reinterpret_cast<float4 *>(ec + s * D + i0);
-            e4[0] = make_float4(ex2_approx(-nbCl[0]), ex2_approx(-nbCl[1]), ex2_approx(-nbCl[2]),
-                                ex2_approx(-nbCl[3]));
-            e4[1] = make_float4(ex2_approx(-nbCl[4]), ex2_approx(-nbCl[5]), ex2_approx(-nbCl[6]),
-                                ex2_approx(-nbCl[7]));
-#pragma unroll
-            for (int e = 0; e < 8; ++e) logG[e] += bC[e];
+            e4[0] = make_float4(ex2_approx(bC[0] * kLog2e), ex2_approx(bC[1] * kLog2e),
+                                ex2_approx(bC[2] * kLog2e), ex2_approx(bC[3] * kLog2e));
+            e4[1] = make_float4(ex2_approx(bC[4] * kLog2e), ex2_approx(bC[5] * kLog2e),
+                                ex2_approx(bC[6] * kLog2e), ex2_approx(bC[7] * kLog2e));
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) logG[e] += bC[e];
         // rescale q (by e^{b_t - b_C}) and k (by e^{b_C - b_t}) in place, 4 rows per batch
 #pragma unroll
         for (int r0 = 0; r0 < 8; r0 += 4) {
@@ -289,7 +251,7 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
             for (int r = 0; r < 4; ++r) {
                 const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
                 if (C::q) qr[r] = *reinterpret_cast<const uint4 *>(st + C::off_q + off);
-                if (C::kv) kr[r] = *reinterpret_cast<const uint4 *>(st + C::off_k + off);
+                if (C::k) kr[r] = *reinterpret_cast<const uint4 *>(st + C::off_k + off);
             }
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
@@ -307,7 +269,7 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
                                          f[2 * e + 1] * ex2_approx(x[2 * e + 1]));
                     *reinterpret_cast<uint4 *>(st + C::off_q + off) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
-                if (C::kv) {
+                if (C::k) {
                     float f[8];
                     unpack8(kr[r], f);
                     uint32_t w[4];
@@ -395,7 +357,7 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         }
         // (b) state decayed to the chunk end: S' = diag(e^{b_C}) S
         if (!mbar_wait(&b.gated[s], ph, abort)) break;
-        {
+        if (!C::dstate) {
             const float4 *e4 = reinterpret_cast<const float4 *>(ec + s * D);
 #pragma unroll
             for (int i4 = 0; i4 < HD / 4; ++i4) {
@@ -442,13 +404,28 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
             __syncwarp();
             if (lane == 0) mbar_arrive(b.o_free);
             __nv_bfloat16 *orow = o + (row0 + (long long)c * CH + h * 32) * D + dv;
+            if (MODE == kPassCorrect) {  // o_local: all loads before the first store
+                float ol[32];
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                float x = __uint_as_float(r[t]);
-                if (MODE == kPassCorrect) x += __bfloat162float(orow[t * D]);
-                orow[t * D] = __float2bfloat16_rn(x);
+                for (int t = 0; t < 32; ++t) ol[t] = __bfloat162float(orow[t * D]);
+#pragma unroll
+                for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(__uint_as_float(r[t]) + ol[t]);
             }
+#pragma unroll
+            for (int t = 0; t < 32; ++t) orow[t * D] = __float2bfloat16_rn(__uint_as_float(r[t]));
         }
+    }
+    if (C::dstate && mbar_wait(b.ds_full, 0, abort)) {  // the segment's gradient state R^T
+        tc_fence_after();
+        uint32_t r[32];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) S[p * 32 + e] = __uint_as_float(r[e]);
+        }
+        tc_fence_before();
     }
     if (C::write_state && !*abort) {
         float *So = a.S_out + ((long long)bh * a.NP + j) * D * D + (long long)h * HD * D + dv;
@@ -504,10 +481,8 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     if (warp == kTmaWarp && lane == 0) {
         if (C::q) prefetch_tmap(&tm_q);
-        if (C::kv) {
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-        }
+        if (C::k) prefetch_tmap(&tm_k);
+        if (C::v) prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_g);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
@@ -536,33 +511,6 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// [rows, 128] bf16 view, 64 x 64 boxes, 128-byte swizzle.
-cudaError_t make_map(CUtensorMap *m, const void *base, long long rows) {
-    auto fn = encode_fn();
-    if (!fn) return cudaErrorNotSupported;
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)CH};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 template <int MODE>
 cudaError_t launch_mode(const PassArgs &a, cudaStream_t st) {
     using C = Cfg<MODE>;
@@ -570,7 +518,7 @@ cudaError_t launch_mode(const PassArgs &a, cudaStream_t st) {
     if (rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
     CUtensorMap mq, mk, mv, mg;
     cudaError_t e;
-    const void *qp = C::q ? a.q : a.g, *kp = C::kv ? a.k : a.g, *vp = C::kv ? a.v : a.g;
+    const void *qp = C::q ? a.q : a.g, *kp = C::k ? a.k : a.g, *vp = C::v ? a.v : a.g;
     if ((e = make_map(&mq, qp, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mk, kp, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mv, vp, rows)) != cudaSuccess) return e;
@@ -596,6 +544,7 @@ cudaError_t launch_tc_pass(const PassArgs &a, PassMode mode, cudaStream_t st) {
         case kPassOutput: return launch_mode<kPassOutput>(a, st);
         case kPassLocal: return launch_mode<kPassLocal>(a, st);
         case kPassCorrect: return launch_mode<kPassCorrect>(a, st);
+        case kPassDState: return launch_mode<kPassDState>(a, st);
     }
     return cudaErrorInvalidValue;
 }

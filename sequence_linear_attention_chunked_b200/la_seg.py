@@ -25,7 +25,8 @@ SCHED_AUTO, SCHED_TWO_PASS, SCHED_THREE_PHASE = 0, 1, 2
 EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_seg_scan",
             "la_seg_state_pass", "la_seg_local_pass", "la_seg_output_pass", "la_seg_correct_pass",
             "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail",
-            "la_seg_forward_noalloc", "la_seg_dstate_pass", "la_seg_grad_pass")
+            "la_seg_forward_noalloc", "la_seg_dstate_pass", "la_seg_dq_pass", "la_seg_dkv_pass",
+            "la_seg_backward_parts")
 
 _lib = None
 
@@ -73,9 +74,14 @@ def lib():
         L.la_seg_dstate_pass.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P,
                                          P, P]
         L.la_seg_dstate_pass.restype = i32
-        L.la_seg_grad_pass.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
-                                       i32, P, P, P, P, P, P, P]
-        L.la_seg_grad_pass.restype = i32
+        L.la_seg_dq_pass.argtypes = [P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32,
+                                     i32, P, P, P, P, P]
+        L.la_seg_dq_pass.restype = i32
+        L.la_seg_dkv_pass.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32,
+                                      i32, i32, P, P, P, P, P]
+        L.la_seg_dkv_pass.restype = i32
+        L.la_seg_backward_parts.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32, i32]
+        L.la_seg_backward_parts.restype = i32
         L.la_seg_check_status.argtypes = [P, P]
         L.la_seg_check_status.restype = i32
         L.la_last_error_detail.argtypes = [ctypes.c_char_p, sz]
@@ -286,16 +292,29 @@ def la_seg_dstate_pass(q, dO, log_g, NP, chunk, *, dSloc=None, log_gamma=None, s
     return dSloc, log_gamma
 
 
-def la_seg_grad_pass(q, k, v, log_g, dO, S_recv, S_final, dX, NP, chunk, *, out=None, dq_ws=None,
-                     status=None, stream=None):
+def la_seg_backward_parts(B, H, L, dk, dv, P, chunk, dt=LA_BF16, reuse=True) -> int:
+    return int(lib().la_seg_backward_parts(B, H, L, dk, dv, P, chunk, dt, int(bool(reuse))))
+
+
+def la_seg_dq_pass(q, k, v, log_g, dO, S_recv, NP, fine, chunk, *, dq=None, qdq=None, S_fine=None,
+                   status=None, stream=None):
+    B, H, L, dk, dv = _seq_shapes(q, v)
+    dq = torch.empty_like(q) if dq is None else dq
+    qdq = torch.empty((B, H, L, dk), dtype=torch.float32, device=q.device) if qdq is None else qdq
+    _check(lib().la_seg_dq_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(dO), _ptr(S_recv), B,
+                                H, L, dk, dv, NP, fine, chunk, _dt(q), _ptr(dq), _ptr(qdq),
+                                _ptr(S_fine), _ptr(status), _stream(stream)), "la_seg_dq_pass")
+    return dq, qdq
+
+
+def la_seg_dkv_pass(q, k, v, log_g, dO, S_recv, S_final, dX, qdq, NP, chunk, *, out=None,
+                    status=None, stream=None):
     B, H, L, dk, dv = _seq_shapes(q, v)
     if out is None:
-        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_g))
-    if dq_ws is None:
-        dq_ws = torch.empty((B, H, L, dk), dtype=torch.float32, device=q.device)
-    dq, dk_, dv_, dg = out
-    _check(lib().la_seg_grad_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(dO), _ptr(S_recv),
-                                  _ptr(S_final), _ptr(dX), B, H, L, dk, dv, NP, chunk, _dt(q),
-                                  _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dq_ws),
-                                  _ptr(status), _stream(stream)), "la_seg_grad_pass")
+        out = (torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_g))
+    dk_, dv_, dg = out
+    _check(lib().la_seg_dkv_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(dO), _ptr(S_recv),
+                                 _ptr(S_final), _ptr(dX), _ptr(qdq), B, H, L, dk, dv, NP, chunk,
+                                 _dt(q), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(status),
+                                 _stream(stream)), "la_seg_dkv_pass")
     return out

@@ -65,16 +65,17 @@ def test_small_backward(cuda_device, shape, reuse):
 
 
 def test_reuse_matches_recompute(cuda_device):
-    """Reusing the forward's received states (ZeCO review, "forward implications") gives the
-    same gradients as recomputing them."""
+    """Reusing the forward's received states (ZeCO review, "forward implications") and
+    recomputing them both give the oracle's gradients."""
     w = WORKLOADS["C1"].with_(H=2, L=4096, P=4, backward=True)
     x = make_inputs(w, cuda_device, with_s0=True)
     _, _, Sr = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], x["S0"], w.P, w.chunk,
                                      want_S_recv=True)
-    a = run_bwd(x, w, None)
-    b = run_bwd(x, w, Sr)
-    for n, ga, gb in zip(NAMES, a, b):
-        assert rel_err(ga, gb.double().cpu().numpy()) <= 1e-2, n
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["log_g"], x["dO"], x["S0"])
+    for saved in (None, Sr):
+        got = run_bwd(x, w, saved)
+        for n, g, r in zip(NAMES, got, ref):
+            assert rel_err(g, r) <= 2e-2, (n, saved is None)
 
 
 def test_backward_empty(cuda_device):
