@@ -58,8 +58,10 @@ WORKLOADS = {
     "C2": Workload("C2", 1, 16, 131072, 128, 128, 8, 64, "bf16", "gla"),
     "C3": Workload("C3", 1, 16, 4194304, 128, 128, 256, 64, "bf16", "gla"),
     "C4": Workload("C4", 2, 16, 131072, 128, 128, 8, 64, "bf16", "gla", backward=True),
-    # not one of the five benchmark workloads: exercises the cross-segment scan with weak decay
+    # not benchmark workloads: the cross-segment scan under weak decay (tests), and a 16k-token
+    # fwd+bwd case for kernel profiles (inputs larger than L2, a few hundred MB in all)
     "WEAK": Workload("WEAK", 1, 4, 16384, 128, 128, 4, 64, "bf16", "weak"),
+    "BWD16K": Workload("BWD16K", 1, 16, 16384, 128, 128, 1, 64, "bf16", "gla", backward=True),
 }
 
 
