@@ -31,9 +31,10 @@ constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
 namespace dqs {
 
 constexpr uint32_t kColDS = 0, kColDQ = 128, kColSA = 192, kColM = 256;
-constexpr int kStages = 3;
-constexpr int off_k = 0, off_v = kTileBytes, off_do = 2 * kTileBytes, off_g = 3 * kTileBytes;
-constexpr int kStageBytes = 4 * kTileBytes;
+constexpr int kStages = 2;
+constexpr int off_k = 0, off_v = kTileBytes, off_do = 2 * kTileBytes, off_g = 3 * kTileBytes,
+              off_q = 4 * kTileBytes;  // q only feeds the epilogue's q . dq
+constexpr int kStageBytes = 5 * kTileBytes;
 constexpr int off_m = kStages * kStageBytes;
 constexpr int off_ec = off_m + CH * CH * 2;
 constexpr int off_bar = off_ec + kStages * D * 4;
@@ -50,7 +51,7 @@ struct Bars {
 
 __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tk,
                          const CUtensorMap *tv, const CUtensorMap *tdo, const CUtensorMap *tg,
-                         long long row0, int nchunks) {
+                         const CUtensorMap *tq, long long row0, int nchunks) {
     int issued = 0;
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % kStages;
@@ -66,6 +67,8 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
         tma_load_2d(st + off_do + kHalfBytes, tdo, 64, y, &b.full[s]);
         tma_load_2d(st + off_g, tg, 0, y, &b.full[s]);
         tma_load_2d(st + off_g + kHalfBytes, tg, 64, y, &b.full[s]);
+        tma_load_2d(st + off_q, tq, 0, y, &b.full[s]);
+        tma_load_2d(st + off_q + kHalfBytes, tq, 64, y, &b.full[s]);
         issued = c + 1;
     }
     if (*abort)
@@ -214,7 +217,6 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
     const int i = quarter * 32 + lane;
     const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
     const float *ec = reinterpret_cast<const float *>(smem + off_ec);
-    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
     __nv_bfloat16 *dq = static_cast<__nv_bfloat16 *>(a.dq_out);
 
     float S[HD];  // S[i][64h + e]
@@ -307,19 +309,14 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         if (lane == 0) mbar_arrive(b.dq_free);
         const long long t0 = row0 + (long long)c * CH + h * 32;
         const __nv_bfloat16 *fcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_g);
+        const __nv_bfloat16 *qcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_q);
 #pragma unroll
-        for (int t8 = 0; t8 < 32; t8 += 8) {
-            float qv[8];  // a batch's loads before its stores: none waits behind a possible alias
-#pragma unroll
-            for (int t = 0; t < 8; ++t) qv[t] = __bfloat162float(q[(t0 + t8 + t) * D + i]);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const float f = __bfloat162float(fcol[tile_off(h * 32 + t8 + t, i) >> 1]);
-                const float v = __uint_as_float(r[t8 + t]) * f;
-                const long long idx = (t0 + t8 + t) * D + i;
-                dq[idx] = __float2bfloat16_rn(v);
-                a.dq_ws[idx] = qv[t] * v;
-            }
+        for (int t = 0; t < 32; ++t) {
+            const uint32_t off = tile_off(h * 32 + t, i) >> 1;
+            const float v = __uint_as_float(r[t]) * __bfloat162float(fcol[off]);
+            const long long idx = (t0 + t) * D + i;
+            dq[idx] = __float2bfloat16_rn(v);
+            a.dq_ws[idx] = __bfloat162float(qcol[off]) * v;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.empty[s]);
@@ -329,7 +326,7 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
 __global__ void __launch_bounds__(kThreads, 1)
 tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_g,
-             const BwdArgs a) {
+             const __grid_constant__ CUtensorMap tm_q, const BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -371,6 +368,7 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_g);
+        prefetch_tmap(&tm_q);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -378,7 +376,7 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (warp == kTmaWarp) {
-        if (lane == 0) producer(smem, b, abort, &tm_k, &tm_v, &tm_do, &tm_g, row0, nchunks);
+        if (lane == 0) producer(smem, b, abort, &tm_k, &tm_v, &tm_do, &tm_g, &tm_q, row0, nchunks);
     } else if (warp == kMmaWarp) {
         if (lane == 0) mma_issuer(smem, b, abort, tmem, nchunks);
     } else if (warp >= kEpiWarps) {
@@ -671,7 +669,6 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
     const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
     const float *ec = reinterpret_cast<const float *>(smem + off_ec);
     float *xb = reinterpret_cast<float *>(smem + off_x);  // [2 sets][2 halves][128]
-    const __nv_bfloat16 *kin = static_cast<const __nv_bfloat16 *>(a.k);
     __nv_bfloat16 *dk = static_cast<__nv_bfloat16 *>(a.dk_out);
     __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv_out);
     __nv_bfloat16 *dg = static_cast<__nv_bfloat16 *>(a.dg_out);
@@ -715,6 +712,10 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         const int c = nchunks - 1 - it;
         uint8_t *st = smem + s * kStageBytes;
         uint32_t r[32];
+        const long long t0 = row0 + (long long)c * CH + h * 32;
+        float qdq[32];  // q . dq of this thread's tokens, in flight while the MMAs run
+#pragma unroll
+        for (int t = 0; t < 32; ++t) qdq[t] = a.dq_ws[(t0 + t) * D + i];
         // (a) masked M and A tiles
         if (!mbar_wait(b.mm_full, it & 1, abort)) break;
         tc_fence_after();
@@ -763,27 +764,18 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(b.dk_free);
-        const long long t0 = row0 + (long long)c * CH + h * 32;
         const __nv_bfloat16 *fcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_g);
+        const __nv_bfloat16 *kcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_k);
         float tot = 0.f;
 #pragma unroll
-        for (int t8 = 0; t8 < 32; t8 += 8) {
-            float qdq[8], kr[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const long long idx = (t0 + t8 + t) * D + i;
-                qdq[t] = a.dq_ws[idx];
-                kr[t] = __bfloat162float(kin[idx]);
-            }
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const float f = __bfloat162float(fcol[tile_off(h * 32 + t8 + t, i) >> 1]);
-                const float dkv = __uint_as_float(r[t8 + t]) * f;
-                dk[(t0 + t8 + t) * D + i] = __float2bfloat16_rn(dkv);
-                const float cg = qdq[t] - kr[t] * dkv;
-                r[t8 + t] = __float_as_uint(cg);  // contribution, kept for the suffix sums
-                tot += cg;
-            }
+        for (int t = 0; t < 32; ++t) {
+            // dk = e^{b_C - b_s} acc and k . dk = Ktil . acc (Ktil = k e^{b_C - b_s}, the MMA operand)
+            const uint32_t off = tile_off(h * 32 + t, i) >> 1;
+            const float acc = __uint_as_float(r[t]);
+            dk[(t0 + t) * D + i] = __float2bfloat16_rn(acc * __bfloat162float(fcol[off]));
+            const float cg = qdq[t] - __bfloat162float(kcol[off]) * acc;
+            r[t] = __float_as_uint(cg);  // contribution, kept for the suffix sums
+            tot += cg;
         }
         float *xs = xb + ((it + 1) & 1) * 2 * D;
         xs[h * D + i] = tot;
@@ -921,18 +913,19 @@ bool tc_bwd_supported(const BwdArgs &a) {
 
 cudaError_t launch_tc_dq(const BwdArgs &a, cudaStream_t st) {
     const long long rows = (long long)a.BH * a.L;
-    CUtensorMap mk, mv, mdo, mg;
+    CUtensorMap mk, mv, mdo, mg, mq;
     cudaError_t e;
     if ((e = make_map(&mk, a.k, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mdo, a.dO, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mq, a.q, rows)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(dqs::tc_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dqs::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long nblk = (long long)a.BH * a.NP;
     if (nblk == 0) return cudaSuccess;
-    dqs::tc_dq_kernel<<<(unsigned)nblk, kThreads, dqs::kSmemBytes, st>>>(mk, mv, mdo, mg, a);
+    dqs::tc_dq_kernel<<<(unsigned)nblk, kThreads, dqs::kSmemBytes, st>>>(mk, mv, mdo, mg, mq, a);
     return cudaGetLastError();
 }
 
