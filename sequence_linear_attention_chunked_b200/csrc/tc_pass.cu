@@ -38,7 +38,7 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
-constexpr int kEpiWarps = 8, kGateWarps = 4;
+constexpr int kStateWarps = 4, kOutWarps = 4, kEpiWarps = kStateWarps + kOutWarps, kGateWarps = 4;
 constexpr int kTmaWarp = 12, kMmaWarp = 13;
 constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
 
@@ -109,6 +109,8 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
 }
 
 // ------------------------------------------------------------------ MMA issuer (1 thread)
+// Per chunk: QK^T (output modes); the state increment accumulated straight onto the decayed
+// state S' that the state warps left in TMEM (S = S' + dS); PV and S'^T Qbar'^T into O^T.
 template <int MODE>
 __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
                            int nchunks) {
@@ -133,18 +135,20 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
                 mma_ss(tmem + kColQK, desc_kmajor(qa, kk), desc_kmajor(ka, kk), i_qk, kk > 0);
             mma_commit(b.qk_full);
         }
-        if (C::dstate) {  // R^T += dO^T Qhat, accumulated over the whole segment
+        if (C::dstate) {  // R^T += dO^T Qhat, accumulated over the whole segment from zero
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(qa, kk), i_ds,
                        (c > 0 || kk > 0) ? 1u : 0u);
         }
-        if (C::kv) {  // chunk state increment dS^T = V^T Ktil
-            if (c > 0 && !mbar_wait(b.ds_free, (c - 1) & 1, abort)) break;
+        if (!C::dstate) {  // S' and its bf16 copy are in place
+            if (!mbar_wait(b.sa_full, c & 1, abort)) break;
             tc_fence_after();
+        }
+        if (C::kv) {  // S^T = S'^T + V^T Ktil
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(ka, kk), i_ds, kk > 0);
+                mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(ka, kk), i_ds, 1u);
             mma_commit(b.ds_full);
         }
         if (C::out) {
@@ -157,8 +161,6 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
                     mma_ss(tmem + kColO, desc_mnmajor(va, kk),
                            smem_desc_sw128(p_addr + kk * 32, 16, 1024), i_pv, kk > 0);
             }
-            if (!mbar_wait(b.sa_full, c & 1, abort)) break;
-            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // O^T += S'^T Qbar'^T, A from tensor memory
                 mma_ts(tmem + kColO, tmem + kColSA + kk * 8, desc_kmajor(qa, kk), i_qs,
@@ -293,116 +295,156 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
     if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
 }
 
-// ------------------------------------------------------------------ epilogue warps (256 threads)
-// Warp w reads TMEM lane quarter q = w % 4, so thread (w, lane) owns d_v column dv = 32q+lane;
-// half h = w / 4 selects which 64 key dims of that state column it keeps (fp32, registers),
-// which 32 of the 64 P / O columns it handles.
+// ------------------------------------------------------------------ state warps (0-3)
+// Thread dv (= TMEM lane) owns row dv of the transposed fp32 state S^T, which lives in TMEM.
+// Per chunk it scales the row by the chunk's decay (S' = diag(e^{b_C}) S), stores S' back
+// for the MMA to accumulate the chunk's increment onto, and (output modes) stores the bf16
+// copy that is the A operand of O^T += S'^T Qbar'^T.
 template <int MODE>
-__device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
-                              const PassArgs &a, uint32_t tmem, int bh, int j, long long row0,
-                              int nchunks) {
+__device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
+                           uint32_t tmem, int bh, int j, int nchunks) {
     using C = Cfg<MODE>;
-    constexpr int HD = D / 2;  // key dims per thread
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quarter = warp & 3, h = warp >> 2;
-    const int dv = quarter * 32 + lane;
-    const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
-    const float *ec = reinterpret_cast<const float *>(smem + C::off_ec) + h * HD;
-    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
-
-    float S[HD];  // S^T[dv][h*64 + e] = S[h*64 + e][dv]
-    if (C::init_state && a.S_init) {
-        const float *Si = a.S_init + ((long long)bh * a.NP + j) * D * D + (long long)h * HD * D + dv;
+    const int dv = warp * 32 + lane;
+    const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+    const float *ec = reinterpret_cast<const float *>(smem + C::off_ec);
+    uint32_t r0[32], r1[32];
+    if (!C::dstate) {  // initial state: the received state (output / correction passes) or zero
+        const float *Si = (C::init_state && a.S_init)
+                              ? a.S_init + ((long long)bh * a.NP + j) * D * D + dv : nullptr;
 #pragma unroll
-        for (int e = 0; e < HD; ++e) S[e] = Si[e * D];
-    } else {
+        for (int p = 0; p < 4; ++p) {
 #pragma unroll
-        for (int e = 0; e < HD; ++e) S[e] = 0.f;
+            for (int e = 0; e < 32; ++e) r0[e] = __float_as_uint(Si ? Si[(p * 32 + e) * D] : 0.f);
+            tmem_st32(tmem + lrow + kColDS + p * 32, r0);
+        }
+        tmem_wait_st();
+        tc_fence_before();
     }
-
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % C::stages;
-        const uint32_t ph = (c / C::stages) & 1;
-        uint32_t r[32];
-        if (C::qk) {  // (a) scores -> causal mask -> bf16 P tile (K-major, swizzled rows)
+        if (!mbar_wait(&b.gated[s], (c / C::stages) & 1, abort)) break;
+        if (!C::dstate) {
+            if (C::kv && c > 0 && !mbar_wait(b.ds_full, (c - 1) & 1, abort)) break;
+            if (C::out && c > 0 && !mbar_wait(b.sa_free, (c - 1) & 1, abort)) break;
+            tc_fence_after();
+            const float *e_s = ec + s * D;
+#pragma unroll
+            for (int p2 = 0; p2 < 2; ++p2) {
+                tmem_ld32(tmem + lrow + kColDS + p2 * 64, r0);
+                tmem_ld32(tmem + lrow + kColDS + p2 * 64 + 32, r1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 f0 = *reinterpret_cast<const float4 *>(e_s + p2 * 64 + 4 * e4);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(e_s + p2 * 64 + 32 + 4 * e4);
+                    r0[4 * e4 + 0] = __float_as_uint(__uint_as_float(r0[4 * e4 + 0]) * f0.x);
+                    r0[4 * e4 + 1] = __float_as_uint(__uint_as_float(r0[4 * e4 + 1]) * f0.y);
+                    r0[4 * e4 + 2] = __float_as_uint(__uint_as_float(r0[4 * e4 + 2]) * f0.z);
+                    r0[4 * e4 + 3] = __float_as_uint(__uint_as_float(r0[4 * e4 + 3]) * f0.w);
+                    r1[4 * e4 + 0] = __float_as_uint(__uint_as_float(r1[4 * e4 + 0]) * f1.x);
+                    r1[4 * e4 + 1] = __float_as_uint(__uint_as_float(r1[4 * e4 + 1]) * f1.y);
+                    r1[4 * e4 + 2] = __float_as_uint(__uint_as_float(r1[4 * e4 + 2]) * f1.z);
+                    r1[4 * e4 + 3] = __float_as_uint(__uint_as_float(r1[4 * e4 + 3]) * f1.w);
+                }
+                if (C::kv || C::out) {  // the correction pass keeps the decayed received state
+                    tmem_st32(tmem + lrow + kColDS + p2 * 64, r0);
+                    tmem_st32(tmem + lrow + kColDS + p2 * 64 + 32, r1);
+                }
+                if (C::out) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        pk[e] = pack_bf16(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+                        pk[16 + e] = pack_bf16(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+                    }
+                    tmem_st32(tmem + lrow + kColSA + p2 * 32, pk);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&b.empty[s]);
+            if (!C::dstate) mbar_arrive(b.sa_full);
+        }
+    }
+    if (C::write_state && !*abort) {
+        const uint32_t last = C::dstate ? 0u : (uint32_t)((nchunks - 1) & 1);
+        if (mbar_wait(b.ds_full, last, abort)) {
+            tc_fence_after();
+            float *So = a.S_out + ((long long)bh * a.NP + j) * D * D + dv;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                tmem_ld32(tmem + lrow + kColDS + p * 32, r0);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) So[(p * 32 + e) * D] = __uint_as_float(r0[e]);
+            }
+            tc_fence_before();
+        }
+    }
+}
+
+// ------------------------------------------------------------------ output warps (4-7)
+// (a) the intra-chunk scores -> causal mask -> bf16 P tile; (d) the chunk's outputs.
+template <int MODE>
+__device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
+                         uint32_t tmem, long long row0, int nchunks) {
+    using C = Cfg<MODE>;
+    if (!C::out) return;
+    const int quarter = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
+    const int dv = quarter * 32 + lane;
+    const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
+    uint32_t r[32];
+    for (int c = 0; c < nchunks; ++c) {
+        if (C::qk) {  // M=64 accumulator: lanes 0-15 of each quarter hold rows 16 quarter + lane
             if (!mbar_wait(b.qk_full, c & 1, abort)) break;
             tc_fence_after();
-            tmem_ld32(tmem + lrow + kColQK + h * 32, r);  // columns s = 32h .. 32h+31
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b.qk_free);
-            if (lane < 16) {  // M=64 accumulator: lanes 0-15 of each quarter hold rows 16q+l
-                const int t = quarter * 16 + lane;
-                uint8_t *prow = smem + C::off_p + t * 128;
+            const int t = quarter * 16 + lane;
+            uint8_t *prow = smem + C::off_p + t * 128;
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    uint32_t w4[4];
+            for (int h = 0; h < 2; ++h) {
+                tmem_ld32(tmem + lrow + kColQK + h * 32, r);
+                tmem_wait_ld();
+                if (h == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b.qk_free);
+                }
+                if (lane < 16) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int sl = jj * 8 + 2 * e;  // local column; key index 32h + sl
-                        const int s0 = h * 32 + sl;
-                        const float x0 = s0 <= t ? __uint_as_float(r[sl]) : 0.f;
-                        const float x1 = s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f;
-                        w4[e] = pack_bf16(x0, x1);
+                    for (int jj = 0; jj < 4; ++jj) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int sl = jj * 8 + 2 * e, s0 = h * 32 + sl;
+                            w4[e] = pack_bf16(s0 <= t ? __uint_as_float(r[sl]) : 0.f,
+                                              s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f);
+                        }
+                        *reinterpret_cast<uint4 *>(prow + (((h * 4 + jj) ^ (t & 7)) << 4)) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
-                    const int chunk16 = h * 4 + jj;
-                    *reinterpret_cast<uint4 *>(prow + ((chunk16 ^ (t & 7)) << 4)) =
-                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(b.p_full);
         }
-        // (b) state decayed to the chunk end: S' = diag(e^{b_C}) S
-        if (!mbar_wait(&b.gated[s], ph, abort)) break;
-        if (!C::dstate) {
-            const float4 *e4 = reinterpret_cast<const float4 *>(ec + s * D);
+        // (d) outputs: column dv of the chunk's 64 rows
+        if (!mbar_wait(b.o_full, c & 1, abort)) break;
+        tc_fence_after();
 #pragma unroll
-            for (int i4 = 0; i4 < HD / 4; ++i4) {
-                const float4 e = e4[i4];
-                S[4 * i4 + 0] *= e.x;
-                S[4 * i4 + 1] *= e.y;
-                S[4 * i4 + 2] *= e.z;
-                S[4 * i4 + 3] *= e.w;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b.empty[s]);
-        if (C::out) {  // bf16 S'^T into tensor memory: A operand of the inter-chunk MMA
-            if (c > 0 && !mbar_wait(b.sa_free, (c - 1) & 1, abort)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = pack_bf16(S[2 * e], S[2 * e + 1]);
-            tmem_st32(tmem + lrow + kColSA + h * 32, r);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b.sa_full);
-        }
-        if (C::kv) {  // (c) S = S' + dS
-            if (!mbar_wait(b.ds_full, c & 1, abort)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) S[p * 32 + e] += __uint_as_float(r[e]);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b.ds_free);
-        }
-        if (C::out) {  // (d) outputs: rows t = 32h .. 32h+31 of column dv
-            if (!mbar_wait(b.o_full, c & 1, abort)) break;
-            tc_fence_after();
+        for (int h = 0; h < 2; ++h) {
             tmem_ld32(tmem + lrow + kColO + h * 32, r);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b.o_free);
+            if (h == 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b.o_free);
+            }
             __nv_bfloat16 *orow = o + (row0 + (long long)c * CH + h * 32) * D + dv;
             if (MODE == kPassCorrect) {  // o_local: all loads before the first store
                 float ol[32];
@@ -414,23 +456,6 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
 #pragma unroll
             for (int t = 0; t < 32; ++t) orow[t * D] = __float2bfloat16_rn(__uint_as_float(r[t]));
         }
-    }
-    if (C::dstate && mbar_wait(b.ds_full, 0, abort)) {  // the segment's gradient state R^T
-        tc_fence_after();
-        uint32_t r[32];
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) S[p * 32 + e] = __uint_as_float(r[e]);
-        }
-        tc_fence_before();
-    }
-    if (C::write_state && !*abort) {
-        float *So = a.S_out + ((long long)bh * a.NP + j) * D * D + (long long)h * HD * D + dv;
-#pragma unroll
-        for (int e = 0; e < HD; ++e) So[e * D] = S[e];
     }
 }
 
@@ -464,17 +489,17 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int s = 0; s < C::stages; ++s) {
             mbar_init(&b.full[s], 1);
             mbar_init(&b.gated[s], kGateWarps);
-            mbar_init(&b.empty[s], 1 + kEpiWarps);
+            mbar_init(&b.empty[s], 1 + kStateWarps);
         }
         mbar_init(b.qk_full, 1);
-        mbar_init(b.qk_free, kEpiWarps);
-        mbar_init(b.p_full, kEpiWarps);
+        mbar_init(b.qk_free, kOutWarps);
+        mbar_init(b.p_full, kOutWarps);
         mbar_init(b.ds_full, 1);
-        mbar_init(b.ds_free, kEpiWarps);
-        mbar_init(b.sa_full, kEpiWarps);
+        mbar_init(b.ds_free, 1);
+        mbar_init(b.sa_full, kStateWarps);
         mbar_init(b.sa_free, 1);
         mbar_init(b.o_full, 1);
-        mbar_init(b.o_free, kEpiWarps);
+        mbar_init(b.o_free, kOutWarps);
         mbar_init(b.fin, 1);
         *abort = 0;
         mbar_fence_init();
@@ -497,8 +522,10 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (lane == 0) mma_issuer<MODE>(smem, b, abort, tmem, nchunks);
     } else if (warp >= kEpiWarps) {
         gate_role<MODE>(smem, b, abort, a, bh, j, nchunks);
+    } else if (warp < kStateWarps) {
+        state_role<MODE>(smem, b, abort, a, tmem, bh, j, nchunks);
     } else {
-        epilogue_role<MODE>(smem, b, abort, a, tmem, bh, j, row0, nchunks);
+        out_role<MODE>(smem, b, abort, a, tmem, row0, nchunks);
     }
 
     tc_fence_before();
