@@ -21,12 +21,7 @@ constexpr int kHalfBytes = CH * 64 * 2;  // one 64-column swizzle half of a tile
 constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Tensor-memory columns (fp32 accumulators; SA holds bf16 pairs).
-constexpr uint32_t kColDS = 0;    // dS^T         128 lanes x 128 cols
-constexpr uint32_t kColO = 128;   // O^T          128 lanes x 64 cols
-constexpr uint32_t kColSA = 192;  // bf16 S'^T    128 lanes x 64 cols (128 values)
-constexpr uint32_t kColQK = 256;  // Qbar' Ktil^T M=64 layout, 64 cols
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 512;  // every tensor-core kernel allocates all of it
 
 // Byte offset of element (t, i) of a [64 x 128] bf16 tile TMA-loaded as two 64-column halves
 // with the 128-byte swizzle (16-byte chunk index XOR row % 8).

@@ -11,18 +11,17 @@
 //   O^T = V^T P^T + S'^T Qbar'^T,  S' = diag(e^{b_C}) S    M=128 (dv) N=64  (t)  K=64 / 128
 //   dS^T = V^T Ktil,  S <- S' + dS                         M=128 (dv) N=128 (i)  K=64  (s)
 //
-// The outputs and the state are kept transposed (d_v on the TMEM lanes) so that each pair of
-// the 256 epilogue threads owns one d_v column: each keeps half of that column of the fp32
-// state in registers, scales it by the decay (per-row factors from shared memory), and writes its bf16
-// copy straight into tensor memory as the A operand of the inter-chunk MMA -- the state never
-// goes through shared memory.  q and k tiles are rescaled in place by the gate warps (one
-// thread per key dimension runs the sequential cumsum), so every MMA operand has the layout
-// TMA wrote.
+// The outputs and the state are kept transposed (d_v on the TMEM lanes).  The fp32 state S^T
+// stays in tensor memory for the whole segment: per chunk a state warp thread scales its row
+// by the chunk's decay (S' = diag(e^{b_C}) S, per-key factors from shared memory), stores S'
+// back for the MMA to accumulate the increment onto, and stores the bf16 copy that is the A
+// operand of the inter-chunk MMA -- the state never goes through shared memory.  q and k tiles
+// are rescaled in place by the gate warps, so every MMA operand has the layout TMA wrote.
 //
-// Warp roles (448 threads): 0-7 epilogue (TMEM lane quarter = warp % 4; warps 0-3 own key
-// dims 0-63 of the state column, warps 4-7 key dims 64-127), 8-11 gates, 12 TMA producer,
-// 13 MMA issuer / TMEM owner.  Every wait is bounded (about a second of clock), after
-// which the CTA stops, drains what it issued, frees its TMEM and reports kStatusTimeout.
+// Warp roles (576 threads): 0-3 state (TMEM lane quarter = warp), 4-7 output (P tile and O
+// read-out, quarter = warp - 4), 8-15 gates, 16 TMA producer, 17 MMA issuer / TMEM owner.
+// Every wait is bounded (about a second of clock), after which the CTA stops, drains what it
+// issued, frees its TMEM and reports kStatusTimeout.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -38,9 +37,13 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
-constexpr int kStateWarps = 4, kOutWarps = 4, kEpiWarps = kStateWarps + kOutWarps, kGateWarps = 4;
-constexpr int kTmaWarp = 12, kMmaWarp = 13;
-constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
+constexpr int kStateWarps = 4, kOutWarps = 4, kEpiWarps = kStateWarps + kOutWarps, kGateWarps = 8;
+constexpr int kTmaWarp = kEpiWarps + kGateWarps, kMmaWarp = kTmaWarp + 1;
+constexpr int kThreads = 32 * (kMmaWarp + 1);
+
+// Tensor-memory columns: the fp32 state, two O^T buffers, two bf16 S'^T buffers (bf16 pairs),
+// the M=64 score tile.
+constexpr uint32_t kColDS = 0, kColO = 128, kColSA = 256, kColQK = 384;
 
 template <int MODE>
 struct Cfg {
@@ -59,20 +62,26 @@ struct Cfg {
     static constexpr int off_v = off_k + (k ? kTileBytes : 0);
     static constexpr int off_g = off_v + (v ? kTileBytes : 0);
     static constexpr int stage_bytes = off_g + kTileBytes;
-    static constexpr int off_p = stages * stage_bytes;
-    static constexpr int off_ec = off_p + (qk ? CH * CH * 2 : 0);
+    static constexpr int off_p = stages * stage_bytes;           // two bf16 P tiles
+    static constexpr int off_ec = off_p + (qk ? 2 * CH * CH * 2 : 0);
     static constexpr int off_bar = off_ec + stages * D * 4;
-    static constexpr int n_bars = 3 * stages + 10;
+    static constexpr int n_bars = 3 * stages + 13;
     static constexpr int off_misc = off_bar + n_bars * 8;
     static constexpr int smem_bytes = off_misc + 16 + 1024;  // + slack to align the base to 1 KB
     static_assert(smem_bytes <= 232448, "shared memory budget");
 };
 
+// Ring barriers per stage; the rest come in pairs where the resource is double-buffered
+// (P tile, O^T and S'^T), so that no waiter can fall two phases behind its barrier.
 struct Bars {
     uint64_t *full, *gated, *empty;
-    uint64_t *qk_full, *qk_free, *p_full, *ds_full, *ds_free, *sa_full, *sa_free, *o_full,
-        *o_free, *fin;
+    uint64_t *qk_full, *qk_free, *p_full, *ds_full, *sa_full, *sa_free, *o_full, *o_free, *fin;
 };
+
+// Waits by a whole warp; the answer is the same in every lane.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort));
+}
 
 // ------------------------------------------------------------------ TMA producer (1 thread)
 template <int MODE>
@@ -108,9 +117,11 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
             wait_drain(&b.full[c % C::stages], (c / C::stages) & 1);
 }
 
-// ------------------------------------------------------------------ MMA issuer (1 thread)
-// Per chunk: QK^T (output modes); the state increment accumulated straight onto the decayed
-// state S' that the state warps left in TMEM (S = S' + dS); PV and S'^T Qbar'^T into O^T.
+// ------------------------------------------------------------------ MMA issuer (1 warp)
+// The whole warp walks the loop and waits; one elected lane issues.  Per chunk c: the state
+// increment accumulated straight onto the decayed state S' that the state warps left in TMEM
+// (S = S' + dS); then, in the output modes, the scores of chunk c+1 (so that the output warps
+// build P(c+1) while the tensor cores finish chunk c); then PV and S'^T Qbar'^T into O^T.
 template <int MODE>
 __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
                            int nchunks) {
@@ -119,76 +130,114 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
     constexpr uint32_t i_pv = idesc_bf16_f32(128, 64, 1, 0);
     constexpr uint32_t i_qs = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t i_ds = idesc_bf16_f32(128, 128, 1, 1);
-    const uint32_t p_addr = smem_u32(smem + C::off_p);
-    for (int c = 0; c < nchunks; ++c) {
-        const int s = c % C::stages;
-        const uint32_t ph = (c / C::stages) & 1;
-        if (!mbar_wait(&b.gated[s], ph, abort)) break;
-        tc_fence_after();
-        const uint32_t st = smem_u32(smem + s * C::stage_bytes);
-        const uint32_t qa = st + C::off_q, ka = st + C::off_k, va = st + C::off_v;
-        if (C::qk) {  // intra-chunk scores
-            if (c > 0 && !mbar_wait(b.qk_free, (c - 1) & 1, abort)) break;
-            tc_fence_after();
+    const uint32_t base = smem_u32(smem);
+    const uint32_t p_addr = base + C::off_p;
+    auto stage = [&](int c) { return base + (uint32_t)((c % C::stages) * C::stage_bytes); };
+    auto issue_qk = [&](int c) {  // intra-chunk scores of chunk c
+        const uint32_t st = stage(c);
+        if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + kColQK, desc_kmajor(qa, kk), desc_kmajor(ka, kk), i_qk, kk > 0);
+                mma_ss(tmem + kColQK, desc_kmajor(st + C::off_q, kk), desc_kmajor(st + C::off_k, kk),
+                       i_qk, kk > 0);
             mma_commit(b.qk_full);
         }
-        if (C::dstate) {  // R^T += dO^T Qhat, accumulated over the whole segment from zero
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(qa, kk), i_ds,
-                       (c > 0 || kk > 0) ? 1u : 0u);
+        __syncwarp();
+    };
+    bool ok = true;
+    if (C::qk && nchunks > 0) {
+        ok = warp_wait(&b.gated[0], 0, abort);
+        tc_fence_after();
+        if (ok) issue_qk(0);
+    }
+    for (int c = 0; ok && c < nchunks; ++c) {
+        const int s = c % C::stages;
+        const uint32_t st = stage(c);
+        const uint32_t qa = st + C::off_q, ka = st + C::off_k, va = st + C::off_v;
+        if (!C::qk) {  // (output modes waited for this chunk's tiles before its scores)
+            if (!(ok = warp_wait(&b.gated[s], (c / C::stages) & 1, abort))) break;
+            tc_fence_after();
         }
-        if (!C::dstate) {  // S' and its bf16 copy are in place
-            if (!mbar_wait(b.sa_full, c & 1, abort)) break;
+        if (C::dstate) {  // R^T += dO^T Qhat, accumulated over the whole segment from zero
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(qa, kk), i_ds,
+                           (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            __syncwarp();
+        } else {  // S' and its bf16 copy are in place
+            if (!(ok = warp_wait(b.sa_full, c & 1, abort))) break;
             tc_fence_after();
         }
         if (C::kv) {  // S^T = S'^T + V^T Ktil
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(ka, kk), i_ds, 1u);
-            mma_commit(b.ds_full);
-        }
-        if (C::out) {
-            if (c > 0 && !mbar_wait(b.o_free, (c - 1) & 1, abort)) break;
-            if (C::qk) {  // O^T = V^T P^T
-                if (!mbar_wait(b.p_full, c & 1, abort)) break;
-                tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tmem + kColO, desc_mnmajor(va, kk),
-                           smem_desc_sw128(p_addr + kk * 32, 16, 1024), i_pv, kk > 0);
+                    mma_ss(tmem + kColDS, desc_mnmajor(va, kk), desc_mnmajor(ka, kk), i_ds, 1u);
+                mma_commit(b.ds_full);
             }
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // O^T += S'^T Qbar'^T, A from tensor memory
-                mma_ts(tmem + kColO, tmem + kColSA + kk * 8, desc_kmajor(qa, kk), i_qs,
-                       (C::qk || kk > 0) ? 1u : 0u);
-            mma_commit(b.o_full);
-            mma_commit(b.sa_free);
+            __syncwarp();
         }
-        mma_commit(&b.empty[s]);
+        if (C::qk && c + 1 < nchunks) {  // scores of the next chunk
+            if (!(ok = warp_wait(&b.gated[(c + 1) % C::stages], ((c + 1) / C::stages) & 1, abort)))
+                break;
+            if (!(ok = warp_wait(b.qk_free, c & 1, abort))) break;
+            tc_fence_after();
+            issue_qk(c + 1);
+        }
+        if (C::out) {
+            const int ob = c & 1;
+            const uint32_t o_col = tmem + kColO + ob * 64;
+            if (c >= 2 && !(ok = warp_wait(&b.o_free[ob], ((c >> 1) - 1) & 1, abort))) break;
+            if (C::qk && !(ok = warp_wait(&b.p_full[ob], (c >> 1) & 1, abort))) break;
+            tc_fence_after();
+            if (elect_one()) {
+                if (C::qk) {  // O^T = V^T P^T
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(o_col, desc_mnmajor(va, kk),
+                               smem_desc_sw128(p_addr + ob * (CH * CH * 2) + kk * 32, 16, 1024),
+                               i_pv, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // O^T += S'^T Qbar'^T, A from tensor memory
+                    mma_ts(o_col, tmem + kColSA + ob * 64 + kk * 8, desc_kmajor(qa, kk), i_qs,
+                           (C::qk || kk > 0) ? 1u : 0u);
+                mma_commit(&b.o_full[ob]);
+                mma_commit(&b.sa_free[ob]);
+            }
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(&b.empty[s]);
+        __syncwarp();
     }
-    if (C::dstate) mma_commit(b.ds_full);
-    mma_commit(b.fin);  // nothing of this CTA may still run on the tensor cores at dealloc
+    if (elect_one()) {
+        if (C::dstate) mma_commit(b.ds_full);
+        mma_commit(b.fin);  // nothing of this CTA may still run on the tensor cores at dealloc
+    }
+    __syncwarp();
     wait_drain(b.fin, 0);
 }
 
-// ------------------------------------------------------------------ gate warps (128 threads)
-// Warp gw owns key dims 32gw .. 32gw+31.  Lane = 4*tg + ig: token group tg (rows 8tg .. 8tg+7)
-// and 16-byte key chunk ig (key dims 32gw + 8ig .. +7), so every shared-memory access moves one
-// swizzled 16-byte chunk.  The in-chunk cumsum of log_g runs down each thread's 8 rows, then
-// a 3-step shuffle scan across the 8 token groups adds the earlier groups' totals; the last
-// group's inclusive value is b_C.  Then q and k are rescaled in place in batches of 4 rows.
+// ------------------------------------------------------------------ gate warps (256 threads)
+// Warp gw owns key dims 16gw .. 16gw+15.  Lane = 2*tg + ig: token group tg (rows 4tg .. 4tg+3)
+// and 16-byte key chunk ig (key dims 16gw + 8ig .. +7), so every shared-memory access moves one
+// swizzled 16-byte chunk.  A thread visits its rows in the order 4tg + (k ^ sw), sw = tg & 2:
+// the rows of one warp-wide access then take four values of row % 8, which with the two key
+// chunks covers all eight 16-byte bank groups of the 128-byte swizzle (4 wavefronts for the
+// 512 bytes, the minimum).  The in-chunk cumsum of log_g is formed from the two row-pair sums,
+// then a 4-step shuffle scan across the 16 token groups adds the earlier groups' totals; the
+// last group's inclusive value is b_C.  Then q and k are rescaled in place, 2 rows per batch.
 template <int MODE>
 __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
                           int bh, int j, int nchunks) {
     using C = Cfg<MODE>;
     const int gw = (threadIdx.x >> 5) - kEpiWarps;
     const int lane = threadIdx.x & 31;
-    const int tg = lane >> 2, ig = lane & 3;
-    const int i0 = gw * 32 + ig * 8;  // first key dim of this thread's chunk
+    const int tg = lane >> 1, ig = lane & 1;
+    const int i0 = gw * 16 + ig * 8;  // first key dim of this thread's chunk
+    const int sw = tg & 2;            // step k visits row 4tg + (k ^ sw)
     float *ec = reinterpret_cast<float *>(smem + C::off_ec);
     float logG[8];  // running sum of the chunk totals: log-decay from the segment start
 #pragma unroll
@@ -198,40 +247,48 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
         const int s = c % C::stages;
         if (!mbar_wait(&b.full[s], (c / C::stages) & 1, abort)) break;
         uint8_t *st = smem + s * C::stage_bytes;
-        // local inclusive cumsum down rows 8tg .. 8tg+7
-        float bt[8][8];
+        // bk[k]: inclusive cumsum, from the group's first row, of the row visited at step k
+        float bk[4][8], tot[8];
         {
-            uint4 graw[8];
+            uint4 graw[4];
 #pragma unroll
-            for (int r = 0; r < 8; ++r)
-                graw[r] = *reinterpret_cast<const uint4 *>(st + C::off_g + tile_off(tg * 8 + r, i0));
+            for (int k = 0; k < 4; ++k)
+                graw[k] = *reinterpret_cast<const uint4 *>(st + C::off_g + tile_off(tg * 4 + (k ^ sw), i0));
+            float f[4][8];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                float f[8];
-                unpack8(graw[r], f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) bt[r][e] = (r ? bt[r - 1][e] : 0.f) + f[e];
-            }
-        }
-        // inclusive scan of the group totals across tg (lanes ig, ig+4, ..., ig+28)
-        float incl[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) incl[e] = bt[7][e];
-#pragma unroll
-        for (int d = 1; d < 8; d <<= 1) {
+            for (int k = 0; k < 4; ++k) unpack8(graw[k], f[k]);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float up = __shfl_up_sync(0xFFFFFFFFu, incl[e], 4 * d);
+                // steps (0,1) and (2,3) each visit one row pair in order; the pair visited
+                // first (rows 4tg, 4tg+1) is at steps 0,1 when sw == 0, at steps 2,3 otherwise
+                const float p01 = f[0][e] + f[1][e], p23 = f[2][e] + f[3][e];
+                const float o01 = sw ? p23 : 0.f, o23 = sw ? 0.f : p01;
+                bk[0][e] = f[0][e] + o01;
+                bk[1][e] = p01 + o01;
+                bk[2][e] = f[2][e] + o23;
+                bk[3][e] = p23 + o23;
+                tot[e] = p01 + p23;
+            }
+        }
+        // inclusive scan of the group totals across tg (lanes ig, ig+2, ..., ig+30)
+        float incl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) incl[e] = tot[e];
+#pragma unroll
+        for (int d = 1; d < 16; d <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float up = __shfl_up_sync(0xFFFFFFFFu, incl[e], 2 * d);
                 if (tg >= d) incl[e] += up;
             }
         }
         float bC[8], nbCl[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            bC[e] = __shfl_sync(0xFFFFFFFFu, incl[e], 28 + ig);
-            const float off = incl[e] - bt[7][e];  // exclusive prefix of this token group
+            bC[e] = __shfl_sync(0xFFFFFFFFu, incl[e], 30 + ig);
+            const float off = incl[e] - tot[e];  // exclusive prefix of this token group
 #pragma unroll
-            for (int r = 0; r < 8; ++r) bt[r][e] += off;
+            for (int k = 0; k < 4; ++k) bk[k][e] += off;
             // exponent offset of q's factor: e^{b_t - b_C}, or e^{B_start + b_t} for Qhat
             nbCl[e] = (C::dstate ? logG[e] : -bC[e]) * kLog2e;
             range_bad |= !(fabsf(bC[e]) <= kGateRangeLimit);
@@ -245,22 +302,22 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) logG[e] += bC[e];
-        // rescale q (by e^{b_t - b_C}) and k (by e^{b_C - b_t}) in place, 4 rows per batch
+        // rescale q (by e^{b_t - b_C}) and k (by e^{b_C - b_t}) in place, 2 rows per batch
 #pragma unroll
-        for (int r0 = 0; r0 < 8; r0 += 4) {
-            uint4 qr[4], kr[4];
+        for (int k0 = 0; k0 < 4; k0 += 2) {
+            uint4 qr[2], kr[2];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t off = tile_off(tg * 4 + ((k0 + r) ^ sw), i0);
                 if (C::q) qr[r] = *reinterpret_cast<const uint4 *>(st + C::off_q + off);
                 if (C::k) kr[r] = *reinterpret_cast<const uint4 *>(st + C::off_k + off);
             }
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t off = tile_off(tg * 4 + ((k0 + r) ^ sw), i0);
                 float x[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = fmaf(bt[r0 + r][e], kLog2e, nbCl[e]);
+                for (int e = 0; e < 8; ++e) x[e] = fmaf(bk[k0 + r][e], kLog2e, nbCl[e]);
                 if (C::q) {
                     float f[8];
                     unpack8(qr[r], f);
@@ -297,9 +354,9 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 
 // ------------------------------------------------------------------ state warps (0-3)
 // Thread dv (= TMEM lane) owns row dv of the transposed fp32 state S^T, which lives in TMEM.
-// Per chunk it scales the row by the chunk's decay (S' = diag(e^{b_C}) S), stores S' back
+// Per chunk c it scales the row by the chunk's decay (S' = diag(e^{b_C}) S), stores S' back
 // for the MMA to accumulate the chunk's increment onto, and (output modes) stores the bf16
-// copy that is the A operand of O^T += S'^T Qbar'^T.
+// copy into S'^T buffer c % 2, the A operand of O^T += S'^T Qbar'^T.
 template <int MODE>
 __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
                            uint32_t tmem, int bh, int j, int nchunks) {
@@ -308,15 +365,15 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
     const int dv = warp * 32 + lane;
     const uint32_t lrow = (uint32_t)(warp * 32) << 16;
     const float *ec = reinterpret_cast<const float *>(smem + C::off_ec);
-    uint32_t r0[32], r1[32];
+    uint32_t r[32];
     if (!C::dstate) {  // initial state: the received state (output / correction passes) or zero
         const float *Si = (C::init_state && a.S_init)
                               ? a.S_init + ((long long)bh * a.NP + j) * D * D + dv : nullptr;
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r0[e] = __float_as_uint(Si ? Si[(p * 32 + e) * D] : 0.f);
-            tmem_st32(tmem + lrow + kColDS + p * 32, r0);
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(Si ? Si[(p * 32 + e) * D] : 0.f);
+            tmem_st32(tmem + lrow + kColDS + p * 32, r);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -326,39 +383,32 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
         if (!mbar_wait(&b.gated[s], (c / C::stages) & 1, abort)) break;
         if (!C::dstate) {
             if (C::kv && c > 0 && !mbar_wait(b.ds_full, (c - 1) & 1, abort)) break;
-            if (C::out && c > 0 && !mbar_wait(b.sa_free, (c - 1) & 1, abort)) break;
+            if (C::out && c >= 2 && !mbar_wait(&b.sa_free[c & 1], ((c >> 1) - 1) & 1, abort)) break;
             tc_fence_after();
             const float *e_s = ec + s * D;
+            const uint32_t sa = tmem + lrow + kColSA + (c & 1) * 64;
 #pragma unroll
-            for (int p2 = 0; p2 < 2; ++p2) {
-                tmem_ld32(tmem + lrow + kColDS + p2 * 64, r0);
-                tmem_ld32(tmem + lrow + kColDS + p2 * 64 + 32, r1);
+            for (int p = 0; p < 4; ++p) {  // key dims 32p .. 32p+31
+                tmem_ld32(tmem + lrow + kColDS + p * 32, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 f0 = *reinterpret_cast<const float4 *>(e_s + p2 * 64 + 4 * e4);
-                    const float4 f1 = *reinterpret_cast<const float4 *>(e_s + p2 * 64 + 32 + 4 * e4);
-                    r0[4 * e4 + 0] = __float_as_uint(__uint_as_float(r0[4 * e4 + 0]) * f0.x);
-                    r0[4 * e4 + 1] = __float_as_uint(__uint_as_float(r0[4 * e4 + 1]) * f0.y);
-                    r0[4 * e4 + 2] = __float_as_uint(__uint_as_float(r0[4 * e4 + 2]) * f0.z);
-                    r0[4 * e4 + 3] = __float_as_uint(__uint_as_float(r0[4 * e4 + 3]) * f0.w);
-                    r1[4 * e4 + 0] = __float_as_uint(__uint_as_float(r1[4 * e4 + 0]) * f1.x);
-                    r1[4 * e4 + 1] = __float_as_uint(__uint_as_float(r1[4 * e4 + 1]) * f1.y);
-                    r1[4 * e4 + 2] = __float_as_uint(__uint_as_float(r1[4 * e4 + 2]) * f1.z);
-                    r1[4 * e4 + 3] = __float_as_uint(__uint_as_float(r1[4 * e4 + 3]) * f1.w);
+                    const ulonglong2 f = *reinterpret_cast<const ulonglong2 *>(e_s + p * 32 + 4 * e4);
+                    const uint64_t x0 = mul_f32x2(((uint64_t)r[4 * e4 + 1] << 32) | r[4 * e4], f.x);
+                    const uint64_t x1 = mul_f32x2(((uint64_t)r[4 * e4 + 3] << 32) | r[4 * e4 + 2], f.y);
+                    r[4 * e4 + 0] = (uint32_t)x0;
+                    r[4 * e4 + 1] = (uint32_t)(x0 >> 32);
+                    r[4 * e4 + 2] = (uint32_t)x1;
+                    r[4 * e4 + 3] = (uint32_t)(x1 >> 32);
                 }
-                if (C::kv || C::out) {  // the correction pass keeps the decayed received state
-                    tmem_st32(tmem + lrow + kColDS + p2 * 64, r0);
-                    tmem_st32(tmem + lrow + kColDS + p2 * 64 + 32, r1);
-                }
+                // the correction pass keeps the decayed received state
+                if (C::kv || C::out) tmem_st32(tmem + lrow + kColDS + p * 32, r);
                 if (C::out) {
-                    uint32_t pk[32];
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        pk[e] = pack_bf16(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
-                        pk[16 + e] = pack_bf16(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
-                    }
-                    tmem_st32(tmem + lrow + kColSA + p2 * 32, pk);
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+                    tmem_st16(sa + p * 16, pk);
                 }
             }
             tmem_wait_st();
@@ -377,10 +427,10 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
             float *So = a.S_out + ((long long)bh * a.NP + j) * D * D + dv;
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-                tmem_ld32(tmem + lrow + kColDS + p * 32, r0);
+                tmem_ld32(tmem + lrow + kColDS + p * 32, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) So[(p * 32 + e) * D] = __uint_as_float(r0[e]);
+                for (int e = 0; e < 32; ++e) So[(p * 32 + e) * D] = __uint_as_float(r[e]);
             }
             tc_fence_before();
         }
@@ -388,7 +438,9 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
 }
 
 // ------------------------------------------------------------------ output warps (4-7)
-// (a) the intra-chunk scores -> causal mask -> bf16 P tile; (d) the chunk's outputs.
+// (a) the intra-chunk scores -> causal mask -> bf16 P tile (buffer c % 2); (d) the chunk's
+// outputs from O^T buffer c % 2.  The scores of chunk c+1 are turned into P before the
+// outputs of chunk c are read, since the tensor cores wait for P and not for the read-out.
 template <int MODE>
 __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
                          uint32_t tmem, long long row0, int nchunks) {
@@ -399,51 +451,56 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
     const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
     uint32_t r[32];
-    for (int c = 0; c < nchunks; ++c) {
-        if (C::qk) {  // M=64 accumulator: lanes 0-15 of each quarter hold rows 16 quarter + lane
-            if (!mbar_wait(b.qk_full, c & 1, abort)) break;
-            tc_fence_after();
-            const int t = quarter * 16 + lane;
-            uint8_t *prow = smem + C::off_p + t * 128;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                tmem_ld32(tmem + lrow + kColQK + h * 32, r);
-                tmem_wait_ld();
-                if (h == 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(b.qk_free);
-                }
-                if (lane < 16) {
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int sl = jj * 8 + 2 * e, s0 = h * 32 + sl;
-                            w4[e] = pack_bf16(s0 <= t ? __uint_as_float(r[sl]) : 0.f,
-                                              s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f);
-                        }
-                        *reinterpret_cast<uint4 *>(prow + (((h * 4 + jj) ^ (t & 7)) << 4)) =
-                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b.p_full);
-        }
-        // (d) outputs: column dv of the chunk's 64 rows
-        if (!mbar_wait(b.o_full, c & 1, abort)) break;
+    // M=64 accumulator: lanes 0-15 of each quarter hold rows 16 quarter + lane
+    auto make_p = [&](int c) -> bool {
+        if (!mbar_wait(b.qk_full, c & 1, abort)) return false;
         tc_fence_after();
+        const int t = quarter * 16 + lane, pb = c & 1;
+        uint8_t *prow = smem + C::off_p + pb * (CH * CH * 2) + t * 128;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            tmem_ld32(tmem + lrow + kColO + h * 32, r);
+            tmem_ld32(tmem + lrow + kColQK + h * 32, r);
             tmem_wait_ld();
             if (h == 1) {
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(b.o_free);
+                if (lane == 0) mbar_arrive(b.qk_free);
+            }
+            if (lane < 16) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int sl = jj * 8 + 2 * e, s0 = h * 32 + sl;
+                        w4[e] = pack_bf16(s0 <= t ? __uint_as_float(r[sl]) : 0.f,
+                                          s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f);
+                    }
+                    *reinterpret_cast<uint4 *>(prow + (((h * 4 + jj) ^ (t & 7)) << 4)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.p_full[pb]);
+        return true;
+    };
+    if (C::qk && nchunks > 0 && !make_p(0)) return;
+    for (int c = 0; c < nchunks; ++c) {
+        if (C::qk && c + 1 < nchunks && !make_p(c + 1)) break;
+        // (d) outputs: column dv of the chunk's 64 rows
+        const int ob = c & 1;
+        if (!mbar_wait(&b.o_full[ob], (c >> 1) & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            tmem_ld32(tmem + lrow + kColO + ob * 64 + h * 32, r);
+            tmem_wait_ld();
+            if (h == 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&b.o_free[ob]);
             }
             __nv_bfloat16 *orow = o + (row0 + (long long)c * CH + h * 32) * D + dv;
             if (MODE == kPassCorrect) {  // o_local: all loads before the first store
@@ -475,8 +532,8 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     b.gated = bar + C::stages;
     b.empty = bar + 2 * C::stages;
     uint64_t *x = bar + 3 * C::stages;
-    b.qk_full = x + 0; b.qk_free = x + 1; b.p_full = x + 2; b.ds_full = x + 3; b.ds_free = x + 4;
-    b.sa_full = x + 5; b.sa_free = x + 6; b.o_full = x + 7; b.o_free = x + 8; b.fin = x + 9;
+    b.qk_full = x + 0; b.qk_free = x + 1; b.p_full = x + 2; b.ds_full = x + 4; b.sa_full = x + 5;
+    b.sa_free = x + 6; b.o_full = x + 8; b.o_free = x + 10; b.fin = x + 12;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::off_misc + 4);
 
@@ -493,13 +550,14 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         mbar_init(b.qk_full, 1);
         mbar_init(b.qk_free, kOutWarps);
-        mbar_init(b.p_full, kOutWarps);
         mbar_init(b.ds_full, 1);
-        mbar_init(b.ds_free, 1);
         mbar_init(b.sa_full, kStateWarps);
-        mbar_init(b.sa_free, 1);
-        mbar_init(b.o_full, 1);
-        mbar_init(b.o_free, kOutWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&b.p_full[i], kOutWarps);
+            mbar_init(&b.sa_free[i], 1);
+            mbar_init(&b.o_full[i], 1);
+            mbar_init(&b.o_free[i], kOutWarps);
+        }
         mbar_init(b.fin, 1);
         *abort = 0;
         mbar_fence_init();
@@ -519,7 +577,7 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp == kTmaWarp) {
         if (lane == 0) producer<MODE>(smem, b, abort, &tm_q, &tm_k, &tm_v, &tm_g, row0, nchunks);
     } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_issuer<MODE>(smem, b, abort, tmem, nchunks);
+        mma_issuer<MODE>(smem, b, abort, tmem, nchunks);
     } else if (warp >= kEpiWarps) {
         gate_role<MODE>(smem, b, abort, a, bh, j, nchunks);
     } else if (warp < kStateWarps) {
