@@ -85,39 +85,52 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
     const uint32_t m_addr = smem_u32(smem + off_m);
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % kStages;
-        if (!mbar_wait(&b.gated[s], (c / kStages) & 1, abort)) break;
+        if (!warp_wait(&b.gated[s], (c / kStages) & 1, abort)) break;
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * kStageBytes);
         const uint32_t ka = st + off_k, va = st + off_v, da = st + off_do;
-        if (c > 0 && !mbar_wait(b.m_free, (c - 1) & 1, abort)) break;
+        if (c > 0 && !warp_wait(b.m_free, (c - 1) & 1, abort)) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // M = dO V^T
-            mma_ss(tmem + kColM, desc_kmajor(da, kk), desc_kmajor(va, kk), i_m, kk > 0);
-        mma_commit(b.m_full);
-        if (c > 0 && !mbar_wait(b.ds_free, (c - 1) & 1, abort)) break;
+            for (int kk = 0; kk < 8; ++kk)  // M = dO V^T
+                mma_ss(tmem + kColM, desc_kmajor(da, kk), desc_kmajor(va, kk), i_m, kk > 0);
+            mma_commit(b.m_full);
+        }
+        __syncwarp();
+        if (c > 0 && !warp_wait(b.ds_free, (c - 1) & 1, abort)) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // dS = Ktil^T V
-            mma_ss(tmem + kColDS, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), i_ds, kk > 0);
-        mma_commit(b.ds_full);
-        if (c > 0 && !mbar_wait(b.dq_free, (c - 1) & 1, abort)) break;
-        if (!mbar_wait(b.p_full, c & 1, abort)) break;
+            for (int kk = 0; kk < 4; ++kk)  // dS = Ktil^T V
+                mma_ss(tmem + kColDS, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), i_ds, kk > 0);
+            mma_commit(b.ds_full);
+        }
+        __syncwarp();
+        if (c > 0 && !warp_wait(b.dq_free, (c - 1) & 1, abort)) break;
+        if (!warp_wait(b.p_full, c & 1, abort)) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // dq^T = Ktil^T M^T
-            mma_ss(tmem + kColDQ, desc_mnmajor(ka, kk), smem_desc_sw128(m_addr + kk * 32, 16, 1024),
-                   i_dqb, kk > 0);
-        if (!mbar_wait(b.sa_full, c & 1, abort)) break;
+            for (int kk = 0; kk < 4; ++kk)  // dq^T = Ktil^T M^T
+                mma_ss(tmem + kColDQ, desc_mnmajor(ka, kk), smem_desc_sw128(m_addr + kk * 32, 16, 1024),
+                       i_dqb, kk > 0);
+        }
+        __syncwarp();
+        if (!warp_wait(b.sa_full, c & 1, abort)) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dq^T += S' dO^T, A from tensor memory
-            mma_ts(tmem + kColDQ, tmem + kColSA + kk * 8, desc_kmajor(da, kk), i_dqa, 1u);
-        mma_commit(b.dq_full);
-        mma_commit(b.sa_free);
-        mma_commit(&b.empty[s]);
+            for (int kk = 0; kk < 8; ++kk)  // dq^T += S' dO^T, A from tensor memory
+                mma_ts(tmem + kColDQ, tmem + kColSA + kk * 8, desc_kmajor(da, kk), i_dqa, 1u);
+            mma_commit(b.dq_full);
+            mma_commit(b.sa_free);
+            mma_commit(&b.empty[s]);
+        }
+        __syncwarp();
     }
-    mma_commit(b.fin);
+    if (elect_one()) mma_commit(b.fin);
+    __syncwarp();
     wait_drain(b.fin, 0);
 }
 
@@ -378,7 +391,7 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (warp == kTmaWarp) {
         if (lane == 0) producer(smem, b, abort, &tm_k, &tm_v, &tm_do, &tm_g, &tm_q, row0, nchunks);
     } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_issuer(smem, b, abort, tmem, nchunks);
+        mma_issuer(smem, b, abort, tmem, nchunks);
     } else if (warp >= kEpiWarps) {
         gate_role(smem, b, abort, a, nchunks);
     } else {
@@ -399,39 +412,43 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 // Per chunk, last to first, with dS the gradient of the state at the chunk's end (rows = key
 // dims; starts at dX of the part), Qbar'_t = q_t e^{b_t - b_C}, Ktil_s = k_s e^{b_C - b_s}:
 //
-//   M     = dO V^T,  A = Qbar' Ktil^T   M=64 (t) N=64 (s) K=128          -> masked s <= t, bf16
+//   M     = dO V^T,  A = Qbar' Ktil^T   M=64  (t) N=64 (s) K=128          -> masked s <= t, bf16
 //   dk^T  = Qbar'^T M + dS V^T          M=128 (i) N=64 (s) K=64 (t) / 128 (j)
-//   dv    = A^T dO + Ktil dS            M=64 (s) N=128 (j) K=64 (t) / 128 (i)
+//   dv^T  = dO^T A + dS^T Ktil^T        M=128 (j) N=64 (s) K=64 (t) / 128 (i)
 //   dS   += Qbar'^T dO                  M=128 (i) N=128 (j) K=64 (t), accumulated in TMEM
 //   dk[s,i] = e^{b_C,i - b_s,i} dk^T[i,s];   dS <- diag(e^{b_C}) dS
 //   dlog_g_s = rowsum(S_end . dX) + sum_{u >= s in the part} (q_u dq_u - k_u dk_u)
 //
-// The fp32 dS lives in tensor memory (the MMA accumulates Qbar'^T dO onto it; the epilogue
-// applies the decay); its bf16 copy lives in one shared tile ([i][j] rows, 128-byte swizzle)
-// read as the K-major A operand of dS V^T and as the MN-major B operand of Ktil dS.
+// Roles (448 threads): warps 0-3 carry dS -- the fp32 dS lives in tensor memory (row i on lane
+// i), they apply the decay, write its bf16 copy into a shared [i][j] tile (read by the MMAs as
+// the K-major A operand of dS V^T and the MN-major A operand of dS^T Ktil^T) and turn M and A
+// into masked bf16 tiles (double-buffered); warps 4-7 read dk^T and dv^T (double-buffered in
+// TMEM; thread x owns key / value dim x for all 64 tokens of the chunk, so the dlog_g suffix
+// sums need no exchange), stage dk, dlog_g and dv in the stage's v, q and dO tiles (free by then)
+// and write them with TMA stores; warps 8-11 gates; 12 TMA; 13 MMA.
 namespace dkv {
 
-constexpr uint32_t kColM = 0, kColA = 64, kColDK = 128, kColDV = 192, kColDS = 320;
+constexpr int kStateWarps = 4, kOutWarps = 4;
+constexpr uint32_t kColM = 0, kColA = 64, kColDK = 128, kColDV = 256, kColDS = 384;
 constexpr int kStages = 2;
 constexpr int off_q = 0, off_k = kTileBytes, off_v = 2 * kTileBytes, off_do = 3 * kTileBytes,
               off_g = 4 * kTileBytes;
 constexpr int kStageBytes = 5 * kTileBytes;
-constexpr int kDsHalf = 128 * 128;  // one 64-column half of the [128 x 128] bf16 dS tile
-constexpr int off_m = kStages * kStageBytes;
-constexpr int off_a = off_m + CH * CH * 2;
-constexpr int off_ds = off_a + CH * CH * 2;
+constexpr int kDsHalf = 128 * 128;            // one 64-column half of the [128 x 128] bf16 dS tile
+constexpr int kMaskBytes = CH * CH * 2;       // one masked 64 x 64 bf16 tile
+constexpr int off_ma = kStages * kStageBytes;  // 2 buffers x (M tile, A tile)
+constexpr int off_ds = off_ma + 4 * kMaskBytes;
 constexpr int off_ec = off_ds + 2 * kDsHalf;
-constexpr int off_x = off_ec + kStages * D * 4;  // half-row exchange between the two epilogue halves
-constexpr int off_bar = off_x + 4 * D * 4;
-constexpr int kBars = 3 * kStages + 16;
+constexpr int off_bar = off_ec + kStages * D * 4;
+constexpr int kBars = 3 * kStages + 15;
 constexpr int off_misc = off_bar + kBars * 8;
 constexpr int kSmemBytes = off_misc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Bars {
     uint64_t *full, *gated, *empty;
-    uint64_t *mm_full, *mm_free, *aa_full, *aa_free, *p_full, *dst_full, *dk_full, *dk_free,
-        *dv_full, *dv_free, *dsn_full, *dsn_free, *xchg, *fin;
+    uint64_t *mm_full, *mm_free, *p_full, *dst_full, *dk_full, *dk_free, *dv_full, *dv_free,
+        *dsn_full, *osync, *fin;
 };
 
 // [128 rows][128 cols] bf16 tile as two 64-column halves of 16 KiB, 128-byte swizzle.
@@ -442,11 +459,13 @@ __device__ __forceinline__ uint32_t ds_off(int row, int col) {
 
 __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tq,
                          const CUtensorMap *tk, const CUtensorMap *tv, const CUtensorMap *tdo,
-                         const CUtensorMap *tg, long long row0, int nchunks) {
+                         const CUtensorMap *tg, const float *qdq, long long row0, int nchunks) {
     int issued = 0;
     for (int it = 0; it < nchunks; ++it) {
         const int s = it % kStages;
         const int c = nchunks - 1 - it;  // last chunk first
+        // the chunk's q . dq rows (read with plain loads by the output warps) on their way to L2
+        bulk_prefetch_l2(qdq + (row0 + (long long)c * CH) * D, CH * D * 4);
         if (it >= kStages && !mbar_wait(&b.empty[s], ((it / kStages) - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&b.full[s], kStageBytes);
         uint8_t *st = smem + s * kStageBytes;
@@ -468,69 +487,86 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
             wait_drain(&b.full[it % kStages], (it / kStages) & 1);
 }
 
+// The whole warp walks the loop; one elected lane issues.  Per chunk: dk^T and dv^T into
+// buffer it % 2 after the dS update (so that dk_full also frees the q tile), then the next
+// chunk's M and A (so that they are ready when the dS warps finish the decay).
 __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
                            int nchunks) {
     constexpr uint32_t i_sq = idesc_bf16_f32(64, 64, 0, 0);      // M, A
     constexpr uint32_t i_dsn = idesc_bf16_f32(128, 128, 1, 1);   // Qbar'^T dO
     constexpr uint32_t i_dka = idesc_bf16_f32(128, 64, 1, 1);    // Qbar'^T M
     constexpr uint32_t i_dkb = idesc_bf16_f32(128, 64, 0, 0);    // dS V^T
-    constexpr uint32_t i_dva = idesc_bf16_f32(64, 128, 1, 1);    // A^T dO
-    constexpr uint32_t i_dvb = idesc_bf16_f32(64, 128, 0, 1);    // Ktil dS
-    const uint32_t m_addr = smem_u32(smem + off_m), a_addr = smem_u32(smem + off_a);
-    const uint32_t ds_addr = smem_u32(smem + off_ds);
-    for (int it = 0; it < nchunks; ++it) {
-        const int s = it % kStages;
-        if (!mbar_wait(&b.gated[s], (it / kStages) & 1, abort)) break;
-        tc_fence_after();
-        const uint32_t st = smem_u32(smem + s * kStageBytes);
+    constexpr uint32_t i_dva = idesc_bf16_f32(128, 64, 1, 1);    // dO^T A
+    constexpr uint32_t i_dvb = idesc_bf16_f32(128, 64, 1, 0);    // dS^T Ktil^T
+    const uint32_t base = smem_u32(smem);
+    const uint32_t ma_addr = base + off_ma, ds_addr = base + off_ds;
+    auto stage = [&](int it) { return base + (uint32_t)((it % kStages) * kStageBytes); };
+    auto issue_ma = [&](int it) {
+        const uint32_t st = stage(it);
+        if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // M = dO V^T
+                mma_ss(tmem + kColM, desc_kmajor(st + off_do, kk), desc_kmajor(st + off_v, kk), i_sq,
+                       kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // A = Qbar' Ktil^T
+                mma_ss(tmem + kColA, desc_kmajor(st + off_q, kk), desc_kmajor(st + off_k, kk), i_sq,
+                       kk > 0);
+            mma_commit(b.mm_full);
+        }
+        __syncwarp();
+    };
+    bool ok = nchunks > 0 && warp_wait(&b.gated[0], 0, abort);
+    tc_fence_after();
+    if (ok) issue_ma(0);
+    for (int it = 0; ok && it < nchunks; ++it) {
+        const int s = it % kStages, bb = it & 1;
+        const uint32_t st = stage(it);
         const uint32_t qa = st + off_q, ka = st + off_k, va = st + off_v, da = st + off_do;
-        const uint32_t pf = (it - 1) & 1;  // phase of the previous chunk's "free" barriers
-        if (it > 0 && !mbar_wait(b.mm_free, pf, abort)) break;
+        const uint32_t mt = ma_addr + bb * 2 * kMaskBytes, at = mt + kMaskBytes;
+        if (!(ok = warp_wait(b.p_full, it & 1, abort))) break;
+        if (!(ok = warp_wait(b.dst_full, it & 1, abort))) break;
+        if (it >= 2) {
+            if (!(ok = warp_wait(&b.dk_free[bb], ((it >> 1) - 1) & 1, abort))) break;
+            if (!(ok = warp_wait(&b.dv_free[bb], ((it >> 1) - 1) & 1, abort))) break;
+        }
         tc_fence_after();
+        if (elect_one()) {
+            const uint32_t dk_col = tmem + kColDK + bb * 64, dv_col = tmem + kColDV + bb * 64;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // M = dO V^T
-            mma_ss(tmem + kColM, desc_kmajor(da, kk), desc_kmajor(va, kk), i_sq, kk > 0);
-        mma_commit(b.mm_full);
-        if (it > 0 && !mbar_wait(b.aa_free, pf, abort)) break;
-        tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)  // dS += Qbar'^T dO  (dk and dv read the old dS tile)
+                mma_ss(tmem + kColDS, desc_mnmajor(qa, kk), desc_mnmajor(da, kk), i_dsn, 1u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // A = Qbar' Ktil^T
-            mma_ss(tmem + kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), i_sq, kk > 0);
-        mma_commit(b.aa_full);
-        if (!mbar_wait(b.p_full, it & 1, abort)) break;
-        if (!mbar_wait(b.dst_full, it & 1, abort)) break;
-        if (it > 0 && !mbar_wait(b.dk_free, pf, abort)) break;
-        tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)  // dk^T = Qbar'^T M   (B: M tile read MN-major)
+                mma_ss(dk_col, desc_mnmajor(qa, kk), smem_desc_sw128(mt + kk * 2048, kHalfBytes, 1024),
+                       i_dka, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // dk^T = Qbar'^T M   (B: M tile read MN-major)
-            mma_ss(tmem + kColDK, desc_mnmajor(qa, kk), smem_desc_sw128(m_addr + kk * 2048, kHalfBytes, 1024),
-                   i_dka, kk > 0);
+            for (int kk = 0; kk < 8; ++kk)  // dk^T += dS V^T   (A: dS tile K-major, 128 rows)
+                mma_ss(dk_col, smem_desc_sw128(ds_addr + (kk >> 2) * kDsHalf + (kk & 3) * 32, 16, 1024),
+                       desc_kmajor(va, kk), i_dkb, 1u);
+            mma_commit(&b.dk_full[bb]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dk^T += dS V^T   (A: dS tile K-major, 128 rows)
-            mma_ss(tmem + kColDK,
-                   smem_desc_sw128(ds_addr + (kk >> 2) * kDsHalf + (kk & 3) * 32, 16, 1024),
-                   desc_kmajor(va, kk), i_dkb, 1u);
-        mma_commit(b.dk_full);
-        if (it > 0 && !mbar_wait(b.dv_free, pf, abort)) break;
-        tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)  // dv^T = dO^T A   (B: A tile read MN-major)
+                mma_ss(dv_col, desc_mnmajor(da, kk), smem_desc_sw128(at + kk * 2048, kHalfBytes, 1024),
+                       i_dva, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // dv = A^T dO   (A: A tile read MN-major)
-            mma_ss(tmem + kColDV, smem_desc_sw128(a_addr + kk * 2048, kHalfBytes, 1024),
-                   desc_mnmajor(da, kk), i_dva, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dv += Ktil dS   (B: dS tile MN-major)
-            mma_ss(tmem + kColDV, desc_kmajor(ka, kk),
-                   smem_desc_sw128(ds_addr + kk * 2048, kDsHalf, 1024), i_dvb, 1u);
-        mma_commit(b.dv_full);
-        if (it > 0 && !mbar_wait(b.dsn_free, pf, abort)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // dS += Qbar'^T dO  (after dk and dv read the old dS)
-            mma_ss(tmem + kColDS, desc_mnmajor(qa, kk), desc_mnmajor(da, kk), i_dsn, 1u);
-        mma_commit(b.dsn_full);
-        mma_commit(&b.empty[s]);
+            for (int kk = 0; kk < 8; ++kk)  // dv^T += dS^T Ktil^T   (A: dS tile read MN-major)
+                mma_ss(dv_col, smem_desc_sw128(ds_addr + kk * 2048, kDsHalf, 1024), desc_kmajor(ka, kk),
+                       i_dvb, 1u);
+            mma_commit(&b.dv_full[bb]);
+            mma_commit(b.dsn_full);  // the dS tile is read out as well
+            mma_commit(&b.empty[s]);
+        }
+        __syncwarp();
+        if (it + 1 < nchunks) {  // the next chunk's M and A, once its tiles are gated
+            if (!(ok = warp_wait(&b.gated[(it + 1) % kStages], ((it + 1) / kStages) & 1, abort))) break;
+            if (!(ok = warp_wait(b.mm_free, it & 1, abort))) break;
+            tc_fence_after();
+            issue_ma(it + 1);
+        }
     }
-    mma_commit(b.fin);
+    if (elect_one()) mma_commit(b.fin);
+    __syncwarp();
     wait_drain(b.fin, 0);
 }
 
@@ -649,34 +685,130 @@ __device__ __forceinline__ void masked_tile(uint8_t *tile, const uint32_t (&r)[3
     }
 }
 
-// Exchange point of the 8 epilogue warps (bounded like every other wait): returns false when
-// the CTA is aborting.
-__device__ __forceinline__ bool epi_exchange(const Bars &b, volatile int *abort, int k, int lane) {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(b.xchg);
-    return mbar_wait(b.xchg, k & 1, abort);
+// Warps 0-3: thread i owns row i of dS (TMEM lane i).  Per chunk: the decay by the previous
+// chunk's e^{b_C} (S_new = diag(e^{b_C}) (dS + Qbar'^T dO), the sum formed by the MMA), the
+// bf16 copy of row i into the dS tile, then the masked M and A tiles of the chunk.
+__device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
+                           uint32_t tmem, int bh, int j, int nchunks) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = warp * 32 + lane;
+    const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+    const float *ec = reinterpret_cast<const float *>(smem + off_ec);
+    uint32_t r[32];
+    {  // dS at the part's end: dX
+        const float4 *x4 = reinterpret_cast<const float4 *>(a.dX + ((long long)bh * a.NP + j) * D * D +
+                                                            (long long)i * D);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 v = x4[p * 8 + e4];
+                r[4 * e4] = __float_as_uint(v.x); r[4 * e4 + 1] = __float_as_uint(v.y);
+                r[4 * e4 + 2] = __float_as_uint(v.z); r[4 * e4 + 3] = __float_as_uint(v.w);
+            }
+            tmem_st32(tmem + lrow + kColDS + p * 32, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+    }
+    for (int it = 0; it < nchunks; ++it) {
+        // (1) dS of this chunk's end: decayed unless it is the part's end
+        if (it > 0) {
+            if (!mbar_wait(b.dsn_full, (it - 1) & 1, abort)) break;
+        }
+        tc_fence_after();
+        const uint64_t e2 = it > 0 ? (uint64_t)__float_as_uint(ec[((it - 1) % kStages) * D + i]) * 0x100000001ull
+                                   : 0ull;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            tmem_ld32(tmem + lrow + kColDS + p * 32, r);
+            tmem_wait_ld();
+            if (it > 0) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const uint64_t x = mul_f32x2(((uint64_t)r[2 * e + 1] << 32) | r[2 * e], e2);
+                    r[2 * e] = (uint32_t)x;
+                    r[2 * e + 1] = (uint32_t)(x >> 32);
+                }
+                tmem_st32(tmem + lrow + kColDS + p * 32, r);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint32_t *x = r + jj * 8;
+                *reinterpret_cast<uint4 *>(smem + off_ds + ds_off(i, p * 32 + jj * 8)) =
+                    make_uint4(pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                               pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
+                               pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
+                               pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
+            }
+        }
+        if (it > 0) tmem_wait_st();
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(b.dst_full);
+            if (it > 0) mbar_arrive(&b.empty[(it - 1) % kStages]);  // its e^{b_C} is used
+        }
+        // (2) masked M and A tiles of this chunk (M=64 layout: lanes 0-15 hold row 16 warp + lane)
+        if (!mbar_wait(b.mm_full, it & 1, abort)) break;
+        tc_fence_after();
+        uint8_t *mt = smem + off_ma + (it & 1) * 2 * kMaskBytes;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {  // M half 0, M half 1, A half 0, A half 1
+            tmem_ld32(tmem + lrow + (t < 2 ? kColM : kColA) + (t & 1) * 32, r);
+            tmem_wait_ld();
+            if (t == 3) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b.mm_free);
+            }
+            masked_tile(mt + (t >> 1) * kMaskBytes, r, warp, t & 1, lane);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.p_full);
+    }
 }
 
-// Epilogue warps: thread (w, lane) owns key dim i = 32 (w % 4) + lane and value dims
-// 64h .. 64h+63 (h = w / 4) of the running state gradient dS, and tokens 32h .. 32h+31 of
-// each chunk for dk and dlog_g; for dv (M=64 accumulator) lanes 0-15 own token 16 (w % 4) + lane.
-__device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
-                              uint32_t tmem, int bh, int j, long long row0, int nchunks) {
-    constexpr int HD = D / 2;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quarter = warp & 3, h = warp >> 2;
-    const int i = quarter * 32 + lane;
-    const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
-    const float *ec = reinterpret_cast<const float *>(smem + off_ec);
-    float *xb = reinterpret_cast<float *>(smem + off_x);  // [2 sets][2 halves][128]
-    __nv_bfloat16 *dk = static_cast<__nv_bfloat16 *>(a.dk_out);
-    __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv_out);
-    __nv_bfloat16 *dg = static_cast<__nv_bfloat16 *>(a.dg_out);
-    const long long sidx = ((long long)bh * a.NP + j) * D * D;
+// Stores the bf16 values of tokens s and s+1 of this lane's dim x into a [64 x 128] swizzled
+// tile.  Lanes x and x^1 swap one value so that each writes one 4-byte word (dims x & ~1 and
+// x | 1): the even lane row s, the odd lane row s+1.  Two-byte stores would put two lanes on
+// each 4-byte word and take two shared-memory wavefronts per instruction.
+// The shared-memory accesses of the output warps are explicit instructions in program order;
+// they carry no compiler memory clobber, so the compiler may schedule other work around them.
+// Their buffers are disjoint: factors and Ktil are read from the g and k tiles, outputs go to
+// the v, q and dO tiles, which no MMA reads any more.
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
+}
 
-    // dS (gradient of the state at the current chunk's end) lives in TMEM: row i, columns
-    // 64h .. 64h+63 of this thread.  Start: dX of the part; carry: rowsum(S_end . dX).
-    float carry;
+__device__ __forceinline__ void store_pair(uint32_t tile, int s, int x, float a, float b) {
+    const uint32_t p = pack_bf16(a, b);  // low half: token s, high half: token s+1
+    const bool odd = x & 1;
+    const uint32_t send = odd ? (p & 0xFFFFu) : (p >> 16);
+    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+    const uint32_t w = odd ? (recv | (p & 0xFFFF0000u)) : ((p & 0xFFFFu) | (recv << 16));
+    sts_u32(tile + tile_off(s + (odd ? 1 : 0), x & ~1), w);
+}
+
+// Warps 4-7: thread x = 32 (warp - 4) + lane owns key dim x of dk / dlog_g and value dim x of
+// dv for all 64 tokens of the chunk.
+__device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
+                         uint32_t tmem, int bh, int j, long long row0, int nchunks,
+                         const CUtensorMap *tdk, const CUtensorMap *tdv, const CUtensorMap *tdg) {
+    const int quarter = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
+    const int x = quarter * 32 + lane;
+    const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+    const bool storer = threadIdx.x == 32 * kStateWarps;
+    const long long sidx = ((long long)bh * a.NP + j) * D * D;
+    // carry: rowsum(S_end . dX), the gradient reaching this part from its end state
+    float carry = 0.f;
     {
         const float *Se = nullptr;
         if (j < a.NP - 1) {
@@ -684,162 +816,130 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         } else if (a.S_fin) {
             Se = a.S_fin + (long long)bh * D * D;
         }
-        float part = 0.f;
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            uint32_t w[32];
-            const float4 *x4 = reinterpret_cast<const float4 *>(a.dX + sidx + (long long)i * D + h * HD + p * 32);
-            const float4 *s4 = Se ? reinterpret_cast<const float4 *>(Se + (long long)i * D + h * HD + p * 32) : nullptr;
-#pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-                const float4 v = x4[e4];
-                w[4 * e4] = __float_as_uint(v.x); w[4 * e4 + 1] = __float_as_uint(v.y);
-                w[4 * e4 + 2] = __float_as_uint(v.z); w[4 * e4 + 3] = __float_as_uint(v.w);
-                if (s4) {
-                    const float4 u = s4[e4];
-                    part += u.x * v.x + u.y * v.y + u.z * v.z + u.w * v.w;
-                }
+        if (Se) {
+            const float4 *x4 = reinterpret_cast<const float4 *>(a.dX + sidx + (long long)x * D);
+            const float4 *s4 = reinterpret_cast<const float4 *>(Se + (long long)x * D);
+#pragma unroll 8
+            for (int e4 = 0; e4 < D / 4; ++e4) {
+                const float4 v = x4[e4], u = s4[e4];
+                carry += u.x * v.x + u.y * v.y + u.z * v.z + u.w * v.w;
             }
-            tmem_st32(tmem + lrow + kColDS + h * HD + p * 32, w);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        xb[h * D + i] = part;
-        carry = epi_exchange(b, abort, 0, lane) ? xb[i] + xb[D + i] : 0.f;
     }
+    uint32_t r[16];
+    float qv[16], qn[16];
     for (int it = 0; it < nchunks; ++it) {
-        const int s = it % kStages;
+        const int s = it % kStages, bb = it & 1;
         const int c = nchunks - 1 - it;
         uint8_t *st = smem + s * kStageBytes;
-        uint32_t r[32];
-        const long long t0 = row0 + (long long)c * CH + h * 32;
-        float qdq[32];  // q . dq of this thread's tokens, in flight while the MMAs run
+        const float *qdq = a.dq_ws + (row0 + (long long)c * CH) * D + x;
+        // q . dq of the chunk's last 16 tokens (L2-prefetched with the chunk's tiles), in flight
+        // while this thread waits for dk; each later group is loaded one group ahead
 #pragma unroll
-        for (int t = 0; t < 32; ++t) qdq[t] = a.dq_ws[(t0 + t) * D + i];
-        // (a) masked M and A tiles
-        if (!mbar_wait(b.mm_full, it & 1, abort)) break;
+        for (int t = 0; t < 16; ++t) qn[t] = qdq[(48 + t) * D];
+        if (it > 0 && storer) {  // the previous chunk's output tiles are read out: release its stage
+            bulk_wait_read();
+            mbar_arrive(&b.empty[(it - 1) % kStages]);
+        }
+        // (1) dk and the dlog_g suffix sums: tokens last to first, 16 at a time.  dk_full also
+        // means the dS update is done, so the v and q tiles are free for dk and dlog_g.
+        if (!mbar_wait(&b.dk_full[bb], (it >> 1) & 1, abort)) break;
         tc_fence_after();
-        tmem_ld32(tmem + lrow + kColM + h * 32, r);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b.mm_free);
-        masked_tile(smem + off_m, r, quarter, h, lane);
-        if (!mbar_wait(b.aa_full, it & 1, abort)) break;
-        tc_fence_after();
-        tmem_ld32(tmem + lrow + kColA + h * 32, r);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b.aa_free);
-        masked_tile(smem + off_a, r, quarter, h, lane);
-        // (b) bf16 dS into the shared tile (row i, columns 64h .. 64h+63)
-        tc_fence_after();
+        const uint32_t sa = smem_u32(st);
+        uint32_t fk[16];  // next group's factors and Ktil, bf16 pairs (f low, Ktil high)
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
-            tmem_wait_ld();
+        for (int t = 0; t < 16; ++t) {
+            const uint32_t off = tile_off(48 + t, x);
+            fk[t] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_k + off) << 16);
+        }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t *x = r + jj * 8;
-                *reinterpret_cast<uint4 *>(smem + off_ds + ds_off(i, h * HD + p * 32 + jj * 8)) =
-                    make_uint4(pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
-                               pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
-                               pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
-                               pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
+        for (int g = 3; g >= 0; --g) {
+            tmem_ld16(tmem + lrow + kColDK + bb * 64 + g * 16, r);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) qv[t] = qn[t];
+            if (g > 0) {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) qn[t] = qdq[((g - 1) * 16 + t) * D];
             }
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(b.p_full);
-            mbar_arrive(b.dst_full);
-        }
-        // (c) dk for tokens 32h .. 32h+31 of the chunk; dlog_g suffix sums
-        if (!mbar_wait(b.dk_full, it & 1, abort)) break;
-        tc_fence_after();
-        tmem_ld32(tmem + lrow + kColDK + h * 32, r);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b.dk_free);
-        const __nv_bfloat16 *fcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_g);
-        const __nv_bfloat16 *kcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_k);
-        float tot = 0.f;
+            // dk = e^{b_C - b_s} acc and the contribution q . dq - k . dk (k . dk = Ktil . acc,
+            // Ktil = k e^{b_C - b_s} the MMA operand); then the suffix sums
+            float f[16], c[16];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            // dk = e^{b_C - b_s} acc and k . dk = Ktil . acc (Ktil = k e^{b_C - b_s}, the MMA operand)
-            const uint32_t off = tile_off(h * 32 + t, i) >> 1;
-            const float acc = __uint_as_float(r[t]);
-            dk[(t0 + t) * D + i] = __float2bfloat16_rn(acc * __bfloat162float(fcol[off]));
-            const float cg = qdq[t] - __bfloat162float(kcol[off]) * acc;
-            r[t] = __float_as_uint(cg);  // contribution, kept for the suffix sums
-            tot += cg;
-        }
-        float *xs = xb + ((it + 1) & 1) * 2 * D;
-        xs[h * D + i] = tot;
-        if (!epi_exchange(b, abort, it + 1, lane)) break;
-        const float later = h == 0 ? xs[D + i] : 0.f;  // the second half's tokens come later
-        float acc = carry + later;
+            for (int t = 0; t < 16; ++t) {
+                f[t] = __uint_as_float(fk[t] << 16);
+                c[t] = __uint_as_float(fk[t] & 0xFFFF0000u);
+            }
+            if (g > 0) {  // the next group's loads go out before this group's stores
 #pragma unroll
-        for (int t = 31; t >= 0; --t) {
-            acc += __uint_as_float(r[t]);
-            dg[(t0 + t) * D + i] = __float2bfloat16_rn(acc);
-        }
-        carry += xs[i] + xs[D + i];
-        // (d) dv rows 16q + lane (lanes 0-15), value dims 64h .. 64h+63
-        if (!mbar_wait(b.dv_full, it & 1, abort)) break;
-        tc_fence_after();
-        {
-            uint4 *drow = reinterpret_cast<uint4 *>(
-                dv + (row0 + (long long)c * CH + quarter * 16 + lane) * D + h * HD);
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                tmem_ld32(tmem + lrow + kColDV + h * HD + p * 32, r);
-                tmem_wait_ld();
-                if (lane < 16) {
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        const uint32_t *src = r + q8 * 8;
-                        drow[p * 4 + q8] =
-                            make_uint4(pack_bf16(__uint_as_float(src[0]), __uint_as_float(src[1])),
-                                       pack_bf16(__uint_as_float(src[2]), __uint_as_float(src[3])),
-                                       pack_bf16(__uint_as_float(src[4]), __uint_as_float(src[5])),
-                                       pack_bf16(__uint_as_float(src[6]), __uint_as_float(src[7])));
-                    }
+                for (int t = 0; t < 16; ++t) {
+                    const uint32_t off = tile_off((g - 1) * 16 + t, x);
+                    fk[t] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_k + off) << 16);
                 }
             }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b.dv_free);
-        // (e) dS <- diag(e^{b_C}) (dS + Qbar'^T dO), the sum already formed by the MMA
-        if (!mbar_wait(b.dsn_full, it & 1, abort)) break;
-        tc_fence_after();
-        const float e_i = ec[s * D + i];
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            tmem_ld32(tmem + lrow + kColDS + h * HD + p * 32, r);
             tmem_wait_ld();
+            if (g == 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&b.dk_free[bb]);
+            }
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(e_i * __uint_as_float(r[e]));
-            tmem_st32(tmem + lrow + kColDS + h * HD + p * 32, r);
+            for (int t = 0; t < 16; ++t) {
+                const float acc = __uint_as_float(r[t]);
+                f[t] *= acc;                  // dk
+                c[t] = qv[t] - c[t] * acc;    // contribution
+            }
+#pragma unroll
+            for (int t = 15; t >= 0; --t) {
+                carry += c[t];
+                c[t] = carry;                 // dlog_g
+            }
+#pragma unroll
+            for (int t = 0; t < 16; t += 2) {
+                store_pair(sa + off_v, g * 16 + t, x, f[t], f[t + 1]);
+                store_pair(sa + off_q, g * 16 + t, x, c[t], c[t + 1]);
+            }
         }
-        tmem_wait_st();
-        tc_fence_before();
+        // (2) dv into the dO tile (its last readers, the dv MMAs, are done)
+        if (!mbar_wait(&b.dv_full[bb], (it >> 1) & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {
+            tmem_ld16(tmem + lrow + kColDV + bb * 64 + g * 16, r);
+            tmem_wait_ld();
+            if (g == 3) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&b.dv_free[bb]);
+            }
+#pragma unroll
+            for (int t = 0; t < 16; t += 2)
+                store_pair(sa + off_do, g * 16 + t, x, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
+        }
+        // (3) once all four warps' values are in the tiles, one thread stores them
+        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(b.dsn_free);
-            mbar_arrive(&b.empty[s]);
+        if (lane == 0) mbar_arrive(b.osync);
+        if (!mbar_wait(b.osync, it & 1, abort)) break;
+        if (storer) {
+            const int y = (int)(row0 + (long long)c * CH);
+            tma_store_2d(tdk, 0, y, st + off_v);
+            tma_store_2d(tdk, 64, y, st + off_v + kHalfBytes);
+            tma_store_2d(tdg, 0, y, st + off_q);
+            tma_store_2d(tdg, 64, y, st + off_q + kHalfBytes);
+            tma_store_2d(tdv, 0, y, st + off_do);
+            tma_store_2d(tdv, 64, y, st + off_do + kHalfBytes);
+            bulk_commit();
         }
     }
+    if (storer) bulk_wait_all();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-              const __grid_constant__ CUtensorMap tm_g, const BwdArgs a) {
+              const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_dk,
+              const __grid_constant__ CUtensorMap tm_dv, const __grid_constant__ CUtensorMap tm_dg,
+              const BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -849,9 +949,9 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     b.gated = bar + kStages;
     b.empty = bar + 2 * kStages;
     uint64_t *x = bar + 3 * kStages;
-    b.mm_full = x + 0; b.mm_free = x + 1; b.aa_full = x + 2; b.aa_free = x + 3; b.p_full = x + 4;
-    b.dst_full = x + 5; b.dk_full = x + 6; b.dk_free = x + 7; b.dv_full = x + 8; b.dv_free = x + 9;
-    b.dsn_full = x + 10; b.dsn_free = x + 11; b.xchg = x + 12; b.fin = x + 13;
+    b.mm_full = x + 0; b.mm_free = x + 1; b.p_full = x + 2; b.dst_full = x + 3; b.dk_full = x + 4;
+    b.dk_free = x + 6; b.dv_full = x + 8; b.dv_free = x + 10; b.dsn_full = x + 12; b.osync = x + 13;
+    b.fin = x + 14;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -862,13 +962,15 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&b.full[s], 1);
             mbar_init(&b.gated[s], kGateWarps);
-            mbar_init(&b.empty[s], 1 + kEpiWarps);
+            mbar_init(&b.empty[s], 1 + kStateWarps + 1);  // MMA, dS warps, output storer
         }
-        uint64_t *one[] = {b.mm_full, b.aa_full, b.dk_full, b.dv_full, b.dsn_full, b.fin};
-        uint64_t *epi[] = {b.mm_free, b.aa_free, b.p_full, b.dst_full, b.dk_free, b.dv_free,
-                           b.dsn_free, b.xchg};
+        uint64_t *one[] = {b.mm_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dv_full + 1,
+                           b.dsn_full, b.fin};
+        uint64_t *st4[] = {b.mm_free, b.p_full, b.dst_full};
+        uint64_t *out4[] = {b.dk_free, b.dk_free + 1, b.dv_free, b.dv_free + 1, b.osync};
         for (uint64_t *p : one) mbar_init(p, 1);
-        for (uint64_t *p : epi) mbar_init(p, kEpiWarps);
+        for (uint64_t *p : st4) mbar_init(p, kStateWarps);
+        for (uint64_t *p : out4) mbar_init(p, kOutWarps);
         *abort = 0;
         mbar_fence_init();
     }
@@ -878,6 +980,9 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_g);
+        prefetch_tmap(&tm_dk);
+        prefetch_tmap(&tm_dv);
+        prefetch_tmap(&tm_dg);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -885,13 +990,16 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (warp == kTmaWarp) {
-        if (lane == 0) producer(smem, b, abort, &tm_q, &tm_k, &tm_v, &tm_do, &tm_g, row0, nchunks);
+        if (lane == 0)
+            producer(smem, b, abort, &tm_q, &tm_k, &tm_v, &tm_do, &tm_g, a.dq_ws, row0, nchunks);
     } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_issuer(smem, b, abort, tmem, nchunks);
+        mma_issuer(smem, b, abort, tmem, nchunks);
     } else if (warp >= kEpiWarps) {
         gate_role(smem, b, abort, a, nchunks);
+    } else if (warp < kStateWarps) {
+        state_role(smem, b, abort, a, tmem, bh, j, nchunks);
     } else {
-        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks);
+        out_role(smem, b, abort, a, tmem, bh, j, row0, nchunks, &tm_dk, &tm_dv, &tm_dg);
     }
     tc_fence_before();
     __syncthreads();
@@ -931,19 +1039,23 @@ cudaError_t launch_tc_dq(const BwdArgs &a, cudaStream_t st) {
 
 cudaError_t launch_tc_dkv(const BwdArgs &a, cudaStream_t st) {
     const long long rows = (long long)a.BH * a.L;
-    CUtensorMap mq, mk, mv, mdo, mg;
+    CUtensorMap mq, mk, mv, mdo, mg, mdk, mdv, mdg;
     cudaError_t e;
     if ((e = make_map(&mq, a.q, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mk, a.k, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mdo, a.dO, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mdk, a.dk_out, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mdv, a.dv_out, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mdg, a.dg_out, rows)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(dkv::tc_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dkv::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long nblk = (long long)a.BH * a.NP;
     if (nblk == 0) return cudaSuccess;
-    dkv::tc_dkv_kernel<<<(unsigned)nblk, kThreads, dkv::kSmemBytes, st>>>(mq, mk, mv, mdo, mg, a);
+    dkv::tc_dkv_kernel<<<(unsigned)nblk, kThreads, dkv::kSmemBytes, st>>>(mq, mk, mv, mdo, mg, mdk,
+                                                                          mdv, mdg, a);
     return cudaGetLastError();
 }
 

@@ -44,6 +44,11 @@ __device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity) {
     return mbar_wait(bar, parity, &dummy);
 }
 
+// Waits by a whole warp; the answer is the same in every lane.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

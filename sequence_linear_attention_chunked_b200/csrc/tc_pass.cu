@@ -78,11 +78,6 @@ struct Bars {
     uint64_t *qk_full, *qk_free, *p_full, *ds_full, *sa_full, *sa_free, *o_full, *o_free, *fin;
 };
 
-// Waits by a whole warp; the answer is the same in every lane.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort));
-}
-
 // ------------------------------------------------------------------ TMA producer (1 thread)
 template <int MODE>
 __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tq,
