@@ -27,6 +27,32 @@ constexpr int kEpiWarps = 8, kGateWarps = 4;
 constexpr int kTmaWarp = 12, kMmaWarp = 13;
 constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
 
+// Shared-memory accesses of the output stages as explicit instructions in program order; they
+// carry no compiler memory clobber, so the compiler may schedule other work around them.  Each
+// kernel reads its factors from tiles it does not write and stages its outputs in tiles that no
+// MMA reads any more.
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
+}
+
+// Stores the bf16 values of tokens s and s+1 of this lane's dim x into a [64 x 128] swizzled
+// tile.  Lanes x and x^1 swap one value so that each writes one 4-byte word (dims x & ~1 and
+// x | 1): the even lane row s, the odd lane row s+1.  Two-byte stores would put two lanes on
+// each 4-byte word and take two shared-memory wavefronts per instruction.
+__device__ __forceinline__ void store_pair(uint32_t tile, int s, int x, float a, float b) {
+    const uint32_t p = pack_bf16(a, b);  // low half: token s, high half: token s+1
+    const bool odd = x & 1;
+    const uint32_t send = odd ? (p & 0xFFFFu) : (p >> 16);
+    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+    const uint32_t w = odd ? (recv | (p & 0xFFFF0000u)) : ((p & 0xFFFFu) | (recv << 16));
+    sts_u32(tile + tile_off(s + (odd ? 1 : 0), x & ~1), w);
+}
+
 // ------------------------------------------------------------------ dq sweep
 namespace dqs {
 
@@ -38,7 +64,7 @@ constexpr int kStageBytes = 5 * kTileBytes;
 constexpr int off_m = kStages * kStageBytes;
 constexpr int off_ec = off_m + CH * CH * 2;
 constexpr int off_bar = off_ec + kStages * D * 4;
-constexpr int kBars = 3 * kStages + 12;
+constexpr int kBars = 3 * kStages + 13;
 constexpr int off_misc = off_bar + kBars * 8;
 constexpr int kSmemBytes = off_misc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -46,7 +72,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 struct Bars {
     uint64_t *full, *gated, *empty;
     uint64_t *m_full, *m_free, *p_full, *ds_full, *ds_free, *sa_full, *sa_free, *dq_full,
-        *dq_free, *fin;
+        *dq_free, *osync, *fin;
 };
 
 __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tk,
@@ -223,14 +249,15 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 // Epilogue warps: thread (w, lane) owns key dim i = 32 (w % 4) + lane (its TMEM lane) and the
 // half h = w / 4 of the state row (value dims 64h .. 64h+63) and of each chunk's 64 tokens.
 __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
-                              uint32_t tmem, int bh, int j, long long row0, int nchunks) {
+                              uint32_t tmem, int bh, int j, long long row0, int nchunks,
+                              const CUtensorMap *tdq, const CUtensorMap *tqdq) {
     constexpr int HD = D / 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3, h = warp >> 2;
     const int i = quarter * 32 + lane;
     const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
     const float *ec = reinterpret_cast<const float *>(smem + off_ec);
-    __nv_bfloat16 *dq = static_cast<__nv_bfloat16 *>(a.dq_out);
+    const bool storer = threadIdx.x == 0;  // issues the chunk's TMA stores of dq and q . dq
 
     float S[HD];  // S[i][64h + e]
     if (a.S_recv) {
@@ -250,6 +277,10 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         const int s = c % kStages;
         uint8_t *st = smem + s * kStageBytes;
         uint32_t r[32];
+        if (c > 0 && storer) {  // the previous chunk's staged outputs are read out: release its stage
+            bulk_wait_read();
+            mbar_arrive(&b.empty[(c - 1) % kStages]);
+        }
         if (a.S_fine && c % cpf == 0) {  // the state entering fine part c / cpf
             float4 *Sf = reinterpret_cast<float4 *>(
                 a.S_fine + (((long long)bh * a.NP + j) * a.fine + c / cpf) * D * D + (long long)i * D + h * HD);
@@ -312,34 +343,65 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(b.ds_free);
-        // (d) dq rows t = 32h .. 32h+31, column i; q . dq for the reverse sweep
+        // (d) dq rows t = 32h .. 32h+31, column i, staged in the k tile (bf16) and q . dq in the
+        // v and dO tiles (fp32, four 32-column boxes): no MMA reads them once dq_full has fired
         if (!mbar_wait(b.dq_full, c & 1, abort)) break;
         tc_fence_after();
-        tmem_ld32(tmem + lrow + kColDQ + h * 32, r);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b.dq_free);
-        const long long t0 = row0 + (long long)c * CH + h * 32;
-        const __nv_bfloat16 *fcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_g);
-        const __nv_bfloat16 *qcol = reinterpret_cast<const __nv_bfloat16 *>(st + off_q);
+        const uint32_t sa = smem_u32(st);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const uint32_t off = tile_off(h * 32 + t, i) >> 1;
-            const float v = __uint_as_float(r[t]) * __bfloat162float(fcol[off]);
-            const long long idx = (t0 + t) * D + i;
-            dq[idx] = __float2bfloat16_rn(v);
-            a.dq_ws[idx] = __bfloat162float(qcol[off]) * v;
+        for (int hh = 0; hh < 2; ++hh) {
+            uint32_t r16[16];
+            tmem_ld16(tmem + lrow + kColDQ + h * 32 + hh * 16, r16);
+            tmem_wait_ld();
+            if (hh == 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b.dq_free);
+            }
+#pragma unroll
+            for (int t0 = 0; t0 < 16; t0 += 8) {
+                uint32_t fq[8];  // factor e^{b_t - b_C} (low half) and q (high half), bf16
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t off = tile_off(h * 32 + hh * 16 + t0 + e, i);
+                    fq[e] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_q + off) << 16);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const int t = h * 32 + hh * 16 + t0 + e;
+                    const float v0 = __uint_as_float(r16[t0 + e]) * __uint_as_float(fq[e] << 16);
+                    const float v1 = __uint_as_float(r16[t0 + e + 1]) * __uint_as_float(fq[e + 1] << 16);
+                    store_pair(sa + off_k, t, i, v0, v1);
+                    sts_u32(sa + off_v + tile_off32(t, i),
+                            __float_as_uint(__uint_as_float(fq[e] & 0xFFFF0000u) * v0));
+                    sts_u32(sa + off_v + tile_off32(t + 1, i),
+                            __float_as_uint(__uint_as_float(fq[e + 1] & 0xFFFF0000u) * v1));
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.osync);
+        if (!mbar_wait(b.osync, c & 1, abort)) break;
+        if (storer) {
+            const int y = (int)(row0 + (long long)c * CH);
+            tma_store_2d(tdq, 0, y, st + off_k);
+            tma_store_2d(tdq, 64, y, st + off_k + kHalfBytes);
+#pragma unroll
+            for (int xb = 0; xb < 4; ++xb) tma_store_2d(tqdq, 32 * xb, y, st + off_v + xb * 8192);
+            bulk_commit();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&b.empty[s]);
+        if (lane == 0 && warp != 0) mbar_arrive(&b.empty[s]);  // warp 0 releases it after the reads
     }
+    if (storer) bulk_wait_all();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_g,
-             const __grid_constant__ CUtensorMap tm_q, const BwdArgs a) {
+             const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dq,
+             const __grid_constant__ CUtensorMap tm_qdq, const BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -350,7 +412,8 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     b.empty = bar + 2 * kStages;
     uint64_t *x = bar + 3 * kStages;
     b.m_full = x + 0; b.m_free = x + 1; b.p_full = x + 2; b.ds_full = x + 3; b.ds_free = x + 4;
-    b.sa_full = x + 5; b.sa_free = x + 6; b.dq_full = x + 7; b.dq_free = x + 8; b.fin = x + 9;
+    b.sa_full = x + 5; b.sa_free = x + 6; b.dq_full = x + 7; b.dq_free = x + 8; b.osync = x + 9;
+    b.fin = x + 10;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -372,6 +435,7 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         mbar_init(b.sa_free, 1);
         mbar_init(b.dq_full, 1);
         mbar_init(b.dq_free, kEpiWarps);
+        mbar_init(b.osync, kEpiWarps);
         mbar_init(b.fin, 1);
         *abort = 0;
         mbar_fence_init();
@@ -382,6 +446,8 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_g);
         prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_dq);
+        prefetch_tmap(&tm_qdq);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -395,7 +461,7 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     } else if (warp >= kEpiWarps) {
         gate_role(smem, b, abort, a, nchunks);
     } else {
-        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks);
+        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks, &tm_dq, &tm_qdq);
     }
     tc_fence_before();
     __syncthreads();
@@ -771,32 +837,6 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
     }
 }
 
-// Stores the bf16 values of tokens s and s+1 of this lane's dim x into a [64 x 128] swizzled
-// tile.  Lanes x and x^1 swap one value so that each writes one 4-byte word (dims x & ~1 and
-// x | 1): the even lane row s, the odd lane row s+1.  Two-byte stores would put two lanes on
-// each 4-byte word and take two shared-memory wavefronts per instruction.
-// The shared-memory accesses of the output warps are explicit instructions in program order;
-// they carry no compiler memory clobber, so the compiler may schedule other work around them.
-// Their buffers are disjoint: factors and Ktil are read from the g and k tiles, outputs go to
-// the v, q and dO tiles, which no MMA reads any more.
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-    uint16_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-    return v;
-}
-__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
-}
-
-__device__ __forceinline__ void store_pair(uint32_t tile, int s, int x, float a, float b) {
-    const uint32_t p = pack_bf16(a, b);  // low half: token s, high half: token s+1
-    const bool odd = x & 1;
-    const uint32_t send = odd ? (p & 0xFFFFu) : (p >> 16);
-    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-    const uint32_t w = odd ? (recv | (p & 0xFFFF0000u)) : ((p & 0xFFFFu) | (recv << 16));
-    sts_u32(tile + tile_off(s + (odd ? 1 : 0), x & ~1), w);
-}
-
 // Warps 4-7: thread x = 32 (warp - 4) + lane owns key dim x of dk / dlog_g and value dim x of
 // dv for all 64 tokens of the chunk.
 __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
@@ -1021,19 +1061,22 @@ bool tc_bwd_supported(const BwdArgs &a) {
 
 cudaError_t launch_tc_dq(const BwdArgs &a, cudaStream_t st) {
     const long long rows = (long long)a.BH * a.L;
-    CUtensorMap mk, mv, mdo, mg, mq;
+    CUtensorMap mk, mv, mdo, mg, mq, mdq, mqdq;
     cudaError_t e;
     if ((e = make_map(&mk, a.k, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mdo, a.dO, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mq, a.q, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mdq, a.dq_out, rows)) != cudaSuccess) return e;
+    if ((e = make_map_f32(&mqdq, a.dq_ws, rows)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(dqs::tc_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dqs::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long nblk = (long long)a.BH * a.NP;
     if (nblk == 0) return cudaSuccess;
-    dqs::tc_dq_kernel<<<(unsigned)nblk, kThreads, dqs::kSmemBytes, st>>>(mk, mv, mdo, mg, mq, a);
+    dqs::tc_dq_kernel<<<(unsigned)nblk, kThreads, dqs::kSmemBytes, st>>>(mk, mv, mdo, mg, mq, mdq,
+                                                                        mqdq, a);
     return cudaGetLastError();
 }
 
