@@ -138,13 +138,14 @@ class ClockSampler:
 class Step:
     """One pass of the whole path through the C ABI's per-step entry points, with CUDA events
     between the phases on the launching stream.  Forward: state pass, state scan, output pass
-    (or local pass, scan, correction pass); backward (fwd+bwd workloads): gradient-state pass,
-    reverse scan, gradient pass, reusing the forward's received states."""
+    (or local pass, scan, correction pass); backward (fwd+bwd workloads): dq pass (which also
+    forms the gradient states), reverse scan, dk/dv/dlog_g pass, reusing the forward's received
+    states."""
 
     KERNEL_KEYS = {"state pass": "state_pass", "output pass": "output_pass",
                    "local pass": "local_pass", "correction pass": "correct_pass",
-                   "state scan": "scan", "dq pass": "dq_pass", "dstate pass": "dstate_pass",
-                   "reverse scan": "scan", "dkv pass": "dkv_pass"}
+                   "state scan": "scan", "dq pass": "dq_pass", "reverse scan": "scan",
+                   "dkv pass": "dkv_pass"}
 
     def __init__(self, w: Workload, x, schedule: str, device):
         from sequence_linear_attention_chunked_b200 import la_seg
@@ -168,7 +169,7 @@ class Step:
             self.NPF = la_seg.la_seg_backward_parts(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt,
                                                     False)
             self.fine = self.NPF // NP
-            self.phases += ["dq pass", "dstate pass", "reverse scan", "dkv pass"]
+            self.phases += ["dq pass", "reverse scan", "dkv pass"]
             NPF = self.NPF
             self.S_fine = torch.empty((B, H, NPF, dk, dv), **f32)
             self.dSloc = torch.empty((B, H, NPF, dk, dv), **f32)
@@ -209,19 +210,16 @@ class Step:
             return
         la.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_recv, NP, self.fine,
                           w.chunk, dq=self.grads[0], qdq=self.qdq, S_fine=self.S_fine,
-                          status=self.status)
+                          dSloc=self.dSloc, log_gamma=self.logG_b, status=self.status)
         rec(4)
         NPF = self.NPF
-        la.la_seg_dstate_pass(x["q"], x["dO"], x["log_g"], NPF, w.chunk, dSloc=self.dSloc,
-                              log_gamma=self.logG_b, status=self.status)
-        rec(5)
         la._check(la.lib().la_seg_scan(la._ptr(self.dSloc), la._ptr(self.logG_b), None, BH, NPF,
                                        w.dk, w.dv, 1, la._ptr(self.dX), la._ptr(self.dS0),
                                        la._stream(None)), "la_seg_scan")
-        rec(6)
+        rec(5)
         la.la_seg_dkv_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_fine, None, self.dX,
                            self.qdq, NPF, w.chunk, out=self.grads[1:], status=self.status)
-        rec(7)
+        rec(6)
 
     def phase_ms(self):
         return [self.events[i].elapsed_time(self.events[i + 1]) for i in range(len(self.phases))]
@@ -244,8 +242,9 @@ class Step:
         if w.backward:
             stf = w.B * w.H * self.NPF * w.dk * w.dv * 4
             lgf = w.B * w.H * self.NPF * w.dk * 4
-            ab["dq pass"] = th * (3 * w.dk + 2 * w.dv + w.dk) * e + st + stf
-            ab["dstate pass"] = th * (2 * w.dk + w.dv) * e + stf + lgf
+            # reads q, k, v, dO, log_g and the received states; writes dq, S_fine, dSloc and
+            # log_gamma (the fp32 q . dq hand-over to the dkv pass is not counted)
+            ab["dq pass"] = th * (3 * w.dk + 2 * w.dv + w.dk) * e + st + 2 * stf + lgf
             ab["reverse scan"] = 2 * stf + lgf + fin
             ab["dkv pass"] = th * (3 * w.dk + 2 * w.dv + 2 * w.dk + w.dv) * e + 2 * stf
         return ab
@@ -261,8 +260,7 @@ class Step:
         else:
             fl = {"local pass": th * (intra + 2 * dd), "state scan": 0, "correction pass": th * dd}
         if w.backward:
-            fl["dq pass"] = th * (2 * C * dv + 2 * C * dk + 2 * dd)
-            fl["dstate pass"] = th * dd
+            fl["dq pass"] = th * (2 * C * dv + 2 * C * dk + 3 * dd)
             fl["reverse scan"] = 0
             fl["dkv pass"] = th * (3 * dd + 2 * C * (3 * dk + 2 * dv))
         return fl

@@ -158,7 +158,7 @@ LA_API la_status la_seg_correct_pass(const void *q, const void *log_g, const flo
                                      int B, int H, long long L, int dk, int dv, int NP, int chunk,
                                      la_dtype dt, void *o, int *status, void *cuda_stream);
 
-/* Gradient-state pass (backward step 3): dSloc[b,h,p] = sum over segment p of
+/* Gradient-state pass (what the backward's dq pass also forms): dSloc[b,h,p] = sum over segment p of
  * diag(exp(B_t)) q_t^T dO_t, B_t the inclusive cumsum of log_g from the segment's first token,
  * fp32 [B,H,NP,dk,dv]; log_gamma[b,h,p] = sum of log_g over segment p, fp32 [B,H,NP,dk]. */
 LA_API la_status la_seg_dstate_pass(const void *q, const void *dO, const void *log_g, int B,
@@ -171,19 +171,22 @@ LA_API la_status la_seg_dstate_pass(const void *q, const void *dO, const void *l
  * [B,H,L,dk], read by la_seg_dkv_pass for dlog_g).  S_fine (nullable, fp32
  * [B,H,NP*fine,dk,dv]) receives the state entering each of the `fine` equal parts of every
  * segment ((L/NP) % fine == 0, parts of whole chunks): the received states of the finer split
- * la_seg_dkv_pass runs on. */
+ * la_seg_dkv_pass runs on.  dSloc and log_gamma (both or neither; fp32 [B,H,NP*fine,dk,dv] and
+ * [B,H,NP*fine,dk]) receive what la_seg_dstate_pass computes over that finer split, formed in
+ * the same sweep (its q, dO and log_g tiles are already on chip). */
 LA_API la_status la_seg_dq_pass(const void *q, const void *k, const void *v, const void *log_g,
                                 const void *dO, const float *S_recv, int B, int H, long long L,
                                 int dk, int dv, int NP, int fine, int chunk, la_dtype dt,
-                                void *dq, float *qdq, float *S_fine, int *status,
-                                void *cuda_stream);
+                                void *dq, float *qdq, float *S_fine, float *dSloc,
+                                float *log_gamma, int *status, void *cuda_stream);
 
-/* dk/dv pass (backward step 5): the reverse chunk sweep of every segment p of NP: dk, dv and
+/* dk/dv pass (backward step 4): the reverse chunk sweep of every segment p of NP: dk, dv and
  * dlog_g (dtype dt).  S_recv: the states the segments receive (fp32 [B,H,NP,dk,dv]; they give
  * each segment's end state for the dlog_g carry rowsum(S_end . dX); null = no carry), S_final
  * (fp32 [B,H,dk,dv], the last segment's end state; null when dS_final is zero), dX: gradient of
- * every segment's end state (la_seg_scan with reverse = 1 over la_seg_dstate_pass's states,
- * initialised with dS_final), qdq: la_seg_dq_pass's q . dq. */
+ * every segment's end state (la_seg_scan with reverse = 1 over the gradient states of
+ * la_seg_dstate_pass or la_seg_dq_pass, initialised with dS_final), qdq: la_seg_dq_pass's
+ * q . dq. */
 LA_API la_status la_seg_dkv_pass(const void *q, const void *k, const void *v, const void *log_g,
                                  const void *dO, const float *S_recv, const float *S_final,
                                  const float *dX, const float *qdq, int B, int H, long long L,

@@ -20,8 +20,17 @@ cudaError_t launch_bwd_dstate(const BwdArgs &a, cudaStream_t st) {
     return launch_simt_dstate(a, st);
 }
 
+// The tensor-core dq sweep also forms the fine parts' gradient states when a.dSloc and a.logG
+// are given; the CUDA-core path runs the gradient-state pass over the fine split after it.
 cudaError_t launch_bwd_dq(const BwdArgs &a, cudaStream_t st) {
-    return tc_bwd_supported(a) ? launch_tc_dq(a, st) : launch_simt_dq(a, st);
+    if (tc_bwd_supported(a)) return launch_tc_dq(a, st);
+    cudaError_t e = launch_simt_dq(a, st);
+    if (e != cudaSuccess || !a.dSloc || !a.logG) return e;
+    BwdArgs f = a;
+    f.NP = a.NP * a.fine;
+    f.T = a.T / a.fine;
+    f.fine = 1;
+    return launch_bwd_dstate(f, st);
 }
 
 cudaError_t launch_bwd_dkv(const BwdArgs &a, cudaStream_t st) {

@@ -283,18 +283,21 @@ la_status la_seg_dstate_pass(const void *q, const void *dO, const void *log_g, i
 la_status la_seg_dq_pass(const void *q, const void *k, const void *v, const void *log_g,
                          const void *dO, const float *S_recv, int B, int H, long long L, int dk,
                          int dv, int NP, int fine, int chunk, la_dtype dt, void *dq, float *qdq,
-                         float *S_fine, int *status, void *cuda_stream) {
+                         float *S_fine, float *dSloc, float *log_gamma, int *status,
+                         void *cuda_stream) {
     la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
                               {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {dO, "dO"},
                                {dq, "dq"}, {qdq, "qdq"}},
-                              {{S_recv, "S_recv"}, {S_fine, "S_fine"}});
+                              {{S_recv, "S_recv"}, {S_fine, "S_fine"}, {dSloc, "dSloc"},
+                               {log_gamma, "log_gamma"}});
     if (st != LA_OK) return st;
+    if (!dSloc != !log_gamma) return fail(LA_ERR_ARG, "dSloc and log_gamma go together");
     if (fine < 1 || (L > 0 && ((L / NP) % fine != 0 || ((L / NP) / fine) % chunk != 0)))
         return fail(LA_ERR_SHAPE, "fine=%d must cut each segment into whole chunks", fine);
     if (L == 0) return LA_OK;
     la::BwdArgs b = {};
     b.q = q; b.k = k; b.v = v; b.g = log_g; b.dO = dO; b.dq_out = dq; b.dq_ws = qdq;
-    b.S_recv = S_recv; b.S_fine = S_fine; b.status = status;
+    b.S_recv = S_recv; b.S_fine = S_fine; b.dSloc = dSloc; b.logG = log_gamma; b.status = status;
     b.L = L; b.T = L / NP; b.BH = B * H; b.NP = NP; b.dk = dk; b.dv = dv; b.chunk = chunk;
     b.fine = fine; b.dt = dt;
     cudaError_t e = la::launch_bwd_dq(b, static_cast<cudaStream_t>(cuda_stream));
@@ -462,18 +465,17 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     b.S_recv = recv; b.S_fine = S_fine; b.S_end_next = S_fine; b.S_fin = reuse ? nullptr : S_fin;
     b.dX = dX; b.dq_ws = qdq; b.dSloc = dSloc; b.logG = logG_f; b.status = status;
     b.L = L; b.BH = s.BH; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
-    // 2. dq sweep over the segments; records the state entering each of their r fine parts
+    // 2. dq sweep over the segments; records the state entering each of their r fine parts,
+    //    and forms every fine part's gradient state and log-decay sum
     b.NP = s.NP; b.T = s.T; b.fine = r;
     if ((e = la::launch_bwd_dq(b, stream)) != cudaSuccess) return cuda_fail(e, "dq pass");
-    // 3-5 run over the fine parts
+    // 3-4 run over the fine parts
     b.NP = s.NP * r; b.T = s.T / r; b.fine = 1;
-    // 3. per-part gradient states and log-decay sums
-    if ((e = la::launch_bwd_dstate(b, stream)) != cudaSuccess) return cuda_fail(e, "gradient-state pass");
-    // 4. reverse exclusive decayed scan: gradient of every part's end state, and dS0
+    // 3. reverse exclusive decayed scan: gradient of every part's end state, and dS0
     if ((e = la::launch_scan(dSloc, logG_f, dS_final, s.BH, b.NP, dk, dv, 1, dX, dS0, stream)) !=
         cudaSuccess)
         return cuda_fail(e, "reverse state scan");
-    // 5. dk, dv, dlog_g per part
+    // 4. dk, dv, dlog_g per part
     if ((e = la::launch_bwd_dkv(b, stream)) != cudaSuccess) return cuda_fail(e, "dkv pass");
     return LA_OK;
 }

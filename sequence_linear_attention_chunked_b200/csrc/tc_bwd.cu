@@ -56,15 +56,17 @@ __device__ __forceinline__ void store_pair(uint32_t tile, int s, int x, float a,
 // ------------------------------------------------------------------ dq sweep
 namespace dqs {
 
-constexpr uint32_t kColDS = 0, kColDQ = 128, kColSA = 192, kColM = 256;
+// R^T: the gradient-state sum of the current fine part (when the sweep also produces it).
+constexpr uint32_t kColDS = 0, kColDQ = 128, kColSA = 192, kColM = 256, kColR = 320;
 constexpr int kStages = 2;
 constexpr int off_k = 0, off_v = kTileBytes, off_do = 2 * kTileBytes, off_g = 3 * kTileBytes,
-              off_q = 4 * kTileBytes;  // q only feeds the epilogue's q . dq
-constexpr int kStageBytes = 5 * kTileBytes;
+              off_q = 4 * kTileBytes,   // q only feeds the epilogue's q . dq
+              off_qh = 5 * kTileBytes;  // Qhat = q e^{B + b_t}, B: log-decay since the part's start
+constexpr int kStageBytes = 6 * kTileBytes;
 constexpr int off_m = kStages * kStageBytes;
 constexpr int off_ec = off_m + CH * CH * 2;
 constexpr int off_bar = off_ec + kStages * D * 4;
-constexpr int kBars = 3 * kStages + 13;
+constexpr int kBars = 3 * kStages + 15;
 constexpr int off_misc = off_bar + kBars * 8;
 constexpr int kSmemBytes = off_misc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -72,7 +74,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 struct Bars {
     uint64_t *full, *gated, *empty;
     uint64_t *m_full, *m_free, *p_full, *ds_full, *ds_free, *sa_full, *sa_free, *dq_full,
-        *dq_free, *osync, *fin;
+        *dq_free, *osync, *r_full, *r_free, *fin;
 };
 
 __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tk,
@@ -82,7 +84,7 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % kStages;
         if (c >= kStages && !mbar_wait(&b.empty[s], ((c / kStages) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&b.full[s], kStageBytes);
+        mbar_arrive_expect_tx(&b.full[s], 5 * kTileBytes);
         uint8_t *st = smem + s * kStageBytes;
         const int y = (int)(row0 + (long long)c * CH);
         tma_load_2d(st + off_k, tk, 0, y, &b.full[s]);
@@ -103,7 +105,7 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
 }
 
 __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
-                           int nchunks) {
+                           int nchunks, bool dstate, int cpf) {
     constexpr uint32_t i_m = idesc_bf16_f32(64, 64, 0, 0);
     constexpr uint32_t i_ds = idesc_bf16_f32(128, 128, 1, 1);
     constexpr uint32_t i_dqb = idesc_bf16_f32(128, 64, 1, 0);
@@ -133,6 +135,20 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
             mma_commit(b.ds_full);
         }
         __syncwarp();
+        if (dstate) {  // R^T += dO^T Qhat over the fine part; before dq so that dq_full covers it
+            const int part = c / cpf;
+            const bool first = c % cpf == 0;
+            if (first && part > 0 && !warp_wait(b.r_free, (part - 1) & 1, abort)) break;
+            tc_fence_after();
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem + kColR, desc_mnmajor(da, kk), desc_mnmajor(st + off_qh, kk), i_ds,
+                           (!first || kk > 0) ? 1u : 0u);
+                if (c % cpf == cpf - 1) mma_commit(b.r_full);
+            }
+            __syncwarp();
+        }
         if (c > 0 && !warp_wait(b.dq_free, (c - 1) & 1, abort)) break;
         if (!warp_wait(b.p_full, c & 1, abort)) break;
         tc_fence_after();
@@ -161,15 +177,20 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
 }
 
 // Gate warps: cumsum as in the forward pass, Ktil in place of k, e^{b_t - b_C} in place of
-// log_g, e^{b_C} per key dim for the state decay.
+// log_g, e^{b_C} per key dim for the state decay; with the gradient-state sum, also
+// Qhat = q e^{B + b_t} (B: log-decay from the fine part's start to the chunk's start, so that
+// e^{B + b_t} = e^{B + b_C} e^{b_t - b_C}) and each part's log-decay sum.
 __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
-                          int nchunks) {
+                          int nchunks, bool dstate, int cpf, int bh, int j) {
     const int gw = (threadIdx.x >> 5) - kEpiWarps;
     const int lane = threadIdx.x & 31;
     const int tg = lane >> 2, ig = lane & 3;
     const int i0 = gw * 32 + ig * 8;
     float *ec = reinterpret_cast<float *>(smem + off_ec);
     bool range_bad = false;
+    float logB[8];  // log-decay from the fine part's start through the current chunk
+#pragma unroll
+    for (int e = 0; e < 8; ++e) logB[e] = 0.f;
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % kStages;
         if (!mbar_wait(&b.full[s], (c / kStages) & 1, abort)) break;
@@ -199,7 +220,8 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
                 if (tg >= d) incl[e] += up;
             }
         }
-        float nbCl[8];
+        float nbCl[8], eB[8];
+        const bool part_start = c % cpf == 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float bC = __shfl_sync(0xFFFFFFFFu, incl[e], 28 + ig);
@@ -208,6 +230,14 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
             for (int r = 0; r < 8; ++r) bt[r][e] += off;
             nbCl[e] = -bC * kLog2e;
             range_bad |= !(fabsf(bC) <= kGateRangeLimit);
+            logB[e] = (part_start ? 0.f : logB[e]) + bC;
+            eB[e] = dstate ? ex2_approx(logB[e] * kLog2e) : 0.f;
+        }
+        if (dstate && c % cpf == cpf - 1 && tg == 0) {  // the part's log-decay sum
+            const long long jf = (long long)j * a.fine + c / cpf;
+            float4 *lg = reinterpret_cast<float4 *>(a.logG + ((long long)bh * a.NP * a.fine + jf) * D + i0);
+            lg[0] = make_float4(logB[0], logB[1], logB[2], logB[3]);
+            lg[1] = make_float4(logB[4], logB[5], logB[6], logB[7]);
         }
         if (tg == 0) {
             float4 *e4 = reinterpret_cast<float4 *>(ec + s * D + i0);
@@ -217,26 +247,36 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
                                 ex2_approx(-nbCl[7]));
         }
 #pragma unroll
-        for (int r0 = 0; r0 < 8; r0 += 4) {
-            uint4 kr[4];
+        for (int r0 = 0; r0 < 8; r0 += 2) {
+            uint4 kr[2], qr[2];
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-                kr[r] = *reinterpret_cast<const uint4 *>(st + off_k + tile_off(tg * 8 + r0 + r, i0));
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+                kr[r] = *reinterpret_cast<const uint4 *>(st + off_k + off);
+                if (dstate) qr[r] = *reinterpret_cast<const uint4 *>(st + off_q + off);
+            }
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < 2; ++r) {
                 const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
                 float x[8], f[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = fmaf(bt[r0 + r][e], kLog2e, nbCl[e]);
                 unpack8(kr[r], f);
-                uint32_t wk[4], wf[4];
+                uint32_t wk[4], wf[4], wq[4];
+                float fq[8];
+                if (dstate) unpack8(qr[r], fq);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
+                    const float u0 = ex2_approx(x[2 * e]), u1 = ex2_approx(x[2 * e + 1]);
                     wk[e] = pack_bf16(f[2 * e] * ex2_approx(-x[2 * e]), f[2 * e + 1] * ex2_approx(-x[2 * e + 1]));
-                    wf[e] = pack_bf16(ex2_approx(x[2 * e]), ex2_approx(x[2 * e + 1]));
+                    wf[e] = pack_bf16(u0, u1);
+                    if (dstate)
+                        wq[e] = pack_bf16(fq[2 * e] * u0 * eB[2 * e], fq[2 * e + 1] * u1 * eB[2 * e + 1]);
                 }
                 *reinterpret_cast<uint4 *>(st + off_k + off) = make_uint4(wk[0], wk[1], wk[2], wk[3]);
                 *reinterpret_cast<uint4 *>(st + off_g + off) = make_uint4(wf[0], wf[1], wf[2], wf[3]);
+                if (dstate)
+                    *reinterpret_cast<uint4 *>(st + off_qh + off) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
             }
         }
         fence_proxy_async_smem();
@@ -250,7 +290,7 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 // half h = w / 4 of the state row (value dims 64h .. 64h+63) and of each chunk's 64 tokens.
 __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
                               uint32_t tmem, int bh, int j, long long row0, int nchunks,
-                              const CUtensorMap *tdq, const CUtensorMap *tqdq) {
+                              const CUtensorMap *tdq, const CUtensorMap *tqdq, bool dstate) {
     constexpr int HD = D / 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3, h = warp >> 2;
@@ -393,6 +433,23 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         }
         __syncwarp();
         if (lane == 0 && warp != 0) mbar_arrive(&b.empty[s]);  // warp 0 releases it after the reads
+        if (dstate && c % cpf == cpf - 1) {  // the fine part's gradient state R[i'][j] = R^T[j][i']
+            if (!mbar_wait(b.r_full, (c / cpf) & 1, abort)) break;
+            tc_fence_after();
+            const long long jf = (long long)j * a.fine + c / cpf;
+            float *Ro = a.dSloc + ((long long)bh * a.NP * a.fine + jf) * D * D + (h * HD) * D + i;
+#pragma unroll 1
+            for (int p = 0; p < 4; ++p, Ro += 16 * D) {  // key dims h HD + 16p .. +15
+                uint32_t r16[16];
+                tmem_ld16(tmem + lrow + kColR + h * HD + p * 16, r16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) Ro[e * D] = __uint_as_float(r16[e]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.r_free);
+        }
     }
     if (storer) bulk_wait_all();
 }
@@ -413,13 +470,15 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     uint64_t *x = bar + 3 * kStages;
     b.m_full = x + 0; b.m_free = x + 1; b.p_full = x + 2; b.ds_full = x + 3; b.ds_free = x + 4;
     b.sa_full = x + 5; b.sa_free = x + 6; b.dq_full = x + 7; b.dq_free = x + 8; b.osync = x + 9;
-    b.fin = x + 10;
+    b.r_full = x + 10; b.r_free = x + 11; b.fin = x + 12;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x / a.NP, j = blockIdx.x % a.NP;
     const long long row0 = (long long)bh * a.L + (long long)j * a.T;
     const int nchunks = (int)(a.T / CH);
+    const bool dstate = a.dSloc && a.logG;  // also the fine parts' gradient states
+    const int cpf = nchunks / a.fine;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&b.full[s], 1);
@@ -436,6 +495,8 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         mbar_init(b.dq_full, 1);
         mbar_init(b.dq_free, kEpiWarps);
         mbar_init(b.osync, kEpiWarps);
+        mbar_init(b.r_full, 1);
+        mbar_init(b.r_free, kEpiWarps);
         mbar_init(b.fin, 1);
         *abort = 0;
         mbar_fence_init();
@@ -457,11 +518,11 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (warp == kTmaWarp) {
         if (lane == 0) producer(smem, b, abort, &tm_k, &tm_v, &tm_do, &tm_g, &tm_q, row0, nchunks);
     } else if (warp == kMmaWarp) {
-        mma_issuer(smem, b, abort, tmem, nchunks);
+        mma_issuer(smem, b, abort, tmem, nchunks, dstate, cpf);
     } else if (warp >= kEpiWarps) {
-        gate_role(smem, b, abort, a, nchunks);
+        gate_role(smem, b, abort, a, nchunks, dstate, cpf, bh, j);
     } else {
-        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks, &tm_dq, &tm_qdq);
+        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks, &tm_dq, &tm_qdq, dstate);
     }
     tc_fence_before();
     __syncthreads();

@@ -75,7 +75,7 @@ def lib():
                                          P, P]
         L.la_seg_dstate_pass.restype = i32
         L.la_seg_dq_pass.argtypes = [P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32,
-                                     i32, P, P, P, P, P]
+                                     i32, P, P, P, P, P, P, P]
         L.la_seg_dq_pass.restype = i32
         L.la_seg_dkv_pass.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32,
                                       i32, i32, P, P, P, P, P]
@@ -297,13 +297,16 @@ def la_seg_backward_parts(B, H, L, dk, dv, P, chunk, dt=LA_BF16, reuse=True) -> 
 
 
 def la_seg_dq_pass(q, k, v, log_g, dO, S_recv, NP, fine, chunk, *, dq=None, qdq=None, S_fine=None,
-                   status=None, stream=None):
+                   dSloc=None, log_gamma=None, status=None, stream=None):
+    """dq and q . dq; optionally (dSloc and log_gamma given, both or neither) the fine parts'
+    gradient states and log-decay sums, as la_seg_dstate_pass over NP * fine parts."""
     B, H, L, dk, dv = _seq_shapes(q, v)
     dq = torch.empty_like(q) if dq is None else dq
     qdq = torch.empty((B, H, L, dk), dtype=torch.float32, device=q.device) if qdq is None else qdq
     _check(lib().la_seg_dq_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(dO), _ptr(S_recv), B,
                                 H, L, dk, dv, NP, fine, chunk, _dt(q), _ptr(dq), _ptr(qdq),
-                                _ptr(S_fine), _ptr(status), _stream(stream)), "la_seg_dq_pass")
+                                _ptr(S_fine), _ptr(dSloc), _ptr(log_gamma), _ptr(status),
+                                _stream(stream)), "la_seg_dq_pass")
     return dq, qdq
 
 

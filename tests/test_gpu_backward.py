@@ -146,3 +146,27 @@ def test_c4_full_sampled(cuda_device):
         for n, g, r in zip(NAMES, grads, ref):
             e = rel_err(g[b, h, t0:t1], r)
             assert e <= 2e-2, (n, b, h, t0, e)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2048, 128, 2, 64, "bf16", 4), (2, 1, 512, 32, 2, 16, "f32", 2)],
+                         ids=["tcgen05", "simt"])
+def test_dq_pass_gradient_states(cuda_device, shape):
+    """The dq pass forms every fine part's gradient state -- the gradient of that part's outputs
+    with respect to its start state, which is the oracle's dS0 on the part alone -- and the
+    part's log-decay sum."""
+    B, H, L, d, NP, C, dt, fine = shape
+    w = Workload("dq-dstate", B, H, L, d, d, NP, C, dt, "gla" if dt == "bf16" else "toy",
+                 backward=True, seed=7)
+    x = make_inputs(w, cuda_device)
+    NPF = NP * fine
+    dSloc = torch.empty((B, H, NPF, d, d), device=cuda_device)
+    lg = torch.empty((B, H, NPF, d), device=cuda_device)
+    la_seg.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], None, NP, fine, C,
+                          dSloc=dSloc, log_gamma=lg)
+    T = L // NPF
+    for p in range(NPF):
+        sl = slice(p * T, (p + 1) * T)
+        part = [x[n][:, :, sl] for n in ("q", "k", "v", "log_g", "dO")]
+        ref = oracle.backward(*part)
+        assert rel_err(dSloc[:, :, p], ref[4]) <= TOL[w.torch_dtype], p
+        assert rel_err(lg[:, :, p], x["log_g"][:, :, sl].double().sum(2).cpu()) <= 1e-5, p
