@@ -66,7 +66,7 @@ constexpr int kStageBytes = 6 * kTileBytes;
 constexpr int off_m = kStages * kStageBytes;
 constexpr int off_ec = off_m + CH * CH * 2;
 constexpr int off_bar = off_ec + kStages * D * 4;
-constexpr int kBars = 3 * kStages + 15;
+constexpr int kBars = 3 * kStages + 14;
 constexpr int off_misc = off_bar + kBars * 8;
 constexpr int kSmemBytes = off_misc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -74,7 +74,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 struct Bars {
     uint64_t *full, *gated, *empty;
     uint64_t *m_full, *m_free, *p_full, *ds_full, *ds_free, *sa_full, *sa_free, *dq_full,
-        *dq_free, *osync, *r_full, *r_free, *fin;
+        *dq_free, *r_full, *r_free, *fin;
 };
 
 __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tk,
@@ -113,19 +113,20 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
     const uint32_t m_addr = smem_u32(smem + off_m);
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % kStages;
-        if (!warp_wait(&b.gated[s], (c / kStages) & 1, abort)) break;
-        tc_fence_after();
         const uint32_t st = smem_u32(smem + s * kStageBytes);
         const uint32_t ka = st + off_k, va = st + off_v, da = st + off_do;
+        // M = dO V^T reads untouched tiles: it runs while the gate warps rescale k
+        if (!warp_wait(&b.full[s], (c / kStages) & 1, abort)) break;
         if (c > 0 && !warp_wait(b.m_free, (c - 1) & 1, abort)) break;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // M = dO V^T
+            for (int kk = 0; kk < 8; ++kk)
                 mma_ss(tmem + kColM, desc_kmajor(da, kk), desc_kmajor(va, kk), i_m, kk > 0);
             mma_commit(b.m_full);
         }
         __syncwarp();
+        if (!warp_wait(&b.gated[s], (c / kStages) & 1, abort)) break;
         if (c > 0 && !warp_wait(b.ds_free, (c - 1) & 1, abort)) break;
         tc_fence_after();
         if (elect_one()) {
@@ -290,14 +291,13 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 // half h = w / 4 of the state row (value dims 64h .. 64h+63) and of each chunk's 64 tokens.
 __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
                               uint32_t tmem, int bh, int j, long long row0, int nchunks,
-                              const CUtensorMap *tdq, const CUtensorMap *tqdq, bool dstate) {
+                              bool dstate) {
     constexpr int HD = D / 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3, h = warp >> 2;
     const int i = quarter * 32 + lane;
     const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
     const float *ec = reinterpret_cast<const float *>(smem + off_ec);
-    const bool storer = threadIdx.x == 0;  // issues the chunk's TMA stores of dq and q . dq
 
     float S[HD];  // S[i][64h + e]
     if (a.S_recv) {
@@ -317,10 +317,7 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         const int s = c % kStages;
         uint8_t *st = smem + s * kStageBytes;
         uint32_t r[32];
-        if (c > 0 && storer) {  // the previous chunk's staged outputs are read out: release its stage
-            bulk_wait_read();
-            mbar_arrive(&b.empty[(c - 1) % kStages]);
-        }
+
         if (a.S_fine && c % cpf == 0) {  // the state entering fine part c / cpf
             float4 *Sf = reinterpret_cast<float4 *>(
                 a.S_fine + (((long long)bh * a.NP + j) * a.fine + c / cpf) * D * D + (long long)i * D + h * HD);
@@ -383,11 +380,14 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(b.ds_free);
-        // (d) dq rows t = 32h .. 32h+31, column i, staged in the k tile (bf16) and q . dq in the
-        // v and dO tiles (fp32, four 32-column boxes): no MMA reads them once dq_full has fired
+        // (d) dq rows t = 32h .. 32h+31, column i, and q . dq, stored straight from registers:
+        // q . dq (fp32) as one 128-byte line per warp and token, dq (bf16) as 4-byte words
+        // (lanes i and i^1 swap one token, so each writes dims i & ~1, i | 1 of one token)
         if (!mbar_wait(b.dq_full, c & 1, abort)) break;
         tc_fence_after();
         const uint32_t sa = smem_u32(st);
+        const long long tok0 = row0 + (long long)c * CH + h * 32;
+        __nv_bfloat16 *dq = static_cast<__nv_bfloat16 *>(a.dq_out);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             uint32_t r16[16];
@@ -408,31 +408,21 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
                 }
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
-                    const int t = h * 32 + hh * 16 + t0 + e;
+                    const long long t = tok0 + hh * 16 + t0 + e;
                     const float v0 = __uint_as_float(r16[t0 + e]) * __uint_as_float(fq[e] << 16);
                     const float v1 = __uint_as_float(r16[t0 + e + 1]) * __uint_as_float(fq[e + 1] << 16);
-                    store_pair(sa + off_k, t, i, v0, v1);
-                    sts_u32(sa + off_v + tile_off32(t, i),
-                            __float_as_uint(__uint_as_float(fq[e] & 0xFFFF0000u) * v0));
-                    sts_u32(sa + off_v + tile_off32(t + 1, i),
-                            __float_as_uint(__uint_as_float(fq[e + 1] & 0xFFFF0000u) * v1));
+                    a.dq_ws[t * D + i] = __uint_as_float(fq[e] & 0xFFFF0000u) * v0;
+                    a.dq_ws[(t + 1) * D + i] = __uint_as_float(fq[e + 1] & 0xFFFF0000u) * v1;
+                    const uint32_t p = pack_bf16(v0, v1);  // low: token t, high: token t+1
+                    const bool odd = i & 1;
+                    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, odd ? (p & 0xFFFFu) : (p >> 16), 1);
+                    const uint32_t w = odd ? (recv | (p & 0xFFFF0000u)) : ((p & 0xFFFFu) | (recv << 16));
+                    *reinterpret_cast<uint32_t *>(dq + (t + (odd ? 1 : 0)) * D + (i & ~1)) = w;
                 }
             }
         }
-        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(b.osync);
-        if (!mbar_wait(b.osync, c & 1, abort)) break;
-        if (storer) {
-            const int y = (int)(row0 + (long long)c * CH);
-            tma_store_2d(tdq, 0, y, st + off_k);
-            tma_store_2d(tdq, 64, y, st + off_k + kHalfBytes);
-#pragma unroll
-            for (int xb = 0; xb < 4; ++xb) tma_store_2d(tqdq, 32 * xb, y, st + off_v + xb * 8192);
-            bulk_commit();
-        }
-        __syncwarp();
-        if (lane == 0 && warp != 0) mbar_arrive(&b.empty[s]);  // warp 0 releases it after the reads
+        if (lane == 0) mbar_arrive(&b.empty[s]);  // this warp's reads of the stage are done
         if (dstate && c % cpf == cpf - 1) {  // the fine part's gradient state R[i'][j] = R^T[j][i']
             if (!mbar_wait(b.r_full, (c / cpf) & 1, abort)) break;
             tc_fence_after();
@@ -451,14 +441,12 @@ __device__ void epilogue_role(uint8_t *smem, const Bars &b, volatile int *abort,
             if (lane == 0) mbar_arrive(b.r_free);
         }
     }
-    if (storer) bulk_wait_all();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_g,
-             const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dq,
-             const __grid_constant__ CUtensorMap tm_qdq, const BwdArgs a) {
+             const __grid_constant__ CUtensorMap tm_q, const BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -469,8 +457,8 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     b.empty = bar + 2 * kStages;
     uint64_t *x = bar + 3 * kStages;
     b.m_full = x + 0; b.m_free = x + 1; b.p_full = x + 2; b.ds_full = x + 3; b.ds_free = x + 4;
-    b.sa_full = x + 5; b.sa_free = x + 6; b.dq_full = x + 7; b.dq_free = x + 8; b.osync = x + 9;
-    b.r_full = x + 10; b.r_free = x + 11; b.fin = x + 12;
+    b.sa_full = x + 5; b.sa_free = x + 6; b.dq_full = x + 7; b.dq_free = x + 8;
+    b.r_full = x + 9; b.r_free = x + 10; b.fin = x + 11;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -494,7 +482,6 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         mbar_init(b.sa_free, 1);
         mbar_init(b.dq_full, 1);
         mbar_init(b.dq_free, kEpiWarps);
-        mbar_init(b.osync, kEpiWarps);
         mbar_init(b.r_full, 1);
         mbar_init(b.r_free, kEpiWarps);
         mbar_init(b.fin, 1);
@@ -507,8 +494,6 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_g);
         prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_dq);
-        prefetch_tmap(&tm_qdq);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -522,7 +507,7 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     } else if (warp >= kEpiWarps) {
         gate_role(smem, b, abort, a, nchunks, dstate, cpf, bh, j);
     } else {
-        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks, &tm_dq, &tm_qdq, dstate);
+        epilogue_role(smem, b, abort, a, tmem, bh, j, row0, nchunks, dstate);
     }
     tc_fence_before();
     __syncthreads();
@@ -1122,22 +1107,19 @@ bool tc_bwd_supported(const BwdArgs &a) {
 
 cudaError_t launch_tc_dq(const BwdArgs &a, cudaStream_t st) {
     const long long rows = (long long)a.BH * a.L;
-    CUtensorMap mk, mv, mdo, mg, mq, mdq, mqdq;
+    CUtensorMap mk, mv, mdo, mg, mq;
     cudaError_t e;
     if ((e = make_map(&mk, a.k, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mdo, a.dO, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mq, a.q, rows)) != cudaSuccess) return e;
-    if ((e = make_map(&mdq, a.dq_out, rows)) != cudaSuccess) return e;
-    if ((e = make_map_f32(&mqdq, a.dq_ws, rows)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(dqs::tc_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dqs::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long nblk = (long long)a.BH * a.NP;
     if (nblk == 0) return cudaSuccess;
-    dqs::tc_dq_kernel<<<(unsigned)nblk, kThreads, dqs::kSmemBytes, st>>>(mk, mv, mdo, mg, mq, mdq,
-                                                                        mqdq, a);
+    dqs::tc_dq_kernel<<<(unsigned)nblk, kThreads, dqs::kSmemBytes, st>>>(mk, mv, mdo, mg, mq, a);
     return cudaGetLastError();
 }
 

@@ -96,25 +96,5 @@ inline cudaError_t make_map(CUtensorMap *m, const void *base, long long rows) {
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// fp32 [rows x 128] tensor (e.g. q . dq) in 32-column boxes of 64 rows with the 128-byte swizzle.
-inline cudaError_t make_map_f32(CUtensorMap *m, const void *base, long long rows) {
-    auto fn = encode_fn();
-    if (!fn) return cudaErrorNotSupported;
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 4};
-    const cuuint32_t box[2] = {32, (cuuint32_t)CH};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-// Byte offset of element (t, i) of a [64 x 128] fp32 tile stored as four 32-column boxes of
-// 64 rows (8 KiB each) with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t tile_off32(int t, int i) {
-    return (uint32_t)((i >> 5) * 8192 + t * 128 + ((((i & 31) >> 2) ^ (t & 7)) << 4) + ((i & 3) << 2));
-}
-
 }  // namespace tc
 }  // namespace la
