@@ -16,19 +16,6 @@ constexpr int kEpiWarps = 8, kGateWarps = 4;
 constexpr int kTmaWarp = 12, kMmaWarp = 13;
 constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
 
-// Stores the bf16 values of tokens s and s+1 of this lane's dim x into a [64 x 128] swizzled
-// tile.  Lanes x and x^1 swap one value so that each writes one 4-byte word (dims x & ~1 and
-// x | 1): the even lane row s, the odd lane row s+1.  Two-byte stores would put two lanes on
-// each 4-byte word and take two shared-memory wavefronts per instruction.
-__device__ __forceinline__ void store_pair(uint32_t tile, int s, int x, float a, float b) {
-    const uint32_t p = pack_bf16(a, b);  // low half: token s, high half: token s+1
-    const bool odd = x & 1;
-    const uint32_t send = odd ? (p & 0xFFFFu) : (p >> 16);
-    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-    const uint32_t w = odd ? (recv | (p & 0xFFFF0000u)) : ((p & 0xFFFFu) | (recv << 16));
-    sts_u32(tile + tile_off(s + (odd ? 1 : 0), x & ~1), w);
-}
-
 // ------------------------------------------------------------------ reverse sweep
 // Per chunk, last to first, with dS the gradient of the state at the chunk's end (rows = key
 // dims; starts at dX of the part), Qbar'_t = q_t e^{b_t - b_C}, Ktil_s = k_s e^{b_C - b_s}:
@@ -61,7 +48,7 @@ constexpr int off_ma = kStages * kStageBytes;  // 2 buffers x (M tile, A tile)
 constexpr int off_ds = off_ma + 4 * kMaskBytes;
 constexpr int off_ec = off_ds + 2 * kDsHalf;
 constexpr int off_bar = off_ec + kStages * D * 4;
-constexpr int kBars = 3 * kStages + 15;
+constexpr int kBars = 3 * kStages + 14;
 constexpr int off_misc = off_bar + kBars * 8;
 constexpr int kSmemBytes = off_misc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -69,7 +56,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 struct Bars {
     uint64_t *full, *gated, *empty;
     uint64_t *mm_full, *mm_free, *p_full, *dst_full, *dk_full, *dk_free, *dv_full, *dv_free,
-        *dsn_full, *osync, *fin;
+        *dsn_full, *fin;
 };
 
 // [128 rows][128 cols] bf16 tile as two 64-column halves of 16 KiB, 128-byte swizzle.
@@ -392,15 +379,27 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
     }
 }
 
+// Stores the bf16 values of tokens t and t+1 of this lane's dim x into a [tokens, 128] bf16
+// tensor: lanes x and x^1 swap one value so that each writes one 4-byte word (dims x & ~1 and
+// x | 1), the even lane row t, the odd lane row t+1.  `row` points at word (x & ~1) / 2 of row
+// t for even lanes and of row t+1 for odd lanes.
+__device__ __forceinline__ void stg_pair(uint32_t *row, bool odd, float a, float b) {
+    const uint32_t p = pack_bf16(a, b);  // low half: token t, high half: token t+1
+    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, odd ? (p & 0xFFFFu) : (p >> 16), 1);
+    *row = odd ? (recv | (p & 0xFFFF0000u)) : ((p & 0xFFFFu) | (recv << 16));
+}
+
 // Warps 4-7: thread x = 32 (warp - 4) + lane owns key dim x of dk / dlog_g and value dim x of
-// dv for all 64 tokens of the chunk.
+// dv for all 64 tokens of the chunk; the outputs go straight from registers to HBM, and each
+// warp releases the stage as soon as it has read the chunk's factors and Ktil.
 __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
-                         uint32_t tmem, int bh, int j, long long row0, int nchunks,
-                         const CUtensorMap *tdk, const CUtensorMap *tdv, const CUtensorMap *tdg) {
+                         uint32_t tmem, int bh, int j, long long row0, int nchunks) {
     const int quarter = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
     const int x = quarter * 32 + lane;
     const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
-    const bool storer = threadIdx.x == 32 * kStateWarps;
+    __nv_bfloat16 *dk = static_cast<__nv_bfloat16 *>(a.dk_out);
+    __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv_out);
+    __nv_bfloat16 *dg = static_cast<__nv_bfloat16 *>(a.dg_out);
     const long long sidx = ((long long)bh * a.NP + j) * D * D;
     // carry: rowsum(S_end . dX), the gradient reaching this part from its end state
     float carry = 0.f;
@@ -432,12 +431,7 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
         // while this thread waits for dk; each later group is loaded one group ahead
 #pragma unroll
         for (int t = 0; t < 16; ++t) qn[t] = qdq[(48 + t) * D];
-        if (it > 0 && storer) {  // the previous chunk's output tiles are read out: release its stage
-            bulk_wait_read();
-            mbar_arrive(&b.empty[(it - 1) % kStages]);
-        }
-        // (1) dk and the dlog_g suffix sums: tokens last to first, 16 at a time.  dk_full also
-        // means the dS update is done, so the v and q tiles are free for dk and dlog_g.
+        // (1) dk and the dlog_g suffix sums: tokens last to first, 16 at a time
         if (!mbar_wait(&b.dk_full[bb], (it >> 1) & 1, abort)) break;
         tc_fence_after();
         const uint32_t sa = smem_u32(st);
@@ -458,11 +452,11 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
             }
             // dk = e^{b_C - b_s} acc and the contribution q . dq - k . dk (k . dk = Ktil . acc,
             // Ktil = k e^{b_C - b_s} the MMA operand); then the suffix sums
-            float f[16], c[16];
+            float fd[16], cg[16];  // dk, then contributions / dlog_g
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
-                f[t] = __uint_as_float(fk[t] << 16);
-                c[t] = __uint_as_float(fk[t] & 0xFFFF0000u);
+                fd[t] = __uint_as_float(fk[t] << 16);
+                cg[t] = __uint_as_float(fk[t] & 0xFFFF0000u);
             }
             if (g > 0) {  // the next group's loads go out before this group's stores
 #pragma unroll
@@ -480,21 +474,25 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
                 const float acc = __uint_as_float(r[t]);
-                f[t] *= acc;                  // dk
-                c[t] = qv[t] - c[t] * acc;    // contribution
+                fd[t] *= acc;                  // dk
+                cg[t] = qv[t] - cg[t] * acc;    // contribution
             }
 #pragma unroll
             for (int t = 15; t >= 0; --t) {
-                carry += c[t];
-                c[t] = carry;                 // dlog_g
+                carry += cg[t];
+                cg[t] = carry;                 // dlog_g
             }
+            const long long w0 = ((row0 + (long long)c * CH + g * 16 + (x & 1)) * D + (x & ~1)) / 2;
+            uint32_t *dkw = reinterpret_cast<uint32_t *>(dk) + w0, *dgw = reinterpret_cast<uint32_t *>(dg) + w0;
 #pragma unroll
-            for (int t = 0; t < 16; t += 2) {
-                store_pair(sa + off_v, g * 16 + t, x, f[t], f[t + 1]);
-                store_pair(sa + off_q, g * 16 + t, x, c[t], c[t + 1]);
+            for (int t = 0; t < 16; t += 2) {  // row stride: D / 2 words
+                stg_pair(dkw + t * (D / 2), x & 1, fd[t], fd[t + 1]);
+                stg_pair(dgw + t * (D / 2), x & 1, cg[t], cg[t + 1]);
             }
         }
-        // (2) dv into the dO tile (its last readers, the dv MMAs, are done)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.empty[s]);  // this warp's reads of the stage are done
+        // (2) dv
         if (!mbar_wait(&b.dv_full[bb], (it >> 1) & 1, abort)) break;
         tc_fence_after();
 #pragma unroll 1
@@ -506,35 +504,19 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&b.dv_free[bb]);
             }
+            uint32_t *dvw = reinterpret_cast<uint32_t *>(dv) +
+                            ((row0 + (long long)c * CH + g * 16 + (x & 1)) * D + (x & ~1)) / 2;
 #pragma unroll
             for (int t = 0; t < 16; t += 2)
-                store_pair(sa + off_do, g * 16 + t, x, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
-        }
-        // (3) once all four warps' values are in the tiles, one thread stores them
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b.osync);
-        if (!mbar_wait(b.osync, it & 1, abort)) break;
-        if (storer) {
-            const int y = (int)(row0 + (long long)c * CH);
-            tma_store_2d(tdk, 0, y, st + off_v);
-            tma_store_2d(tdk, 64, y, st + off_v + kHalfBytes);
-            tma_store_2d(tdg, 0, y, st + off_q);
-            tma_store_2d(tdg, 64, y, st + off_q + kHalfBytes);
-            tma_store_2d(tdv, 0, y, st + off_do);
-            tma_store_2d(tdv, 64, y, st + off_do + kHalfBytes);
-            bulk_commit();
+                stg_pair(dvw + t * (D / 2), x & 1, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
         }
     }
-    if (storer) bulk_wait_all();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-              const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_dk,
-              const __grid_constant__ CUtensorMap tm_dv, const __grid_constant__ CUtensorMap tm_dg,
-              const BwdArgs a) {
+              const __grid_constant__ CUtensorMap tm_g, const BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -545,8 +527,7 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     b.empty = bar + 2 * kStages;
     uint64_t *x = bar + 3 * kStages;
     b.mm_full = x + 0; b.mm_free = x + 1; b.p_full = x + 2; b.dst_full = x + 3; b.dk_full = x + 4;
-    b.dk_free = x + 6; b.dv_full = x + 8; b.dv_free = x + 10; b.dsn_full = x + 12; b.osync = x + 13;
-    b.fin = x + 14;
+    b.dk_free = x + 6; b.dv_full = x + 8; b.dv_free = x + 10; b.dsn_full = x + 12; b.fin = x + 13;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -557,12 +538,12 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&b.full[s], 1);
             mbar_init(&b.gated[s], kGateWarps);
-            mbar_init(&b.empty[s], 1 + kStateWarps + 1);  // MMA, dS warps, output storer
+            mbar_init(&b.empty[s], 1 + kStateWarps + kOutWarps);
         }
         uint64_t *one[] = {b.mm_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dv_full + 1,
                            b.dsn_full, b.fin};
         uint64_t *st4[] = {b.mm_free, b.p_full, b.dst_full};
-        uint64_t *out4[] = {b.dk_free, b.dk_free + 1, b.dv_free, b.dv_free + 1, b.osync};
+        uint64_t *out4[] = {b.dk_free, b.dk_free + 1, b.dv_free, b.dv_free + 1};
         for (uint64_t *p : one) mbar_init(p, 1);
         for (uint64_t *p : st4) mbar_init(p, kStateWarps);
         for (uint64_t *p : out4) mbar_init(p, kOutWarps);
@@ -575,9 +556,6 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_g);
-        prefetch_tmap(&tm_dk);
-        prefetch_tmap(&tm_dv);
-        prefetch_tmap(&tm_dg);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -594,7 +572,7 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     } else if (warp < kStateWarps) {
         state_role(smem, b, abort, a, tmem, bh, j, nchunks);
     } else {
-        out_role(smem, b, abort, a, tmem, bh, j, row0, nchunks, &tm_dk, &tm_dv, &tm_dg);
+        out_role(smem, b, abort, a, tmem, bh, j, row0, nchunks);
     }
     tc_fence_before();
     __syncthreads();
@@ -616,23 +594,19 @@ bool tc_bwd_supported(const BwdArgs &a) {
 
 cudaError_t launch_tc_dkv(const BwdArgs &a, cudaStream_t st) {
     const long long rows = (long long)a.BH * a.L;
-    CUtensorMap mq, mk, mv, mdo, mg, mdk, mdv, mdg;
+    CUtensorMap mq, mk, mv, mdo, mg;
     cudaError_t e;
     if ((e = make_map(&mq, a.q, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mk, a.k, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mdo, a.dO, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
-    if ((e = make_map(&mdk, a.dk_out, rows)) != cudaSuccess) return e;
-    if ((e = make_map(&mdv, a.dv_out, rows)) != cudaSuccess) return e;
-    if ((e = make_map(&mdg, a.dg_out, rows)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(dkv::tc_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dkv::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long nblk = (long long)a.BH * a.NP;
     if (nblk == 0) return cudaSuccess;
-    dkv::tc_dkv_kernel<<<(unsigned)nblk, kThreads, dkv::kSmemBytes, st>>>(mq, mk, mv, mdo, mg, mdk,
-                                                                          mdv, mdg, a);
+    dkv::tc_dkv_kernel<<<(unsigned)nblk, kThreads, dkv::kSmemBytes, st>>>(mq, mk, mv, mdo, mg, a);
     return cudaGetLastError();
 }
 
