@@ -380,13 +380,12 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
 }
 
 // Stores the bf16 values of tokens t and t+1 of this lane's dim x into a [tokens, 128] bf16
-// tensor: lanes x and x^1 swap one value so that each writes one 4-byte word (dims x & ~1 and
-// x | 1), the even lane row t, the odd lane row t+1.  `row` points at word (x & ~1) / 2 of row
-// t for even lanes and of row t+1 for odd lanes.
-__device__ __forceinline__ void stg_pair(uint32_t *row, bool odd, float a, float b) {
+// tensor (one conversion, two 2-byte stores).  `at` points at element (t, x).
+__device__ __forceinline__ void stg_pair(__nv_bfloat16 *at, float a, float b) {
     const uint32_t p = pack_bf16(a, b);  // low half: token t, high half: token t+1
-    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, odd ? (p & 0xFFFFu) : (p >> 16), 1);
-    *row = odd ? (recv | (p & 0xFFFF0000u)) : ((p & 0xFFFFu) | (recv << 16));
+    unsigned short *h = reinterpret_cast<unsigned short *>(at);
+    h[0] = (unsigned short)(p & 0xFFFFu);
+    h[D] = (unsigned short)(p >> 16);
 }
 
 // Warps 4-7: thread x = 32 (warp - 4) + lane owns key dim x of dk / dlog_g and value dim x of
@@ -482,12 +481,11 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                 carry += cg[t];
                 cg[t] = carry;                 // dlog_g
             }
-            const long long w0 = ((row0 + (long long)c * CH + g * 16 + (x & 1)) * D + (x & ~1)) / 2;
-            uint32_t *dkw = reinterpret_cast<uint32_t *>(dk) + w0, *dgw = reinterpret_cast<uint32_t *>(dg) + w0;
+            const long long e0 = (row0 + (long long)c * CH + g * 16) * D + x;  // element (t0, x)
 #pragma unroll
-            for (int t = 0; t < 16; t += 2) {  // row stride: D / 2 words
-                stg_pair(dkw + t * (D / 2), x & 1, fd[t], fd[t + 1]);
-                stg_pair(dgw + t * (D / 2), x & 1, cg[t], cg[t + 1]);
+            for (int t = 0; t < 16; t += 2) {
+                stg_pair(dk + e0 + t * D, fd[t], fd[t + 1]);
+                stg_pair(dg + e0 + t * D, cg[t], cg[t + 1]);
             }
         }
         __syncwarp();
@@ -504,11 +502,10 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&b.dv_free[bb]);
             }
-            uint32_t *dvw = reinterpret_cast<uint32_t *>(dv) +
-                            ((row0 + (long long)c * CH + g * 16 + (x & 1)) * D + (x & ~1)) / 2;
+            __nv_bfloat16 *dvt = dv + (row0 + (long long)c * CH + g * 16) * D + x;
 #pragma unroll
             for (int t = 0; t < 16; t += 2)
-                stg_pair(dvw + t * (D / 2), x & 1, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
+                stg_pair(dvt + t * D, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
         }
     }
 }

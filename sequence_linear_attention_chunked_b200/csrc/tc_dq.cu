@@ -382,7 +382,7 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
 // ------------------------------------------------------------------ output warps (4-7)
 // (a) M -> causal mask -> bf16 P tile (buffer c % 2); (d) dq^T read-out: thread i owns key dim
 // i; dq = F . dq^T with F = e^{b_t - b_C} from the gates, q . dq in fp32 -- stored straight from
-// registers (q . dq as one 128-byte line per warp and token, dq as lane-paired 4-byte words).
+// registers (q . dq as one 128-byte line per warp and token, dq as 2-byte stores per token).
 // dq of chunk c is read out before M of chunk c+1 is masked: the read-out releases the stage
 // that chunk c+2 loads into, while M(c+1) can only be formed once chunk c+1 has landed.
 __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
@@ -433,7 +433,6 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + s * kStageBytes);
         const long long tok0 = w.row0 + (long long)c * CH;
-        const bool odd = i & 1;
 #pragma unroll 1
         for (int g = 0; g < 4; ++g) {  // tokens 16g .. 16g+15
             uint32_t r16[16];
@@ -460,9 +459,9 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                     a.dq_ws[t * D + i] = __uint_as_float(fq[e] & 0xFFFF0000u) * v0;
                     a.dq_ws[(t + 1) * D + i] = __uint_as_float(fq[e + 1] & 0xFFFF0000u) * v1;
                     const uint32_t p = pack_bf16(v0, v1);  // low: token t, high: token t+1
-                    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, odd ? (p & 0xFFFFu) : (p >> 16), 1);
-                    const uint32_t wd = odd ? (recv | (p & 0xFFFF0000u)) : ((p & 0xFFFFu) | (recv << 16));
-                    *reinterpret_cast<uint32_t *>(dq + (t + (odd ? 1 : 0)) * D + (i & ~1)) = wd;
+                    unsigned short *h = reinterpret_cast<unsigned short *>(dq + t * D + i);
+                    h[0] = (unsigned short)(p & 0xFFFFu);
+                    h[D] = (unsigned short)(p >> 16);
                 }
             }
         }
