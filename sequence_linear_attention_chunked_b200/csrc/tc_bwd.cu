@@ -48,14 +48,14 @@ constexpr int off_ma = kStages * kStageBytes;  // 2 buffers x (M tile, A tile)
 constexpr int off_ds = off_ma + 4 * kMaskBytes;
 constexpr int off_ec = off_ds + 2 * kDsHalf;
 constexpr int off_bar = off_ec + kStages * D * 4;
-constexpr int kBars = 3 * kStages + 14;
+constexpr int kBars = 3 * kStages + 16;
 constexpr int off_misc = off_bar + kBars * 8;
 constexpr int kSmemBytes = off_misc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Bars {
     uint64_t *full, *gated, *empty;
-    uint64_t *mm_full, *mm_free, *p_full, *dst_full, *dk_full, *dk_free, *dv_full, *dv_free,
+    uint64_t *m_full, *m_free, *a_full, *a_free, *p_full, *dst_full, *dk_full, *dk_free, *dv_full, *dv_free,
         *dsn_full, *fin;
 };
 
@@ -109,24 +109,35 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
     const uint32_t base = smem_u32(smem);
     const uint32_t ma_addr = base + off_ma, ds_addr = base + off_ds;
     auto stage = [&](int it) { return base + (uint32_t)((it % kStages) * kStageBytes); };
-    auto issue_ma = [&](int it) {
+    // M = dO V^T reads untouched tiles: issued as soon as the chunk lands, so the dS warps mask
+    // it while the gates work; A = Qbar' Ktil^T once the tiles are gated.
+    auto issue_ma = [&](int it) -> bool {
         const uint32_t st = stage(it);
+        if (!warp_wait(&b.full[it % kStages], (it / kStages) & 1, abort)) return false;
+        if (it > 0 && !warp_wait(b.m_free, (it - 1) & 1, abort)) return false;
+        tc_fence_after();
         if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // M = dO V^T
+            for (int kk = 0; kk < 8; ++kk)
                 mma_ss(tmem + kColM, desc_kmajor(st + off_do, kk), desc_kmajor(st + off_v, kk), i_sq,
                        kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // A = Qbar' Ktil^T
-                mma_ss(tmem + kColA, desc_kmajor(st + off_q, kk), desc_kmajor(st + off_k, kk), i_sq,
-                       kk > 0);
-            mma_commit(b.mm_full);
+            mma_commit(b.m_full);
         }
         __syncwarp();
+        if (!warp_wait(&b.gated[it % kStages], (it / kStages) & 1, abort)) return false;
+        if (it > 0 && !warp_wait(b.a_free, (it - 1) & 1, abort)) return false;
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + kColA, desc_kmajor(st + off_q, kk), desc_kmajor(st + off_k, kk), i_sq,
+                       kk > 0);
+            mma_commit(b.a_full);
+        }
+        __syncwarp();
+        return true;
     };
-    bool ok = nchunks > 0 && warp_wait(&b.gated[0], 0, abort);
-    tc_fence_after();
-    if (ok) issue_ma(0);
+    bool ok = nchunks > 0 && issue_ma(0);
     for (int it = 0; ok && it < nchunks; ++it) {
         const int s = it % kStages, bb = it & 1;
         const uint32_t st = stage(it);
@@ -166,12 +177,7 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
             mma_commit(&b.empty[s]);
         }
         __syncwarp();
-        if (it + 1 < nchunks) {  // the next chunk's M and A, once its tiles are gated
-            if (!(ok = warp_wait(&b.gated[(it + 1) % kStages], ((it + 1) / kStages) & 1, abort))) break;
-            if (!(ok = warp_wait(b.mm_free, it & 1, abort))) break;
-            tc_fence_after();
-            issue_ma(it + 1);
-        }
+        if (it + 1 < nchunks && !(ok = issue_ma(it + 1))) break;  // the next chunk's M and A
     }
     if (elect_one()) mma_commit(b.fin);
     __syncwarp();
@@ -358,21 +364,24 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
             mbar_arrive(b.dst_full);
             if (it > 0) mbar_arrive(&b.empty[(it - 1) % kStages]);  // its e^{b_C} is used
         }
-        // (2) masked M and A tiles of this chunk (M=64 layout: lanes 0-15 hold row 16 warp + lane)
-        if (!mbar_wait(b.mm_full, it & 1, abort)) break;
-        tc_fence_after();
+        // (2) masked M and A tiles of this chunk (M=64 layout: lanes 0-15 hold row 16 warp + lane);
+        // M is ready before the gates finish, A only after
         uint8_t *mt = smem + off_ma + (it & 1) * 2 * kMaskBytes;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {  // M half 0, M half 1, A half 0, A half 1
+            if (t == 0 && !mbar_wait(b.m_full, it & 1, abort)) break;
+            if (t == 2 && !mbar_wait(b.a_full, it & 1, abort)) break;
+            if ((t & 1) == 0) tc_fence_after();
             tmem_ld32(tmem + lrow + (t < 2 ? kColM : kColA) + (t & 1) * 32, r);
             tmem_wait_ld();
-            if (t == 3) {
+            if (t & 1) {
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(b.mm_free);
+                if (lane == 0) mbar_arrive(t == 1 ? b.m_free : b.a_free);
             }
             masked_tile(mt + (t >> 1) * kMaskBytes, r, warp, t & 1, lane);
         }
+        if (*abort) break;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(b.p_full);
@@ -523,8 +532,9 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     b.gated = bar + kStages;
     b.empty = bar + 2 * kStages;
     uint64_t *x = bar + 3 * kStages;
-    b.mm_full = x + 0; b.mm_free = x + 1; b.p_full = x + 2; b.dst_full = x + 3; b.dk_full = x + 4;
+    b.m_full = x + 0; b.m_free = x + 1; b.p_full = x + 2; b.dst_full = x + 3; b.dk_full = x + 4;
     b.dk_free = x + 6; b.dv_full = x + 8; b.dv_free = x + 10; b.dsn_full = x + 12; b.fin = x + 13;
+    b.a_full = x + 14; b.a_free = x + 15;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -537,9 +547,9 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&b.gated[s], kGateWarps);
             mbar_init(&b.empty[s], 1 + kStateWarps + kOutWarps);
         }
-        uint64_t *one[] = {b.mm_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dv_full + 1,
+        uint64_t *one[] = {b.m_full, b.a_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dv_full + 1,
                            b.dsn_full, b.fin};
-        uint64_t *st4[] = {b.mm_free, b.p_full, b.dst_full};
+        uint64_t *st4[] = {b.m_free, b.a_free, b.p_full, b.dst_full};
         uint64_t *out4[] = {b.dk_free, b.dk_free + 1, b.dv_free, b.dv_free + 1};
         for (uint64_t *p : one) mbar_init(p, 1);
         for (uint64_t *p : st4) mbar_init(p, kStateWarps);
