@@ -371,53 +371,84 @@ def bench_e2e(args, w, x, device, world):
     """Same metric through the public entry points with host buffers: per step, pinned host ->
     device copies of the inputs (q, k, v, log_g, and dO for fwd+bwd), la_seg_forward (saving
     the received states), la_seg_backward reusing them, and device -> host copies of the
-    results (o and S_final; dq, dk, dv, dlog_g and dS0 for fwd+bwd)."""
+    results (o and S_final; dq, dk, dv, dlog_g and dS0 for fwd+bwd).  Steps are pipelined over
+    three streams with two sets of device buffers, as a serving loop would run them: step i's
+    inputs are copied in while step i-1 computes and step i-2's results are copied out (PCIe
+    moves both directions at once).  Every step copies all of its inputs in and all of its
+    results out inside the timed region."""
     from sequence_linear_attention_chunked_b200 import la_seg
     names = ("q", "k", "v", "log_g") + (("dO",) if w.backward else ())
     host = {n: x[n].cpu().pin_memory() for n in names}
-    dev = {n: torch.empty_like(x[n]) for n in names}
     dt = la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16
-    ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device)
-    wsb = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, device) if w.backward else None
     f32 = dict(dtype=torch.float32, device=device)
-    o_dev = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype, device=device)
-    Sf = torch.empty((w.B, w.H, w.dk, w.dv), **f32)
-    Sr = torch.empty((w.B, w.H, w.P, w.dk, w.dv), **f32) if w.backward else None
-    outs = [o_dev, Sf]
-    if w.backward:
-        grads = [torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
-                 torch.empty_like(x["log_g"]), torch.empty_like(Sf)]
-        outs += grads
-    outs_host = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+    ws = [la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device) for _ in range(2)]
+    wsb = ([la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, device)
+            for _ in range(2)] if w.backward else [None, None])
+    bufs = []
+    for _ in range(2):  # two sets of device inputs and outputs
+        d = {n: torch.empty_like(x[n]) for n in names}
+        o_dev = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype, device=device)
+        Sf = torch.empty((w.B, w.H, w.dk, w.dv), **f32)
+        Sr = torch.empty((w.B, w.H, w.P, w.dk, w.dv), **f32) if w.backward else None
+        outs = [o_dev, Sf]
+        grads = None
+        if w.backward:
+            grads = [torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
+                     torch.empty_like(x["log_g"]), torch.empty_like(Sf)]
+            outs += grads
+        bufs.append(dict(inp=d, o=o_dev, Sf=Sf, Sr=Sr, grads=grads, outs=outs,
+                         host_out=[torch.empty_like(t, device="cpu").pin_memory() for t in outs]))
     steps = max(3, min(args.steps, 20))
     P = la_seg._ptr
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of a buffer set copied in
+    ev_comp = [torch.cuda.Event() for _ in range(2)]   # step done reading inputs, outputs written
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # outputs of a buffer set copied out
+    used = [False, False]
 
-    def one():
-        for n in names:
-            dev[n].copy_(host[n], non_blocking=True)
+    def one(i):
+        k = i % 2
+        bf = bufs[k]
+        with torch.cuda.stream(s_in):
+            if used[k]:
+                s_in.wait_event(ev_comp[k])  # the step two back has read these inputs
+            for n in names:
+                bf["inp"][n].copy_(host[n], non_blocking=True)
+            ev_in[k].record(s_in)
+        s_comp.wait_event(ev_in[k])
+        if used[k]:
+            s_comp.wait_event(ev_out[k])  # the step two back's results are copied out
+        st = la_seg._stream(s_comp)
+        d = bf["inp"]
         la_seg._check(la_seg.lib().la_seg_forward(
-            P(dev["q"]), P(dev["k"]), P(dev["v"]), P(dev["log_g"]), None, w.B, w.H, w.L, w.dk, w.dv,
-            w.P, w.chunk, dt, P(o_dev), P(Sf), P(Sr), 0, P(ws), ws.numel(), la_seg._stream(None)),
+            P(d["q"]), P(d["k"]), P(d["v"]), P(d["log_g"]), None, w.B, w.H, w.L, w.dk, w.dv,
+            w.P, w.chunk, dt, P(bf["o"]), P(bf["Sf"]), P(bf["Sr"]), 0, P(ws[k]), ws[k].numel(), st),
             "la_seg_forward")
         if w.backward:
+            g = bf["grads"]
             la_seg._check(la_seg.lib().la_seg_backward(
-                P(dev["q"]), P(dev["k"]), P(dev["v"]), P(dev["log_g"]), None, P(Sr), P(dev["dO"]),
-                None, w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, P(grads[0]), P(grads[1]),
-                P(grads[2]), P(grads[3]), P(grads[4]), P(wsb), wsb.numel(), la_seg._stream(None)),
-                "la_seg_backward")
-        for d, h in zip(outs, outs_host):
-            h.copy_(d, non_blocking=True)
+                P(d["q"]), P(d["k"]), P(d["v"]), P(d["log_g"]), None, P(bf["Sr"]), P(d["dO"]),
+                None, w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, P(g[0]), P(g[1]), P(g[2]),
+                P(g[3]), P(g[4]), P(wsb[k]), wsb[k].numel(), st), "la_seg_backward")
+        ev_comp[k].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[k])
+            for dv_, h in zip(bf["outs"], bf["host_out"]):
+                h.copy_(dv_, non_blocking=True)
+            ev_out[k].record(s_out)
+        used[k] = True
 
-    for _ in range(3):
-        one()
+    for i in range(3):
+        one(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    e0.record(s_in)
+    for i in range(steps):
+        one(i)
+    s_out.wait_event(ev_comp[(steps - 1) % 2])
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     t = torch.tensor([ms], dtype=torch.float64, device=device)
@@ -425,11 +456,12 @@ def bench_e2e(args, w, x, device, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = sum(v.numel() * v.element_size() for v in outs_host)
+    d2h = sum(v.numel() * v.element_size() for v in bufs[0]["host_out"])
     api = "la_seg_forward" + (" + la_seg_backward" if w.backward else "")
     return {"value": round(w.B * w.L * world * steps / (ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": f"{api} (C ABI) with pinned host buffers"}
+            "api": f"{api} (C ABI) with pinned host buffers, steps pipelined over copy-in, "
+                   "compute and copy-out streams"}
 
 
 # ----------------------------------------------------------------------------- oracle arm
