@@ -142,7 +142,8 @@ class Step:
     forms the gradient states), reverse scan, dk/dv/dlog_g pass, reusing the forward's received
     states."""
 
-    KERNEL_KEYS = {"state pass": "state_pass", "output pass": "output_pass",
+    KERNEL_KEYS = {"chain reset": "chain_reset", "single pass": "chain_kernel",
+                   "state pass": "state_pass", "output pass": "output_pass",
                    "local pass": "local_pass", "correction pass": "correct_pass",
                    "state scan": "scan", "dq pass": "dq_pass", "reverse scan": "scan",
                    "dkv pass": "dkv_pass"}
@@ -162,8 +163,14 @@ class Step:
         self.S_recv = torch.empty((B, H, NP, dk, dv), **f32)
         self.S_final = torch.empty((B, H, dk, dv), **f32)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
-        self.phases = (["state pass", "state scan", "output pass"] if schedule != "three"
-                       else ["local pass", "state scan", "correction pass"])
+        if schedule == "single":  # the same sub-segments; S_recv saved for the backward
+            self.phases = ["chain reset", "single pass"]
+            self.chain = la_seg.chain_buffers(B, H, dk, dv, device)
+        elif schedule == "three":
+            self.phases = ["local pass", "state scan", "correction pass"]
+        else:
+            self.phases = ["state pass", "state scan", "output pass"]
+        self.n_fwd = len(self.phases)
         if w.backward:
             # the backward's fine split (parts of <= 1024 tokens) under the forward's segments
             self.NPF = la_seg.la_seg_backward_parts(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt,
@@ -188,38 +195,47 @@ class Step:
         rec = (lambda i: ev[i].record()) if record else (lambda i: None)
         BH = w.B * w.H
         rec(0)
-        if self.schedule != "three":
-            la.la_seg_state_pass(x["k"], x["v"], x["log_g"], NP, w.chunk, S_loc=self.S_loc,
-                                 log_gamma=self.logG, status=self.status)
+        if self.schedule == "single":
+            la.la_seg_chain_reset(None, w.B, w.H, w.dk, w.dv, *self.chain)
+            rec(1)
+            la.la_seg_chain_pass(x["q"], x["k"], x["v"], x["log_g"], NP, w.chunk, *self.chain,
+                                 o=self.o, S_final=self.S_final, S_recv_save=self.S_recv,
+                                 save_every=1, status=self.status)
+            rec(2)
         else:
-            la.la_seg_local_pass(x["q"], x["k"], x["v"], x["log_g"], NP, w.chunk, o=self.o,
-                                 S_loc=self.S_loc, log_gamma=self.logG, status=self.status)
-        rec(1)
-        la._check(la.lib().la_seg_scan(la._ptr(self.S_loc), la._ptr(self.logG), None, BH, NP, w.dk,
-                                       w.dv, 0, la._ptr(self.S_recv), la._ptr(self.S_final),
-                                       la._stream(None)), "la_seg_scan")
-        rec(2)
-        if self.schedule != "three":
-            la.la_seg_output_pass(x["q"], x["k"], x["v"], x["log_g"], self.S_recv, NP, w.chunk,
-                                  o=self.o, status=self.status)
-        else:
-            la.la_seg_correct_pass(x["q"], x["log_g"], self.S_recv, NP, w.chunk, self.o,
-                                   status=self.status)
-        rec(3)
+            if self.schedule != "three":
+                la.la_seg_state_pass(x["k"], x["v"], x["log_g"], NP, w.chunk, S_loc=self.S_loc,
+                                     log_gamma=self.logG, status=self.status)
+            else:
+                la.la_seg_local_pass(x["q"], x["k"], x["v"], x["log_g"], NP, w.chunk, o=self.o,
+                                     S_loc=self.S_loc, log_gamma=self.logG, status=self.status)
+            rec(1)
+            la._check(la.lib().la_seg_scan(la._ptr(self.S_loc), la._ptr(self.logG), None, BH, NP,
+                                           w.dk, w.dv, 0, la._ptr(self.S_recv),
+                                           la._ptr(self.S_final), la._stream(None)), "la_seg_scan")
+            rec(2)
+            if self.schedule != "three":
+                la.la_seg_output_pass(x["q"], x["k"], x["v"], x["log_g"], self.S_recv, NP,
+                                      w.chunk, o=self.o, status=self.status)
+            else:
+                la.la_seg_correct_pass(x["q"], x["log_g"], self.S_recv, NP, w.chunk, self.o,
+                                       status=self.status)
+            rec(3)
         if not w.backward:
             return
+        f = self.n_fwd
         la.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_recv, NP, self.fine,
                           w.chunk, dq=self.grads[0], qdq=self.qdq, S_fine=self.S_fine,
                           dSloc=self.dSloc, log_gamma=self.logG_b, status=self.status)
-        rec(4)
+        rec(f + 1)
         NPF = self.NPF
         la._check(la.lib().la_seg_scan(la._ptr(self.dSloc), la._ptr(self.logG_b), None, BH, NPF,
                                        w.dk, w.dv, 1, la._ptr(self.dX), la._ptr(self.dS0),
                                        la._stream(None)), "la_seg_scan")
-        rec(5)
+        rec(f + 2)
         la.la_seg_dkv_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_fine, None, self.dX,
                            self.qdq, NPF, w.chunk, out=self.grads[1:], status=self.status)
-        rec(6)
+        rec(f + 3)
 
     def phase_ms(self):
         return [self.events[i].elapsed_time(self.events[i + 1]) for i in range(len(self.phases))]
@@ -233,7 +249,10 @@ class Step:
         lg = w.B * w.H * self.NP * w.dk * 4
         fin = w.B * w.H * w.dk * w.dv * 4
         scan = 2 * st + lg + fin
-        if self.schedule != "three":
+        if self.schedule == "single":  # inputs read once, o and the saved states written once
+            ab = {"chain reset": 2 * w.B * w.H * w.dk * w.dv * 4,
+                  "single pass": th * (3 * w.dk + 2 * w.dv) * e + st + fin}
+        elif self.schedule != "three":
             ab = {"state pass": th * (2 * w.dk + w.dv) * e + st + lg, "state scan": scan,
                   "output pass": th * (3 * w.dk + 2 * w.dv) * e + st}
         else:
@@ -255,7 +274,9 @@ class Step:
         C, dk, dv = w.chunk, w.dk, w.dv
         intra = 2 * C * dk + 2 * C * dv  # QK^T and PV on full chunk tiles
         dd = 2 * dk * dv                 # one state-sized contraction per token
-        if self.schedule != "three":
+        if self.schedule == "single":
+            fl = {"chain reset": 0, "single pass": th * (intra + 3 * dd)}
+        elif self.schedule != "three":
             fl = {"state pass": th * dd, "state scan": 0, "output pass": th * (intra + 2 * dd)}
         else:
             fl = {"local pass": th * (intra + 2 * dd), "state scan": 0, "correction pass": th * dd}
@@ -274,7 +295,7 @@ def bench_ours(args, rank, world, device):
 
     # The per-step composition must reproduce the public entry point bit for bit.
     sched = {"auto": la_seg.SCHED_AUTO, "two": la_seg.SCHED_TWO_PASS,
-             "three": la_seg.SCHED_THREE_PHASE}[args.schedule]
+             "three": la_seg.SCHED_THREE_PHASE, "single": la_seg.SCHED_SINGLE_PASS}[args.schedule]
     ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk,
                           la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16, False, device)
     o_api, Sf_api, _ = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, w.P,
@@ -528,7 +549,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="C4", choices=sorted(WORKLOADS),
                     help="C4 (fwd+bwd, every step of the path) by default; C0-C3 forward only")
-    ap.add_argument("--schedule", default="auto", choices=["auto", "two", "three"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "two", "three", "single"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

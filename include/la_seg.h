@@ -71,14 +71,24 @@ typedef enum {
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
 
-/* Forward schedules (both compute the same result):
+/* Forward schedules (all compute the same result):
  *  LA_SCHED_AUTO    the library's choice (currently LA_SCHED_TWO_PASS).
  *  LA_SCHED_TWO_PASS ZeCO's own order: a state-only pass over k, v, log_g per segment, the
  *                   exclusive decayed scan, then one output pass per segment that starts from
  *                   the received state (so the q . S_recv term is folded into the chunk loop).
  *  LA_SCHED_THREE_PHASE  local pass (intra-chunk outputs + local states from zero), scan, then
- *                   a separate correction pass o += (q . exp(B_seg)) S_recv. */
-typedef enum { LA_SCHED_AUTO = 0, LA_SCHED_TWO_PASS = 1, LA_SCHED_THREE_PHASE = 2 } la_schedule;
+ *                   a separate correction pass o += (q . exp(B_seg)) S_recv.
+ *  LA_SCHED_SINGLE_PASS  the two-pass order in one kernel (la_seg_chain_pass over the same
+ *                   sub-segments): each sub-segment's state pass, then the scan step chained
+ *                   from its predecessor, then its output pass.  Its workspace holds two states
+ *                   per (b, h) instead of per-sub-segment state arrays.  Needs bf16,
+ *                   dk = dv = 128, chunk = 64; other shapes run LA_SCHED_TWO_PASS. */
+typedef enum {
+    LA_SCHED_AUTO = 0,
+    LA_SCHED_TWO_PASS = 1,
+    LA_SCHED_THREE_PHASE = 2,
+    LA_SCHED_SINGLE_PASS = 3
+} la_schedule;
 
 /* Bytes of workspace la_seg_forward (backward = 0) or la_seg_backward (backward = 1) needs for
  * these sizes.  Returns 0 for sizes the library rejects. */
@@ -157,6 +167,37 @@ LA_API la_status la_seg_output_pass(const void *q, const void *k, const void *v,
 LA_API la_status la_seg_correct_pass(const void *q, const void *log_g, const float *S_recv,
                                      int B, int H, long long L, int dk, int dv, int NP, int chunk,
                                      la_dtype dt, void *o, int *status, void *cuda_stream);
+
+/* Single pass (the two-pass order fused into one kernel, with the scan chained between CTAs):
+ * for every (b, h), the NP sub-segments j = 0 .. NP-1 of L/NP tokens each
+ *   1. form their local state S_j from zero and Gamma_j = diag(exp(sum of log_g over j));
+ *   2. wait until chain_ready[bh] >= j, read S_recv_j from slot j % 2 of chain_states[bh],
+ *      write S_recv_{j+1} = Gamma_j S_recv_j + S_j into slot (j + 1) % 2 (into S_final for the
+ *      last j), then set chain_ready[bh] = j + 1 (the All-Scan update of the ZeCO review's
+ *      "key machinery", chained through the sub-segments);
+ *   3. compute their outputs o from S_recv_j, as la_seg_output_pass does.
+ * Sub-segments are taken in launch order through a ticket counter, so a sub-segment only waits
+ * for ones that are already running.
+ *  chain_states   fp32 [B*H, 2, dk, dv]; slot 0 must hold the state the sequence starts from.
+ *  chain_ready    int [B*H + 1]; [bh] must be 0 and [B*H] (the ticket counter) must be 0.
+ *                 la_seg_chain_reset sets up both; the call leaves them used up.
+ *  S_final        nullable: the state after the last token, fp32 [B,H,dk,dv].
+ *  S_recv_save    nullable: the received state of every save_every-th sub-segment, fp32
+ *                 [B,H,NP/save_every,dk,dv] (save_every divides NP).
+ * A wait on chain_ready is bounded (about a second of GPU clock): when it gives up, the
+ * sub-segment computes no outputs, marks the chain as failed (chain_ready[bh] = 0x7FFFFFF0) so
+ * that its successors stop at once, and ORs 2 into *status (LA_ERR_TIMEOUT from
+ * la_seg_check_status).  Needs bf16, dk = dv = 128 and chunk = 64 (LA_ERR_SHAPE otherwise). */
+LA_API la_status la_seg_chain_pass(const void *q, const void *k, const void *v,
+                                   const void *log_g, int B, int H, long long L, int dk, int dv,
+                                   int NP, int chunk, la_dtype dt, float *chain_states,
+                                   int *chain_ready, void *o, float *S_final, float *S_recv_save,
+                                   int save_every, int *status, void *cuda_stream);
+
+/* Sets up la_seg_chain_pass's chain: slot 0 of chain_states[bh] = S0[bh] (nullable: zeros),
+ * chain_ready[bh] = 0 for every bh < B*H, ticket counter chain_ready[B*H] = 0. */
+LA_API la_status la_seg_chain_reset(const float *S0, int B, int H, int dk, int dv,
+                                    float *chain_states, int *chain_ready, void *cuda_stream);
 
 /* Gradient-state pass (what the backward's dq pass also forms): dSloc[b,h,p] = sum over segment p of
  * diag(exp(B_t)) q_t^T dO_t, B_t the inclusive cumsum of log_g from the segment's first token,

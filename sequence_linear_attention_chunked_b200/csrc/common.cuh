@@ -12,6 +12,10 @@ namespace la {
 // Bits of the device status word kept at the start of the workspace.
 enum : int { kStatusGateRange = 1, kStatusTimeout = 2 };
 
+// Value a sub-segment of the single-pass forward publishes instead of its index when it has no
+// received state to pass on (a wait before it gave up); larger than every index.
+constexpr int kChainPoison = 0x7FFFFFF0;
+
 // |sum of log_g over one chunk| above this makes exp(b_t - b_C) / exp(b_C - b_s) leave the
 // range where the chunk factorisation is accurate; the kernels flag it instead of returning
 // inf/NaN silently.

@@ -53,6 +53,26 @@ struct BwdArgs {
     la_dtype dt;
 };
 
+// The single-pass forward's chain through the sub-segments of every (b, h) sequence.
+struct ChainArgs {
+    float *states;   // [BH, 2, dk, dv]: two slots for the state a sub-segment receives; sub-segment
+                     // j reads slot j % 2 and writes the state after it into slot (j + 1) % 2
+    int *ready;      // [BH + 1]: ready[bh] = the latest sub-segment j whose received state is in
+                     // its slot (kChainPoison after a failure); ready[BH] = ticket counter
+    float *S_final;  // [BH, dk, dv] state after the last sub-segment, or null
+    float *S_save;   // [BH, NP / save_every, dk, dv] received state of every save_every-th
+                     // sub-segment, or null
+    int save_every;
+};
+
+// Single-pass forward (bf16, d = 128, chunk 64): state pass, chained scan and output pass in
+// one kernel.  ready and slot 0 of states must be set up by launch_chain_reset.
+cudaError_t launch_tc_chain(const PassArgs &a, const ChainArgs &ch, cudaStream_t st);
+
+// Slot 0 of every sequence's chain = S0 (or zeros), ready[bh] = 0, ticket counter = 0.
+cudaError_t launch_chain_reset(const float *S0, int BH, int dk, int dv, float *states, int *ready,
+                               cudaStream_t st);
+
 // Backward passes for these arguments (tensor-core kernels where they apply, else SIMT).
 cudaError_t launch_bwd_dstate(const BwdArgs &a, cudaStream_t st);
 cudaError_t launch_bwd_dq(const BwdArgs &a, cudaStream_t st);

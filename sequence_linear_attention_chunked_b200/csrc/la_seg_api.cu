@@ -83,7 +83,7 @@ la::Split make_split(int B, int H, long long L, int P, int chunk) {
 }
 
 struct FwdLayout {
-    size_t status, S_loc, logG, S_recv, total;
+    size_t status, S_loc, logG, S_recv, chain_states, chain_ready, total;
 };
 
 FwdLayout fwd_layout(const la::Split &s, int dk, int dv) {
@@ -94,7 +94,9 @@ FwdLayout fwd_layout(const la::Split &s, int dk, int dv) {
     w.S_loc = 256;
     w.logG = align_up(w.S_loc + states, 256);
     w.S_recv = align_up(w.logG + gam, 256);
-    w.total = align_up(w.S_recv + states, 256);
+    w.chain_states = align_up(w.S_recv + states, 256);
+    w.chain_ready = align_up(w.chain_states + (size_t)s.BH * 2 * dk * dv * sizeof(float), 256);
+    w.total = align_up(w.chain_ready + (size_t)(s.BH + 1) * sizeof(int), 256);
     return w;
 }
 
@@ -347,7 +349,7 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     la_status st = check_shape(B, H, L, dk, dv, P, chunk, dt);
     if (st != LA_OK) return st;
     if (schedule != LA_SCHED_AUTO && schedule != LA_SCHED_TWO_PASS &&
-        schedule != LA_SCHED_THREE_PHASE)
+        schedule != LA_SCHED_THREE_PHASE && schedule != LA_SCHED_SINGLE_PASS)
         return fail(LA_ERR_ARG, "unknown schedule %d", schedule);
     if (L > 0 && (!q || !k || !v || !log_g || !o))
         return fail(LA_ERR_ARG, "q, k, v, log_g and o must be non-null");
@@ -380,6 +382,26 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     float *logG = reinterpret_cast<float *>(at(workspace, w.logG));
     float *S_recv = reinterpret_cast<float *>(at(workspace, w.S_recv));
 
+    if (schedule == LA_SCHED_SINGLE_PASS) {  // same sub-segments as the other schedules
+        la::PassArgs a = pass_args(q, k, v, log_g, o, nullptr, nullptr, nullptr, status, B, H, L,
+                                   dk, dv, s.NP, chunk, dt);
+        if (la::tc_pass_supported(a)) {
+            la::ChainArgs ch;
+            ch.states = reinterpret_cast<float *>(at(workspace, w.chain_states));
+            ch.ready = reinterpret_cast<int *>(at(workspace, w.chain_ready));
+            ch.S_final = S_final;
+            ch.S_save = S_recv_save;
+            ch.save_every = s.m;
+            if ((e = la::launch_chain_reset(S0, s.BH, dk, dv, ch.states, ch.ready, stream)) !=
+                cudaSuccess)
+                return cuda_fail(e, "chain reset");
+            if ((e = la::launch_tc_chain(a, ch, stream)) != cudaSuccess)
+                return cuda_fail(e, "single pass");
+            return LA_OK;
+        }
+        // other shapes: the two-pass order below (same result)
+    }
+
     la::PassArgs a = pass_args(q, k, v, log_g, o, nullptr, S_loc, logG, status, B, H, L, dk, dv,
                                s.NP, chunk, dt);
     const bool three = schedule == LA_SCHED_THREE_PHASE;
@@ -399,6 +421,45 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
             cudaSuccess)
         return cuda_fail(e, "S_recv_save gather");
     return LA_OK;
+}
+
+la_status la_seg_chain_reset(const float *S0, int B, int H, int dk, int dv, float *chain_states,
+                             int *chain_ready, void *cuda_stream) {
+    if (B < 1 || H < 1 || !(dk == 32 || dk == 64 || dk == 128) || dv != dk)
+        return fail(LA_ERR_SHAPE, "need B, H >= 1 and dk == dv in {32, 64, 128}");
+    if (!chain_states || !chain_ready)
+        return fail(LA_ERR_ARG, "chain_states and chain_ready must be non-null");
+    if (!aligned(chain_states, 16) || !aligned(chain_ready, 16) || (S0 && !aligned(S0, 16)))
+        return fail(LA_ERR_ALIGN, "S0, chain_states and chain_ready must be 16-byte aligned");
+    cudaError_t e = la::launch_chain_reset(S0, B * H, dk, dv, chain_states, chain_ready,
+                                           static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, "chain reset");
+}
+
+la_status la_seg_chain_pass(const void *q, const void *k, const void *v, const void *log_g, int B,
+                            int H, long long L, int dk, int dv, int NP, int chunk, la_dtype dt,
+                            float *chain_states, int *chain_ready, void *o, float *S_final,
+                            float *S_recv_save, int save_every, int *status, void *cuda_stream) {
+    la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
+                              {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {o, "o"},
+                               {chain_states, "chain_states"}, {chain_ready, "chain_ready"}},
+                              {{S_final, "S_final"}, {S_recv_save, "S_recv_save"}});
+    if (st != LA_OK) return st;
+    if (save_every < 1 || NP % save_every != 0)
+        return fail(LA_ERR_ARG, "save_every=%d must divide NP=%d", save_every, NP);
+    la::PassArgs a = pass_args(q, k, v, log_g, o, nullptr, nullptr, nullptr, status, B, H, L, dk,
+                               dv, NP, chunk, dt);
+    if (!la::tc_pass_supported(a))
+        return fail(LA_ERR_SHAPE, "the single pass needs bf16, dk = dv = 128 and chunk = 64");
+    if (L == 0) return LA_OK;
+    la::ChainArgs ch;
+    ch.states = chain_states;
+    ch.ready = chain_ready;
+    ch.S_final = S_final;
+    ch.S_save = S_recv_save;
+    ch.save_every = save_every;
+    cudaError_t e = la::launch_tc_chain(a, ch, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, "single pass");
 }
 
 la_status la_seg_backward(const void *q, const void *k, const void *v, const void *log_g,

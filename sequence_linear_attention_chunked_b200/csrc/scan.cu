@@ -122,6 +122,29 @@ cudaError_t launch_copy_state(const float *src, int BH, int dk, int dv, float *d
 
 namespace la {
 namespace {
+__global__ void chain_reset_kernel(const float4 *__restrict__ S0, int BH, long long per4,
+                                   float4 *__restrict__ states, int *__restrict__ ready) {
+    const int bh = blockIdx.x;
+    for (long long e = threadIdx.x; e < per4; e += blockDim.x)
+        states[(long long)bh * 2 * per4 + e] = S0 ? S0[(long long)bh * per4 + e]
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (threadIdx.x == 0) {
+        ready[bh] = 0;
+        if (bh == 0) ready[BH] = 0;
+    }
+}
+}  // namespace
+
+cudaError_t launch_chain_reset(const float *S0, int BH, int dk, int dv, float *states, int *ready,
+                               cudaStream_t st) {
+    if (BH == 0) return cudaSuccess;
+    chain_reset_kernel<<<BH, 256, 0, st>>>(reinterpret_cast<const float4 *>(S0), BH,
+                                           (long long)dk * dv / 4,
+                                           reinterpret_cast<float4 *>(states), ready);
+    return cudaGetLastError();
+}
+
+namespace {
 __global__ void broadcast_state_kernel(const float4 *__restrict__ src, int BH, int P,
                                        long long per4, float4 *__restrict__ dst) {
     const long long n = (long long)BH * P * per4;

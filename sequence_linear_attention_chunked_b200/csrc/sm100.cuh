@@ -114,6 +114,21 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// GPU-scope acquire load and release store of a global int (flags between CTAs).
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Named barrier over `nthreads` threads (a multiple of 32) of the CTA; id 0 is __syncthreads.
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // TMA tile store from shared memory (bulk-group completion).  The writing threads must have
 // made their shared-memory stores visible to the async proxy (fence_proxy_async_smem) and
 // synchronised with the issuing thread first.

@@ -41,6 +41,10 @@ constexpr int kStateWarps = 4, kOutWarps = 4, kEpiWarps = kStateWarps + kOutWarp
 constexpr int kTmaWarp = kEpiWarps + kGateWarps, kMmaWarp = kTmaWarp + 1;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
+// Wait limit of the single-pass kernel's cross-CTA chain, in clock cycles (about a second).
+constexpr long long kChainWaitLimit = 2000000000LL;
+
+
 // Tensor-memory columns: the fp32 state, two O^T buffers, two bf16 S'^T buffers (bf16 pairs),
 // the M=64 score tile.
 constexpr uint32_t kColDS = 0, kColO = 128, kColSA = 256, kColQK = 384;
@@ -91,20 +95,14 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
         mbar_arrive_expect_tx(&b.full[s], C::stage_bytes);
         uint8_t *st = smem + s * C::stage_bytes;
         const int y = (int)(row0 + (long long)c * CH);
-        if (C::q) {
-            tma_load_2d(st + C::off_q, tq, 0, y, &b.full[s]);
-            tma_load_2d(st + C::off_q + kHalfBytes, tq, 64, y, &b.full[s]);
-        }
-        if (C::k) {
-            tma_load_2d(st + C::off_k, tk, 0, y, &b.full[s]);
-            tma_load_2d(st + C::off_k + kHalfBytes, tk, 64, y, &b.full[s]);
-        }
-        if (C::v) {
-            tma_load_2d(st + C::off_v, tv, 0, y, &b.full[s]);
-            tma_load_2d(st + C::off_v + kHalfBytes, tv, 64, y, &b.full[s]);
-        }
-        tma_load_2d(st + C::off_g, tg, 0, y, &b.full[s]);
-        tma_load_2d(st + C::off_g + kHalfBytes, tg, 64, y, &b.full[s]);
+        auto load = [&](int off, const CUtensorMap *m) {  // both 64-column halves of one tile
+            tma_load_2d(st + off, m, 0, y, &b.full[s]);
+            tma_load_2d(st + off + kHalfBytes, m, 64, y, &b.full[s]);
+        };
+        if (C::q) load(C::off_q, tq);
+        if (C::k) load(C::off_k, tk);
+        if (C::v) load(C::off_v, tv);
+        load(C::off_g, tg);
         issued = c + 1;
     }
     if (*abort)  // let every copy this CTA started land before it exits
@@ -226,7 +224,8 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
 // last group's inclusive value is b_C.  Then q and k are rescaled in place, 2 rows per batch.
 template <int MODE>
 __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
-                          int bh, int j, int nchunks) {
+                          int bh, int j, int nchunks, float *lg_smem = nullptr,
+                          uint64_t *lg_full = nullptr) {
     using C = Cfg<MODE>;
     const int gw = (threadIdx.x >> 5) - kEpiWarps;
     const int lane = threadIdx.x & 31;
@@ -339,10 +338,15 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.gated[s]);
     }
-    if (C::write_state && !*abort && tg == 0) {
-        float4 *lg = reinterpret_cast<float4 *>(a.logG + ((long long)bh * a.NP + j) * D + i0);
+    if (C::write_state && !*abort && tg == 0) {  // to shared memory (lg_full) or global
+        float4 *lg = reinterpret_cast<float4 *>(
+            lg_smem ? lg_smem + i0 : a.logG + ((long long)bh * a.NP + j) * D + i0);
         lg[0] = make_float4(logG[0], logG[1], logG[2], logG[3]);
         lg[1] = make_float4(logG[4], logG[5], logG[6], logG[7]);
+    }
+    if (lg_full) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(lg_full);
     }
     if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
 }
@@ -352,16 +356,19 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 // Per chunk c it scales the row by the chunk's decay (S' = diag(e^{b_C}) S), stores S' back
 // for the MMA to accumulate the chunk's increment onto, and (output modes) stores the bf16
 // copy into S'^T buffer c % 2, the A operand of O^T += S'^T Qbar'^T.
+// Flags for the single-pass kernel: the initial state is already in TMEM (kRoleStateLoaded);
+// the final state stays in TMEM and is not written out (kRoleStateKept).
+enum : int { kRoleStateLoaded = 1, kRoleStateKept = 2 };
 template <int MODE>
 __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, const PassArgs &a,
-                           uint32_t tmem, int bh, int j, int nchunks) {
+                           uint32_t tmem, int bh, int j, int nchunks, int flags = 0) {
     using C = Cfg<MODE>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int dv = warp * 32 + lane;
     const uint32_t lrow = (uint32_t)(warp * 32) << 16;
     const float *ec = reinterpret_cast<const float *>(smem + C::off_ec);
     uint32_t r[32];
-    if (!C::dstate) {  // initial state: the received state (output / correction passes) or zero
+    if (!C::dstate && !(flags & kRoleStateLoaded)) {  // initial state: the received state (output / correction passes) or zero
         const float *Si = (C::init_state && a.S_init)
                               ? a.S_init + ((long long)bh * a.NP + j) * D * D + dv : nullptr;
 #pragma unroll
@@ -417,7 +424,7 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
     }
     if (C::write_state && !*abort) {
         const uint32_t last = C::dstate ? 0u : (uint32_t)((nchunks - 1) & 1);
-        if (mbar_wait(b.ds_full, last, abort)) {
+        if (mbar_wait(b.ds_full, last, abort) && !(flags & kRoleStateKept)) {
             tc_fence_after();
             float *So = a.S_out + ((long long)bh * a.NP + j) * D * D + dv;
 #pragma unroll
@@ -511,7 +518,38 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
     }
 }
 
-// ------------------------------------------------------------------ the kernel
+// ------------------------------------------------------------------ the kernels
+// Barrier block of one pass: 3 per stage, then 13 (layout of Bars).
+__device__ Bars carve_bars(uint64_t *bar, int stages) {
+    Bars b;
+    b.full = bar;
+    b.gated = bar + stages;
+    b.empty = bar + 2 * stages;
+    uint64_t *x = bar + 3 * stages;
+    b.qk_full = x + 0; b.qk_free = x + 1; b.p_full = x + 2; b.ds_full = x + 4; b.sa_full = x + 5;
+    b.sa_free = x + 6; b.o_full = x + 8; b.o_free = x + 10; b.fin = x + 12;
+    return b;
+}
+
+__device__ void init_bars(const Bars &b, int stages) {
+    for (int s = 0; s < stages; ++s) {
+        mbar_init(&b.full[s], 1);
+        mbar_init(&b.gated[s], kGateWarps);
+        mbar_init(&b.empty[s], 1 + kStateWarps);
+    }
+    mbar_init(b.qk_full, 1);
+    mbar_init(b.qk_free, kOutWarps);
+    mbar_init(b.ds_full, 1);
+    mbar_init(b.sa_full, kStateWarps);
+    for (int i = 0; i < 2; ++i) {
+        mbar_init(&b.p_full[i], kOutWarps);
+        mbar_init(&b.sa_free[i], 1);
+        mbar_init(&b.o_full[i], 1);
+        mbar_init(&b.o_free[i], kOutWarps);
+    }
+    mbar_init(b.fin, 1);
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -521,14 +559,7 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + C::off_bar);
-    Bars b;
-    b.full = bar;
-    b.gated = bar + C::stages;
-    b.empty = bar + 2 * C::stages;
-    uint64_t *x = bar + 3 * C::stages;
-    b.qk_full = x + 0; b.qk_free = x + 1; b.p_full = x + 2; b.ds_full = x + 4; b.sa_full = x + 5;
-    b.sa_free = x + 6; b.o_full = x + 8; b.o_free = x + 10; b.fin = x + 12;
+    const Bars b = carve_bars(reinterpret_cast<uint64_t *>(smem + C::off_bar), C::stages);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::off_misc + 4);
 
@@ -538,22 +569,7 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int nchunks = (int)(a.T / CH);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::stages; ++s) {
-            mbar_init(&b.full[s], 1);
-            mbar_init(&b.gated[s], kGateWarps);
-            mbar_init(&b.empty[s], 1 + kStateWarps);
-        }
-        mbar_init(b.qk_full, 1);
-        mbar_init(b.qk_free, kOutWarps);
-        mbar_init(b.ds_full, 1);
-        mbar_init(b.sa_full, kStateWarps);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&b.p_full[i], kOutWarps);
-            mbar_init(&b.sa_free[i], 1);
-            mbar_init(&b.o_full[i], 1);
-            mbar_init(&b.o_free[i], kOutWarps);
-        }
-        mbar_init(b.fin, 1);
+        init_bars(b, C::stages);
         *abort = 0;
         mbar_fence_init();
     }
@@ -590,6 +606,178 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (threadIdx.x == 0 && *abort && a.status) atomicOr(a.status, kStatusTimeout);
 }
 
+// ------------------------------------------------------------------ single-pass forward
+// One CTA per (b, h, sub-segment j) does the state pass and then the output pass of its
+// sub-segment, and the decayed scan between them is chained through the sub-segments of each
+// sequence.  The CTAs take (b, h, j) from a ticket counter in launch order -- ticket t is
+// sub-segment j = t / BH of sequence bh = t % BH -- so the CTA a waiting CTA depends on holds
+// an earlier ticket and is already resident: the chain cannot deadlock on scheduling.
+//
+// Phase 1 is the state pass (local state S_j from zero in TMEM, log-decay sum Gamma_j in shared
+// memory).  The state warps then wait until sub-segment j-1 has published S_recv_j (the state
+// this sub-segment receives), publish S_recv_{j+1} = Gamma_j S_recv_j + S_j (the All-Scan
+// update of the ZeCO review's "key machinery", with the accumulated state moving on as referee
+// major comment 4 requires), and load S_recv_j into TMEM as the start state of phase 2, the
+// output pass.  Phase 2's loads, gates and first scores do not depend on S_recv_j, so they run
+// during the wait.  No per-sub-segment state arrays and no separate scan launch are needed: two
+// state slots per sequence suffice, since sub-segment j reads slot j % 2 before it publishes
+// j + 1, and slot j % 2 is next written by sub-segment j + 1 after that.
+constexpr uint32_t kChainBarrier = 1;  // named barrier of the 4 state warps
+
+struct ChainCfg {
+    using A = Cfg<kPassState>;
+    using B = Cfg<kPassOutput>;
+    static constexpr int off_lg = A::off_bar > B::off_bar ? A::off_bar : B::off_bar;
+    static constexpr int off_bar = off_lg + D * 4;
+    static constexpr int n_bars = A::n_bars + B::n_bars + 1;
+    static constexpr int off_misc = off_bar + n_bars * 8;
+    static constexpr int smem_bytes = off_misc + 16 + 1024;
+    static_assert(smem_bytes <= 232448, "shared memory budget");
+};
+
+// State warps, between the phases.  Thread dv owns row dv of S^T in TMEM and column dv of the
+// [dk, dv] states in global memory (coalesced across the warp).
+__device__ void chain_step(const PassArgs &a, const ChainArgs &ch, const float *lg,
+                           uint64_t *lg_full, volatile int *abort, uint32_t tmem, int bh, int j) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int dv = warp * 32 + lane;
+    const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+    int *ready = ch.ready + bh;
+    int seen = -1;
+    if (lane == 0) {  // bounded wait for ready[bh] >= j
+        const long long t0 = clock64();
+        while (true) {
+            seen = ld_acquire_gpu(ready);
+            if (seen >= j || *abort) break;
+            if (clock64() - t0 > kChainWaitLimit) {
+                *abort = 1;
+                break;
+            }
+            __nanosleep(64);
+        }
+    }
+    seen = __shfl_sync(0xFFFFFFFFu, seen, 0);
+    bool ok = seen >= j && seen != kChainPoison;
+    if (ok) (void)ld_acquire_gpu(ready);  // each lane's own acquire before it reads the slot
+    if (ok) ok = warp_wait(lg_full, 0, abort);  // Gamma_j from the gate warps
+    if (ok) {
+        tc_fence_after();
+        const long long per = (long long)D * D;
+        const float *rin = ch.states + ((long long)bh * 2 + (j & 1)) * per + dv;
+        float *rout = j + 1 < a.NP ? ch.states + ((long long)bh * 2 + ((j + 1) & 1)) * per + dv
+                                   : (ch.S_final ? ch.S_final + (long long)bh * per + dv : nullptr);
+        float *save = (ch.S_save && j % ch.save_every == 0)
+                          ? ch.S_save + ((long long)bh * (a.NP / ch.save_every) + j / ch.save_every) * per + dv
+                          : nullptr;
+        uint32_t r[32];
+        float x[32];
+#pragma unroll 1
+        for (int p = 0; p < 4; ++p) {  // key dims 32p .. 32p+31
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = __ldcg(rin + (p * 32 + e) * D);
+            tmem_ld32(tmem + lrow + kColDS + p * 32, r);
+            tmem_wait_ld();
+            if (rout) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    rout[(p * 32 + e) * D] = fmaf(__expf(lg[p * 32 + e]), x[e], __uint_as_float(r[e]));
+            }
+            if (save) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) save[(p * 32 + e) * D] = x[e];
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(x[e]);
+            tmem_st32(tmem + lrow + kColDS + p * 32, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+    } else {
+        *abort = 1;  // no received state: phase 2 does not run, and the successors learn it
+    }
+    __threadfence();
+    named_sync(kChainBarrier, kStateWarps * 32);
+    if (threadIdx.x == 0) st_release_gpu(ready, ok ? j + 1 : kChainPoison);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+tc_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                const PassArgs a, const ChainArgs ch) {
+    using CA = ChainCfg::A;
+    using CB = ChainCfg::B;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + ChainCfg::off_bar);
+    const Bars ba = carve_bars(bar, CA::stages);
+    const Bars bb = carve_bars(bar + CA::n_bars, CB::stages);
+    uint64_t *lg_full = bar + CA::n_bars + CB::n_bars;
+    float *lg = reinterpret_cast<float *>(smem + ChainCfg::off_lg);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + ChainCfg::off_misc);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + ChainCfg::off_misc + 4);
+    int *ticket = reinterpret_cast<int *>(smem + ChainCfg::off_misc + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        init_bars(ba, CA::stages);
+        init_bars(bb, CB::stages);
+        mbar_init(lg_full, kGateWarps);
+        *abort = 0;
+        *ticket = atomicAdd(ch.ready + a.BH, 1);
+        mbar_fence_init();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_g);
+    }
+    if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int t = *ticket;
+    const bool valid = t >= 0 && (long long)t < (long long)a.BH * a.NP;
+    const int bh = valid ? t % a.BH : 0, j = valid ? t / a.BH : 0;
+    const long long row0 = (long long)bh * a.L + (long long)j * a.T;
+    const int nchunks = (int)(a.T / CH);
+
+    if (!valid) {  // ticket counter not reset before the launch: no work, report it
+        if (threadIdx.x == 0) *abort = 1;
+    } else if (warp == kTmaWarp) {
+        if (lane == 0) {
+            producer<kPassState>(smem, ba, abort, &tm_q, &tm_k, &tm_v, &tm_g, row0, nchunks);
+            // phase 2 reuses the stage memory: every stage of phase 1 must be released first
+            bool ok = !*abort;
+            for (int c = nchunks > CA::stages ? nchunks - CA::stages : 0; ok && c < nchunks; ++c)
+                ok = mbar_wait(&ba.empty[c % CA::stages], (c / CA::stages) & 1, abort);
+            if (ok) producer<kPassOutput>(smem, bb, abort, &tm_q, &tm_k, &tm_v, &tm_g, row0, nchunks);
+        }
+    } else if (warp == kMmaWarp) {
+        mma_issuer<kPassState>(smem, ba, abort, tmem, nchunks);
+        mma_issuer<kPassOutput>(smem, bb, abort, tmem, nchunks);
+    } else if (warp >= kEpiWarps) {
+        gate_role<kPassState>(smem, ba, abort, a, bh, j, nchunks, lg, lg_full);
+        gate_role<kPassOutput>(smem, bb, abort, a, bh, j, nchunks);
+    } else if (warp < kStateWarps) {
+        state_role<kPassState>(smem, ba, abort, a, tmem, bh, j, nchunks, kRoleStateKept);
+        chain_step(a, ch, lg, lg_full, abort, tmem, bh, j);
+        state_role<kPassOutput>(smem, bb, abort, a, tmem, bh, j, nchunks, kRoleStateLoaded);
+    } else {
+        out_role<kPassOutput>(smem, bb, abort, a, tmem, row0, nchunks);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort && a.status) atomicOr(a.status, kStatusTimeout);
+}
+
 // ------------------------------------------------------------------ host side
 template <int MODE>
 cudaError_t launch_mode(const PassArgs &a, cudaStream_t st) {
@@ -613,6 +801,24 @@ cudaError_t launch_mode(const PassArgs &a, cudaStream_t st) {
 }
 
 }  // namespace
+
+cudaError_t launch_tc_chain(const PassArgs &a, const ChainArgs &ch, cudaStream_t st) {
+    const long long rows = (long long)a.BH * a.L;
+    if (rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
+    CUtensorMap mq, mk, mv, mg;
+    cudaError_t e;
+    if ((e = make_map(&mq, a.q, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mk, a.k, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ChainCfg::smem_bytes);
+    if (e != cudaSuccess) return e;
+    const long long nblk = (long long)a.BH * a.NP;
+    if (nblk == 0) return cudaSuccess;
+    tc_chain_kernel<<<(unsigned)nblk, kThreads, ChainCfg::smem_bytes, st>>>(mq, mk, mv, mg, a, ch);
+    return cudaGetLastError();
+}
 
 bool tc_pass_supported(const PassArgs &a) {
     return a.dt == LA_BF16 && a.dk == D && a.dv == D && a.chunk == CH && a.T % CH == 0;

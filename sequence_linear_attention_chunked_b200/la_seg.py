@@ -21,12 +21,12 @@ STATUS_NAMES = {0: "LA_OK", -1: "LA_ERR_ARG", -2: "LA_ERR_SHAPE", -3: "LA_ERR_AL
                 -4: "LA_ERR_DTYPE", -5: "LA_ERR_WORKSPACE", -6: "LA_ERR_GATE_RANGE",
                 -7: "LA_ERR_TIMEOUT", -8: "LA_ERR_CUDA"}
 LA_F32, LA_BF16 = 0, 1
-SCHED_AUTO, SCHED_TWO_PASS, SCHED_THREE_PHASE = 0, 1, 2
+SCHED_AUTO, SCHED_TWO_PASS, SCHED_THREE_PHASE, SCHED_SINGLE_PASS = 0, 1, 2, 3
 EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_seg_scan",
             "la_seg_state_pass", "la_seg_local_pass", "la_seg_output_pass", "la_seg_correct_pass",
             "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail",
             "la_seg_forward_noalloc", "la_seg_dstate_pass", "la_seg_dq_pass", "la_seg_dkv_pass",
-            "la_seg_backward_parts")
+            "la_seg_backward_parts", "la_seg_chain_pass", "la_seg_chain_reset")
 
 _lib = None
 
@@ -82,6 +82,11 @@ def lib():
         L.la_seg_dkv_pass.restype = i32
         L.la_seg_backward_parts.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32, i32]
         L.la_seg_backward_parts.restype = i32
+        L.la_seg_chain_pass.argtypes = [P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P,
+                                        P, P, P, i32, P, P]
+        L.la_seg_chain_pass.restype = i32
+        L.la_seg_chain_reset.argtypes = [P, i32, i32, i32, i32, P, P, P]
+        L.la_seg_chain_reset.restype = i32
         L.la_seg_check_status.argtypes = [P, P]
         L.la_seg_check_status.restype = i32
         L.la_last_error_detail.argtypes = [ctypes.c_char_p, sz]
@@ -321,3 +326,37 @@ def la_seg_dkv_pass(q, k, v, log_g, dO, S_recv, S_final, dX, qdq, NP, chunk, *, 
                                  _dt(q), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(status),
                                  _stream(stream)), "la_seg_dkv_pass")
     return out
+
+
+def chain_buffers(B, H, dk, dv, device="cuda"):
+    """Caller-owned chain buffers of la_seg_chain_pass: fp32 [B*H, 2, dk, dv] state slots and
+    int32 [B*H + 1] ready words (the last one the ticket counter)."""
+    states = torch.empty((B * H, 2, dk, dv), dtype=torch.float32, device=device)
+    ready = torch.empty((B * H + 1,), dtype=torch.int32, device=device)
+    return states, ready
+
+
+def la_seg_chain_reset(S0, B, H, dk, dv, states, ready, *, stream=None):
+    """Slot 0 of every sequence's chain = S0 (None: zeros); ready words and ticket = 0."""
+    _need(S0, "S0", torch.float32, (B, H, dk, dv), states.device)
+    _check(lib().la_seg_chain_reset(_ptr(S0), B, H, dk, dv, _ptr(states), _ptr(ready),
+                                    _stream(stream)), "la_seg_chain_reset")
+
+
+def la_seg_chain_pass(q, k, v, log_g, NP, chunk, states, ready, *, o=None, S_final=None,
+                      S_recv_save=None, save_every=1, status=None, stream=None):
+    """One-kernel forward over NP sub-segments per (b, h) with the scan chained between them
+    (la_seg.h); states / ready as la_seg_chain_reset left them.  Returns o."""
+    B, H, L, dk, dv = _seq_shapes(q, v)
+    dev = q.device
+    for t, n, shp in ((q, "q", (B, H, L, dk)), (k, "k", (B, H, L, dk)), (v, "v", (B, H, L, dv)),
+                      (log_g, "log_g", (B, H, L, dk))):
+        _need(t, n, q.dtype, shp, dev)
+    _need(states, "states", torch.float32, (B * H, 2, dk, dv), dev)
+    _need(ready, "ready", torch.int32, (B * H + 1,), dev)
+    o = torch.empty((B, H, L, dv), dtype=q.dtype, device=dev) if o is None else o
+    _check(lib().la_seg_chain_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), B, H, L, dk, dv, NP,
+                                   chunk, _dt(q), _ptr(states), _ptr(ready), _ptr(o),
+                                   _ptr(S_final), _ptr(S_recv_save), int(save_every),
+                                   _ptr(status), _stream(stream)), "la_seg_chain_pass")
+    return o
