@@ -29,15 +29,18 @@ constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
 //
 // Roles (448 threads): warps 0-3 carry dS -- the fp32 dS lives in tensor memory (row i on lane
 // i), they apply the decay, write its bf16 copy into a shared [i][j] tile (read by the MMAs as
-// the K-major A operand of dS V^T and the MN-major A operand of dS^T Ktil^T) and turn M and A
-// into masked bf16 tiles (double-buffered); warps 4-7 read dk^T and dv^T (double-buffered in
-// TMEM; thread x owns key / value dim x for all 64 tokens of the chunk, so the dlog_g suffix
-// sums need no exchange), stage dk, dlog_g and dv in the stage's v, q and dO tiles (free by then)
-// and write them with TMA stores; warps 8-11 gates; 12 TMA; 13 MMA.
+// the K-major A operand of dS V^T and the MN-major A operand of dS^T Ktil^T), turn M and A into
+// masked bf16 tiles (double-buffered); warps 4-7 read dk^T (double-buffered in TMEM) and write
+// dk and dlog_g (thread x owns key dim x for all 64 tokens of the chunk, so the dlog_g suffix
+// sums need no exchange); warps 8-11 gate the chunks and write dv from dv^T; 12 TMA; 13 MMA.  A stage
+// is released once the tensor cores are done with it and the dS and output warps have copied
+// the per-key factors they need into registers or TMEM.
 namespace dkv {
 
 constexpr int kStateWarps = 4, kOutWarps = 4;
-constexpr uint32_t kColM = 0, kColA = 64, kColDK = 128, kColDV = 256, kColDS = 384;
+// Tensor-memory columns: M, A (M=64 layout), dk^T x 2, dv^T, the chunk's (e^{b_C - b_s}, Ktil)
+// pairs for the output warps, dS.
+constexpr uint32_t kColM = 0, kColA = 64, kColDK = 128, kColDV = 256, kColFK = 320, kColDS = 384;
 constexpr int kStages = 2;
 constexpr int off_q = 0, off_k = kTileBytes, off_v = 2 * kTileBytes, off_do = 3 * kTileBytes,
               off_g = 4 * kTileBytes;
@@ -145,13 +148,11 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
         const uint32_t mt = ma_addr + bb * 2 * kMaskBytes, at = mt + kMaskBytes;
         if (!(ok = warp_wait(b.p_full, it & 1, abort))) break;
         if (!(ok = warp_wait(b.dst_full, it & 1, abort))) break;
-        if (it >= 2) {
-            if (!(ok = warp_wait(&b.dk_free[bb], ((it >> 1) - 1) & 1, abort))) break;
-            if (!(ok = warp_wait(&b.dv_free[bb], ((it >> 1) - 1) & 1, abort))) break;
-        }
+        if (it >= 2 && !(ok = warp_wait(&b.dk_free[bb], ((it >> 1) - 1) & 1, abort))) break;
+        if (it >= 1 && !(ok = warp_wait(b.dv_free, (it - 1) & 1, abort))) break;
         tc_fence_after();
         if (elect_one()) {
-            const uint32_t dk_col = tmem + kColDK + bb * 64, dv_col = tmem + kColDV + bb * 64;
+            const uint32_t dk_col = tmem + kColDK + bb * 64, dv_col = tmem + kColDV;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dS += Qbar'^T dO  (dk and dv read the old dS tile)
                 mma_ss(tmem + kColDS, desc_mnmajor(qa, kk), desc_mnmajor(da, kk), i_dsn, 1u);
@@ -172,7 +173,7 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
             for (int kk = 0; kk < 8; ++kk)  // dv^T += dS^T Ktil^T   (A: dS tile read MN-major)
                 mma_ss(dv_col, smem_desc_sw128(ds_addr + kk * 2048, kDsHalf, 1024), desc_kmajor(ka, kk),
                        i_dvb, 1u);
-            mma_commit(&b.dv_full[bb]);
+            mma_commit(b.dv_full);
             mma_commit(b.dsn_full);  // the dS tile is read out as well
             mma_commit(&b.empty[s]);
         }
@@ -184,12 +185,50 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
     wait_drain(b.fin, 0);
 }
 
+// Stores the bf16 values of tokens t and t+1 of this lane's dim x into a [tokens, 128] bf16
+// tensor (one conversion, two 2-byte stores).  `at` points at element (t, x).
+__device__ __forceinline__ void stg_pair(__nv_bfloat16 *at, float a, float b) {
+    const uint32_t p = pack_bf16(a, b);  // low half: token t, high half: token t+1
+    unsigned short *h = reinterpret_cast<unsigned short *>(at);
+    h[0] = (unsigned short)(p & 0xFFFFu);
+    h[D] = (unsigned short)(p >> 16);
+}
+
+// dv of one chunk from dv^T (thread x = TMEM lane x owns value dim x), straight to HBM;
+// releases the accumulator after the last tensor-memory read.  The gate warps run it right after
+// gating the next chunk, before that chunk's masked A tile (and so its dv^T MMA) can exist, so
+// one dv^T buffer suffices.
+__device__ __forceinline__ bool dv_readout(const Bars &b, volatile int *abort, uint32_t tmem,
+                                           uint32_t lrow, int parity, __nv_bfloat16 *dvc,
+                                           int lane) {
+    if (!mbar_wait(b.dv_full, parity, abort)) return false;
+    tc_fence_after();
+    uint32_t r[16];
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+        tmem_ld16(tmem + lrow + kColDV + g * 16, r);
+        tmem_wait_ld();
+        if (g == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.dv_free);
+        }
+#pragma unroll
+        for (int t = 0; t < 16; t += 2)
+            stg_pair(dvc + (g * 16 + t) * D, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
+    }
+    return true;
+}
+
 // Gate warps: Qbar' and Ktil in place of q and k, e^{b_C - b_t} in place of log_g (the dk
-// output factor), e^{b_C} per key dim.
+// output factor), e^{b_C} per key dim; then dv of the previous chunk (warp gw reads TMEM lane
+// quarter gw, value dims 32 gw .. 32 gw + 31).
 __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
-                          int nchunks) {
+                          uint32_t tmem, long long row0, int nchunks) {
     const int gw = (threadIdx.x >> 5) - kEpiWarps;
     const int lane = threadIdx.x & 31;
+    const uint32_t lrow = (uint32_t)(gw * 32) << 16;
+    __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv_out) + row0 * D + gw * 32 + lane;
     const int tg = lane >> 2, ig = lane & 3;
     const int i0 = gw * 32 + ig * 8;
     float *ec = reinterpret_cast<float *>(smem + off_ec);
@@ -274,7 +313,12 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.gated[s]);
+        if (it > 0 && !dv_readout(b, abort, tmem, lrow, (it - 1) & 1,
+                                  dv + (long long)(nchunks - it) * CH * D, lane))
+            break;
     }
+    if (!*abort && nchunks > 0)  // dv of the part's first chunk
+        dv_readout(b, abort, tmem, lrow, (nchunks - 1) & 1, dv, lane);
     if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
 }
 
@@ -301,7 +345,8 @@ __device__ __forceinline__ void masked_tile(uint8_t *tile, const uint32_t (&r)[3
 
 // Warps 0-3: thread i owns row i of dS (TMEM lane i).  Per chunk: the decay by the previous
 // chunk's e^{b_C} (S_new = diag(e^{b_C}) (dS + Qbar'^T dO), the sum formed by the MMA), the
-// bf16 copy of row i into the dS tile, then the masked M and A tiles of the chunk.
+// bf16 copy of row i into the dS tile, the masked M and A tiles; the stage is released as soon
+// as its e^{b_C} is in a register.
 __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
                            uint32_t tmem, int bh, int j, int nchunks) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -325,14 +370,11 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
         tmem_wait_st();
         tc_fence_before();
     }
+    uint64_t e2 = 0;  // e^{b_C,i} of the previous chunk, in both halves
     for (int it = 0; it < nchunks; ++it) {
         // (1) dS of this chunk's end: decayed unless it is the part's end
-        if (it > 0) {
-            if (!mbar_wait(b.dsn_full, (it - 1) & 1, abort)) break;
-        }
+        if (it > 0 && !mbar_wait(b.dsn_full, (it - 1) & 1, abort)) break;
         tc_fence_after();
-        const uint64_t e2 = it > 0 ? (uint64_t)__float_as_uint(ec[((it - 1) % kStages) * D + i]) * 0x100000001ull
-                                   : 0ull;
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             tmem_ld32(tmem + lrow + kColDS + p * 32, r);
@@ -360,14 +402,11 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
         tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(b.dst_full);
-            if (it > 0) mbar_arrive(&b.empty[(it - 1) % kStages]);  // its e^{b_C} is used
-        }
+        if (lane == 0) mbar_arrive(b.dst_full);
         // (2) masked M and A tiles of this chunk (M=64 layout: lanes 0-15 hold row 16 warp + lane);
-        // M is ready before the gates finish, A only after
+        // M is ready before the gates finish, A only after; dv of the previous chunk in between
         uint8_t *mt = smem + off_ma + (it & 1) * 2 * kMaskBytes;
-#pragma unroll
+#pragma unroll 1
         for (int t = 0; t < 4; ++t) {  // M half 0, M half 1, A half 0, A half 1
             if (t == 0 && !mbar_wait(b.m_full, it & 1, abort)) break;
             if (t == 2 && !mbar_wait(b.a_full, it & 1, abort)) break;
@@ -383,30 +422,27 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
         }
         if (*abort) break;
         fence_proxy_async_smem();
+        // the chunk's e^{b_C} is this role's last read of the stage
+        e2 = (uint64_t)__float_as_uint(ec[(it % kStages) * D + i]) * 0x100000001ull;
         __syncwarp();
-        if (lane == 0) mbar_arrive(b.p_full);
+        if (lane == 0) {
+            mbar_arrive(b.p_full);
+            mbar_arrive(&b.empty[it % kStages]);
+        }
     }
 }
 
-// Stores the bf16 values of tokens t and t+1 of this lane's dim x into a [tokens, 128] bf16
-// tensor (one conversion, two 2-byte stores).  `at` points at element (t, x).
-__device__ __forceinline__ void stg_pair(__nv_bfloat16 *at, float a, float b) {
-    const uint32_t p = pack_bf16(a, b);  // low half: token t, high half: token t+1
-    unsigned short *h = reinterpret_cast<unsigned short *>(at);
-    h[0] = (unsigned short)(p & 0xFFFFu);
-    h[D] = (unsigned short)(p >> 16);
-}
-
-// Warps 4-7: thread x = 32 (warp - 4) + lane owns key dim x of dk / dlog_g and value dim x of
-// dv for all 64 tokens of the chunk; the outputs go straight from registers to HBM, and each
-// warp releases the stage as soon as it has read the chunk's factors and Ktil.
+// Warps 4-7: thread x = 32 (warp - 4) + lane owns key dim x of dk and dlog_g for all 64 tokens
+// of the chunk.  As soon as the gates are done with a chunk, each thread copies its dim's 64
+// (e^{b_C - b_s}, Ktil) pairs from the stage into its TMEM lane and releases the stage; the dk
+// loop then reads them back from TMEM beside the dk^T accumulator.  Outputs go straight from
+// registers to HBM.
 __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
                          uint32_t tmem, int bh, int j, long long row0, int nchunks) {
     const int quarter = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
     const int x = quarter * 32 + lane;
     const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
     __nv_bfloat16 *dk = static_cast<__nv_bfloat16 *>(a.dk_out);
-    __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv_out);
     __nv_bfloat16 *dg = static_cast<__nv_bfloat16 *>(a.dg_out);
     const long long sidx = ((long long)bh * a.NP + j) * D * D;
     // carry: rowsum(S_end . dX), the gradient reaching this part from its end state
@@ -428,50 +464,43 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
             }
         }
     }
-    uint32_t r[16];
+    uint32_t r[16], fk[16];
     float qv[16], qn[16];
     for (int it = 0; it < nchunks; ++it) {
         const int s = it % kStages, bb = it & 1;
         const int c = nchunks - 1 - it;
-        uint8_t *st = smem + s * kStageBytes;
         const float *qdq = a.dq_ws + (row0 + (long long)c * CH) * D + x;
+        // (1) the chunk's factors and Ktil into this lane of TMEM; then the stage is released
+        if (!mbar_wait(&b.gated[s], (it / kStages) & 1, abort)) break;
+        const uint32_t sa = smem_u32(smem + s * kStageBytes);
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                const uint32_t off = tile_off(g * 16 + t, x);
+                fk[t] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_k + off) << 16);
+            }
+            tmem_st16(tmem + lrow + kColFK + g * 16, fk);
+        }
+        tmem_wait_st();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.empty[s]);
         // q . dq of the chunk's last 16 tokens (L2-prefetched with the chunk's tiles), in flight
         // while this thread waits for dk; each later group is loaded one group ahead
 #pragma unroll
         for (int t = 0; t < 16; ++t) qn[t] = qdq[(48 + t) * D];
-        // (1) dk and the dlog_g suffix sums: tokens last to first, 16 at a time
+        // (2) dk and the dlog_g suffix sums: tokens last to first, 16 at a time
         if (!mbar_wait(&b.dk_full[bb], (it >> 1) & 1, abort)) break;
         tc_fence_after();
-        const uint32_t sa = smem_u32(st);
-        uint32_t fk[16];  // next group's factors and Ktil, bf16 pairs (f low, Ktil high)
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const uint32_t off = tile_off(48 + t, x);
-            fk[t] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_k + off) << 16);
-        }
 #pragma unroll
         for (int g = 3; g >= 0; --g) {
             tmem_ld16(tmem + lrow + kColDK + bb * 64 + g * 16, r);
+            tmem_ld16(tmem + lrow + kColFK + g * 16, fk);
 #pragma unroll
             for (int t = 0; t < 16; ++t) qv[t] = qn[t];
-            if (g > 0) {
-#pragma unroll
-                for (int t = 0; t < 16; ++t) qn[t] = qdq[((g - 1) * 16 + t) * D];
-            }
-            // dk = e^{b_C - b_s} acc and the contribution q . dq - k . dk (k . dk = Ktil . acc,
-            // Ktil = k e^{b_C - b_s} the MMA operand); then the suffix sums
-            float fd[16], cg[16];  // dk, then contributions / dlog_g
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                fd[t] = __uint_as_float(fk[t] << 16);
-                cg[t] = __uint_as_float(fk[t] & 0xFFFF0000u);
-            }
             if (g > 0) {  // the next group's loads go out before this group's stores
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const uint32_t off = tile_off((g - 1) * 16 + t, x);
-                    fk[t] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_k + off) << 16);
-                }
+                for (int t = 0; t < 16; ++t) qn[t] = qdq[((g - 1) * 16 + t) * D];
             }
             tmem_wait_ld();
             if (g == 0) {
@@ -479,11 +508,14 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&b.dk_free[bb]);
             }
+            // dk = e^{b_C - b_s} acc and the contribution q . dq - k . dk (k . dk = Ktil . acc,
+            // Ktil = k e^{b_C - b_s} the MMA operand); then the suffix sums
+            float fd[16], cg[16];  // dk, then contributions / dlog_g
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
                 const float acc = __uint_as_float(r[t]);
-                fd[t] *= acc;                  // dk
-                cg[t] = qv[t] - cg[t] * acc;    // contribution
+                fd[t] = __uint_as_float(fk[t] << 16) * acc;                        // dk
+                cg[t] = qv[t] - __uint_as_float(fk[t] & 0xFFFF0000u) * acc;       // contribution
             }
 #pragma unroll
             for (int t = 15; t >= 0; --t) {
@@ -496,25 +528,6 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                 stg_pair(dk + e0 + t * D, fd[t], fd[t + 1]);
                 stg_pair(dg + e0 + t * D, cg[t], cg[t + 1]);
             }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b.empty[s]);  // this warp's reads of the stage are done
-        // (2) dv
-        if (!mbar_wait(&b.dv_full[bb], (it >> 1) & 1, abort)) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int g = 0; g < 4; ++g) {
-            tmem_ld16(tmem + lrow + kColDV + bb * 64 + g * 16, r);
-            tmem_wait_ld();
-            if (g == 3) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&b.dv_free[bb]);
-            }
-            __nv_bfloat16 *dvt = dv + (row0 + (long long)c * CH + g * 16) * D + x;
-#pragma unroll
-            for (int t = 0; t < 16; t += 2)
-                stg_pair(dvt + t * D, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
         }
     }
 }
@@ -547,10 +560,10 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&b.gated[s], kGateWarps);
             mbar_init(&b.empty[s], 1 + kStateWarps + kOutWarps);
         }
-        uint64_t *one[] = {b.m_full, b.a_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dv_full + 1,
-                           b.dsn_full, b.fin};
-        uint64_t *st4[] = {b.m_free, b.a_free, b.p_full, b.dst_full};
-        uint64_t *out4[] = {b.dk_free, b.dk_free + 1, b.dv_free, b.dv_free + 1};
+        uint64_t *one[] = {b.m_full, b.a_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dsn_full,
+                           b.fin};
+        uint64_t *st4[] = {b.m_free, b.a_free, b.p_full, b.dst_full, b.dv_free};  // dv_free: gates
+        uint64_t *out4[] = {b.dk_free, b.dk_free + 1};
         for (uint64_t *p : one) mbar_init(p, 1);
         for (uint64_t *p : st4) mbar_init(p, kStateWarps);
         for (uint64_t *p : out4) mbar_init(p, kOutWarps);
@@ -575,7 +588,7 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     } else if (warp == kMmaWarp) {
         mma_issuer(smem, b, abort, tmem, nchunks);
     } else if (warp >= kEpiWarps) {
-        gate_role(smem, b, abort, a, nchunks);
+        gate_role(smem, b, abort, a, tmem, row0, nchunks);
     } else if (warp < kStateWarps) {
         state_role(smem, b, abort, a, tmem, bh, j, nchunks);
     } else {
