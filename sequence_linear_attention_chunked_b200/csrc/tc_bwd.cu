@@ -51,13 +51,13 @@ constexpr int off_ma = kStages * kStageBytes;  // 2 buffers x (M tile, A tile)
 constexpr int off_ds = off_ma + 4 * kMaskBytes;
 constexpr int off_ec = off_ds + 2 * kDsHalf;
 constexpr int off_bar = off_ec + kStages * D * 4;
-constexpr int kBars = 3 * kStages + 16;
+constexpr int kBars = 4 * kStages + 16;
 constexpr int off_misc = off_bar + kBars * 8;
 constexpr int kSmemBytes = off_misc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Bars {
-    uint64_t *full, *gated, *empty;
+    uint64_t *full, *full_b, *gated, *empty;  // full: log_g, q, k (the gates); full_b: v, dO
     uint64_t *m_full, *m_free, *a_full, *a_free, *p_full, *dst_full, *dk_full, *dk_free, *dv_full, *dv_free,
         *dsn_full, *fin;
 };
@@ -78,24 +78,27 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
         // the chunk's q . dq rows (read with plain loads by the output warps) on their way to L2
         bulk_prefetch_l2(qdq + (row0 + (long long)c * CH) * D, CH * D * 4);
         if (it >= kStages && !mbar_wait(&b.empty[s], ((it / kStages) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&b.full[s], kStageBytes);
         uint8_t *st = smem + s * kStageBytes;
         const int y = (int)(row0 + (long long)c * CH);
-        tma_load_2d(st + off_q, tq, 0, y, &b.full[s]);
-        tma_load_2d(st + off_q + kHalfBytes, tq, 64, y, &b.full[s]);
-        tma_load_2d(st + off_k, tk, 0, y, &b.full[s]);
-        tma_load_2d(st + off_k + kHalfBytes, tk, 64, y, &b.full[s]);
-        tma_load_2d(st + off_v, tv, 0, y, &b.full[s]);
-        tma_load_2d(st + off_v + kHalfBytes, tv, 64, y, &b.full[s]);
-        tma_load_2d(st + off_do, tdo, 0, y, &b.full[s]);
-        tma_load_2d(st + off_do + kHalfBytes, tdo, 64, y, &b.full[s]);
-        tma_load_2d(st + off_g, tg, 0, y, &b.full[s]);
-        tma_load_2d(st + off_g + kHalfBytes, tg, 64, y, &b.full[s]);
+        // the gates' tiles first, on their own barrier (the gates start as soon as they land);
+        // v and dO, read only by the tensor cores, behind them
+        const CUtensorMap *maps[5] = {tg, tq, tk, tv, tdo};
+        const int offs[5] = {off_g, off_q, off_k, off_v, off_do};
+        mbar_arrive_expect_tx(&b.full[s], 3 * kTileBytes);
+        mbar_arrive_expect_tx(&b.full_b[s], 2 * kTileBytes);
+#pragma unroll
+        for (int m = 0; m < 5; ++m) {
+            uint64_t *bar = m < 3 ? &b.full[s] : &b.full_b[s];
+            tma_load_2d(st + offs[m], maps[m], 0, y, bar);
+            tma_load_2d(st + offs[m] + kHalfBytes, maps[m], 64, y, bar);
+        }
         issued = it + 1;
     }
     if (*abort)
-        for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it)
+        for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it) {
             wait_drain(&b.full[it % kStages], (it / kStages) & 1);
+            wait_drain(&b.full_b[it % kStages], (it / kStages) & 1);
+        }
 }
 
 // The whole warp walks the loop; one elected lane issues.  Per chunk: dk^T and dv^T into
@@ -116,7 +119,7 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
     // it while the gates work; A = Qbar' Ktil^T once the tiles are gated.
     auto issue_ma = [&](int it) -> bool {
         const uint32_t st = stage(it);
-        if (!warp_wait(&b.full[it % kStages], (it / kStages) & 1, abort)) return false;
+        if (!warp_wait(&b.full_b[it % kStages], (it / kStages) & 1, abort)) return false;  // v, dO
         if (it > 0 && !warp_wait(b.m_free, (it - 1) & 1, abort)) return false;
         tc_fence_after();
         if (elect_one()) {
@@ -544,7 +547,8 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     b.full = bar;
     b.gated = bar + kStages;
     b.empty = bar + 2 * kStages;
-    uint64_t *x = bar + 3 * kStages;
+    b.full_b = bar + 3 * kStages;
+    uint64_t *x = bar + 4 * kStages;
     b.m_full = x + 0; b.m_free = x + 1; b.p_full = x + 2; b.dst_full = x + 3; b.dk_full = x + 4;
     b.dk_free = x + 6; b.dv_full = x + 8; b.dv_free = x + 10; b.dsn_full = x + 12; b.fin = x + 13;
     b.a_full = x + 14; b.a_free = x + 15;
@@ -557,6 +561,7 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&b.full[s], 1);
+            mbar_init(&b.full_b[s], 1);
             mbar_init(&b.gated[s], kGateWarps);
             mbar_init(&b.empty[s], 1 + kStateWarps + kOutWarps);
         }

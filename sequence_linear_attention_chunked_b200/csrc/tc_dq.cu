@@ -41,14 +41,14 @@ constexpr int kStateWarps = 4, kOutWarps = 4, kEpiWarps = kStateWarps + kOutWarp
 constexpr int kTmaWarp = kEpiWarps + kGateWarps, kMmaWarp = kTmaWarp + 1;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
-// Tensor-memory columns: the fp32 state, dq^T, two bf16 S' copies, M (M=64 layout), R^T.
-constexpr uint32_t kColS = 0, kColDQ = 128, kColSA = 192, kColM = 320, kColR = 384;
+// Tensor-memory columns: the fp32 state, dq^T, the bf16 S' copy, the chunk's (F, q) pairs for
+// the output warps, M (M=64 layout), R^T.
+constexpr uint32_t kColS = 0, kColDQ = 128, kColSA = 192, kColFQ = 256, kColM = 320, kColR = 384;
 
 constexpr int kStages = 2;
 constexpr int off_k = 0, off_v = kTileBytes, off_do = 2 * kTileBytes, off_g = 3 * kTileBytes,
               off_q = 4 * kTileBytes,   // read by the output warps (q . dq) and the gates (Qhat)
               off_qh = 5 * kTileBytes;  // Qhat, written by the gates
-constexpr int kLoadBytes = 5 * kTileBytes;
 constexpr int kStageBytes = 6 * kTileBytes;
 constexpr int off_p = kStages * kStageBytes;  // two masked M tiles
 constexpr int off_ec = off_p + 2 * CH * CH * 2;
@@ -62,8 +62,9 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 enum : int {
     kFull = 0, kGated = kFull + kStages, kEmpty = kGated + kStages, kMFull = kEmpty + kStages,
     kMFree, kPFull, kDsFull = kPFull + 2, kSaFull, kSaFree, kDqFull = kSaFree + 2, kDqFree,
-    kRFull, kRFree, kFin, kNumBars
+    kRFull, kRFree, kFin, kFullB, kNumBars = kFullB + kStages
 };
+static_assert(kNumBars <= 24, "barrier area");
 struct Bars {
     uint64_t *base;
     __device__ __forceinline__ uint64_t *operator[](int k) const { return base + k; }
@@ -84,21 +85,27 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
     for (int c = 0; c < w.nchunks; ++c) {
         const int s = c % kStages;
         if (c >= kStages && !mbar_wait(b[kEmpty + s], ((c / kStages) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(b[kFull + s], kLoadBytes);
         uint8_t *st = smem + s * kStageBytes;
         const int y = (int)(w.row0 + (long long)c * CH);
-        const CUtensorMap *maps[5] = {tk, tv, tdo, tg, tq};
-        const int offs[5] = {off_k, off_v, off_do, off_g, off_q};
+        // the gates' tiles first, on their own barrier (the gates start as soon as they land);
+        // dO and v, read only by the tensor cores, behind them
+        const CUtensorMap *maps[5] = {tg, tk, tq, tdo, tv};
+        const int offs[5] = {off_g, off_k, off_q, off_do, off_v};
+        mbar_arrive_expect_tx(b[kFull + s], 3 * kTileBytes);
+        mbar_arrive_expect_tx(b[kFullB + s], 2 * kTileBytes);
 #pragma unroll
         for (int m = 0; m < 5; ++m) {
-            tma_load_2d(st + offs[m], maps[m], 0, y, b[kFull + s]);
-            tma_load_2d(st + offs[m] + kHalfBytes, maps[m], 64, y, b[kFull + s]);
+            uint64_t *bar = b[(m < 3 ? kFull : kFullB) + s];
+            tma_load_2d(st + offs[m], maps[m], 0, y, bar);
+            tma_load_2d(st + offs[m] + kHalfBytes, maps[m], 64, y, bar);
         }
         issued = c + 1;
     }
     if (*abort)  // let every copy this CTA started land before it exits
-        for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
+        for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c) {
             wait_drain(b[kFull + c % kStages], (c / kStages) & 1);
+            wait_drain(b[kFullB + c % kStages], (c / kStages) & 1);
+        }
 }
 
 // ------------------------------------------------------------------ MMA issuer (1 warp)
@@ -117,7 +124,7 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
         const int s = c % kStages, pb = c & 1;
         const uint32_t st = base + (uint32_t)(s * kStageBytes);
         const uint32_t ka = st + off_k, va = st + off_v, da = st + off_do;
-        if (!(ok = warp_wait(b[kFull + s], (c / kStages) & 1, abort))) break;
+        if (!(ok = warp_wait(b[kFullB + s], (c / kStages) & 1, abort))) break;  // dO, v
         if (c > 0 && !(ok = warp_wait(b[kMFree], (c - 1) & 1, abort))) break;
         tc_fence_after();
         if (elect_one()) {
@@ -159,14 +166,13 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
             const uint32_t pa = base + off_p + pb * (CH * CH * 2);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // dq^T = S' dO^T
-                mma_ts(tmem + kColDQ, tmem + kColSA + pb * 64 + kk * 8, desc_kmajor(da, kk), i_qa,
-                       kk > 0);
+                mma_ts(tmem + kColDQ, tmem + kColSA + kk * 8, desc_kmajor(da, kk), i_qa, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dq^T += Ktil^T M^T   (B: masked M tile, K-major)
                 mma_ss(tmem + kColDQ, desc_mnmajor(ka, kk), smem_desc_sw128(pa + kk * 32, 16, 1024),
                        i_qb, 1u);
             mma_commit(b[kDqFull]);
-            mma_commit(b[kSaFree + pb]);
+            mma_commit(b[kSaFree]);
             mma_commit(b[kEmpty + s]);
         }
         __syncwarp();
@@ -323,14 +329,14 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
         const int s = c % kStages;
         if (!mbar_wait(b[kGated + s], (c / kStages) & 1, abort)) break;
         if (c > 0 && !mbar_wait(b[kDsFull], (c - 1) & 1, abort)) break;
-        if (c >= 2 && !mbar_wait(b[kSaFree + (c & 1)], ((c >> 1) - 1) & 1, abort)) break;
+        if (c >= 1 && !mbar_wait(b[kSaFree], (c - 1) & 1, abort)) break;
         tc_fence_after();
         const uint64_t e2 = (uint64_t)__float_as_uint(ec[s * D + i]) * 0x100000001ull;
         float4 *rec = nullptr;  // the state entering a fine part
         if (a.S_fine && c % w.cpf == 0)
             rec = reinterpret_cast<float4 *>(
                 a.S_fine + ((((long long)w.bh * a.NP + w.j) * a.fine + c / w.cpf) * D + i) * D);
-        const uint32_t sa = tmem + lrow + kColSA + (c & 1) * 64;
+        const uint32_t sa = tmem + lrow + kColSA;
 #pragma unroll 1
         for (int p = 0; p < 4; ++p) {  // value dims 32p .. 32p+31
             tmem_ld32(tmem + lrow + kColS + p * 32, r);
@@ -380,11 +386,12 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
 }
 
 // ------------------------------------------------------------------ output warps (4-7)
-// (a) M -> causal mask -> bf16 P tile (buffer c % 2); (d) dq^T read-out: thread i owns key dim
-// i; dq = F . dq^T with F = e^{b_t - b_C} from the gates, q . dq in fp32 -- stored straight from
+// (a) M -> causal mask -> bf16 P tile (buffer c % 2); (b) the chunk's (F, q) pairs copied from
+// the stage into TMEM, which releases the stage; (d) dq^T read-out: thread i owns key dim i;
+// dq = F . dq^T with F = e^{b_t - b_C} from the gates, q . dq in fp32 -- stored straight from
 // registers (q . dq as one 128-byte line per warp and token, dq as 2-byte stores per token).
-// dq of chunk c is read out before M of chunk c+1 is masked: the read-out releases the stage
-// that chunk c+2 loads into, while M(c+1) can only be formed once chunk c+1 has landed.
+// Chunk c's copy and read-out come before M of chunk c+1 is masked, since M(c+1) can only be
+// formed once chunk c+1 has landed.
 __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
                          uint32_t tmem, const Sweep &w) {
     const int quarter = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
@@ -429,14 +436,34 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
     if (w.nchunks > 0 && !make_p(0)) return;
     for (int c = 0; c < w.nchunks; ++c) {
         const int s = c % kStages;
+        // (b) once the gates are done, this dim's 64 (F, q) pairs into its TMEM lane: the
+        // stage is released before the read-out instead of after it
+        if (!mbar_wait(b[kGated + s], (c / kStages) & 1, abort)) break;
+        {
+            const uint32_t sa = smem_u32(smem + s * kStageBytes);
+            uint32_t fq[16];  // factor (low half) and q (high half), bf16
+#pragma unroll 1
+            for (int g = 0; g < 4; ++g) {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const uint32_t off = tile_off(g * 16 + t, i);
+                    fq[t] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_q + off) << 16);
+                }
+                tmem_st16(tmem + lrow + kColFQ + g * 16, fq);
+            }
+            tmem_wait_st();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b[kEmpty + s]);  // this warp's reads of the stage are done
+        // (d) dq and q . dq
         if (!mbar_wait(b[kDqFull], c & 1, abort)) break;
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + s * kStageBytes);
         const long long tok0 = w.row0 + (long long)c * CH;
 #pragma unroll 1
         for (int g = 0; g < 4; ++g) {  // tokens 16g .. 16g+15
-            uint32_t r16[16];
+            uint32_t r16[16], fq[16];
             tmem_ld16(tmem + lrow + kColDQ + g * 16, r16);
+            tmem_ld16(tmem + lrow + kColFQ + g * 16, fq);
             tmem_wait_ld();
             if (g == 3) {
                 tc_fence_before();
@@ -444,29 +471,18 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                 if (lane == 0) mbar_arrive(b[kDqFree]);
             }
 #pragma unroll
-            for (int t0 = 0; t0 < 16; t0 += 8) {
-                uint32_t fq[8];  // factor (low half) and q (high half), bf16
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t off = tile_off(g * 16 + t0 + e, i);
-                    fq[e] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_q + off) << 16);
-                }
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const long long t = tok0 + g * 16 + t0 + e;
-                    const float v0 = __uint_as_float(r16[t0 + e]) * __uint_as_float(fq[e] << 16);
-                    const float v1 = __uint_as_float(r16[t0 + e + 1]) * __uint_as_float(fq[e + 1] << 16);
-                    a.dq_ws[t * D + i] = __uint_as_float(fq[e] & 0xFFFF0000u) * v0;
-                    a.dq_ws[(t + 1) * D + i] = __uint_as_float(fq[e + 1] & 0xFFFF0000u) * v1;
-                    const uint32_t p = pack_bf16(v0, v1);  // low: token t, high: token t+1
-                    unsigned short *h = reinterpret_cast<unsigned short *>(dq + t * D + i);
-                    h[0] = (unsigned short)(p & 0xFFFFu);
-                    h[D] = (unsigned short)(p >> 16);
-                }
+            for (int e = 0; e < 16; e += 2) {
+                const long long t = tok0 + g * 16 + e;
+                const float v0 = __uint_as_float(r16[e]) * __uint_as_float(fq[e] << 16);
+                const float v1 = __uint_as_float(r16[e + 1]) * __uint_as_float(fq[e + 1] << 16);
+                a.dq_ws[t * D + i] = __uint_as_float(fq[e] & 0xFFFF0000u) * v0;
+                a.dq_ws[(t + 1) * D + i] = __uint_as_float(fq[e + 1] & 0xFFFF0000u) * v1;
+                const uint32_t p = pack_bf16(v0, v1);  // low: token t, high: token t+1
+                unsigned short *h = reinterpret_cast<unsigned short *>(dq + t * D + i);
+                h[0] = (unsigned short)(p & 0xFFFFu);
+                h[D] = (unsigned short)(p >> 16);
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b[kEmpty + s]);  // this warp's reads of the stage are done
         if (c + 1 < w.nchunks && !make_p(c + 1)) break;
     }
 }
@@ -497,6 +513,7 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(b[kFull + s], 1);
+            mbar_init(b[kFullB + s], 1);
             mbar_init(b[kGated + s], kGateWarps);
             mbar_init(b[kEmpty + s], 1 + kStateWarps + kOutWarps);
         }

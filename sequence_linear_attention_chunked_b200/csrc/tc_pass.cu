@@ -69,7 +69,7 @@ struct Cfg {
     static constexpr int off_p = stages * stage_bytes;           // two bf16 P tiles
     static constexpr int off_ec = off_p + (qk ? 2 * CH * CH * 2 : 0);
     static constexpr int off_bar = off_ec + stages * D * 4;
-    static constexpr int n_bars = 3 * stages + 13;
+    static constexpr int n_bars = 4 * stages + 13;
     static constexpr int off_misc = off_bar + n_bars * 8;
     static constexpr int smem_bytes = off_misc + 16 + 1024;  // + slack to align the base to 1 KB
     static_assert(smem_bytes <= 232448, "shared memory budget");
@@ -78,7 +78,7 @@ struct Cfg {
 // Ring barriers per stage; the rest come in pairs where the resource is double-buffered
 // (P tile, O^T and S'^T), so that no waiter can fall two phases behind its barrier.
 struct Bars {
-    uint64_t *full, *gated, *empty;
+    uint64_t *full, *full_b, *gated, *empty;  // full: the gates' tiles; full_b: v
     uint64_t *qk_full, *qk_free, *p_full, *ds_full, *sa_full, *sa_free, *o_full, *o_free, *fin;
 };
 
@@ -92,22 +92,27 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % C::stages;
         if (c >= C::stages && !mbar_wait(&b.empty[s], ((c / C::stages) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&b.full[s], C::stage_bytes);
         uint8_t *st = smem + s * C::stage_bytes;
         const int y = (int)(row0 + (long long)c * CH);
-        auto load = [&](int off, const CUtensorMap *m) {  // both 64-column halves of one tile
-            tma_load_2d(st + off, m, 0, y, &b.full[s]);
-            tma_load_2d(st + off + kHalfBytes, m, 64, y, &b.full[s]);
+        auto load = [&](int off, const CUtensorMap *m, uint64_t *bar) {  // both halves of a tile
+            tma_load_2d(st + off, m, 0, y, bar);
+            tma_load_2d(st + off + kHalfBytes, m, 64, y, bar);
         };
-        if (C::q) load(C::off_q, tq);
-        if (C::k) load(C::off_k, tk);
-        if (C::v) load(C::off_v, tv);
-        load(C::off_g, tg);
+        // the gates' tiles first, on their own barrier (the gates start as soon as they land);
+        // v, read only by the tensor cores, behind them
+        mbar_arrive_expect_tx(&b.full[s], C::stage_bytes - (C::v ? kTileBytes : 0));
+        if (C::v) mbar_arrive_expect_tx(&b.full_b[s], kTileBytes);
+        load(C::off_g, tg, &b.full[s]);
+        if (C::q) load(C::off_q, tq, &b.full[s]);
+        if (C::k) load(C::off_k, tk, &b.full[s]);
+        if (C::v) load(C::off_v, tv, &b.full_b[s]);
         issued = c + 1;
     }
     if (*abort)  // let every copy this CTA started land before it exits
-        for (int c = issued > C::stages ? issued - C::stages : 0; c < issued; ++c)
+        for (int c = issued > C::stages ? issued - C::stages : 0; c < issued; ++c) {
             wait_drain(&b.full[c % C::stages], (c / C::stages) & 1);
+            if (C::v) wait_drain(&b.full_b[c % C::stages], (c / C::stages) & 1);
+        }
 }
 
 // ------------------------------------------------------------------ MMA issuer (1 warp)
@@ -151,6 +156,7 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
             if (!(ok = warp_wait(&b.gated[s], (c / C::stages) & 1, abort))) break;
             tc_fence_after();
         }
+        if (C::v && !(ok = warp_wait(&b.full_b[s], (c / C::stages) & 1, abort))) break;
         if (C::dstate) {  // R^T += dO^T Qhat, accumulated over the whole segment from zero
             if (elect_one()) {
 #pragma unroll
@@ -519,13 +525,14 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
 }
 
 // ------------------------------------------------------------------ the kernels
-// Barrier block of one pass: 3 per stage, then 13 (layout of Bars).
+// Barrier block of one pass: 4 per stage, then 13 (layout of Bars).
 __device__ Bars carve_bars(uint64_t *bar, int stages) {
     Bars b;
     b.full = bar;
     b.gated = bar + stages;
     b.empty = bar + 2 * stages;
-    uint64_t *x = bar + 3 * stages;
+    b.full_b = bar + 3 * stages;
+    uint64_t *x = bar + 4 * stages;
     b.qk_full = x + 0; b.qk_free = x + 1; b.p_full = x + 2; b.ds_full = x + 4; b.sa_full = x + 5;
     b.sa_free = x + 6; b.o_full = x + 8; b.o_free = x + 10; b.fin = x + 12;
     return b;
@@ -534,6 +541,7 @@ __device__ Bars carve_bars(uint64_t *bar, int stages) {
 __device__ void init_bars(const Bars &b, int stages) {
     for (int s = 0; s < stages; ++s) {
         mbar_init(&b.full[s], 1);
+        mbar_init(&b.full_b[s], 1);
         mbar_init(&b.gated[s], kGateWarps);
         mbar_init(&b.empty[s], 1 + kStateWarps);
     }
