@@ -118,8 +118,8 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
 // ------------------------------------------------------------------ MMA issuer (1 warp)
 // The whole warp walks the loop and waits; one elected lane issues.  Per chunk c: the state
 // increment accumulated straight onto the decayed state S' that the state warps left in TMEM
-// (S = S' + dS); then, in the output modes, the scores of chunk c+1 (so that the output warps
-// build P(c+1) while the tensor cores finish chunk c); then PV and S'^T Qbar'^T into O^T.
+// (S = S' + dS); then, in the output modes, PV and S'^T Qbar'^T into O^T and the scores of
+// chunk c+1 -- the scores first when chunk c+1 is already gated.
 template <int MODE>
 __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
                            int nchunks) {
@@ -178,12 +178,17 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
             }
             __syncwarp();
         }
-        if (C::qk && c + 1 < nchunks) {  // scores of the next chunk
-            if (!(ok = warp_wait(&b.gated[(c + 1) % C::stages], ((c + 1) / C::stages) & 1, abort)))
-                break;
+        // The scores of the next chunk go first when its tiles are already gated (the output
+        // warps then build P(c+1) while the tensor cores finish chunk c); otherwise chunk c's
+        // outputs go first, so that this stage's release does not wait for the next gates.
+        const int n1 = (c + 1) % C::stages;
+        const uint32_t n1_par = ((c + 1) / C::stages) & 1;
+        bool qk_next = C::qk && c + 1 < nchunks;
+        if (qk_next && __all_sync(0xFFFFFFFFu, mbar_test_wait(&b.gated[n1], n1_par))) {
             if (!(ok = warp_wait(b.qk_free, c & 1, abort))) break;
             tc_fence_after();
             issue_qk(c + 1);
+            qk_next = false;
         }
         if (C::out) {
             const int ob = c & 1;
@@ -210,6 +215,12 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
         }
         if (elect_one()) mma_commit(&b.empty[s]);
         __syncwarp();
+        if (qk_next) {  // the next chunk's scores, after its gates
+            if (!(ok = warp_wait(&b.gated[n1], n1_par, abort))) break;
+            if (!(ok = warp_wait(b.qk_free, c & 1, abort))) break;
+            tc_fence_after();
+            issue_qk(c + 1);
+        }
     }
     if (elect_one()) {
         if (C::dstate) mma_commit(b.ds_full);
