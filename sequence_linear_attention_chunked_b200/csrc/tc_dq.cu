@@ -62,7 +62,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 enum : int {
     kFull = 0, kGated = kFull + kStages, kEmpty = kGated + kStages, kMFull = kEmpty + kStages,
     kMFree, kPFull, kDsFull = kPFull + 2, kSaFull, kSaFree, kDqFull = kSaFree + 2, kDqFree,
-    kRFull, kRFree, kFin, kFullB, kNumBars = kFullB + kStages
+    kRFull, kRFree, kFin, kFullB, kEcFull = kFullB + kStages, kNumBars = kEcFull + kStages
 };
 static_assert(kNumBars <= 24, "barrier area");
 struct Bars {
@@ -267,6 +267,8 @@ __device__ __noinline__ void gate_role(uint8_t *smem, const Bars &b, volatile in
                 lg[1] = make_float4(logB[4], logB[5], logB[6], logB[7]);
             }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b[kEcFull + s]);  // e^{b_C}: the state warps' decay can start
 #pragma unroll
         for (int k = 0; k < 4; ++k) {  // one row at a time, dims in pairs (register budget)
             const uint32_t off = tile_off(tg * 4 + (k ^ sw), i0);
@@ -327,7 +329,8 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
     }
     for (int c = 0; c < w.nchunks; ++c) {
         const int s = c % kStages;
-        if (!mbar_wait(b[kGated + s], (c / kStages) & 1, abort)) break;
+        // the decay needs only e^{b_C}, published by the gates before they rescale the tiles
+        if (!mbar_wait(b[kEcFull + s], (c / kStages) & 1, abort)) break;
         if (c > 0 && !mbar_wait(b[kDsFull], (c - 1) & 1, abort)) break;
         if (c >= 1 && !mbar_wait(b[kSaFree], (c - 1) & 1, abort)) break;
         tc_fence_after();
@@ -514,6 +517,7 @@ tc_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         for (int s = 0; s < kStages; ++s) {
             mbar_init(b[kFull + s], 1);
             mbar_init(b[kFullB + s], 1);
+            mbar_init(b[kEcFull + s], kGateWarps);
             mbar_init(b[kGated + s], kGateWarps);
             mbar_init(b[kEmpty + s], 1 + kStateWarps + kOutWarps);
         }

@@ -69,7 +69,7 @@ struct Cfg {
     static constexpr int off_p = stages * stage_bytes;           // two bf16 P tiles
     static constexpr int off_ec = off_p + (qk ? 2 * CH * CH * 2 : 0);
     static constexpr int off_bar = off_ec + stages * D * 4;
-    static constexpr int n_bars = 4 * stages + 13;
+    static constexpr int n_bars = 5 * stages + 13;
     static constexpr int off_misc = off_bar + n_bars * 8;
     static constexpr int smem_bytes = off_misc + 16 + 1024;  // + slack to align the base to 1 KB
     static_assert(smem_bytes <= 232448, "shared memory budget");
@@ -79,6 +79,7 @@ struct Cfg {
 // (P tile, O^T and S'^T), so that no waiter can fall two phases behind its barrier.
 struct Bars {
     uint64_t *full, *full_b, *gated, *empty;  // full: the gates' tiles; full_b: v
+    uint64_t *ec_full;                        // e^{b_C} written (before the gates rescale)
     uint64_t *qk_full, *qk_free, *p_full, *ds_full, *sa_full, *sa_free, *o_full, *o_free, *fin;
 };
 
@@ -313,6 +314,8 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) logG[e] += bC[e];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.ec_full[s]);  // the state warps' decay can start
         // rescale q (by e^{b_t - b_C}) and k (by e^{b_C - b_t}) in place, 2 rows per batch
 #pragma unroll
         for (int k0 = 0; k0 < 4; k0 += 2) {
@@ -399,7 +402,8 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
     }
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % C::stages;
-        if (!mbar_wait(&b.gated[s], (c / C::stages) & 1, abort)) break;
+        // the decay needs only e^{b_C}, published by the gates before they rescale the tiles
+        if (!mbar_wait(&b.ec_full[s], (c / C::stages) & 1, abort)) break;
         if (!C::dstate) {
             if (C::kv && c > 0 && !mbar_wait(b.ds_full, (c - 1) & 1, abort)) break;
             if (C::out && c >= 2 && !mbar_wait(&b.sa_free[c & 1], ((c >> 1) - 1) & 1, abort)) break;
@@ -536,14 +540,15 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
 }
 
 // ------------------------------------------------------------------ the kernels
-// Barrier block of one pass: 4 per stage, then 13 (layout of Bars).
+// Barrier block of one pass: 5 per stage, then 13 (layout of Bars).
 __device__ Bars carve_bars(uint64_t *bar, int stages) {
     Bars b;
     b.full = bar;
     b.gated = bar + stages;
     b.empty = bar + 2 * stages;
     b.full_b = bar + 3 * stages;
-    uint64_t *x = bar + 4 * stages;
+    b.ec_full = bar + 4 * stages;
+    uint64_t *x = bar + 5 * stages;
     b.qk_full = x + 0; b.qk_free = x + 1; b.p_full = x + 2; b.ds_full = x + 4; b.sa_full = x + 5;
     b.sa_free = x + 6; b.o_full = x + 8; b.o_free = x + 10; b.fin = x + 12;
     return b;
@@ -553,6 +558,7 @@ __device__ void init_bars(const Bars &b, int stages) {
     for (int s = 0; s < stages; ++s) {
         mbar_init(&b.full[s], 1);
         mbar_init(&b.full_b[s], 1);
+        mbar_init(&b.ec_full[s], kGateWarps);
         mbar_init(&b.gated[s], kGateWarps);
         mbar_init(&b.empty[s], 1 + kStateWarps);
     }
