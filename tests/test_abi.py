@@ -140,3 +140,52 @@ def test_backward_workspace_covers_both_splits(lib):
     need = w(2, 16, 131072, 128, 128, 8, 64, la_seg.LA_BF16, True)
     assert need >= 2 * 16 * 131072 * 128 * 4
     assert w(2, 16, 131072, 128, 128, 8, 64, la_seg.LA_BF16, False) < need
+
+
+def _chain(lib, **kw):
+    """Calls la_seg_chain_pass with fake (but aligned) pointers: only argument checks may run."""
+    a = dict(q=0x1000, k=0x2000, v=0x3000, g=0x4000, B=1, H=2, L=1024, d=128, NP=4, chunk=64,
+             dt=la_seg.LA_BF16, states=0x8000, ready=0x9000, o=0x5000, Sf=None, Ss=None, every=1,
+             status=None)
+    a.update(kw)
+    V = ctypes.c_void_p
+    return lib.la_seg_chain_pass(V(a["q"]), V(a["k"]), V(a["v"]), V(a["g"]), a["B"], a["H"],
+                                 a["L"], a["d"], a["d"], a["NP"], a["chunk"], a["dt"],
+                                 V(a["states"]), V(a["ready"]), V(a["o"]), V(a["Sf"]), V(a["Ss"]),
+                                 a["every"], V(a["status"]), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dt=la_seg.LA_F32), -2),      # the single pass exists for bf16, d = 128, chunk 64 only
+    (dict(d=64), -2),
+    (dict(chunk=32), -2),
+    (dict(NP=3), -2),                  # L % NP
+    (dict(states=None), -1),
+    (dict(ready=None), -1),
+    (dict(o=None), -1),
+    (dict(every=0), -1),
+    (dict(every=3), -1),               # save_every must divide NP
+    (dict(states=0x8004), -3),
+    (dict(Sf=0x7008), -3),
+    (dict(dt=9), -4),
+])
+def test_chain_pass_rejects_bad_arguments(lib, kw, status):
+    assert _chain(lib, **kw) == status
+    assert len(la_seg.la_last_error_detail()) > 0
+
+
+def test_chain_reset_rejects_bad_arguments(lib):
+    V = ctypes.c_void_p
+    reset = lib.la_seg_chain_reset
+    assert reset(None, 0, 2, 128, 128, V(0x8000), V(0x9000), None) == -2
+    assert reset(None, 1, 2, 48, 48, V(0x8000), V(0x9000), None) == -2
+    assert reset(None, 1, 2, 128, 128, None, V(0x9000), None) == -1
+    assert reset(None, 1, 2, 128, 128, V(0x8000), None, None) == -1
+    assert reset(V(0x7004), 1, 2, 128, 128, V(0x8000), V(0x9000), None) == -3
+
+
+def test_single_pass_schedule_is_accepted(lib):
+    # an unknown schedule is rejected, the single pass is not (the call then stops at the
+    # workspace check, before any launch)
+    assert _fwd(lib, sched=4) == -1
+    assert _fwd(lib, sched=la_seg.SCHED_SINGLE_PASS, ws=None) == -5
