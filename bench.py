@@ -182,6 +182,7 @@ class Step:
             self.dSloc = torch.empty((B, H, NPF, dk, dv), **f32)
             self.logG_b = torch.empty((B, H, NPF, dk), **f32)
             self.dX = torch.empty((B, H, NPF, dk, dv), **f32)
+            self.carry = torch.empty((B, H, NPF, dk), **f32)  # the parts' dlog_g carries
             self.dS0 = torch.empty_like(self.S_final)
             self.grads = (torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
                           torch.empty_like(x["log_g"]))
@@ -212,7 +213,8 @@ class Step:
             rec(1)
             la._check(la.lib().la_seg_scan(la._ptr(self.S_loc), la._ptr(self.logG), None, BH, NP,
                                            w.dk, w.dv, 0, la._ptr(self.S_recv),
-                                           la._ptr(self.S_final), la._stream(None)), "la_seg_scan")
+                                           la._ptr(self.S_final), None, None, None,
+                                           la._stream(None)), "la_seg_scan")
             rec(2)
             if self.schedule != "three":
                 la.la_seg_output_pass(x["q"], x["k"], x["v"], x["log_g"], self.S_recv, NP,
@@ -231,10 +233,12 @@ class Step:
         NPF = self.NPF
         la._check(la.lib().la_seg_scan(la._ptr(self.dSloc), la._ptr(self.logG_b), None, BH, NPF,
                                        w.dk, w.dv, 1, la._ptr(self.dX), la._ptr(self.dS0),
+                                       la._ptr(self.S_fine), None, la._ptr(self.carry),
                                        la._stream(None)), "la_seg_scan")
         rec(f + 2)
         la.la_seg_dkv_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_fine, None, self.dX,
-                           self.qdq, NPF, w.chunk, out=self.grads[1:], status=self.status)
+                           self.qdq, NPF, w.chunk, carry=self.carry, out=self.grads[1:],
+                           status=self.status)
         rec(f + 3)
 
     def phase_ms(self):

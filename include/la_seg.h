@@ -128,9 +128,15 @@ LA_API la_status la_seg_backward(const void *q, const void *k, const void *v, co
  *   reverse != 0:  acc = init;  for p = NP-1 .. 0:  out[p] = acc;  acc = exp(log_gamma[p][i]) * acc + S_in[p]
  *   final = acc.
  *  S_in, out: fp32 [BH, NP, dk, dv]; log_gamma: fp32 [BH, NP, dk]; init, final: fp32
- *  [BH, dk, dv], init nullable (zero), final nullable.  dv % 4 == 0.  out may not alias S_in. */
+ *  [BH, dk, dv], init nullable (zero), final nullable.  dv % 4 == 0.  out may not alias S_in.
+ *  carry (nullable, fp32 [BH, NP, dk]): also writes carry[p][i] = sum_j S_end_p[i][j] out[p][i][j]
+ *  with S_end_p = S_next[p+1] for p < NP-1 and S_last for p = NP-1 (S_next fp32
+ *  [BH, NP, dk, dv], required with carry; S_last fp32 [BH, dk, dv], nullable: zero) -- for the
+ *  backward's reverse scan, the dlog_g carry rowsum(S_end . dX) of every part, which
+ *  la_seg_dkv_pass then takes instead of forming it.  Needs dv / 4 to divide 32. */
 LA_API la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
                       int NP, int dk, int dv, int reverse, float *out, float *final_state,
+                      const float *S_next, const float *S_last, float *carry,
                       void *cuda_stream);
 
 /* ---- The steps of the path, one entry point each -------------------------------------
@@ -227,12 +233,14 @@ LA_API la_status la_seg_dq_pass(const void *q, const void *k, const void *v, con
  * (fp32 [B,H,dk,dv], the last segment's end state; null when dS_final is zero), dX: gradient of
  * every segment's end state (la_seg_scan with reverse = 1 over the gradient states of
  * la_seg_dstate_pass or la_seg_dq_pass, initialised with dS_final), qdq: la_seg_dq_pass's
- * q . dq. */
+ * q . dq.  carry (nullable, fp32 [B,H,NP,dk]): the dlog_g carries la_seg_scan formed with
+ * S_next = S_recv and S_last = S_final; when given, S_recv and S_final are not read. */
 LA_API la_status la_seg_dkv_pass(const void *q, const void *k, const void *v, const void *log_g,
                                  const void *dO, const float *S_recv, const float *S_final,
-                                 const float *dX, const float *qdq, int B, int H, long long L,
-                                 int dk, int dv, int NP, int chunk, la_dtype dt, void *dk_,
-                                 void *dv_, void *dlog_g, int *status, void *cuda_stream);
+                                 const float *dX, const float *qdq, const float *carry, int B,
+                                 int H, long long L, int dk, int dv, int NP, int chunk,
+                                 la_dtype dt, void *dk_, void *dv_, void *dlog_g, int *status,
+                                 void *cuda_stream);
 
 /* Number of parts la_seg_backward's gradient-state, reverse-scan and dk/dv steps run over
  * (reuse != 0: the caller passes S_recv_saved and no dS_final), or 0 for rejected sizes. */

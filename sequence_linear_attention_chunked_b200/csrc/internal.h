@@ -47,6 +47,7 @@ struct BwdArgs {
     float *dq_ws;             // [BH, L, dk] fp32 q . dq, from the dq sweep to the reverse sweep
     float *dSloc;             // [BH, NP, dk, dv] per-segment gradient states (dstate pass)
     float *logG;              // [BH, NP, dk] per-segment log-decay sums (dstate pass)
+    const float *carry;       // reverse sweep: [BH, NP, dk] dlog_g carry per part (null: computed)
     int *status;
     long long L, T;
     int BH, NP, dk, dv, chunk, fine;
@@ -98,10 +99,14 @@ cudaError_t launch_tc_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
 // The chunk pass for these arguments: the tensor-core kernels where they apply, else SIMT.
 cudaError_t launch_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
 
-// Exclusive decayed scan over NP sub-segments (see la_seg_scan in la_seg.h).
+// Exclusive decayed scan over NP sub-segments (see la_seg_scan in la_seg.h).  With `carry`
+// (fp32 [BH, NP, dk]) it also writes the reverse sweep's dlog_g carry of every part p,
+// rowsum(S_end_p . out[p]), S_end_p = S_next[p+1] for p < NP-1 and S_last (nullable: zero) for
+// the last part.
 cudaError_t launch_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
                         int NP, int dk, int dv, int reverse, float *out, float *final_state,
-                        cudaStream_t st);
+                        cudaStream_t st, const float *S_next = nullptr,
+                        const float *S_last = nullptr, float *carry = nullptr);
 
 // Copies the per-sub-segment states at API-segment boundaries: dst[bh][p] = src[bh][p*m].
 cudaError_t launch_gather_states(const float *src, int BH, int NP, int m, int dk, int dv,

@@ -111,7 +111,7 @@ int fine_factor(long long T, int chunk) {
 }
 
 struct BwdLayout {
-    size_t status, S_loc, logG, S_recv, S_fin, S_fine, dSloc, logG_f, dX, qdq, total;
+    size_t status, S_loc, logG, S_recv, S_fin, S_fine, dSloc, logG_f, dX, carry, qdq, total;
 };
 
 BwdLayout bwd_layout(const la::Split &s, int r, int dk, int dv) {
@@ -128,7 +128,8 @@ BwdLayout bwd_layout(const la::Split &s, int r, int dk, int dv) {
     w.dSloc = align_up(w.S_fine + fine_states, 256);
     w.logG_f = align_up(w.dSloc + fine_states, 256);
     w.dX = align_up(w.logG_f + gam * r, 256);
-    w.qdq = align_up(w.dX + fine_states, 256);
+    w.carry = align_up(w.dX + fine_states, 256);
+    w.qdq = align_up(w.carry + gam * r, 256);
     w.total = align_up(w.qdq + (size_t)s.BH * s.L * dk * sizeof(float), 256);
     return w;
 }
@@ -308,20 +309,21 @@ la_status la_seg_dq_pass(const void *q, const void *k, const void *v, const void
 
 la_status la_seg_dkv_pass(const void *q, const void *k, const void *v, const void *log_g,
                           const void *dO, const float *S_recv, const float *S_final,
-                          const float *dX, const float *qdq, int B, int H, long long L, int dk,
-                          int dv, int NP, int chunk, la_dtype dt, void *dk_, void *dv_,
-                          void *dlog_g, int *status, void *cuda_stream) {
+                          const float *dX, const float *qdq, const float *carry, int B, int H,
+                          long long L, int dk, int dv, int NP, int chunk, la_dtype dt, void *dk_,
+                          void *dv_, void *dlog_g, int *status, void *cuda_stream) {
     la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
                               {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {dO, "dO"},
                                {dX, "dX"}, {qdq, "qdq"}, {dk_, "dk"}, {dv_, "dv"},
                                {dlog_g, "dlog_g"}},
-                              {{S_recv, "S_recv"}, {S_final, "S_final"}});
+                              {{S_recv, "S_recv"}, {S_final, "S_final"}, {carry, "carry"}});
     if (st != LA_OK) return st;
     if (L == 0) return LA_OK;
     la::BwdArgs b = {};
     b.q = q; b.k = k; b.v = v; b.g = log_g; b.dO = dO;
     b.dk_out = dk_; b.dv_out = dv_; b.dg_out = dlog_g;
     b.S_end_next = S_recv; b.S_fin = S_final; b.dX = dX; b.dq_ws = const_cast<float *>(qdq);
+    b.carry = carry;
     b.status = status;
     b.L = L; b.T = L / NP; b.BH = B * H; b.NP = NP; b.dk = dk; b.dv = dv; b.chunk = chunk;
     b.fine = 1; b.dt = dt;
@@ -506,6 +508,7 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     float *dSloc = reinterpret_cast<float *>(at(workspace, w.dSloc));
     float *logG_f = reinterpret_cast<float *>(at(workspace, w.logG_f));
     float *dX = reinterpret_cast<float *>(at(workspace, w.dX));
+    float *carry = reinterpret_cast<float *>(at(workspace, w.carry));
     float *qdq = reinterpret_cast<float *>(at(workspace, w.qdq));
 
     // 1. the states each segment receives: the forward's when given and S_final is not needed
@@ -532,10 +535,12 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     if ((e = la::launch_bwd_dq(b, stream)) != cudaSuccess) return cuda_fail(e, "dq pass");
     // 3-4 run over the fine parts
     b.NP = s.NP * r; b.T = s.T / r; b.fine = 1;
-    // 3. reverse exclusive decayed scan: gradient of every part's end state, and dS0
-    if ((e = la::launch_scan(dSloc, logG_f, dS_final, s.BH, b.NP, dk, dv, 1, dX, dS0, stream)) !=
-        cudaSuccess)
+    // 3. reverse exclusive decayed scan: gradient of every part's end state, dS0, and each
+    //    part's dlog_g carry rowsum(S_end . dX) (S_end: the state entering the next part)
+    if ((e = la::launch_scan(dSloc, logG_f, dS_final, s.BH, b.NP, dk, dv, 1, dX, dS0, stream,
+                             S_fine, b.S_fin, carry)) != cudaSuccess)
         return cuda_fail(e, "reverse state scan");
+    b.carry = carry;
     // 4. dk, dv, dlog_g per part
     if ((e = la::launch_bwd_dkv(b, stream)) != cudaSuccess) return cuda_fail(e, "dkv pass");
     return LA_OK;
@@ -543,6 +548,7 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
 
 la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
                       int NP, int dk, int dv, int reverse, float *out, float *final_state,
+                      const float *S_next, const float *S_last, float *carry,
                       void *cuda_stream) {
     if (BH < 0 || NP < 0 || dk < 1 || dv < 4 || dv % 4)
         return fail(LA_ERR_SHAPE, "need BH, NP >= 0, dk >= 1, dv a positive multiple of 4");
@@ -555,8 +561,19 @@ la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *in
             return fail(LA_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
     if (log_gamma && !aligned(log_gamma, 4)) return fail(LA_ERR_ALIGN, "log_gamma misaligned");
     if (S_in && out == S_in) return fail(LA_ERR_ARG, "out may not alias S_in");
+    if (carry) {
+        if (32 % (dv / 4) || (dk * (dv / 4)) % 32)
+            return fail(LA_ERR_SHAPE, "carry needs dv / 4 to divide 32 (got dv=%d)", dv);
+        if ((long long)BH * NP > 0 && !S_next)
+            return fail(LA_ERR_ARG, "S_next must be non-null with carry");
+        const void *cp[] = {S_next, S_last};
+        for (const void *q : cp)
+            if (q && !aligned(q, 16)) return fail(LA_ERR_ALIGN, "S_next / S_last misaligned");
+        if (!aligned(carry, 4)) return fail(LA_ERR_ALIGN, "carry misaligned");
+    }
     cudaError_t e = la::launch_scan(S_in, log_gamma, init, BH, NP, dk, dv, reverse, out,
-                                    final_state, static_cast<cudaStream_t>(cuda_stream));
+                                    final_state, static_cast<cudaStream_t>(cuda_stream), S_next,
+                                    S_last, carry);
     return e == cudaSuccess ? LA_OK : cuda_fail(e, "scan");
 }
 

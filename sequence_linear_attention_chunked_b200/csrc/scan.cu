@@ -16,13 +16,23 @@
 namespace la {
 namespace {
 
-constexpr int kScanThreads = 256;
+// 128-thread blocks and a 4-deep batch for the carry variant keep it at one wave of blocks
+// (the C4 reverse scan is 1024 blocks, 7 per SM), which 256-thread blocks at its register count
+// would not.
+constexpr int kScanThreads = 128;
 constexpr int kUnroll = 8;
 
+// With `carry` (the backward's reverse scan): carry[bh][p][i] = sum_j S_end_p[i][j] out[p][i][j],
+// S_end_p = S_next[p+1] (p < NP-1) or S_last (p = NP-1; null: zero) -- the dlog_g carry of part
+// p.  The threads of one row i are dv4 consecutive lanes of a warp, so the sum over j is a
+// segmented warp reduction.
+template <bool CARRY>
 __global__ void __launch_bounds__(kScanThreads)
 scan_kernel(const float4 *__restrict__ S_in, const float *__restrict__ log_gamma,
             const float4 *__restrict__ init, int BH, int NP, int dk, int dv4, int reverse,
-            float4 *__restrict__ out, float4 *__restrict__ final_state) {
+            float4 *__restrict__ out, float4 *__restrict__ final_state,
+            const float4 *__restrict__ S_next, const float4 *__restrict__ S_last,
+            float *__restrict__ carry) {
     const long long e = (long long)blockIdx.x * kScanThreads + threadIdx.x;  // (bh, i, j4)
     const long long per_bh = (long long)dk * dv4;
     if (e >= (long long)BH * per_bh) return;
@@ -34,24 +44,36 @@ scan_kernel(const float4 *__restrict__ S_in, const float *__restrict__ log_gamma
     const float *lg = log_gamma + bh * (long long)NP * dk + i;
 
     float4 acc = init ? init[bh * per_bh + ij] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p0 = 0; p0 < NP; p0 += kUnroll) {
-        float4 x[kUnroll];
-        float gm[kUnroll];
+    constexpr int kU = CARRY ? 4 : kUnroll;
+    for (int p0 = 0; p0 < NP; p0 += kU) {
+        float4 x[kU], se[CARRY ? kU : 1];
+        float gm[kU];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < kU; ++u) {
             const int p = p0 + u;
             if (p < NP) {
                 const int pp = reverse ? NP - 1 - p : p;
                 x[u] = __ldcs(src + (long long)pp * per_bh);
                 gm[u] = __expf(lg[(long long)pp * dk]);
+                if (CARRY) {
+                    const float4 *e4 = pp + 1 < NP ? S_next + (bh * NP + pp + 1) * per_bh + ij
+                                                   : (S_last ? S_last + bh * per_bh + ij : nullptr);
+                    se[CARRY ? u : 0] = e4 ? *e4 : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < kU; ++u) {
             const int p = p0 + u;
             if (p < NP) {
                 const int pp = reverse ? NP - 1 - p : p;
                 __stcs(dst + (long long)pp * per_bh, acc);
+                if (CARRY) {
+                    const float4 &v = se[CARRY ? u : 0];
+                    float sum = fmaf(v.w, acc.w, fmaf(v.z, acc.z, fmaf(v.y, acc.y, v.x * acc.x)));
+                    for (int o = 1; o < dv4; o <<= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+                    if (ij % dv4 == 0) carry[(bh * NP + pp) * dk + i] = sum;
+                }
                 acc.x = fmaf(gm[u], acc.x, x[u].x);
                 acc.y = fmaf(gm[u], acc.y, x[u].y);
                 acc.z = fmaf(gm[u], acc.z, x[u].z);
@@ -85,15 +107,24 @@ __global__ void copy_state_kernel(const float4 *__restrict__ src, long long n4,
 
 cudaError_t launch_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
                         int NP, int dk, int dv, int reverse, float *out, float *final_state,
-                        cudaStream_t st) {
+                        cudaStream_t st, const float *S_next, const float *S_last, float *carry) {
+    if (carry && (dv % 4 || 32 % (dv / 4) || (dk * (dv / 4)) % 32)) return cudaErrorInvalidValue;
     const int dv4 = dv / 4;
     const long long n = (long long)BH * dk * dv4;
     if (n == 0) return cudaSuccess;
     const unsigned blocks = (unsigned)((n + kScanThreads - 1) / kScanThreads);
-    scan_kernel<<<blocks, kScanThreads, 0, st>>>(
-        reinterpret_cast<const float4 *>(S_in), log_gamma, reinterpret_cast<const float4 *>(init),
-        BH, NP, dk, dv4, reverse, reinterpret_cast<float4 *>(out),
-        reinterpret_cast<float4 *>(final_state));
+    auto S_in4 = reinterpret_cast<const float4 *>(S_in);
+    auto init4 = reinterpret_cast<const float4 *>(init);
+    auto out4 = reinterpret_cast<float4 *>(out);
+    auto fin4 = reinterpret_cast<float4 *>(final_state);
+    if (carry)  // whole warps per row: dv4 divides 32 and blocks hold whole rows
+        scan_kernel<true><<<blocks, kScanThreads, 0, st>>>(
+            S_in4, log_gamma, init4, BH, NP, dk, dv4, reverse, out4, fin4,
+            reinterpret_cast<const float4 *>(S_next), reinterpret_cast<const float4 *>(S_last), carry);
+    else
+        scan_kernel<false><<<blocks, kScanThreads, 0, st>>>(S_in4, log_gamma, init4, BH, NP, dk,
+                                                            dv4, reverse, out4, fin4, nullptr,
+                                                            nullptr, nullptr);
     return cudaGetLastError();
 }
 

@@ -448,23 +448,33 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
     __nv_bfloat16 *dk = static_cast<__nv_bfloat16 *>(a.dk_out);
     __nv_bfloat16 *dg = static_cast<__nv_bfloat16 *>(a.dg_out);
     const long long sidx = ((long long)bh * a.NP + j) * D * D;
-    // carry: rowsum(S_end . dX), the gradient reaching this part from its end state
+    // carry: rowsum(S_end . dX), the gradient reaching this part from its end state (formed by
+    // the reverse scan when it is given)
     float carry = 0.f;
-    {
+    if (a.carry) {
+        carry = a.carry[((long long)bh * a.NP + j) * D + x];
+    } else {
         const float *Se = nullptr;
         if (j < a.NP - 1) {
             if (a.S_end_next) Se = a.S_end_next + sidx + (long long)D * D;
         } else if (a.S_fin) {
             Se = a.S_fin + (long long)bh * D * D;
         }
-        if (Se) {
+        if (Se) {  // summed in the reverse scan's order (per 4 columns, then a pairwise tree)
             const float4 *x4 = reinterpret_cast<const float4 *>(a.dX + sidx + (long long)x * D);
             const float4 *s4 = reinterpret_cast<const float4 *>(Se + (long long)x * D);
-#pragma unroll 8
+            float part[D / 4];
+#pragma unroll
             for (int e4 = 0; e4 < D / 4; ++e4) {
                 const float4 v = x4[e4], u = s4[e4];
-                carry += u.x * v.x + u.y * v.y + u.z * v.z + u.w * v.w;
+                part[e4] = fmaf(u.w, v.w, fmaf(u.z, v.z, fmaf(u.y, v.y, u.x * v.x)));
             }
+#pragma unroll
+            for (int o = 1; o < D / 4; o <<= 1) {
+#pragma unroll
+                for (int k = 0; k < D / 4; k += 2 * o) part[k] += part[k + o];
+            }
+            carry = part[0];
         }
     }
     uint32_t r[16], fk[16];

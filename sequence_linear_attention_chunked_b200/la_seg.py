@@ -54,7 +54,7 @@ def lib():
         L.la_seg_backward.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
                                       i32, P, P, P, P, P, P, sz, P]
         L.la_seg_backward.restype = i32
-        L.la_seg_scan.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P]
+        L.la_seg_scan.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
         L.la_seg_scan.restype = i32
         L.la_seg_state_pass.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P, P, P]
         L.la_seg_state_pass.restype = i32
@@ -77,7 +77,7 @@ def lib():
         L.la_seg_dq_pass.argtypes = [P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32,
                                      i32, P, P, P, P, P, P, P]
         L.la_seg_dq_pass.restype = i32
-        L.la_seg_dkv_pass.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32,
+        L.la_seg_dkv_pass.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32,
                                       i32, i32, P, P, P, P, P]
         L.la_seg_dkv_pass.restype = i32
         L.la_seg_backward_parts.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32, i32]
@@ -208,19 +208,30 @@ def la_seg_backward(q, k, v, log_g, dO, S0=None, S_recv_saved=None, dS_final=Non
     return dq, dk_, dv_, dg, dS0
 
 
-def la_seg_scan(S_in, log_gamma, init=None, reverse=False, *, want_final=True, stream=None):
-    """out, final = exclusive decayed scan over dim 1 of S_in [BH, NP, dk, dv] (fp32)."""
+def la_seg_scan(S_in, log_gamma, init=None, reverse=False, *, want_final=True, S_next=None,
+                S_last=None, out=None, final=None, carry=None, stream=None):
+    """out, final = exclusive decayed scan over dim 1 of S_in [BH, NP, dk, dv] (fp32).
+
+    With S_next (and optionally S_last) a carry tensor fp32 [BH, NP, dk] is filled too (given,
+    or allocated and returned as a third value): the dlog_g carries of la_seg_dkv_pass."""
     BH, NP, dk, dv = S_in.shape
     dev = S_in.device
     _need(S_in, "S_in", torch.float32, None, dev)
     _need(log_gamma, "log_gamma", torch.float32, (BH, NP, dk), dev)
     _need(init, "init", torch.float32, (BH, dk, dv), dev)
-    out = torch.empty_like(S_in)
-    final = torch.empty((BH, dk, dv), dtype=torch.float32, device=dev) if want_final else None
+    _need(S_next, "S_next", torch.float32, (BH, NP, dk, dv), dev)
+    _need(S_last, "S_last", torch.float32, (BH, dk, dv), dev)
+    out = torch.empty_like(S_in) if out is None else out
+    if final is None and want_final:
+        final = torch.empty((BH, dk, dv), dtype=torch.float32, device=dev)
+    want_carry = S_next is not None
+    if want_carry and carry is None:
+        carry = torch.empty((BH, NP, dk), dtype=torch.float32, device=dev)
     st = lib().la_seg_scan(_ptr(S_in), _ptr(log_gamma), _ptr(init), BH, NP, dk, dv,
-                           int(bool(reverse)), _ptr(out), _ptr(final), _stream(stream))
+                           int(bool(reverse)), _ptr(out), _ptr(final), _ptr(S_next),
+                           _ptr(S_last), _ptr(carry if want_carry else None), _stream(stream))
     _check(st, "la_seg_scan")
-    return out, final
+    return (out, final, carry) if want_carry else (out, final)
 
 
 def la_seg_check_status(ws, stream=None):
@@ -315,14 +326,15 @@ def la_seg_dq_pass(q, k, v, log_g, dO, S_recv, NP, fine, chunk, *, dq=None, qdq=
     return dq, qdq
 
 
-def la_seg_dkv_pass(q, k, v, log_g, dO, S_recv, S_final, dX, qdq, NP, chunk, *, out=None,
-                    status=None, stream=None):
+def la_seg_dkv_pass(q, k, v, log_g, dO, S_recv, S_final, dX, qdq, NP, chunk, *, carry=None,
+                    out=None, status=None, stream=None):
     B, H, L, dk, dv = _seq_shapes(q, v)
     if out is None:
         out = (torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_g))
     dk_, dv_, dg = out
     _check(lib().la_seg_dkv_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(dO), _ptr(S_recv),
-                                 _ptr(S_final), _ptr(dX), _ptr(qdq), B, H, L, dk, dv, NP, chunk,
+                                 _ptr(S_final), _ptr(dX), _ptr(qdq), _ptr(carry), B, H, L, dk, dv,
+                                 NP, chunk,
                                  _dt(q), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(status),
                                  _stream(stream)), "la_seg_dkv_pass")
     return out

@@ -89,12 +89,23 @@ def test_forward_rejects_bad_arguments(lib, kw, status):
     assert len(la_seg.la_last_error_detail()) > 0
 
 
-def test_scan_rejects_bad_arguments(lib):
+def _scan(lib, S_in=0x1000, lg=0x2000, d=32, dv=None, out=0x3000, S_next=None, S_last=None,
+          carry=None):
+    """la_seg_scan with fake (but aligned) pointers: only argument checks may run."""
     V = ctypes.c_void_p
-    assert lib.la_seg_scan(V(0x1000), V(0x2000), None, 1, 2, 32, 30, 0, V(0x3000), None, None) == -2
-    assert lib.la_seg_scan(None, V(0x2000), None, 1, 2, 32, 32, 0, V(0x3000), None, None) == -1
-    assert lib.la_seg_scan(V(0x1004), V(0x2000), None, 1, 2, 32, 32, 0, V(0x3000), None, None) == -3
-    assert lib.la_seg_scan(V(0x1000), V(0x2000), None, 1, 2, 32, 32, 0, V(0x1000), None, None) == -1
+    return lib.la_seg_scan(V(S_in), V(lg), None, 1, 2, d, d if dv is None else dv, 0, V(out),
+                           None, V(S_next), V(S_last), V(carry), None)
+
+
+def test_scan_rejects_bad_arguments(lib):
+    assert _scan(lib, dv=30) == -2
+    assert _scan(lib, S_in=None) == -1
+    assert _scan(lib, S_in=0x1004) == -3
+    assert _scan(lib, out=0x1000) == -1                        # out aliases S_in
+    assert _scan(lib, carry=0x5000) == -1                      # carry needs S_next
+    assert _scan(lib, dv=24, S_next=0x4000, carry=0x5000) == -2  # dv / 4 must divide 32
+    assert _scan(lib, S_next=0x4008, carry=0x5000) == -3
+    assert _scan(lib, S_next=0x4000, S_last=0x6004, carry=0x5000) == -3
 
 
 def test_error_detail_handles_small_buffers(lib):

@@ -170,3 +170,32 @@ def test_dq_pass_gradient_states(cuda_device, shape):
         ref = oracle.backward(*part)
         assert rel_err(dSloc[:, :, p], ref[4]) <= TOL[w.torch_dtype], p
         assert rel_err(lg[:, :, p], x["log_g"][:, :, sl].double().sum(2).cpu()) <= 1e-5, p
+
+
+def test_dkv_pass_carry_from_scan_is_bit_identical(cuda_device):
+    """la_seg_dkv_pass with the reverse scan's carries equals forming them in the pass (both sum
+    each row in the same order), and la_seg_backward composes exactly these steps."""
+    w = Workload("dkv-carry", 1, 2, 4096, 128, 128, 2, 64, "bf16", "gla", seed=9, backward=True)
+    x = make_inputs(w, cuda_device)
+    B, H, L, D = w.B, w.H, w.L, 128
+    NP = la_seg.la_seg_subsegments(B, H, L, D, D, w.P, 64)
+    NPF = la_seg.la_seg_backward_parts(B, H, L, D, D, w.P, 64, la_seg.LA_BF16, False)
+    f32 = dict(dtype=torch.float32, device=cuda_device)
+    _, Sf, _ = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, w.P, 64)
+    S_loc, lgs = la_seg.la_seg_state_pass(x["k"], x["v"], x["log_g"], NP, 64)
+    S_recv, _ = la_seg.la_seg_scan(S_loc.view(B * H, NP, D, D), lgs.view(B * H, NP, D))
+    S_fine = torch.empty((B, H, NPF, D, D), **f32)
+    dSloc = torch.empty_like(S_fine)
+    lgf = torch.empty((B, H, NPF, D), **f32)
+    dq, qdq = la_seg.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"],
+                                    S_recv.view(B, H, NP, D, D), NP, NPF // NP, 64,
+                                    S_fine=S_fine, dSloc=dSloc, log_gamma=lgf)
+    dX, _, carry = la_seg.la_seg_scan(dSloc.view(B * H, NPF, D, D), lgf.view(B * H, NPF, D),
+                                      None, True, S_next=S_fine.view(B * H, NPF, D, D),
+                                      S_last=Sf.view(B * H, D, D))
+    a = la_seg.la_seg_dkv_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], S_fine, Sf, dX, qdq,
+                               NPF, 64)
+    b = la_seg.la_seg_dkv_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], S_fine, Sf, dX, qdq,
+                               NPF, 64, carry=carry)
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)

@@ -78,3 +78,23 @@ def test_scan_empty(cuda_device):
     lg = torch.zeros((0, 4, 32), device=cuda_device)
     out, fin = la_seg.la_seg_scan(S, lg, None)
     assert out.numel() == 0 and fin.numel() == 0
+
+
+def test_scan_carry(cuda_device):
+    """The reverse scan's dlog_g carries: carry[p][i] = sum_j S_end_p[i][j] out[p][i][j], with
+    S_end_p = S_next[p+1] and S_last for the last segment."""
+    g = torch.Generator(device="cpu").manual_seed(5)
+    BH, NP, d = 3, 9, 128
+    S = torch.randn(BH, NP, d, d, generator=g).to(cuda_device)
+    lg = (-torch.rand(BH, NP, d, generator=g)).to(cuda_device)
+    init = torch.randn(BH, d, d, generator=g).to(cuda_device)
+    S_next = torch.randn(BH, NP, d, d, generator=g).to(cuda_device)
+    S_last = torch.randn(BH, d, d, generator=g).to(cuda_device)
+    out, fin, carry = la_seg.la_seg_scan(S, lg, init, True, S_next=S_next, S_last=S_last)
+    out_plain, fin_plain = la_seg.la_seg_scan(S, lg, init, True)
+    assert torch.equal(out, out_plain) and torch.equal(fin, fin_plain)
+    S_end = torch.cat([S_next[:, 1:], S_last[:, None]], dim=1).double()
+    ref = (S_end * out.double()).sum(dim=-1)
+    assert torch.allclose(carry.double(), ref, rtol=1e-5, atol=1e-4 * float(ref.abs().max()))
+    _, _, carry0 = la_seg.la_seg_scan(S, lg, init, True, S_next=S_next)  # no S_last: zero there
+    assert torch.equal(carry0[:, :-1], carry[:, :-1]) and torch.all(carry0[:, -1] == 0)
