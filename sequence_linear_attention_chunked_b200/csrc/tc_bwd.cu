@@ -51,7 +51,7 @@ constexpr int off_ma = kStages * kStageBytes;  // 2 buffers x (M tile, A tile)
 constexpr int off_ds = off_ma + 4 * kMaskBytes;
 constexpr int off_ec = off_ds + 2 * kDsHalf;
 constexpr int off_bar = off_ec + kStages * D * 4;
-constexpr int kBars = 4 * kStages + 16;
+constexpr int kBars = 4 * kStages + 17;
 constexpr int off_misc = off_bar + kBars * 8;
 constexpr int kSmemBytes = off_misc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -59,8 +59,15 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 struct Bars {
     uint64_t *full, *full_b, *gated, *empty;  // full: log_g, q, k (the gates); full_b: v, dO
     uint64_t *m_full, *m_free, *a_full, *a_free, *p_full, *dst_full, *dk_full, *dk_free, *dv_full, *dv_free,
-        *dsn_full, *fin;
+        *dsn_full, *fin, *dx_full;
 };
+
+// At a CTA's start the part's dX (fp32 [128 x 128], 64 KiB) is TMA-loaded as four 32-column
+// boxes with the 128-byte swizzle into the masked-tile and dS-tile area, which the first chunk
+// only writes later: row i of box b at kDxStage + b * 16 KiB + i * 128, 16-byte chunk e stored
+// at chunk e ^ (i % 8), so that the dS warps' row reads are free of bank conflicts.
+constexpr int kDxStage = off_ma;
+static_assert(off_ds + 2 * kDsHalf - off_ma == 4 * 16384, "dX staging area");
 
 // [128 rows][128 cols] bf16 tile as two 64-column halves of 16 KiB, 128-byte swizzle.
 __device__ __forceinline__ uint32_t ds_off(int row, int col) {
@@ -70,7 +77,11 @@ __device__ __forceinline__ uint32_t ds_off(int row, int col) {
 
 __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tq,
                          const CUtensorMap *tk, const CUtensorMap *tv, const CUtensorMap *tdo,
-                         const CUtensorMap *tg, const float *qdq, long long row0, int nchunks) {
+                         const CUtensorMap *tg, const CUtensorMap *tdx, int dx_row,
+                         const float *qdq, long long row0, int nchunks) {
+    mbar_arrive_expect_tx(b.dx_full, 4 * 16384);
+    for (int bx = 0; bx < 4; ++bx)
+        tma_load_2d(smem + kDxStage + bx * 16384, tdx, 32 * bx, dx_row, b.dx_full);
     int issued = 0;
     for (int it = 0; it < nchunks; ++it) {
         const int s = it % kStages;
@@ -94,11 +105,13 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
         }
         issued = it + 1;
     }
-    if (*abort)
+    if (*abort) {
+        wait_drain(b.dx_full, 0);
         for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it) {
             wait_drain(&b.full[it % kStages], (it / kStages) & 1);
             wait_drain(&b.full_b[it % kStages], (it / kStages) & 1);
         }
+    }
 }
 
 // The whole warp walks the loop; one elected lane issues.  Per chunk: dk^T and dv^T into
@@ -357,32 +370,47 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
     const uint32_t lrow = (uint32_t)(warp * 32) << 16;
     const float *ec = reinterpret_cast<const float *>(smem + off_ec);
     uint32_t r[32];
-    {  // dS at the part's end: dX
-        const float4 *x4 = reinterpret_cast<const float4 *>(a.dX + ((long long)bh * a.NP + j) * D * D +
-                                                            (long long)i * D);
+    // dS at the part's end: dX, row i from the swizzled staging boxes.  Column groups go last to
+    // first: the bf16 copy of group p lands on row i of box 2 + p / 2 (the dS tile's halves
+    // overlay boxes 2 and 3), which this thread has read by then; no other thread reads row i.
+    const bool dx_ok = warp_wait(b.dx_full, 0, abort);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
+    for (int p = 3; p >= 0; --p) {
+        if (!dx_ok) break;
+        const uint8_t *row = smem + kDxStage + p * 16384 + i * 128;
 #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-                const float4 v = x4[p * 8 + e4];
-                r[4 * e4] = __float_as_uint(v.x); r[4 * e4 + 1] = __float_as_uint(v.y);
-                r[4 * e4 + 2] = __float_as_uint(v.z); r[4 * e4 + 3] = __float_as_uint(v.w);
-            }
-            tmem_st32(tmem + lrow + kColDS + p * 32, r);
+        for (int e4 = 0; e4 < 8; ++e4) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(row + ((e4 ^ (i & 7)) << 4));
+            r[4 * e4] = v.x; r[4 * e4 + 1] = v.y; r[4 * e4 + 2] = v.z; r[4 * e4 + 3] = v.w;
         }
-        tmem_wait_st();
-        tc_fence_before();
+        tmem_st32(tmem + lrow + kColDS + p * 32, r);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t *x = r + jj * 8;
+            *reinterpret_cast<uint4 *>(smem + off_ds + ds_off(i, p * 32 + jj * 8)) =
+                make_uint4(pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                           pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
+                           pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
+                           pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
+        }
     }
+    tmem_wait_st();
+    tc_fence_before();
+    // the first masked tiles overwrite boxes 0 and 1, whose rows the other dS warps read (every
+    // dS warp reaches this barrier, also when its wait gave up)
+    named_sync(1, kStateWarps * 32);
+    if (!dx_ok) return;
     uint64_t e2 = 0;  // e^{b_C,i} of the previous chunk, in both halves
     for (int it = 0; it < nchunks; ++it) {
-        // (1) dS of this chunk's end: decayed unless it is the part's end
-        if (it > 0 && !mbar_wait(b.dsn_full, (it - 1) & 1, abort)) break;
-        tc_fence_after();
+        // (1) dS of this chunk's end: the decayed dS of the chunk after it (the part's last
+        // chunk starts from dX, stored above)
+        if (it > 0) {
+            if (!mbar_wait(b.dsn_full, (it - 1) & 1, abort)) break;
+            tc_fence_after();
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            tmem_ld32(tmem + lrow + kColDS + p * 32, r);
-            tmem_wait_ld();
-            if (it > 0) {
+            for (int p = 0; p < 4; ++p) {
+                tmem_ld32(tmem + lrow + kColDS + p * 32, r);
+                tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const uint64_t x = mul_f32x2(((uint64_t)r[2 * e + 1] << 32) | r[2 * e], e2);
@@ -390,18 +418,18 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
                     r[2 * e + 1] = (uint32_t)(x >> 32);
                 }
                 tmem_st32(tmem + lrow + kColDS + p * 32, r);
-            }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t *x = r + jj * 8;
-                *reinterpret_cast<uint4 *>(smem + off_ds + ds_off(i, p * 32 + jj * 8)) =
-                    make_uint4(pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
-                               pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
-                               pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
-                               pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t *x = r + jj * 8;
+                    *reinterpret_cast<uint4 *>(smem + off_ds + ds_off(i, p * 32 + jj * 8)) =
+                        make_uint4(pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                                   pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
+                                   pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
+                                   pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
+                }
             }
+            tmem_wait_st();
         }
-        if (it > 0) tmem_wait_st();
         tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
@@ -548,7 +576,8 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
 __global__ void __launch_bounds__(kThreads, 1)
 tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-              const __grid_constant__ CUtensorMap tm_g, const BwdArgs a) {
+              const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_dx,
+              const BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -561,7 +590,7 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint64_t *x = bar + 4 * kStages;
     b.m_full = x + 0; b.m_free = x + 1; b.p_full = x + 2; b.dst_full = x + 3; b.dk_full = x + 4;
     b.dk_free = x + 6; b.dv_full = x + 8; b.dv_free = x + 10; b.dsn_full = x + 12; b.fin = x + 13;
-    b.a_full = x + 14; b.a_free = x + 15;
+    b.a_full = x + 14; b.a_free = x + 15; b.dx_full = x + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -576,7 +605,7 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&b.empty[s], 1 + kStateWarps + kOutWarps);
         }
         uint64_t *one[] = {b.m_full, b.a_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dsn_full,
-                           b.fin};
+                           b.fin, b.dx_full};
         uint64_t *st4[] = {b.m_free, b.a_free, b.p_full, b.dst_full, b.dv_free};  // dv_free: gates
         uint64_t *out4[] = {b.dk_free, b.dk_free + 1};
         for (uint64_t *p : one) mbar_init(p, 1);
@@ -591,6 +620,7 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_g);
+        prefetch_tmap(&tm_dx);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -599,7 +629,8 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
     if (warp == kTmaWarp) {
         if (lane == 0)
-            producer(smem, b, abort, &tm_q, &tm_k, &tm_v, &tm_do, &tm_g, a.dq_ws, row0, nchunks);
+            producer(smem, b, abort, &tm_q, &tm_k, &tm_v, &tm_do, &tm_g, &tm_dx,
+                     (int)(((long long)bh * a.NP + j) * D), a.dq_ws, row0, nchunks);
     } else if (warp == kMmaWarp) {
         mma_issuer(smem, b, abort, tmem, nchunks);
     } else if (warp >= kEpiWarps) {
@@ -636,12 +667,16 @@ cudaError_t launch_tc_dkv(const BwdArgs &a, cudaStream_t st) {
     if ((e = make_map(&mv, a.v, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mdo, a.dO, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mg, a.g, rows)) != cudaSuccess) return e;
+    CUtensorMap mdx;  // dX as [BH * NP * dk rows, dv] fp32
+    if ((long long)a.BH * a.NP * D > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    if ((e = make_map_f32_rows(&mdx, a.dX, (long long)a.BH * a.NP * D)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(dkv::tc_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dkv::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long nblk = (long long)a.BH * a.NP;
     if (nblk == 0) return cudaSuccess;
-    dkv::tc_dkv_kernel<<<(unsigned)nblk, kThreads, dkv::kSmemBytes, st>>>(mq, mk, mv, mdo, mg, a);
+    dkv::tc_dkv_kernel<<<(unsigned)nblk, kThreads, dkv::kSmemBytes, st>>>(mq, mk, mv, mdo, mg, mdx,
+                                                                           a);
     return cudaGetLastError();
 }
 
