@@ -268,8 +268,11 @@ class Step:
             # reads q, k, v, dO, log_g and the received states; writes dq, S_fine, dSloc and
             # log_gamma (the fp32 q . dq hand-over to the dkv pass is not counted)
             ab["dq pass"] = th * (3 * w.dk + 2 * w.dv + w.dk) * e + st + 2 * stf + lgf
-            ab["reverse scan"] = 2 * stf + lgf + fin
-            ab["dkv pass"] = th * (3 * w.dk + 2 * w.dv + 2 * w.dk + w.dv) * e + 2 * stf
+            carry = w.B * w.H * self.NPF * w.dk * 4
+            # reverse scan: the parts' gradient states in, their end-state gradients out, and the
+            # dlog_g carries (end states read, one float per part and key dim written)
+            ab["reverse scan"] = 3 * stf + lgf + fin + carry
+            ab["dkv pass"] = th * (3 * w.dk + 2 * w.dv + 2 * w.dk + w.dv) * e + stf + carry
         return ab
 
     def flops(self):
