@@ -512,17 +512,9 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
         const int c = nchunks - 1 - it;
         const float *qdq = a.dq_ws + (row0 + (long long)c * CH) * D + x;
         // (1) the chunk's factors and Ktil into this lane of TMEM; then the stage is released
-        if (!mbar_wait(&b.gated[s], (it / kStages) & 1, abort)) break;
+        if (!warp_wait(&b.gated[s], (it / kStages) & 1, abort)) break;
         const uint32_t sa = smem_u32(smem + s * kStageBytes);
-#pragma unroll 1
-        for (int g = 0; g < 4; ++g) {
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const uint32_t off = tile_off(g * 16 + t, x);
-                fk[t] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_k + off) << 16);
-            }
-            tmem_st16(tmem + lrow + kColFK + g * 16, fk);
-        }
+        copy_pairs_to_tmem(sa + off_g, sa + off_k, tmem + kColFK, quarter, lane);
         tmem_wait_st();
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.empty[s]);

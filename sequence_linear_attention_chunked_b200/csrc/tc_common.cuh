@@ -69,6 +69,35 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// A chunk's 64 pairs (lo, hi) for each of this warp's 32 key dims, lo from the bf16 stage tile at
+// tile_lo and hi from the one at tile_hi (both [64 tokens][128 dims], tile_off layout), into
+// TMEM as one word lo | hi << 16 per (dim, token): lane = dim (the warp's quarter), column =
+// token from taddr's column.  ldmatrix with .trans gives thread l tokens 2(l%4) and 2(l%4)+1 of
+// dim l/4 in each 8x8 block, which is how the 16x256b store lays its registers out; the eight
+// row reads of one block fall on eight different 16-byte bank groups under the swizzle.
+__device__ __forceinline__ void copy_pairs_to_tmem(uint32_t tile_lo, uint32_t tile_hi,
+                                                   uint32_t taddr, int quarter, int lane) {
+    const int dim0 = quarter * 32 + (lane >> 3) * 8;  // block lane / 8: dims dim0 .. dim0 + 7
+    const int r = lane & 7;                           // the block row this lane addresses
+    const uint32_t row = (uint32_t)((dim0 >> 6) * kHalfBytes + r * 128 +
+                                    ((((dim0 & 63) >> 3) ^ r) << 4));
+#pragma unroll
+    for (int t0 = 0; t0 < CH; t0 += 8) {  // tokens t0 .. t0+7 (row t0 + r, and (t0 + r) % 8 = r)
+        uint32_t a[4], b[4];
+        ldsm_x4_trans(tile_lo + row + t0 * 128, a);
+        ldsm_x4_trans(tile_hi + row + t0 * 128, b);
+        uint32_t w[8];  // per block: the pair of token 2(l%4), then of token 2(l%4)+1
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            w[2 * m] = __byte_perm(a[m], b[m], 0x5410);
+            w[2 * m + 1] = __byte_perm(a[m], b[m], 0x7632);
+        }
+        const uint32_t ta = taddr + ((uint32_t)(quarter * 32) << 16) + (uint32_t)t0;
+        tmem_st_16x256b(ta, w[0], w[1], w[2], w[3]);                // dims +0 .. +15
+        tmem_st_16x256b(ta + (16u << 16), w[4], w[5], w[6], w[7]);  // dims +16 .. +31
+    }
+}
+
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {

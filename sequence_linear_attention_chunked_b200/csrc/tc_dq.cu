@@ -441,19 +441,10 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
         const int s = c % kStages;
         // (b) once the gates are done, this dim's 64 (F, q) pairs into its TMEM lane: the
         // stage is released before the read-out instead of after it
-        if (!mbar_wait(b[kGated + s], (c / kStages) & 1, abort)) break;
-        {
+        if (!warp_wait(b[kGated + s], (c / kStages) & 1, abort)) break;
+        {  // factor (low half) and q (high half), bf16
             const uint32_t sa = smem_u32(smem + s * kStageBytes);
-            uint32_t fq[16];  // factor (low half) and q (high half), bf16
-#pragma unroll 1
-            for (int g = 0; g < 4; ++g) {
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const uint32_t off = tile_off(g * 16 + t, i);
-                    fq[t] = lds_u16(sa + off_g + off) | (lds_u16(sa + off_q + off) << 16);
-                }
-                tmem_st16(tmem + lrow + kColFQ + g * 16, fq);
-            }
+            copy_pairs_to_tmem(sa + off_g, sa + off_q, tmem + kColFQ, quarter, lane);
             tmem_wait_st();
         }
         __syncwarp();
