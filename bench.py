@@ -36,6 +36,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ----------------------------------------------------------------------------- helpers
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of every rank's value: the job's device time is its slowest rank's."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, world: int, steps: int, job_ms: float) -> float:
+    """Units all ranks processed (each rank runs its own replica) per second of job time."""
+    return units_per_rank_step * world * steps / (job_ms / 1e3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -348,13 +361,8 @@ def bench_ours(args, rank, world, device):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    tokens_per_step = w.B * w.L
-    value = tokens_per_step * world * args.steps / (total_ms / 1e3)
+    total_ms = max_over_ranks(sum(step_ms), world, device)
+    value = job_throughput(w.B * w.L, world, args.steps, total_ms)
 
     # phases and the dominant kernel's roofline
     mean_phase = [statistics.fmean(p[i] for p in phase_ms) for i in range(len(step.phases))]
@@ -478,15 +486,13 @@ def bench_e2e(args, w, x, device, world):
     s_out.wait_event(ev_comp[(steps - 1) % 2])
     e1.record(s_out)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=device)
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+        dist.barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = sum(v.numel() * v.element_size() for v in bufs[0]["host_out"])
     api = "la_seg_forward" + (" + la_seg_backward" if w.backward else "")
-    return {"value": round(w.B * w.L * world * steps / (ms / 1e3), 1), "unit": "tokens/s",
+    return {"value": round(job_throughput(w.B * w.L, world, steps, ms), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "api": f"{api} (C ABI) with pinned host buffers, steps pipelined over copy-in, "
                    "compute and copy-out streams"}
