@@ -110,7 +110,11 @@ LA_API la_status la_seg_forward(const void *q, const void *k, const void *v, con
 
 /* Backward pass for loss = <o, dO> + <S_final, dS_final>.
  *  S_recv_saved    nullable: the forward's S_recv_save (reused, as the ZeCO review's "forward
- *                  implications" describe); when NULL the states are recomputed.
+ *                  implications" describe); when NULL the states are recomputed.  With saved
+ *                  states the dq sweep runs one CTA per saved segment.  The gradients do not
+ *                  depend on P, so a caller whose B*H*P leaves the GPU's last wave part-empty
+ *                  can pass P = la_seg_subsegments(...) to both calls: the sweep then runs on
+ *                  the library's own split.
  *  dS_final        nullable: zero.
  *  dq, dk_, dv_, dlog_g  outputs (dtype dt), fully overwritten.
  *  dS0             nullable: gradient with respect to S0, fp32 [B,H,dk,dv]. */

@@ -78,6 +78,23 @@ def test_reuse_matches_recompute(cuda_device):
             assert rel_err(g, r) <= 2e-2, (n, saved is None)
 
 
+def test_reuse_on_the_library_split(cuda_device):
+    """P = la_seg_subsegments(...) for both calls gives the same forward bit for bit and the
+    oracle's gradients: the segment count only picks which received states are saved."""
+    w = WORKLOADS["C1"].with_(H=4, L=8192, P=2, backward=True)
+    x = make_inputs(w, cuda_device)
+    NP = la_seg.la_seg_subsegments(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk)
+    assert NP > w.P
+    o1, Sf1, _ = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, w.P, w.chunk)
+    o2, Sf2, Sr = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, NP, w.chunk,
+                                        want_S_recv=True)
+    assert torch.equal(o1, o2) and torch.equal(Sf1, Sf2)
+    got = run_bwd(x, w.with_(P=NP), Sr)
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["log_g"], x["dO"])
+    for n, g, r in zip(NAMES, got, ref):
+        assert rel_err(g, r) <= 2e-2, n
+
+
 def test_backward_empty(cuda_device):
     w = Workload("empty", 1, 2, 0, 32, 32, 2, 16, "f32", "toy", backward=True)
     x = make_inputs(w, cuda_device, with_s0=True)
