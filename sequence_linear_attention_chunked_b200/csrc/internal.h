@@ -23,8 +23,8 @@ struct PassArgs {
     const void *q, *k, *v, *g;
     void *o;
     const float *S_init;  // [BH, NP, dk, dv] or null (zero)
-    float *S_out;         // [BH, NP, dk, dv] (kPassState / kPassLocal)
-    float *logG;          // [BH, NP, dk]    (kPassState / kPassLocal)
+    float *S_out;         // [BH, NP, dk, dv] (kPassState / kPassLocal; null: not written)
+    float *logG;          // [BH, NP, dk]    (kPassState / kPassLocal; null: not written)
     int *status;
     long long L, T;       // tokens per (b, h), tokens per sub-segment
     int BH, NP, dk, dv, chunk;

@@ -134,6 +134,36 @@ BwdLayout bwd_layout(const la::Split &s, int r, int dk, int dv) {
     return w;
 }
 
+// LA_SCHED_OVERLAP's second stream (highest priority, so that the scan's blocks are placed
+// beside the local pass's CTAs as SMs free up) and its fork / join events: one set per host
+// thread and device, created on first use and kept for the thread's lifetime.
+struct Aux {
+    int device = -1;
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+cudaError_t aux_streams(Aux **out) {
+    static thread_local Aux per_device[16];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
+    Aux &x = per_device[dev];
+    if (x.device != dev) {
+        int lo = 0, hi = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithPriority(&x.stream, cudaStreamNonBlocking, hi)) != cudaSuccess)
+            return e;
+        if ((e = cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming)) != cudaSuccess ||
+            (e = cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming)) != cudaSuccess)
+            return e;
+        x.device = dev;
+    }
+    *out = &x;
+    return cudaSuccess;
+}
+
 la::Split whole_segments(const la::Split &s) {
     la::Split w = s;
     w.m = 1;
@@ -235,9 +265,10 @@ la_status la_seg_local_pass(const void *q, const void *k, const void *v, const v
                             void *o, float *S_loc, float *log_gamma, int *status,
                             void *cuda_stream) {
     la_status st = check_pass(B, H, L, dk, dv, NP, chunk, dt,
-                              {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {o, "o"},
-                               {S_loc, "S_loc"}, {log_gamma, "log_gamma"}}, {});
+                              {{q, "q"}, {k, "k"}, {v, "v"}, {log_g, "log_g"}, {o, "o"}},
+                              {{S_loc, "S_loc"}, {log_gamma, "log_gamma"}});
     if (st != LA_OK) return st;
+    if (!S_loc != !log_gamma) return fail(LA_ERR_ARG, "S_loc and log_gamma go together");
     return run_pass(pass_args(q, k, v, log_g, o, nullptr, S_loc, log_gamma, status, B, H, L, dk, dv,
                               NP, chunk, dt),
                     la::kPassLocal, static_cast<cudaStream_t>(cuda_stream), "local pass");
@@ -351,7 +382,8 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     la_status st = check_shape(B, H, L, dk, dv, P, chunk, dt);
     if (st != LA_OK) return st;
     if (schedule != LA_SCHED_AUTO && schedule != LA_SCHED_TWO_PASS &&
-        schedule != LA_SCHED_THREE_PHASE && schedule != LA_SCHED_SINGLE_PASS)
+        schedule != LA_SCHED_THREE_PHASE && schedule != LA_SCHED_SINGLE_PASS &&
+        schedule != LA_SCHED_OVERLAP)
         return fail(LA_ERR_ARG, "unknown schedule %d", schedule);
     if (L > 0 && (!q || !k || !v || !log_g || !o))
         return fail(LA_ERR_ARG, "q, k, v, log_g and o must be non-null");
@@ -406,6 +438,38 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
 
     la::PassArgs a = pass_args(q, k, v, log_g, o, nullptr, S_loc, logG, status, B, H, L, dk, dv,
                                s.NP, chunk, dt);
+    if (schedule == LA_SCHED_OVERLAP) {
+        Aux *aux = nullptr;
+        if ((e = aux_streams(&aux)) != cudaSuccess) return cuda_fail(e, "second stream");
+        // 1. local states (state pass) on the caller's stream
+        if ((e = la::launch_pass(a, la::kPassState, stream)) != cudaSuccess)
+            return cuda_fail(e, "state pass");
+        // 2. fork: the scan on the second stream, the local outputs on the caller's
+        if ((e = cudaEventRecord(aux->fork, stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(aux->stream, aux->fork, 0)) != cudaSuccess)
+            return cuda_fail(e, "stream fork");
+        if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_final,
+                                 aux->stream)) != cudaSuccess)
+            return cuda_fail(e, "state scan");
+        if ((e = cudaEventRecord(aux->join, aux->stream)) != cudaSuccess)
+            return cuda_fail(e, "stream join");
+        la::PassArgs loc = a;
+        loc.S_out = nullptr;  // the state pass has them; the scan reads them meanwhile
+        loc.logG = nullptr;
+        if ((e = la::launch_pass(loc, la::kPassLocal, stream)) != cudaSuccess)
+            return cuda_fail(e, "local pass");
+        // 3. join, then the q . S_recv correction
+        if ((e = cudaStreamWaitEvent(stream, aux->join, 0)) != cudaSuccess)
+            return cuda_fail(e, "stream join");
+        a.S_init = S_recv;
+        if ((e = la::launch_pass(a, la::kPassCorrect, stream)) != cudaSuccess)
+            return cuda_fail(e, "correction pass");
+        if (S_recv_save &&
+            (e = la::launch_gather_states(S_recv, s.BH, s.NP, s.m, dk, dv, S_recv_save, stream)) !=
+                cudaSuccess)
+            return cuda_fail(e, "S_recv_save gather");
+        return LA_OK;
+    }
     const bool three = schedule == LA_SCHED_THREE_PHASE;
     // 1. per sub-segment: local state from zero (+ intra-chunk outputs for three-phase)
     if ((e = la::launch_pass(a, three ? la::kPassLocal : la::kPassState, stream)) != cudaSuccess)

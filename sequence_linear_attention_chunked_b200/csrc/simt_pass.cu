@@ -148,11 +148,11 @@ __global__ void __launch_bounds__(kThreads) simt_pass_kernel(PassArgs a) {
         }
     }
     __syncthreads();
-    if (kWritesState) {
+    if (kWritesState && a.S_out) {  // null: a local pass whose states are not wanted
         float *Sout = a.S_out + ((long long)bh * a.NP + j) * DK * DV;
         for (int idx = tid; idx < DK * DV; idx += kThreads) Sout[idx] = sS[idx];
-        if (tid < DK) a.logG[((long long)bh * a.NP + j) * DK + tid] = logG;
     }
+    if (kWritesState && a.logG && tid < DK) a.logG[((long long)bh * a.NP + j) * DK + tid] = logG;
     if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
 }
 

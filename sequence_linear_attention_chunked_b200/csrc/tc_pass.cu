@@ -69,7 +69,7 @@ struct Cfg {
     static constexpr int off_p = stages * stage_bytes;           // two bf16 P tiles
     static constexpr int off_ec = off_p + (qk ? 2 * CH * CH * 2 : 0);
     static constexpr int off_bar = off_ec + stages * D * 4;
-    static constexpr int n_bars = 5 * stages + 13;
+    static constexpr int n_bars = 5 * stages + 14;
     static constexpr int off_misc = off_bar + n_bars * 8;
     static constexpr int smem_bytes = off_misc + 16 + 1024;  // + slack to align the base to 1 KB
     static_assert(smem_bytes <= 232448, "shared memory budget");
@@ -81,6 +81,10 @@ struct Bars {
     uint64_t *full, *full_b, *gated, *empty;  // full: the gates' tiles; full_b: v
     uint64_t *ec_full;                        // e^{b_C} written (before the gates rescale)
     uint64_t *qk_full, *qk_free, *p_full, *ds_full, *sa_full, *sa_free, *o_full, *o_free, *fin;
+    // sa_full[c % 2]: S' of chunk c (and its bf16 copy c % 2) in place, 4 arrivals.  One per
+    // copy buffer: in the correction pass nothing holds a state warp back for a whole chunk
+    // (no state increment to wait for), and a warp one chunk ahead must not count towards the
+    // chunk the others are still writing.
 };
 
 // ------------------------------------------------------------------ TMA producer (1 thread)
@@ -167,7 +171,7 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
             }
             __syncwarp();
         } else {  // S' and its bf16 copy are in place
-            if (!(ok = warp_wait(b.sa_full, c & 1, abort))) break;
+            if (!(ok = warp_wait(&b.sa_full[c & 1], (c >> 1) & 1, abort))) break;
             tc_fence_after();
         }
         if (C::kv) {  // S^T = S'^T + V^T Ktil
@@ -358,7 +362,7 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.gated[s]);
     }
-    if (C::write_state && !*abort && tg == 0) {  // to shared memory (lg_full) or global
+    if (C::write_state && !*abort && tg == 0 && (lg_smem || a.logG)) {  // shared (lg_full) or global
         float4 *lg = reinterpret_cast<float4 *>(
             lg_smem ? lg_smem + i0 : a.logG + ((long long)bh * a.NP + j) * D + i0);
         lg[0] = make_float4(logG[0], logG[1], logG[2], logG[3]);
@@ -440,12 +444,12 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
         __syncwarp();
         if (lane == 0) {
             mbar_arrive(&b.empty[s]);
-            if (!C::dstate) mbar_arrive(b.sa_full);
+            if (!C::dstate) mbar_arrive(&b.sa_full[c & 1]);
         }
     }
     if (C::write_state && !*abort) {
         const uint32_t last = C::dstate ? 0u : (uint32_t)((nchunks - 1) & 1);
-        if (mbar_wait(b.ds_full, last, abort) && !(flags & kRoleStateKept)) {
+        if (mbar_wait(b.ds_full, last, abort) && !(flags & kRoleStateKept) && a.S_out) {
             tc_fence_after();
             float *So = a.S_out + ((long long)bh * a.NP + j) * D * D + dv;
 #pragma unroll
@@ -540,7 +544,7 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
 }
 
 // ------------------------------------------------------------------ the kernels
-// Barrier block of one pass: 5 per stage, then 13 (layout of Bars).
+// Barrier block of one pass: 5 per stage, then 14 (layout of Bars).
 __device__ Bars carve_bars(uint64_t *bar, int stages) {
     Bars b;
     b.full = bar;
@@ -550,7 +554,7 @@ __device__ Bars carve_bars(uint64_t *bar, int stages) {
     b.ec_full = bar + 4 * stages;
     uint64_t *x = bar + 5 * stages;
     b.qk_full = x + 0; b.qk_free = x + 1; b.p_full = x + 2; b.ds_full = x + 4; b.sa_full = x + 5;
-    b.sa_free = x + 6; b.o_full = x + 8; b.o_free = x + 10; b.fin = x + 12;
+    b.sa_free = x + 7; b.o_full = x + 9; b.o_free = x + 11; b.fin = x + 13;
     return b;
 }
 
@@ -565,8 +569,8 @@ __device__ void init_bars(const Bars &b, int stages) {
     mbar_init(b.qk_full, 1);
     mbar_init(b.qk_free, kOutWarps);
     mbar_init(b.ds_full, 1);
-    mbar_init(b.sa_full, kStateWarps);
     for (int i = 0; i < 2; ++i) {
+        mbar_init(&b.sa_full[i], kStateWarps);
         mbar_init(&b.p_full[i], kOutWarps);
         mbar_init(&b.sa_free[i], 1);
         mbar_init(&b.o_full[i], 1);

@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "LA_OK", -1: "LA_ERR_ARG", -2: "LA_ERR_SHAPE", -3: "LA_ERR_AL
                 -4: "LA_ERR_DTYPE", -5: "LA_ERR_WORKSPACE", -6: "LA_ERR_GATE_RANGE",
                 -7: "LA_ERR_TIMEOUT", -8: "LA_ERR_CUDA"}
 LA_F32, LA_BF16 = 0, 1
-SCHED_AUTO, SCHED_TWO_PASS, SCHED_THREE_PHASE, SCHED_SINGLE_PASS = 0, 1, 2, 3
+SCHED_AUTO, SCHED_TWO_PASS, SCHED_THREE_PHASE, SCHED_SINGLE_PASS, SCHED_OVERLAP = 0, 1, 2, 3, 4
 EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_seg_scan",
             "la_seg_state_pass", "la_seg_local_pass", "la_seg_output_pass", "la_seg_correct_pass",
             "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail",
@@ -265,13 +265,19 @@ def la_seg_state_pass(k, v, log_g, NP, chunk, *, S_loc=None, log_gamma=None, sta
 
 
 def la_seg_local_pass(q, k, v, log_g, NP, chunk, *, o=None, S_loc=None, log_gamma=None,
-                      status=None, stream=None):
+                      want_states=True, status=None, stream=None):
+    """Segment-local outputs; with want_states=False the local states are not written (and
+    S_loc, log_gamma come back as None)."""
     B, H, L, dk, dv = _seq_shapes(q, v)
     dev = q.device
     o = torch.empty((B, H, L, dv), dtype=q.dtype, device=dev) if o is None else o
-    S_loc = torch.empty((B, H, NP, dk, dv), dtype=torch.float32, device=dev) if S_loc is None else S_loc
-    log_gamma = (torch.empty((B, H, NP, dk), dtype=torch.float32, device=dev)
-                 if log_gamma is None else log_gamma)
+    if want_states:
+        S_loc = (torch.empty((B, H, NP, dk, dv), dtype=torch.float32, device=dev)
+                 if S_loc is None else S_loc)
+        log_gamma = (torch.empty((B, H, NP, dk), dtype=torch.float32, device=dev)
+                     if log_gamma is None else log_gamma)
+    else:
+        S_loc = log_gamma = None
     _check(lib().la_seg_local_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), B, H, L, dk, dv, NP,
                                    chunk, _dt(q), _ptr(o), _ptr(S_loc), _ptr(log_gamma),
                                    _ptr(status), _stream(stream)), "la_seg_local_pass")

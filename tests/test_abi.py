@@ -195,8 +195,20 @@ def test_chain_reset_rejects_bad_arguments(lib):
     assert reset(V(0x7004), 1, 2, 128, 128, V(0x8000), V(0x9000), None) == -3
 
 
-def test_single_pass_schedule_is_accepted(lib):
-    # an unknown schedule is rejected, the single pass is not (the call then stops at the
-    # workspace check, before any launch)
-    assert _fwd(lib, sched=4) == -1
+def test_single_pass_and_overlap_schedules_are_accepted(lib):
+    # an unknown schedule is rejected, the single pass and the overlap schedule are not (the
+    # call then stops at the workspace check, before any launch)
+    assert _fwd(lib, sched=5) == -1
+    assert _fwd(lib, sched=-1) == -1
     assert _fwd(lib, sched=la_seg.SCHED_SINGLE_PASS, ws=None) == -5
+    assert _fwd(lib, sched=la_seg.SCHED_OVERLAP, ws=None) == -5
+
+
+def test_local_pass_states_go_together(lib):
+    # S_loc without log_gamma (or the reverse) is an argument error, found before any launch
+    V, L_ = ctypes.c_void_p, ctypes.c_longlong
+    f = lib.la_seg_local_pass
+    for sl, lgm in ((0x6000, None), (None, 0x7000)):
+        st = f(V(0x1000), V(0x2000), V(0x3000), V(0x4000), 1, 1, L_(64), 32, 32, 1, 16, 0,
+               V(0x5000), V(sl) if sl else None, V(lgm) if lgm else None, None, None)
+        assert st == -1

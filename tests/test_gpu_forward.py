@@ -10,7 +10,7 @@ from tests.parity import TOL, oracle_window, rel_err
 
 pytestmark = pytest.mark.gpu
 
-SCHEDULES = [la_seg.SCHED_TWO_PASS, la_seg.SCHED_THREE_PHASE]
+SCHEDULES = [la_seg.SCHED_TWO_PASS, la_seg.SCHED_THREE_PHASE, la_seg.SCHED_OVERLAP]
 
 
 def run(x, w, schedule=la_seg.SCHED_AUTO, want_recv=True):
@@ -98,6 +98,26 @@ def test_schedules_agree(cuda_device):
     b = run(x, w, la_seg.SCHED_THREE_PHASE)
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])  # same state path
     assert rel_err(a[0], b[0].double().cpu().numpy()) <= 2e-2
+    c = run(x, w, la_seg.SCHED_OVERLAP)  # three-phase with the scan on a second stream
+    for u, v in zip(b, c):
+        assert torch.equal(u, v)
+
+
+def test_overlap_on_a_user_stream(cuda_device):
+    """The overlap schedule forks from and joins back into the caller's stream: launched on a
+    side stream, repeatedly, it matches the three-phase result."""
+    w = WORKLOADS["C1"].with_(H=4, L=8192, P=2)
+    x = make_inputs(w, cuda_device)
+    ref = run(x, w, la_seg.SCHED_THREE_PHASE)
+    side = torch.cuda.Stream(device=cuda_device)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        outs = [run(x, w, la_seg.SCHED_OVERLAP) for _ in range(3)]
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    for got in outs:
+        for u, v in zip(ref, got):
+            assert torch.equal(u, v)
 
 
 def test_gate_range_flagged(cuda_device):
@@ -134,17 +154,51 @@ def test_c1_full(cuda_device):
 
 @pytest.mark.parametrize("name", ["C2", "C3"])
 def test_large_sampled(cuda_device, name):
-    """C2 / C3 at full size: sampled windows (including segment starts) against the oracle."""
+    """C2 / C3 at full size: sampled windows (including segment starts) against the oracle.  At
+    C2 the three-phase and overlap schedules are checked on the same windows too (64
+    sub-segments of 32 chunks: the correction pass at scale)."""
     w = WORKLOADS[name]
     x = make_inputs(w, cuda_device)
-    o, Sf, _ = run(x, w, want_recv=False)
+    scheds = [la_seg.SCHED_AUTO]
+    if name == "C2":
+        scheds += [la_seg.SCHED_THREE_PHASE, la_seg.SCHED_OVERLAP]
+    outs = [run(x, w, sc, want_recv=False)[0] for sc in scheds]
     T = w.L // w.P
     rng = np.random.default_rng(7)
     for h in (0, w.H - 1):
         for p in (0, 1, w.P - 1, int(rng.integers(1, w.P))):
             for t0 in (p * T, p * T + int(rng.integers(0, T - 512)) // 64 * 64):
                 ref = oracle_window(x, 0, h, t0, t0 + 512)
-                got = o[0, h, t0:t0 + 512]
-                assert rel_err(got, ref) <= 2e-2, (name, h, p, t0)
-    del x, o
+                for sc, o in zip(scheds, outs):
+                    assert rel_err(o[0, h, t0:t0 + 512], ref) <= 2e-2, (name, sc, h, p, t0)
+    del x, outs
+    torch.cuda.empty_cache()
+
+
+def test_correction_pass_exact_at_scale(cuda_device):
+    """The correction pass over C2's 64 sub-segments of 32 chunks: the term of zero received
+    states leaves o bit for bit, repeated corrections agree bit for bit, and so do repeated
+    three-phase and overlap forwards."""
+    w = WORKLOADS["C2"]
+    x = make_inputs(w, cuda_device)
+    NP = la_seg.la_seg_subsegments(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk)
+    o_loc, S_loc, lg = la_seg.la_seg_local_pass(x["q"], x["k"], x["v"], x["log_g"], NP, w.chunk)
+    Sr, _ = la_seg.la_seg_scan(S_loc.view(-1, NP, w.dk, w.dv), lg.view(-1, NP, w.dk))
+    Sr = Sr.view(w.B, w.H, NP, w.dk, w.dv)
+    oz = o_loc.clone()
+    la_seg.la_seg_correct_pass(x["q"], x["log_g"], torch.zeros_like(Sr), NP, w.chunk, oz)
+    assert torch.equal(oz, o_loc)
+    first = None
+    for _ in range(3):
+        oc = o_loc.clone()
+        la_seg.la_seg_correct_pass(x["q"], x["log_g"], Sr, NP, w.chunk, oc)
+        if first is None:
+            first = oc
+        assert torch.equal(oc, first)
+    for sc in (la_seg.SCHED_THREE_PHASE, la_seg.SCHED_OVERLAP):
+        a = run(x, w, sc, want_recv=False)[0]
+        b = run(x, w, sc, want_recv=False)[0]
+        assert torch.equal(a, b), sc
+        assert torch.equal(a, first), sc
+    del x
     torch.cuda.empty_cache()
