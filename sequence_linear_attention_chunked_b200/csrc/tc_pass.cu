@@ -60,10 +60,14 @@ struct Cfg {
     static constexpr bool out = MODE != kPassState && !dstate;
     static constexpr bool write_state = MODE == kPassState || MODE == kPassLocal || dstate;
     static constexpr bool init_state = MODE == kPassOutput || MODE == kPassCorrect;
+    // the correction pass reads the local outputs o through the ring (in the k slot, on the
+    // second barrier), so the output warps find them on chip and release the stage after them
+    static constexpr bool ol = MODE == kPassCorrect;
     static constexpr int stages = (MODE == kPassOutput || MODE == kPassLocal) ? 3 : 4;
     static constexpr int off_q = 0;
-    static constexpr int off_k = off_q + (q ? kTileBytes : 0);
-    static constexpr int off_v = off_k + (k ? kTileBytes : 0);
+    static constexpr int off_k = off_q + (q ? kTileBytes : 0);  // k, or o in the correction pass
+    static constexpr int off_v = off_k + ((k || ol) ? kTileBytes : 0);
+    static constexpr int empty_count = 1 + kStateWarps + (ol ? kOutWarps : 0);
     static constexpr int off_g = off_v + (v ? kTileBytes : 0);
     static constexpr int stage_bytes = off_g + kTileBytes;
     static constexpr int off_p = stages * stage_bytes;           // two bf16 P tiles
@@ -105,18 +109,19 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
         };
         // the gates' tiles first, on their own barrier (the gates start as soon as they land);
         // v, read only by the tensor cores, behind them
-        mbar_arrive_expect_tx(&b.full[s], C::stage_bytes - (C::v ? kTileBytes : 0));
-        if (C::v) mbar_arrive_expect_tx(&b.full_b[s], kTileBytes);
+        mbar_arrive_expect_tx(&b.full[s], C::stage_bytes - ((C::v || C::ol) ? kTileBytes : 0));
+        if (C::v || C::ol) mbar_arrive_expect_tx(&b.full_b[s], kTileBytes);
         load(C::off_g, tg, &b.full[s]);
         if (C::q) load(C::off_q, tq, &b.full[s]);
         if (C::k) load(C::off_k, tk, &b.full[s]);
         if (C::v) load(C::off_v, tv, &b.full_b[s]);
+        if (C::ol) load(C::off_k, tk, &b.full_b[s]);  // the local outputs (tk maps o here)
         issued = c + 1;
     }
     if (*abort)  // let every copy this CTA started land before it exits
         for (int c = issued > C::stages ? issued - C::stages : 0; c < issued; ++c) {
             wait_drain(&b.full[c % C::stages], (c / C::stages) & 1);
-            if (C::v) wait_drain(&b.full_b[c % C::stages], (c / C::stages) & 1);
+            if (C::v || C::ol) wait_drain(&b.full_b[c % C::stages], (c / C::stages) & 1);
         }
 }
 
@@ -519,6 +524,7 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
         // (d) outputs: column dv of the chunk's 64 rows
         const int ob = c & 1;
         if (!mbar_wait(&b.o_full[ob], (c >> 1) & 1, abort)) break;
+        if (C::ol && !mbar_wait(&b.full_b[c % C::stages], (c / C::stages) & 1, abort)) break;
         tc_fence_after();
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -530,15 +536,19 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                 if (lane == 0) mbar_arrive(&b.o_free[ob]);
             }
             __nv_bfloat16 *orow = o + (row0 + (long long)c * CH + h * 32) * D + dv;
-            if (MODE == kPassCorrect) {  // o_local: all loads before the first store
-                float ol[32];
+            if (C::ol) {  // o_local of these 32 rows, from the stage
+                const uint32_t ot = smem_u32(smem + (c % C::stages) * C::stage_bytes + C::off_k);
 #pragma unroll
-                for (int t = 0; t < 32; ++t) ol[t] = __bfloat162float(orow[t * D]);
-#pragma unroll
-                for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(__uint_as_float(r[t]) + ol[t]);
+                for (int t = 0; t < 32; ++t)
+                    r[t] = __float_as_uint(__uint_as_float(r[t]) +
+                                           __uint_as_float(lds_u16(ot + tile_off(h * 32 + t, dv)) << 16));
             }
 #pragma unroll
             for (int t = 0; t < 32; ++t) orow[t * D] = __float2bfloat16_rn(__uint_as_float(r[t]));
+        }
+        if (C::ol) {  // this warp's reads of the stage are done
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&b.empty[c % C::stages]);
         }
     }
 }
@@ -558,13 +568,13 @@ __device__ Bars carve_bars(uint64_t *bar, int stages) {
     return b;
 }
 
-__device__ void init_bars(const Bars &b, int stages) {
+__device__ void init_bars(const Bars &b, int stages, int empty_count) {
     for (int s = 0; s < stages; ++s) {
         mbar_init(&b.full[s], 1);
         mbar_init(&b.full_b[s], 1);
         mbar_init(&b.ec_full[s], kGateWarps);
         mbar_init(&b.gated[s], kGateWarps);
-        mbar_init(&b.empty[s], 1 + kStateWarps);
+        mbar_init(&b.empty[s], empty_count);
     }
     mbar_init(b.qk_full, 1);
     mbar_init(b.qk_free, kOutWarps);
@@ -598,7 +608,7 @@ tc_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int nchunks = (int)(a.T / CH);
 
     if (threadIdx.x == 0) {
-        init_bars(b, C::stages);
+        init_bars(b, C::stages, C::empty_count);
         *abort = 0;
         mbar_fence_init();
     }
@@ -749,8 +759,8 @@ tc_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        init_bars(ba, CA::stages);
-        init_bars(bb, CB::stages);
+        init_bars(ba, CA::stages, CA::empty_count);
+        init_bars(bb, CB::stages, CB::empty_count);
         mbar_init(lg_full, kGateWarps);
         *abort = 0;
         *ticket = atomicAdd(ch.ready + a.BH, 1);
@@ -815,7 +825,8 @@ cudaError_t launch_mode(const PassArgs &a, cudaStream_t st) {
     if (rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
     CUtensorMap mq, mk, mv, mg;
     cudaError_t e;
-    const void *qp = C::q ? a.q : a.g, *kp = C::k ? a.k : a.g, *vp = C::v ? a.v : a.g;
+    const void *qp = C::q ? a.q : a.g, *vp = C::v ? a.v : a.g;
+    const void *kp = C::k ? a.k : (C::ol ? a.o : a.g);
     if ((e = make_map(&mq, qp, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mk, kp, rows)) != cudaSuccess) return e;
     if ((e = make_map(&mv, vp, rows)) != cudaSuccess) return e;
