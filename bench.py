@@ -229,7 +229,8 @@ class Step:
             la._check(la.lib().la_seg_scan(la._ptr(self.S_loc), la._ptr(self.logG), None, BH, NP,
                                            w.dk, w.dv, 0, la._ptr(self.S_recv),
                                            la._ptr(self.S_final), None, None, None,
-                                           la._stream(self.side)), "la_seg_scan")
+                                           la._ptr(self.status), la._stream(self.side)),
+                      "la_seg_scan")
             if record:
                 self.scan_ev[1].record(self.side)
             self.join.record(self.side)
@@ -259,7 +260,7 @@ class Step:
             la._check(la.lib().la_seg_scan(la._ptr(self.S_loc), la._ptr(self.logG), None, BH, NP,
                                            w.dk, w.dv, 0, la._ptr(self.S_recv),
                                            la._ptr(self.S_final), None, None, None,
-                                           la._stream(None)), "la_seg_scan")
+                                           la._ptr(self.status), la._stream(None)), "la_seg_scan")
             rec(2)
             if self.schedule != "three":
                 la.la_seg_output_pass(x["q"], x["k"], x["v"], x["log_g"], self.S_recv, NP,
@@ -279,7 +280,7 @@ class Step:
         la._check(la.lib().la_seg_scan(la._ptr(self.dSloc), la._ptr(self.logG_b), None, BH, NPF,
                                        w.dk, w.dv, 1, la._ptr(self.dX), la._ptr(self.dS0),
                                        la._ptr(self.S_fine), None, la._ptr(self.carry),
-                                       la._stream(None)), "la_seg_scan")
+                                       la._ptr(self.status), la._stream(None)), "la_seg_scan")
         rec(f + 2)
         la.la_seg_dkv_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_fine, None, self.dX,
                            self.qdq, NPF, w.chunk, carry=self.carry, out=self.grads[1:],

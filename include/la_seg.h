@@ -145,10 +145,14 @@ LA_API la_status la_seg_backward(const void *q, const void *k, const void *v, co
  *  with S_end_p = S_next[p+1] for p < NP-1 and S_last for p = NP-1 (S_next fp32
  *  [BH, NP, dk, dv], required with carry; S_last fp32 [BH, dk, dv], nullable: zero) -- for the
  *  backward's reverse scan, the dlog_g carry rowsum(S_end . dX) of every part, which
- *  la_seg_dkv_pass then takes instead of forming it.  Needs dv / 4 to divide 32. */
+ *  la_seg_dkv_pass then takes instead of forming it.  Needs dv / 4 to divide 32.
+ *  status (nullable device int): without a carry, and for states of whole 1024-float slices
+ *  with dk % 4 == 0 and a 16-byte aligned log_gamma, the scan streams the states through
+ *  shared memory by bulk copies and ORs 2 (LA_ERR_TIMEOUT, see la_seg_check_status) into
+ *  *status if one of its bounded waits gives up. */
 LA_API la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
                       int NP, int dk, int dv, int reverse, float *out, float *final_state,
-                      const float *S_next, const float *S_last, float *carry,
+                      const float *S_next, const float *S_last, float *carry, int *status,
                       void *cuda_stream);
 
 /* ---- The steps of the path, one entry point each -------------------------------------

@@ -102,11 +102,14 @@ cudaError_t launch_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
 // Exclusive decayed scan over NP sub-segments (see la_seg_scan in la_seg.h).  With `carry`
 // (fp32 [BH, NP, dk]) it also writes the reverse sweep's dlog_g carry of every part p,
 // rowsum(S_end_p . out[p]), S_end_p = S_next[p+1] for p < NP-1 and S_last (nullable: zero) for
-// the last part.
+// the last part.  Without a carry (and for d_k x d_v states of whole 1024-float slices) the
+// scan streams the states by bulk copies; a wait there that gives up sets kStatusTimeout in
+// *status (nullable).
 cudaError_t launch_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
                         int NP, int dk, int dv, int reverse, float *out, float *final_state,
                         cudaStream_t st, const float *S_next = nullptr,
-                        const float *S_last = nullptr, float *carry = nullptr);
+                        const float *S_last = nullptr, float *carry = nullptr,
+                        int *status = nullptr);
 
 // Copies the per-sub-segment states at API-segment boundaries: dst[bh][p] = src[bh][p*m].
 cudaError_t launch_gather_states(const float *src, int BH, int NP, int m, int dk, int dv,

@@ -449,7 +449,7 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
             (e = cudaStreamWaitEvent(aux->stream, aux->fork, 0)) != cudaSuccess)
             return cuda_fail(e, "stream fork");
         if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_final,
-                                 aux->stream)) != cudaSuccess)
+                                 aux->stream, nullptr, nullptr, nullptr, status)) != cudaSuccess)
             return cuda_fail(e, "state scan");
         if ((e = cudaEventRecord(aux->join, aux->stream)) != cudaSuccess)
             return cuda_fail(e, "stream join");
@@ -475,7 +475,8 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     if ((e = la::launch_pass(a, three ? la::kPassLocal : la::kPassState, stream)) != cudaSuccess)
         return cuda_fail(e, three ? "local pass" : "state pass");
     // 2. exclusive decayed scan across sub-segments
-    if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_final, stream)) !=
+    if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_final, stream,
+                             nullptr, nullptr, nullptr, status)) !=
         cudaSuccess)
         return cuda_fail(e, "state scan");
     // 3. outputs from the received states (two-pass) or the q . S_recv correction (three-phase)
@@ -583,7 +584,8 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
                                    H, L, dk, dv, s.NP, chunk, dt);
         if ((e = la::launch_pass(a, la::kPassState, stream)) != cudaSuccess)
             return cuda_fail(e, "backward state pass");
-        if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_fin, stream)) !=
+        if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_fin, stream,
+                                 nullptr, nullptr, nullptr, status)) !=
             cudaSuccess)
             return cuda_fail(e, "backward state scan");
     }
@@ -612,7 +614,7 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
 
 la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
                       int NP, int dk, int dv, int reverse, float *out, float *final_state,
-                      const float *S_next, const float *S_last, float *carry,
+                      const float *S_next, const float *S_last, float *carry, int *status,
                       void *cuda_stream) {
     if (BH < 0 || NP < 0 || dk < 1 || dv < 4 || dv % 4)
         return fail(LA_ERR_SHAPE, "need BH, NP >= 0, dk >= 1, dv a positive multiple of 4");
@@ -637,7 +639,7 @@ la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *in
     }
     cudaError_t e = la::launch_scan(S_in, log_gamma, init, BH, NP, dk, dv, reverse, out,
                                     final_state, static_cast<cudaStream_t>(cuda_stream), S_next,
-                                    S_last, carry);
+                                    S_last, carry, status);
     return e == cudaSuccess ? LA_OK : cuda_fail(e, "scan");
 }
 

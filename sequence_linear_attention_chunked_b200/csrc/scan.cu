@@ -12,9 +12,12 @@
 // element's chain is the same whatever the block split.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace la {
 namespace {
+
+using namespace sm100;
 
 // 128-thread blocks and a 4-deep batch for the carry variant keep it at one wave of blocks
 // (the C4 reverse scan is 1024 blocks, 7 per SM), which 256-thread blocks at its register count
@@ -84,6 +87,109 @@ scan_kernel(const float4 *__restrict__ S_in, const float *__restrict__ log_gamma
     if (final_state) final_state[bh * per_bh + ij] = acc;
 }
 
+// ---- the forward form (no carry), fed by bulk copies ----------------------------------------
+// One CTA per (bh, slice of kSlice consecutive floats of the dk x dv state).  A producer thread
+// streams each segment's slice and the log-decays of the slice's rows into a kSliceStages-deep
+// ring of shared memory with bulk copies: the copy engine keeps the bytes of many segments in
+// flight, where per-thread loads capped a 16-head scan at about half the bandwidth a plain
+// copy reaches.  Thread t of the 128 carries elements 8t .. 8t+7 of the slice (one row, since
+// dv >= 32) through the recurrence and stores out[p] straight to HBM.  12 stages (51 KiB)
+// keep four CTAs per SM resident, so a 32-head grid of 512 CTAs is a single wave.
+constexpr int kSlice = 1024, kSliceStages = 12, kSliceThreads = 128;
+constexpr int kSliceBytes = kSlice * 4, kLgBytes = 128;  // a slice has kSlice / dv <= 32 rows
+constexpr int kSliceStage = kSliceBytes + kLgBytes;
+constexpr int kSliceSmem = kSliceStages * kSliceStage + 2 * kSliceStages * 8 + 16;
+
+__device__ __forceinline__ float4 vfma4(float g, const float4 &a, const float4 &x) {
+    return make_float4(fmaf(g, a.x, x.x), fmaf(g, a.y, x.y), fmaf(g, a.z, x.z), fmaf(g, a.w, x.w));
+}
+
+__global__ void __launch_bounds__(kSliceThreads + 32)
+scan_bulk_kernel(const float *__restrict__ S_in, const float *__restrict__ log_gamma,
+                 const float *__restrict__ init, int NP, int dk, int dv, int reverse,
+                 float *__restrict__ out, float *__restrict__ final_state, int *status) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + kSliceStages * kSliceStage);
+    uint64_t *empty = full + kSliceStages;
+    volatile int *abort = reinterpret_cast<volatile int *>(empty + kSliceStages);
+    const int nsl = dk * dv / kSlice;
+    const long long bh = blockIdx.x / nsl;
+    const int sl = blockIdx.x % nsl;
+    const int rows = kSlice / dv, row0 = sl * rows;
+    const long long state = (long long)dk * dv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSliceStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kSliceThreads / 32);
+        }
+        *abort = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (warp == kSliceThreads / 32) {  // the producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int p = 0; p < NP; ++p) {
+                const int s = p % kSliceStages;
+                if (p >= kSliceStages &&
+                    !mbar_wait(&empty[s], ((p / kSliceStages) - 1) & 1, abort))
+                    break;
+                const long long pp = reverse ? NP - 1 - p : p;
+                uint8_t *st = sm + s * kSliceStage;
+                mbar_arrive_expect_tx(&full[s], kSliceBytes + rows * 4);
+                bulk_load(st, S_in + (bh * NP + pp) * state + (long long)sl * kSlice, kSliceBytes,
+                          &full[s]);
+                bulk_load(st + kSliceBytes, log_gamma + (bh * NP + pp) * dk + row0, rows * 4,
+                          &full[s]);
+                issued = p + 1;
+            }
+            if (*abort) {  // let the copies this CTA started land before it exits
+                int ignore = 0;
+                for (int p = issued > kSliceStages ? issued - kSliceStages : 0; p < issued; ++p)
+                    mbar_wait(&full[p % kSliceStages], (p / kSliceStages) & 1, &ignore);
+            }
+        }
+        return;
+    }
+    const int e0 = threadIdx.x * 8;
+    const int r = e0 / dv;
+    const long long gofs = (long long)sl * kSlice + e0;
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    if (init) {
+        const float4 *ip = reinterpret_cast<const float4 *>(init + bh * state + gofs);
+        a0 = ip[0];
+        a1 = ip[1];
+    }
+    bool ok = true;
+    for (int p = 0; p < NP; ++p) {
+        const int s = p % kSliceStages;
+        if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (p / kSliceStages) & 1, abort))))
+            break;
+        const long long pp = reverse ? NP - 1 - p : p;
+        const uint8_t *st = sm + s * kSliceStage;
+        const float4 x0 = *reinterpret_cast<const float4 *>(st + e0 * 4);
+        const float4 x1 = *reinterpret_cast<const float4 *>(st + e0 * 4 + 16);
+        const float g = __expf(*reinterpret_cast<const float *>(st + kSliceBytes + r * 4));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // this warp's reads of the stage are done
+        float4 *op = reinterpret_cast<float4 *>(out + (bh * NP + pp) * state + gofs);
+        __stcs(op, a0);
+        __stcs(op + 1, a1);
+        a0 = vfma4(g, a0, x0);
+        a1 = vfma4(g, a1, x1);
+    }
+    if (!ok) {
+        if (status && lane == 0) atomicOr(status, kStatusTimeout);
+        return;
+    }
+    if (final_state) {
+        float4 *fp = reinterpret_cast<float4 *>(final_state + bh * state + gofs);
+        fp[0] = a0;
+        fp[1] = a1;
+    }
+}
+
 __global__ void gather_states_kernel(const float4 *__restrict__ src, int BH, int NP, int m,
                                      long long per_state4, float4 *__restrict__ dst) {
     const int P = NP / m;
@@ -107,7 +213,23 @@ __global__ void copy_state_kernel(const float4 *__restrict__ src, long long n4,
 
 cudaError_t launch_scan(const float *S_in, const float *log_gamma, const float *init, int BH,
                         int NP, int dk, int dv, int reverse, float *out, float *final_state,
-                        cudaStream_t st, const float *S_next, const float *S_last, float *carry) {
+                        cudaStream_t st, const float *S_next, const float *S_last, float *carry,
+                        int *status) {
+    if (!carry && dk % 4 == 0 && (dk * dv) % kSlice == 0 && kSlice % dv == 0 &&
+        kSlice / dv * 4 <= kLgBytes && reinterpret_cast<uintptr_t>(log_gamma) % 16 == 0) {
+        const long long nblk = (long long)BH * (dk * dv / kSlice);
+        if (nblk == 0 || NP == 0) {
+            if (NP == 0 && final_state && BH > 0)  // no segments: the final state is the start
+                return launch_copy_state(init, BH, dk, dv, final_state, st);
+            return cudaSuccess;
+        }
+        cudaError_t e = cudaFuncSetAttribute(scan_bulk_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSliceSmem);
+        if (e != cudaSuccess) return e;
+        scan_bulk_kernel<<<(unsigned)nblk, kSliceThreads + 32, kSliceSmem, st>>>(
+            S_in, log_gamma, init, NP, dk, dv, reverse, out, final_state, status);
+        return cudaGetLastError();
+    }
     if (carry && (dv % 4 || 32 % (dv / 4) || (dk * (dv / 4)) % 32)) return cudaErrorInvalidValue;
     const int dv4 = dv / 4;
     const long long n = (long long)BH * dk * dv4;

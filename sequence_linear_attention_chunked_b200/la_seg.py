@@ -54,7 +54,7 @@ def lib():
         L.la_seg_backward.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
                                       i32, P, P, P, P, P, P, sz, P]
         L.la_seg_backward.restype = i32
-        L.la_seg_scan.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
+        L.la_seg_scan.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P, P]
         L.la_seg_scan.restype = i32
         L.la_seg_state_pass.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P, P, P]
         L.la_seg_state_pass.restype = i32
@@ -209,7 +209,7 @@ def la_seg_backward(q, k, v, log_g, dO, S0=None, S_recv_saved=None, dS_final=Non
 
 
 def la_seg_scan(S_in, log_gamma, init=None, reverse=False, *, want_final=True, S_next=None,
-                S_last=None, out=None, final=None, carry=None, stream=None):
+                S_last=None, out=None, final=None, carry=None, status=None, stream=None):
     """out, final = exclusive decayed scan over dim 1 of S_in [BH, NP, dk, dv] (fp32).
 
     With S_next (and optionally S_last) a carry tensor fp32 [BH, NP, dk] is filled too (given,
@@ -229,7 +229,8 @@ def la_seg_scan(S_in, log_gamma, init=None, reverse=False, *, want_final=True, S
         carry = torch.empty((BH, NP, dk), dtype=torch.float32, device=dev)
     st = lib().la_seg_scan(_ptr(S_in), _ptr(log_gamma), _ptr(init), BH, NP, dk, dv,
                            int(bool(reverse)), _ptr(out), _ptr(final), _ptr(S_next),
-                           _ptr(S_last), _ptr(carry if want_carry else None), _stream(stream))
+                           _ptr(S_last), _ptr(carry if want_carry else None), _ptr(status),
+                           _stream(stream))
     _check(st, "la_seg_scan")
     return (out, final, carry) if want_carry else (out, final)
 

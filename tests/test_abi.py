@@ -94,7 +94,7 @@ def _scan(lib, S_in=0x1000, lg=0x2000, d=32, dv=None, out=0x3000, S_next=None, S
     """la_seg_scan with fake (but aligned) pointers: only argument checks may run."""
     V = ctypes.c_void_p
     return lib.la_seg_scan(V(S_in), V(lg), None, 1, 2, d, d if dv is None else dv, 0, V(out),
-                           None, V(S_next), V(S_last), V(carry), None)
+                           None, V(S_next), V(S_last), V(carry), None, None)
 
 
 def test_scan_rejects_bad_arguments(lib):
