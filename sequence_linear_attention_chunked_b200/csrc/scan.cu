@@ -87,31 +87,47 @@ scan_kernel(const float4 *__restrict__ S_in, const float *__restrict__ log_gamma
     if (final_state) final_state[bh * per_bh + ij] = acc;
 }
 
-// ---- the forward form (no carry), fed by bulk copies ----------------------------------------
+// ---- the scan fed by bulk copies ------------------------------------------------------------
 // One CTA per (bh, slice of kSlice consecutive floats of the dk x dv state).  A producer thread
-// streams each segment's slice and the log-decays of the slice's rows into a kSliceStages-deep
-// ring of shared memory with bulk copies: the copy engine keeps the bytes of many segments in
-// flight, where per-thread loads capped a 16-head scan at about half the bandwidth a plain
-// copy reaches.  Thread t of the 128 carries elements 8t .. 8t+7 of the slice (one row, since
-// dv >= 32) through the recurrence and stores out[p] straight to HBM.  12 stages (51 KiB)
-// keep four CTAs per SM resident, so a 32-head grid of 512 CTAs is a single wave.
-constexpr int kSlice = 1024, kSliceStages = 12, kSliceThreads = 128;
+// streams each segment's slice and the log-decays of the slice's rows (and, for the carry, the
+// matching slice of the segment's end state) into a ring of shared memory with bulk copies: the
+// copy engine keeps the bytes of many segments in flight, where per-thread loads capped a
+// 16-head scan at about half the bandwidth a plain copy reaches.  Thread t of the 128 carries
+// elements 8t .. 8t+7 of the slice (one row, since dv >= 32) through the recurrence and stores
+// out[p] straight to HBM.  12 stages (6 with the end states) keep four CTAs per SM resident, so
+// a 32-head grid of 512 CTAs is a single wave.
+constexpr int kSlice = 1024, kSliceThreads = 128;
 constexpr int kSliceBytes = kSlice * 4, kLgBytes = 128;  // a slice has kSlice / dv <= 32 rows
-constexpr int kSliceStage = kSliceBytes + kLgBytes;
-constexpr int kSliceSmem = kSliceStages * kSliceStage + 2 * kSliceStages * 8 + 16;
+
+template <bool CARRY> struct SliceRing {
+    static constexpr int stages = CARRY ? 6 : 12;
+    static constexpr int off_end = kSliceBytes;                       // end-state slice (carry)
+    static constexpr int off_lg = kSliceBytes * (CARRY ? 2 : 1);
+    static constexpr int stage = off_lg + kLgBytes;
+    static constexpr int smem = stages * stage + 2 * stages * 8 + 16;
+};
 
 __device__ __forceinline__ float4 vfma4(float g, const float4 &a, const float4 &x) {
     return make_float4(fmaf(g, a.x, x.x), fmaf(g, a.y, x.y), fmaf(g, a.z, x.z), fmaf(g, a.w, x.w));
 }
 
+// With CARRY (the backward's reverse scan): carry[bh][p][i] = sum_j S_end_p[i][j] out[p][i][j],
+// S_end_p = S_next[p+1] (p < NP-1) or S_last (p = NP-1; null: zero), summed in the order of the
+// per-thread kernel: a 4-term fma chain per group of 4 columns, then a pairwise tree over the
+// row's groups (the thread's two groups first, then across the dv / 8 lanes of the row), which
+// la_seg_dkv_pass reproduces when it forms the carry itself.
+template <bool CARRY>
 __global__ void __launch_bounds__(kSliceThreads + 32)
 scan_bulk_kernel(const float *__restrict__ S_in, const float *__restrict__ log_gamma,
                  const float *__restrict__ init, int NP, int dk, int dv, int reverse,
-                 float *__restrict__ out, float *__restrict__ final_state, int *status) {
+                 float *__restrict__ out, float *__restrict__ final_state,
+                 const float *__restrict__ S_next, const float *__restrict__ S_last,
+                 float *__restrict__ carry, int *status) {
+    using R = SliceRing<CARRY>;
     extern __shared__ __align__(128) uint8_t sm[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + kSliceStages * kSliceStage);
-    uint64_t *empty = full + kSliceStages;
-    volatile int *abort = reinterpret_cast<volatile int *>(empty + kSliceStages);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + R::stages * R::stage);
+    uint64_t *empty = full + R::stages;
+    volatile int *abort = reinterpret_cast<volatile int *>(empty + R::stages);
     const int nsl = dk * dv / kSlice;
     const long long bh = blockIdx.x / nsl;
     const int sl = blockIdx.x % nsl;
@@ -119,7 +135,7 @@ scan_bulk_kernel(const float *__restrict__ S_in, const float *__restrict__ log_g
     const long long state = (long long)dk * dv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kSliceStages; ++s) {
+        for (int s = 0; s < R::stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kSliceThreads / 32);
         }
@@ -131,23 +147,27 @@ scan_bulk_kernel(const float *__restrict__ S_in, const float *__restrict__ log_g
         if (lane == 0) {
             int issued = 0;
             for (int p = 0; p < NP; ++p) {
-                const int s = p % kSliceStages;
-                if (p >= kSliceStages &&
-                    !mbar_wait(&empty[s], ((p / kSliceStages) - 1) & 1, abort))
+                const int s = p % R::stages;
+                if (p >= R::stages && !mbar_wait(&empty[s], ((p / R::stages) - 1) & 1, abort))
                     break;
                 const long long pp = reverse ? NP - 1 - p : p;
-                uint8_t *st = sm + s * kSliceStage;
-                mbar_arrive_expect_tx(&full[s], kSliceBytes + rows * 4);
+                uint8_t *st = sm + s * R::stage;
+                const float *end = nullptr;
+                if (CARRY)
+                    end = pp + 1 < NP ? S_next + (bh * NP + pp + 1) * state
+                                      : (S_last ? S_last + bh * state : nullptr);
+                mbar_arrive_expect_tx(&full[s], kSliceBytes + rows * 4 + (end ? kSliceBytes : 0));
                 bulk_load(st, S_in + (bh * NP + pp) * state + (long long)sl * kSlice, kSliceBytes,
                           &full[s]);
-                bulk_load(st + kSliceBytes, log_gamma + (bh * NP + pp) * dk + row0, rows * 4,
+                bulk_load(st + R::off_lg, log_gamma + (bh * NP + pp) * dk + row0, rows * 4,
                           &full[s]);
+                if (end) bulk_load(st + R::off_end, end + (long long)sl * kSlice, kSliceBytes, &full[s]);
                 issued = p + 1;
             }
             if (*abort) {  // let the copies this CTA started land before it exits
                 int ignore = 0;
-                for (int p = issued > kSliceStages ? issued - kSliceStages : 0; p < issued; ++p)
-                    mbar_wait(&full[p % kSliceStages], (p / kSliceStages) & 1, &ignore);
+                for (int p = issued > R::stages ? issued - R::stages : 0; p < issued; ++p)
+                    mbar_wait(&full[p % R::stages], (p / R::stages) & 1, &ignore);
             }
         }
         return;
@@ -161,21 +181,33 @@ scan_bulk_kernel(const float *__restrict__ S_in, const float *__restrict__ log_g
         a0 = ip[0];
         a1 = ip[1];
     }
+    const int row_lanes = dv / 8;  // lanes that share a row: a power of two dividing 32
     bool ok = true;
     for (int p = 0; p < NP; ++p) {
-        const int s = p % kSliceStages;
-        if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (p / kSliceStages) & 1, abort))))
+        const int s = p % R::stages;
+        if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (p / R::stages) & 1, abort))))
             break;
         const long long pp = reverse ? NP - 1 - p : p;
-        const uint8_t *st = sm + s * kSliceStage;
+        const uint8_t *st = sm + s * R::stage;
         const float4 x0 = *reinterpret_cast<const float4 *>(st + e0 * 4);
         const float4 x1 = *reinterpret_cast<const float4 *>(st + e0 * 4 + 16);
-        const float g = __expf(*reinterpret_cast<const float *>(st + kSliceBytes + r * 4));
+        const float g = __expf(*reinterpret_cast<const float *>(st + R::off_lg + r * 4));
+        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+        if (CARRY && (pp + 1 < NP || S_last)) {
+            v0 = *reinterpret_cast<const float4 *>(st + R::off_end + e0 * 4);
+            v1 = *reinterpret_cast<const float4 *>(st + R::off_end + e0 * 4 + 16);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);  // this warp's reads of the stage are done
         float4 *op = reinterpret_cast<float4 *>(out + (bh * NP + pp) * state + gofs);
         __stcs(op, a0);
         __stcs(op + 1, a1);
+        if (CARRY) {
+            float sum = fmaf(v0.w, a0.w, fmaf(v0.z, a0.z, fmaf(v0.y, a0.y, v0.x * a0.x))) +
+                        fmaf(v1.w, a1.w, fmaf(v1.z, a1.z, fmaf(v1.y, a1.y, v1.x * a1.x)));
+            for (int o = 1; o < row_lanes; o <<= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+            if ((lane & (row_lanes - 1)) == 0) carry[(bh * NP + pp) * dk + row0 + r] = sum;
+        }
         a0 = vfma4(g, a0, x0);
         a1 = vfma4(g, a1, x1);
     }
@@ -215,7 +247,9 @@ cudaError_t launch_scan(const float *S_in, const float *log_gamma, const float *
                         int NP, int dk, int dv, int reverse, float *out, float *final_state,
                         cudaStream_t st, const float *S_next, const float *S_last, float *carry,
                         int *status) {
-    if (!carry && dk % 4 == 0 && (dk * dv) % kSlice == 0 && kSlice % dv == 0 &&
+    // bulk path: whole slices of whole rows, >= 4 rows per slice (16-byte log-decay copies; a
+    // row's lanes within one warp), 16-byte aligned log-decay rows
+    if (dk % 4 == 0 && (dk * dv) % kSlice == 0 && kSlice % dv == 0 && kSlice / dv >= 4 &&
         kSlice / dv * 4 <= kLgBytes && reinterpret_cast<uintptr_t>(log_gamma) % 16 == 0) {
         const long long nblk = (long long)BH * (dk * dv / kSlice);
         if (nblk == 0 || NP == 0) {
@@ -223,11 +257,13 @@ cudaError_t launch_scan(const float *S_in, const float *log_gamma, const float *
                 return launch_copy_state(init, BH, dk, dv, final_state, st);
             return cudaSuccess;
         }
-        cudaError_t e = cudaFuncSetAttribute(scan_bulk_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSliceSmem);
+        auto kern = carry ? scan_bulk_kernel<true> : scan_bulk_kernel<false>;
+        const int smem = carry ? SliceRing<true>::smem : SliceRing<false>::smem;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        scan_bulk_kernel<<<(unsigned)nblk, kSliceThreads + 32, kSliceSmem, st>>>(
-            S_in, log_gamma, init, NP, dk, dv, reverse, out, final_state, status);
+        kern<<<(unsigned)nblk, kSliceThreads + 32, smem, st>>>(S_in, log_gamma, init, NP, dk, dv,
+                                                              reverse, out, final_state, S_next,
+                                                              S_last, carry, status);
         return cudaGetLastError();
     }
     if (carry && (dv % 4 || 32 % (dv / 4) || (dk * (dv / 4)) % 32)) return cudaErrorInvalidValue;
