@@ -98,3 +98,26 @@ def test_scan_carry(cuda_device):
     assert torch.allclose(carry.double(), ref, rtol=1e-5, atol=1e-4 * float(ref.abs().max()))
     _, _, carry0 = la_seg.la_seg_scan(S, lg, init, True, S_next=S_next)  # no S_last: zero there
     assert torch.equal(carry0[:, :-1], carry[:, :-1]) and torch.all(carry0[:, -1] == 0)
+
+
+@pytest.mark.parametrize("dk,dv", [(6, 32), (4, 512), (128, 128)])
+def test_scan_both_kernels(cuda_device, dk, dv):
+    """Whole 1024-float slices of >= 4 rows with 16-byte aligned log-decays take the bulk-copy
+    kernel, other shapes the per-thread one; a log_gamma view one float off alignment sends the
+    same sizes to the per-thread kernel, and the two agree bit for bit (same fma order)."""
+    g = torch.Generator(device=cuda_device).manual_seed(dk + dv)
+    BH, NP = 3, 7
+    S = torch.randn((BH, NP, dk, dv), generator=g, device=cuda_device)
+    lg = -torch.rand((BH, NP, dk), generator=g, device=cuda_device)
+    init = torch.randn((BH, dk, dv), generator=g, device=cuda_device)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    for reverse in (False, True):
+        out, fin = la_seg.la_seg_scan(S, lg, init, reverse, status=status)
+        ref_out, ref_fin = ref_scan(S, lg, init, reverse)
+        assert rel_err(out, ref_out) <= 1e-6 and rel_err(fin, ref_fin) <= 1e-6
+        buf = torch.empty(lg.numel() + 1, device=cuda_device)
+        lg_off = buf[1:].view(BH, NP, dk)
+        lg_off.copy_(lg)
+        out2, fin2 = la_seg.la_seg_scan(S, lg_off, init, reverse, status=status)
+        assert torch.equal(out, out2) and torch.equal(fin, fin2)
+    assert int(status.item()) == 0
