@@ -5,11 +5,14 @@
 //
 //   acc = init;  for p in order:  out[p] = acc;  acc = exp(log_gamma[p][i]) * acc + S_in[p]
 //
-// Rows i (and columns j) are independent, so the scan is element-parallel over
-// (bh, i, j/4) and sequential over p.  It is HBM-bound: every thread streams float4 states,
-// with the loads of UNROLL segments issued before the dependent FMA chain consumes them.
-// Splitting d_k into blocks (the review's K blocks of All-Scan) changes nothing here: each
-// element's chain is the same whatever the block split.
+// Rows i (and columns j) are independent, so the scan is element-parallel over (bh, i, j) and
+// sequential over p.  It is HBM-bound.  The main kernel (scan_bulk_kernel, below) streams the
+// states through shared memory by bulk copies; the per-thread kernel (scan_kernel) takes the
+// shapes its 1024-float slices do not cover, each thread streaming float4 states with the loads
+// of kUnroll segments issued before the dependent FMA chain consumes them.  Both keep one fma
+// per element and segment in the same order, so they agree bit for bit.  Splitting d_k into
+// blocks (the review's K blocks of All-Scan) changes nothing here: each element's chain is the
+// same whatever the block split.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -19,9 +22,8 @@ namespace {
 
 using namespace sm100;
 
-// 128-thread blocks and a 4-deep batch for the carry variant keep it at one wave of blocks
-// (the C4 reverse scan is 1024 blocks, 7 per SM), which 256-thread blocks at its register count
-// would not.
+// Per-thread kernel: 128-thread blocks, and a 4-deep batch for the carry variant, so that a
+// grid of ~7 blocks per SM stays at one wave.
 constexpr int kScanThreads = 128;
 constexpr int kUnroll = 8;
 

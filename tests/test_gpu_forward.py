@@ -202,3 +202,22 @@ def test_correction_pass_exact_at_scale(cuda_device):
         assert torch.equal(a, first), sc
     del x
     torch.cuda.empty_cache()
+
+
+def test_segmentation_invariance(cuda_device):
+    """Any segmentation P and chunk size gives the P = 1 result (the linear-decomposition
+    identity the scan rests on; ZeCO review, "key machinery"): fp32 CUDA-core path over every
+    chunk size and several P within 1e-4, the bf16 tensor-core path over P within 2e-2."""
+    w = Workload("pinv-f32", 1, 2, 512, 32, 32, 1, 16, "f32", "toy", seed=21)
+    x = make_inputs(w, cuda_device, with_s0=True)
+    base = run(x, w)[0].double().cpu().numpy()
+    for P in (1, 2, 4, 8):
+        for C in (16, 32, 64):
+            o = run(x, w.with_(P=P, chunk=C))[0]
+            assert rel_err(o, base) <= 1e-4, (P, C)
+    w = WORKLOADS["C1"].with_(H=2, L=8192)
+    x = make_inputs(w, cuda_device, with_s0=True)
+    base = run(x, w)[0].double().cpu().numpy()
+    for P in (2, 4, 8):
+        o = run(x, w.with_(P=P))[0]
+        assert rel_err(o, base) <= 2e-2, P
