@@ -293,6 +293,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
+// 16 lanes x 256 bits, 4 times along the columns: r[4k .. 4k+3] of thread l hold columns
+// 8k + 2(l%4) and 8k + 2(l%4) + 1 of lane l/4 (r[4k], r[4k+1]) and of lane l/4 + 8 (r[4k+2],
+// r[4k+3]), from the lane and column of taddr (inside the warp's 32-lane quarter).
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 // 16 lanes x 256 bits: thread l writes lane l/4 (r0, r1) and lane l/4 + 8 (r2, r3) at columns
 // 2(l%4) and 2(l%4)+1 from the lane and column of taddr (inside the warp's 32-lane quarter).
 __device__ __forceinline__ void tmem_st_16x256b(uint32_t taddr, uint32_t r0, uint32_t r1,

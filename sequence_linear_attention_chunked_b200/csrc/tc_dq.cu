@@ -335,21 +335,37 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
         if (c >= 1 && !mbar_wait(b[kSaFree], (c - 1) & 1, abort)) break;
         tc_fence_after();
         const uint64_t e2 = (uint64_t)__float_as_uint(ec[s * D + i]) * 0x100000001ull;
-        float4 *rec = nullptr;  // the state entering a fine part
-        if (a.S_fine && c % w.cpf == 0)
-            rec = reinterpret_cast<float4 *>(
-                a.S_fine + ((((long long)w.bh * a.NP + w.j) * a.fine + c / w.cpf) * D + i) * D);
+        if (a.S_fine && c % w.cpf == 0) {  // the state entering a fine part, to HBM
+            // read through the 16x256b shape, so that one warp-wide store covers whole 32-byte
+            // sectors of 8 rows (thread l: rows r and r + 8, two adjacent columns per 8), where
+            // a thread writing its own row spread every store over 32 rows
+            float *rec = a.S_fine + (((long long)w.bh * a.NP + w.j) * a.fine + c / w.cpf) * D * D;
+            const int c2 = 2 * (lane & 3);
+#pragma unroll 1
+            for (int hq = 0; hq < 2; ++hq) {
+                const int ra = warp * 32 + 16 * hq + (lane >> 2);
+#pragma unroll 1
+                for (int p = 0; p < 4; ++p) {
+                    uint32_t q16[16];
+                    tmem_ld_16x256b_x4(tmem + ((uint32_t)(warp * 32 + 16 * hq) << 16) + kColS + p * 32,
+                                       q16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int col = p * 32 + 8 * k + c2;
+                        *reinterpret_cast<float2 *>(rec + (long long)ra * D + col) =
+                            make_float2(__uint_as_float(q16[4 * k]), __uint_as_float(q16[4 * k + 1]));
+                        *reinterpret_cast<float2 *>(rec + (long long)(ra + 8) * D + col) =
+                            make_float2(__uint_as_float(q16[4 * k + 2]), __uint_as_float(q16[4 * k + 3]));
+                    }
+                }
+            }
+        }
         const uint32_t sa = tmem + lrow + kColSA;
 #pragma unroll 1
         for (int p = 0; p < 4; ++p) {  // value dims 32p .. 32p+31
             tmem_ld32(tmem + lrow + kColS + p * 32, r);
             tmem_wait_ld();
-            if (rec) {
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4)
-                    rec[p * 8 + e4] = make_float4(__uint_as_float(r[4 * e4]), __uint_as_float(r[4 * e4 + 1]),
-                                                  __uint_as_float(r[4 * e4 + 2]), __uint_as_float(r[4 * e4 + 3]));
-            }
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const uint64_t x = mul_f32x2(((uint64_t)r[2 * e + 1] << 32) | r[2 * e], e2);
