@@ -1,6 +1,6 @@
 """bench.py's N > 1 plumbing on the CPU: two gloo ranks on 127.0.0.1 take the job time as the
 slowest rank's and report the throughput of all replicas; a rank other than 0 of the reference
-arm leaves without work or output."""
+arm leaves without work or output, and rank 0 of it prints one line of the bench contract."""
 import datetime
 import os
 import socket
@@ -71,3 +71,23 @@ def test_reference_arm_other_ranks_exit_without_work():
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout == ""
+
+
+def test_reference_arm_rank0_prints_one_contract_line():
+    import json
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "C0", "--steps", "2", "--warmup", "3",
+                        "--cpu-seconds", "0.2"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = r.stdout.strip().splitlines()
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["higher_is_better"]
+    assert d["steps"] == 2 and d["warmup"] == 3 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert "C0" in d["config"]["workload"]
