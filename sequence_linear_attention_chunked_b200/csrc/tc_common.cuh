@@ -1,6 +1,7 @@
 // tc_common.cuh -- pieces shared by the tcgen05 chunk kernels (forward and backward):
 // tile geometry, swizzled-tile addressing, UMMA descriptors for the two operand majors,
-// bf16 packing, the fast exp2, and the TMA tensor-map encoder.
+// bf16 packing, the fast exp2, the copy of interleaved token pairs into tensor memory, and the
+// TMA tensor-map encoder.
 #pragma once
 
 #include <cuda.h>
