@@ -34,9 +34,16 @@
  *             asynchronous on it; nothing blocks the host except la_seg_check_status.
  *  Errors     Argument checks run on the host before any launch and return a negative
  *             la_status; la_last_error_detail then describes the failure.  Conditions found
- *             on the device (a gate range the chunk factorisation cannot represent) set a
- *             status word inside the workspace, read by la_seg_check_status.  No C++
- *             exception crosses this boundary.
+ *             on the device set a status word inside the workspace, read by
+ *             la_seg_check_status.  No C++ exception crosses this boundary.
+ *  Gates      The chunk kernels scale q and k by exp(+-(b_t - b_C)) (b the in-chunk cumsum of
+ *             log_g, b_C its total).  That is exact enough in fp32 / bf16 while no log_g of a
+ *             chunk is positive and |b_C| <= 80 in every key dim.  la_seg_forward and
+ *             la_seg_backward recompute every segment that holds another chunk -- a positive
+ *             log_g, a decay beyond e^-80 over one chunk (down to a = 0), a non-finite value --
+ *             with the token recurrence itself on the CUDA cores (exact, slower), so any gates
+ *             give the recurrence's result.  The per-step entry points have no such path:
+ *             they report such a chunk in their status word (LA_ERR_GATE_RANGE).
  *  Sizes      dk == dv in {32, 64, 128}; chunk in {16, 32, 64}; L % P == 0 and (L / P) % chunk
  *             == 0; B, H, P >= 1.  L == 0 is legal and does nothing but write S_final = S0.
  *  Determinism Identical inputs give bit-identical outputs (no atomics on data).
@@ -63,8 +70,9 @@ typedef enum {
     LA_ERR_ALIGN = -3,      /* a pointer is not 16-byte aligned (workspace: 256-byte)         */
     LA_ERR_DTYPE = -4,      /* unknown la_dtype                                               */
     LA_ERR_WORKSPACE = -5,  /* workspace missing or smaller than la_seg_workspace_bytes       */
-    LA_ERR_GATE_RANGE = -6, /* |sum of log_g over one chunk| > 80 in some key dim: outputs of  */
-                            /* that chunk are not reliable (reported by la_seg_check_status)  */
+    LA_ERR_GATE_RANGE = -6, /* a per-step call met a chunk with a positive log_g or with      */
+                            /* |sum of log_g| > 80 in some key dim: the outputs of its        */
+                            /* segment are not reliable (see "Gates" above)                   */
     LA_ERR_TIMEOUT = -7,    /* a bounded device-side wait gave up                             */
     LA_ERR_CUDA = -8        /* a CUDA runtime call failed (launch, attribute, memset)         */
 } la_status;
@@ -160,8 +168,9 @@ LA_API la_status la_seg_scan(const float *S_in, const float *log_gamma, const fl
  * schedule (e.g. replace the on-device scan by a cross-device one) and time each step.  Each
  * cuts every (b, h) sequence into NP equal segments of L/NP tokens (L % NP == 0, (L/NP) %
  * chunk == 0) and processes every segment independently, chunk by chunk, in one CTA.
- * status: nullable device int; a kernel that meets a chunk whose |sum of log_g| exceeds the
- * factorisation range ORs 1 into it (see LA_ERR_GATE_RANGE). */
+ * status: nullable device int; a kernel that meets a chunk outside the chunk factorisation's
+ * range (a positive log_g, or |sum of log_g| > 80 in some key dim) ORs 1 into it (see
+ * LA_ERR_GATE_RANGE and "Gates" above); these entry points do not recompute such segments. */
 
 /* State pass (ZeCO Alg. 1, "local state stored to HBM"; GLA chunk-state update):
  * S_loc[b,h,p] = state after segment p from a zero start, fp32 [B,H,NP,dk,dv];
@@ -260,6 +269,13 @@ LA_API la_status la_seg_dkv_pass(const void *q, const void *k, const void *v, co
                                  la_dtype dt, void *dk_, void *dv_, void *dlog_g, int *status,
                                  void *cuda_stream);
 
+/* The received states at API-segment boundaries, as la_seg_forward saves them for the
+ * backward (S_recv_save): dst[bh][p] = src[bh][p * m] for p < NP / m, with src fp32
+ * [BH, NP, dk, dv] the states every one of NP sub-segments receives and dst fp32
+ * [BH, NP / m, dk, dv]; m divides NP, dv % 4 == 0. */
+LA_API la_status la_seg_gather_states(const float *src, int BH, int NP, int m, int dk, int dv,
+                                      float *dst, void *cuda_stream);
+
 /* Number of parts la_seg_backward's gradient-state, reverse-scan and dk/dv steps run over
  * (reuse != 0: the caller passes S_recv_saved and no dS_final), or 0 for rejected sizes. */
 LA_API int la_seg_backward_parts(int B, int H, long long L, int dk, int dv, int P, int chunk,
@@ -282,13 +298,16 @@ LA_API int la_seg_subsegments(int B, int H, long long L, int dk, int dv, int P, 
  *
  * Same arguments and result as la_seg_forward, without the workspace.  Sizes whose
  * workspace (la_seg_workspace_bytes) exceeds LA_NOALLOC_SCRATCH_BYTES are rejected with
- * LA_ERR_WORKSPACE before anything runs.  The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress, with that device current); make that first
- * call before any stream capture.  Every call on a device shares the one array, which keeps
- * the last call's contents (the status word is cleared at the start of each call): calls
- * that overlap on the GPU -- on different streams, or from different host threads -- race
- * on it and must be serialised by the caller.  Device-side conditions (LA_ERR_GATE_RANGE)
- * are not reported by this entry point. */
+ * LA_ERR_WORKSPACE before anything runs.  The call looks up the array's device address
+ * (cudaGetSymbolAddress, with the device current) on its first use on each device, and again
+ * after the device's context has been re-created (cudaDeviceReset reloads the module, and the
+ * array may then sit elsewhere; the library notices through the context's unique id); make
+ * those calls before any stream capture.  Devices 0 .. 63 are served.  Every call on a device
+ * shares the one array, which keeps the last call's contents (the status word is cleared at
+ * the start of each call): calls that overlap on the GPU -- on different streams, or from
+ * different host threads -- race on it and must be serialised by the caller.  Device-side
+ * conditions (LA_ERR_TIMEOUT) land in the array's status word, which
+ * la_seg_noalloc_check_status reads. */
 #define LA_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 LA_API la_status la_seg_forward_noalloc(const void *q, const void *k, const void *v,
@@ -297,8 +316,16 @@ LA_API la_status la_seg_forward_noalloc(const void *q, const void *k, const void
                                         la_dtype dt, void *o, float *S_final, float *S_recv_save,
                                         int schedule, void *cuda_stream);
 
+/* la_seg_check_status for la_seg_forward_noalloc: synchronises cuda_stream and returns the
+ * status word that the last no-alloc call on the current device left in the static scratch
+ * (LA_OK or LA_ERR_TIMEOUT), or LA_ERR_CUDA.  Allocates nothing.  A later no-alloc call on the
+ * same device clears the word again. */
+LA_API la_status la_seg_noalloc_check_status(void *cuda_stream);
+
 /* Synchronises cuda_stream and returns the device status word a previous call left in
- * workspace (LA_OK, LA_ERR_GATE_RANGE or LA_ERR_TIMEOUT), or LA_ERR_CUDA. */
+ * workspace (LA_OK or LA_ERR_TIMEOUT after la_seg_forward / la_seg_backward, which compute
+ * every gate range; LA_ERR_GATE_RANGE only from a workspace a caller's per-step status word
+ * shares), or LA_ERR_CUDA. */
 LA_API la_status la_seg_check_status(void *workspace, void *cuda_stream);
 
 /* Copies a NUL-terminated description of the calling thread's last failure into buf (at most

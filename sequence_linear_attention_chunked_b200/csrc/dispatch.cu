@@ -13,7 +13,7 @@ cudaError_t launch_pass(const PassArgs &a, PassMode mode, cudaStream_t st) {
 cudaError_t launch_bwd_dstate(const BwdArgs &a, cudaStream_t st) {
     PassArgs p = {};
     p.q = a.q; p.v = a.dO; p.g = a.g;  // the gradient-state pass reads dO through the v slot
-    p.S_out = a.dSloc; p.logG = a.logG; p.status = a.status;
+    p.S_out = a.dSloc; p.logG = a.logG; p.status = a.status; p.flags = a.flags;
     p.L = a.L; p.T = a.T; p.BH = a.BH; p.NP = a.NP; p.dk = a.dk; p.dv = a.dv; p.chunk = a.chunk;
     p.dt = a.dt;
     if (tc_pass_supported(p)) return launch_tc_pass(p, kPassDState, st);

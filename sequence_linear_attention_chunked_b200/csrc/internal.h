@@ -26,6 +26,7 @@ struct PassArgs {
     float *S_out;         // [BH, NP, dk, dv] (kPassState / kPassLocal; null: not written)
     float *logG;          // [BH, NP, dk]    (kPassState / kPassLocal; null: not written)
     int *status;
+    int *flags;           // [BH, NP] units met outside the factorisation's range (null: status)
     long long L, T;       // tokens per (b, h), tokens per sub-segment
     int BH, NP, dk, dv, chunk;
     la_dtype dt;
@@ -49,6 +50,8 @@ struct BwdArgs {
     float *logG;              // [BH, NP, dk] per-segment log-decay sums (dstate pass)
     const float *carry;       // reverse sweep: [BH, NP, dk] dlog_g carry per part (null: computed)
     int *status;
+    int *flags;               // [BH, NP * fine] fine parts met outside the factorisation's range
+                              // (null: status); the dq sweep marks every part of its segment
     long long L, T;
     int BH, NP, dk, dv, chunk, fine;
     la_dtype dt;
@@ -98,6 +101,20 @@ cudaError_t launch_tc_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
 
 // The chunk pass for these arguments: the tensor-core kernels where they apply, else SIMT.
 cudaError_t launch_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
+
+// The exact token-by-token path (exact.cu) over the units a chunk kernel marked in a.flags:
+//  launch_exact_pass      units (bh, j) of a chunk pass: kPassState rewrites S_out and logG,
+//                         kPassOutput / kPassCorrect rewrite o from S_init[j] (the whole output),
+//                         kPassLocal rewrites o, S_out and logG from zero;
+//  launch_exact_sequence  every (b, h) with a marked sub-segment, from S0 over all L tokens: o,
+//                         S_final and the state entering every save_every-th sub-segment;
+//  launch_exact_dq        segments with a marked fine part: dq, q . dq, S_fine, dSloc, logG;
+//  launch_exact_dkv       marked fine parts: dk, dv, dlog_g (needs a.carry).
+cudaError_t launch_exact_pass(const PassArgs &a, PassMode mode, cudaStream_t st);
+cudaError_t launch_exact_sequence(const PassArgs &a, const float *S0, float *S_final,
+                                  float *S_save, int save_every, cudaStream_t st);
+cudaError_t launch_exact_dq(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_exact_dkv(const BwdArgs &a, cudaStream_t st);
 
 // Exclusive decayed scan over NP sub-segments (see la_seg_scan in la_seg.h).  With `carry`
 // (fp32 [BH, NP, dk]) it also writes the reverse sweep's dlog_g carry of every part p,

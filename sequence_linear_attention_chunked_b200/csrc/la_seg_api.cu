@@ -82,8 +82,10 @@ la::Split make_split(int B, int H, long long L, int P, int chunk) {
     return s;
 }
 
+// Both layouts start with the status word and the flag arrays of the exact path, which each
+// call clears with one memset of the bytes before S_loc.
 struct FwdLayout {
-    size_t status, S_loc, logG, S_recv, chain_states, chain_ready, total;
+    size_t status, flags, S_loc, logG, S_recv, chain_states, chain_ready, total;
 };
 
 FwdLayout fwd_layout(const la::Split &s, int dk, int dv) {
@@ -91,7 +93,8 @@ FwdLayout fwd_layout(const la::Split &s, int dk, int dv) {
     const size_t states = (size_t)s.BH * s.NP * dk * dv * sizeof(float);
     const size_t gam = (size_t)s.BH * s.NP * dk * sizeof(float);
     w.status = 0;
-    w.S_loc = 256;
+    w.flags = 256;  // [BH, NP] sub-segments marked for the exact path
+    w.S_loc = align_up(w.flags + (size_t)s.BH * s.NP * sizeof(int), 256);
     w.logG = align_up(w.S_loc + states, 256);
     w.S_recv = align_up(w.logG + gam, 256);
     w.chain_states = align_up(w.S_recv + states, 256);
@@ -111,7 +114,8 @@ int fine_factor(long long T, int chunk) {
 }
 
 struct BwdLayout {
-    size_t status, S_loc, logG, S_recv, S_fin, S_fine, dSloc, logG_f, dX, carry, qdq, total;
+    size_t status, flags_s, flags_f, S_loc, logG, S_recv, S_fin, S_fine, dSloc, logG_f, dX, carry,
+        qdq, total;
 };
 
 BwdLayout bwd_layout(const la::Split &s, int r, int dk, int dv) {
@@ -120,7 +124,9 @@ BwdLayout bwd_layout(const la::Split &s, int r, int dk, int dv) {
     const size_t fine_states = states * r;
     const size_t gam = (size_t)s.BH * s.NP * dk * sizeof(float);
     w.status = 0;
-    w.S_loc = 256;
+    w.flags_s = 256;  // [BH, NP] segments of the recomputed state pass marked for the exact path
+    w.flags_f = align_up(w.flags_s + (size_t)s.BH * s.NP * sizeof(int), 256);  // [BH, NP * r] fine parts
+    w.S_loc = align_up(w.flags_f + (size_t)s.BH * s.NP * r * sizeof(int), 256);
     w.logG = align_up(w.S_loc + states, 256);
     w.S_recv = align_up(w.logG + gam, 256);
     w.S_fin = align_up(w.S_recv + states, 256);
@@ -144,11 +150,11 @@ struct Aux {
 };
 
 cudaError_t aux_streams(Aux **out) {
-    static thread_local Aux per_device[16];
+    static thread_local Aux per_device[la::kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
+    if (dev < 0 || dev >= la::kMaxDevices) return cudaErrorInvalidDevice;
     Aux &x = per_device[dev];
     if (x.device != dev) {
         int lo = 0, hi = 0;
@@ -231,7 +237,7 @@ la_status check_pass(int B, int H, long long L, int dk, int dv, int NP, int chun
 la::PassArgs pass_args(const void *q, const void *k, const void *v, const void *g, void *o,
                        const float *S_init, float *S_out, float *logG, int *status, int B, int H,
                        long long L, int dk, int dv, int NP, int chunk, la_dtype dt) {
-    la::PassArgs a;
+    la::PassArgs a = {};
     a.q = q; a.k = k; a.v = v; a.g = g; a.o = o;
     a.S_init = S_init; a.S_out = S_out; a.logG = logG; a.status = status;
     a.L = L; a.T = NP > 0 ? L / NP : 0; a.BH = B * H; a.NP = NP;
@@ -400,7 +406,8 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     if (!aligned(workspace, 256)) return fail(LA_ERR_ALIGN, "workspace is not 256-byte aligned");
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     int *status = reinterpret_cast<int *>(at(workspace, w.status));
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
+    int *flags = reinterpret_cast<int *>(at(workspace, w.flags));
+    cudaError_t e = cudaMemsetAsync(status, 0, w.S_loc, stream);  // status word and flags
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
 
     if (L == 0) {
@@ -416,9 +423,13 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     float *logG = reinterpret_cast<float *>(at(workspace, w.logG));
     float *S_recv = reinterpret_cast<float *>(at(workspace, w.S_recv));
 
+    // Every chunk pass below marks the sub-segments whose chunks the factorisation cannot hold
+    // in `flags`; the exact path then rewrites what those sub-segments produced: their local
+    // states before the scan reads them, their outputs after the last pass.
     if (schedule == LA_SCHED_SINGLE_PASS) {  // same sub-segments as the other schedules
         la::PassArgs a = pass_args(q, k, v, log_g, o, nullptr, nullptr, nullptr, status, B, H, L,
                                    dk, dv, s.NP, chunk, dt);
+        a.flags = flags;
         if (la::tc_pass_supported(a)) {
             la::ChainArgs ch;
             ch.states = reinterpret_cast<float *>(at(workspace, w.chain_states));
@@ -431,6 +442,9 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
                 return cuda_fail(e, "chain reset");
             if ((e = la::launch_tc_chain(a, ch, stream)) != cudaSuccess)
                 return cuda_fail(e, "single pass");
+            // a marked sub-segment's state runs on through the chain: its whole sequence again
+            if ((e = la::launch_exact_sequence(a, S0, S_final, S_recv_save, s.m, stream)) != cudaSuccess)
+                return cuda_fail(e, "exact path (sequences)");
             return LA_OK;
         }
         // other shapes: the two-pass order below (same result)
@@ -438,12 +452,19 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
 
     la::PassArgs a = pass_args(q, k, v, log_g, o, nullptr, S_loc, logG, status, B, H, L, dk, dv,
                                s.NP, chunk, dt);
+    a.flags = flags;
     if (schedule == LA_SCHED_OVERLAP) {
         Aux *aux = nullptr;
-        if ((e = aux_streams(&aux)) != cudaSuccess) return cuda_fail(e, "second stream");
+        if ((e = aux_streams(&aux)) != cudaSuccess)
+            return e == cudaErrorInvalidDevice
+                       ? fail(LA_ERR_ARG, "LA_SCHED_OVERLAP: the current device is beyond the %d "
+                              "devices this library serves", la::kMaxDevices)
+                       : cuda_fail(e, "second stream");
         // 1. local states (state pass) on the caller's stream
         if ((e = la::launch_pass(a, la::kPassState, stream)) != cudaSuccess)
             return cuda_fail(e, "state pass");
+        if ((e = la::launch_exact_pass(a, la::kPassState, stream)) != cudaSuccess)
+            return cuda_fail(e, "exact path (states)");
         // 2. fork: the scan on the second stream, the local outputs on the caller's
         if ((e = cudaEventRecord(aux->fork, stream)) != cudaSuccess ||
             (e = cudaStreamWaitEvent(aux->stream, aux->fork, 0)) != cudaSuccess)
@@ -464,6 +485,8 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
         a.S_init = S_recv;
         if ((e = la::launch_pass(a, la::kPassCorrect, stream)) != cudaSuccess)
             return cuda_fail(e, "correction pass");
+        if ((e = la::launch_exact_pass(a, la::kPassCorrect, stream)) != cudaSuccess)
+            return cuda_fail(e, "exact path (outputs)");
         if (S_recv_save &&
             (e = la::launch_gather_states(S_recv, s.BH, s.NP, s.m, dk, dv, S_recv_save, stream)) !=
                 cudaSuccess)
@@ -474,6 +497,8 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     // 1. per sub-segment: local state from zero (+ intra-chunk outputs for three-phase)
     if ((e = la::launch_pass(a, three ? la::kPassLocal : la::kPassState, stream)) != cudaSuccess)
         return cuda_fail(e, three ? "local pass" : "state pass");
+    if ((e = la::launch_exact_pass(a, la::kPassState, stream)) != cudaSuccess)
+        return cuda_fail(e, "exact path (states)");
     // 2. exclusive decayed scan across sub-segments
     if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_final, stream,
                              nullptr, nullptr, nullptr, status)) !=
@@ -483,6 +508,8 @@ la_status la_seg_forward(const void *q, const void *k, const void *v, const void
     a.S_init = S_recv;
     if ((e = la::launch_pass(a, three ? la::kPassCorrect : la::kPassOutput, stream)) != cudaSuccess)
         return cuda_fail(e, three ? "correction pass" : "output pass");
+    if ((e = la::launch_exact_pass(a, la::kPassOutput, stream)) != cudaSuccess)
+        return cuda_fail(e, "exact path (outputs)");
     if (S_recv_save &&
         (e = la::launch_gather_states(S_recv, s.BH, s.NP, s.m, dk, dv, S_recv_save, stream)) !=
             cudaSuccess)
@@ -558,7 +585,9 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     if (!aligned(workspace, 256)) return fail(LA_ERR_ALIGN, "workspace is not 256-byte aligned");
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     int *status = reinterpret_cast<int *>(at(workspace, w.status));
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
+    int *flags_s = reinterpret_cast<int *>(at(workspace, w.flags_s));
+    int *flags_f = reinterpret_cast<int *>(at(workspace, w.flags_f));
+    cudaError_t e = cudaMemsetAsync(status, 0, w.S_loc, stream);  // status word and flags
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
     if (L == 0) {  // no tokens: S_final = S0, so dS0 = dS_final
         if (dS0 && (e = la::launch_copy_state(dS_final, s.BH, dk, dv, dS0, stream)) != cudaSuccess)
@@ -582,8 +611,11 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     if (!reuse) {
         la::PassArgs a = pass_args(nullptr, k, v, log_g, nullptr, nullptr, S_loc, logG, status, B,
                                    H, L, dk, dv, s.NP, chunk, dt);
+        a.flags = flags_s;
         if ((e = la::launch_pass(a, la::kPassState, stream)) != cudaSuccess)
             return cuda_fail(e, "backward state pass");
+        if ((e = la::launch_exact_pass(a, la::kPassState, stream)) != cudaSuccess)
+            return cuda_fail(e, "exact path (states)");
         if ((e = la::launch_scan(S_loc, logG, S0, s.BH, s.NP, dk, dv, 0, S_recv, S_fin, stream,
                                  nullptr, nullptr, nullptr, status)) !=
             cudaSuccess)
@@ -594,11 +626,13 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     b.dq_out = dq; b.dk_out = dk_; b.dv_out = dv_; b.dg_out = dlog_g;
     b.S_recv = recv; b.S_fine = S_fine; b.S_end_next = S_fine; b.S_fin = reuse ? nullptr : S_fin;
     b.dX = dX; b.dq_ws = qdq; b.dSloc = dSloc; b.logG = logG_f; b.status = status;
+    b.flags = flags_f;  // fine parts whose chunks the factorisation cannot hold: the exact path
     b.L = L; b.BH = s.BH; b.dk = dk; b.dv = dv; b.chunk = chunk; b.dt = dt;
     // 2. dq sweep over the segments; records the state entering each of their r fine parts,
     //    and forms every fine part's gradient state and log-decay sum
     b.NP = s.NP; b.T = s.T; b.fine = r;
     if ((e = la::launch_bwd_dq(b, stream)) != cudaSuccess) return cuda_fail(e, "dq pass");
+    if ((e = la::launch_exact_dq(b, stream)) != cudaSuccess) return cuda_fail(e, "exact path (dq)");
     // 3-4 run over the fine parts
     b.NP = s.NP * r; b.T = s.T / r; b.fine = 1;
     // 3. reverse exclusive decayed scan: gradient of every part's end state, dS0, and each
@@ -609,6 +643,7 @@ la_status la_seg_backward(const void *q, const void *k, const void *v, const voi
     b.carry = carry;
     // 4. dk, dv, dlog_g per part
     if ((e = la::launch_bwd_dkv(b, stream)) != cudaSuccess) return cuda_fail(e, "dkv pass");
+    if ((e = la::launch_exact_dkv(b, stream)) != cudaSuccess) return cuda_fail(e, "exact path (dkv)");
     return LA_OK;
 }
 
@@ -643,6 +678,19 @@ la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *in
     return e == cudaSuccess ? LA_OK : cuda_fail(e, "scan");
 }
 
+la_status la_seg_gather_states(const float *src, int BH, int NP, int m, int dk, int dv, float *dst,
+                               void *cuda_stream) {
+    if (BH < 0 || NP < 0 || m < 1 || (NP % m) != 0 || dk < 1 || dv < 4 || dv % 4)
+        return fail(LA_ERR_SHAPE, "need BH, NP >= 0, m >= 1 dividing NP, dk >= 1, dv a multiple of 4");
+    if ((long long)BH * NP > 0 && (!src || !dst))
+        return fail(LA_ERR_ARG, "src and dst must be non-null");
+    if ((src && !aligned(src, 16)) || (dst && !aligned(dst, 16)))
+        return fail(LA_ERR_ALIGN, "src and dst must be 16-byte aligned");
+    cudaError_t e = la::launch_gather_states(src, BH, NP, m, dk, dv, dst,
+                                             static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e, "state gather");
+}
+
 la_status la_seg_check_status(void *workspace, void *cuda_stream) {
     if (!workspace) return fail(LA_ERR_ARG, "workspace is null");
     int h = 0;
@@ -653,7 +701,8 @@ la_status la_seg_check_status(void *workspace, void *cuda_stream) {
     if (h & la::kStatusTimeout) return fail(LA_ERR_TIMEOUT, "a device-side wait gave up");
     if (h & la::kStatusGateRange)
         return fail(LA_ERR_GATE_RANGE,
-                    "some chunk has |sum of log_g| > %.0f in a key dimension; use a smaller chunk",
+                    "some chunk has a positive log_g or |sum of log_g| > %.0f in a key dimension; "
+                    "la_seg_forward / la_seg_backward compute such chunks exactly",
                     (double)la::kGateRangeLimit);
     return LA_OK;
 }

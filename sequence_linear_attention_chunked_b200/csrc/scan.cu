@@ -30,7 +30,10 @@ constexpr int kUnroll = 8;
 // With `carry` (the backward's reverse scan): carry[bh][p][i] = sum_j S_end_p[i][j] out[p][i][j],
 // S_end_p = S_next[p+1] (p < NP-1) or S_last (p = NP-1; null: zero) -- the dlog_g carry of part
 // p.  The threads of one row i are dv4 consecutive lanes of a warp, so the sum over j is a
-// segmented warp reduction.
+// segmented warp reduction.  The xor butterfly over offsets below dv4 keeps to one row only
+// when dv4 = dv / 4 is a power of two that divides 32 (dv in {4, 8, .., 128}) and rows start
+// on dv4-lane boundaries (dk * dv4 a multiple of 32); launch_scan and la_seg_scan refuse any
+// other dv with a carry.
 template <bool CARRY>
 __global__ void __launch_bounds__(kScanThreads)
 scan_kernel(const float4 *__restrict__ S_in, const float *__restrict__ log_gamma,

@@ -72,7 +72,9 @@ __global__ void __launch_bounds__(kThreads) simt_dstate_kernel(BwdArgs a) {
             float acc = sB0[tid];
             const float start = acc;
             for (int t = 0; t < C; ++t) {
-                acc += sg[t * DKP + tid];
+                const float x = sg[t * DKP + tid];
+                range_bad |= !(x <= 0.f);  // a positive (or NaN) gate exponent
+                acc += x;
                 sg[t * DKP + tid] = acc;
             }
             range_bad |= !(fabsf(acc - start) <= kGateRangeLimit);
@@ -95,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) simt_dstate_kernel(BwdArgs a) {
     float *R = a.dSloc + ((long long)bh * a.NP + j) * DK * DV;
     for (int idx = tid; idx < DK * DV; idx += kThreads) R[idx] = sR[idx];
     if (tid < DK) a.logG[((long long)bh * a.NP + j) * DK + tid] = sB0[tid];
-    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
+    if (range_bad) flag_range(a.flags, (long long)blockIdx.x, 1, a.status);
 }
 
 // ------------------------------------------------------------------ gradient pass
@@ -139,15 +141,19 @@ __global__ void __launch_bounds__(kThreads) simt_dq_kernel(BwdArgs a) {
     const long long sidx = ((long long)bh * a.NP + j) * DK * DV;
 
     // cumsum of the chunk's log-gates (threads < DK), then e^{b_C}; returns after a barrier
+    bool range_bad = false;
     auto gates = [&](long long r0) {
         if (tid < DK) {
             float acc = 0.f;
             for (int t = 0; t < C; ++t) {
-                acc += sb[t * DKP + tid];
+                const float x = sb[t * DKP + tid];
+                range_bad |= !(x <= 0.f);  // a positive (or NaN) gate exponent
+                acc += x;
                 sb[t * DKP + tid] = acc;
             }
             sbC[tid] = acc;
             seC[tid] = __expf(acc);
+            range_bad |= !(fabsf(acc) <= kGateRangeLimit);
         }
         __syncthreads();
     };
@@ -203,7 +209,8 @@ __global__ void __launch_bounds__(kThreads) simt_dq_kernel(BwdArgs a) {
         }
     }
     __syncthreads();
-
+    if (range_bad)  // every fine part of the segment: the state runs through them
+        flag_range(a.flags, ((long long)bh * a.NP + j) * a.fine, a.fine, a.status);
 }
 
 template <typename T, int DK, int DV, int C>
@@ -226,15 +233,19 @@ __global__ void __launch_bounds__(kThreads) simt_dkv_kernel(BwdArgs a) {
     const long long sidx = ((long long)bh * a.NP + j) * DK * DV;
 
     // cumsum of the chunk's log-gates (threads < DK), then e^{b_C}; returns after a barrier
+    bool range_bad = false;
     auto gates = [&](long long r0) {
         if (tid < DK) {
             float acc = 0.f;
             for (int t = 0; t < C; ++t) {
-                acc += sb[t * DKP + tid];
+                const float x = sb[t * DKP + tid];
+                range_bad |= !(x <= 0.f);  // a positive (or NaN) gate exponent
+                acc += x;
                 sb[t * DKP + tid] = acc;
             }
             sbC[tid] = acc;
             seC[tid] = __expf(acc);
+            range_bad |= !(fabsf(acc) <= kGateRangeLimit);
         }
         __syncthreads();
     };
@@ -322,6 +333,7 @@ __global__ void __launch_bounds__(kThreads) simt_dkv_kernel(BwdArgs a) {
             sS[idx] = acc * seC[i];
         }
     }
+    if (range_bad) flag_range(a.flags, (long long)blockIdx.x, 1, a.status);
 }
 
 template <typename Kern>

@@ -12,8 +12,9 @@
 //   S       = S' + Ktil^T V
 //
 // Qbar'_t Ktil_s = sum_i q_ti k_si exp(b_ti - b_si), and Qbar'_t S' = (q_t . exp(b_t)) S,
-// which is the token recurrence summed over the chunk.  Every exponent is bounded by the
-// chunk's |b_C|; above kGateRangeLimit the status word gets kStatusGateRange.
+// which is the token recurrence summed over the chunk.  With log_g <= 0 every exponent is
+// bounded by the chunk's |b_C|; a chunk with a positive log_g or |b_C| > kGateRangeLimit is
+// flagged (flag_range).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -90,7 +91,9 @@ __global__ void __launch_bounds__(kThreads) simt_pass_kernel(PassArgs a) {
         if (tid < DK) {
             float acc = 0.f;
             for (int t = 0; t < C; ++t) {
-                acc += sg[t * DKP + tid];
+                const float x = sg[t * DKP + tid];
+                range_bad |= !(x <= 0.f);  // a positive (or NaN) gate exponent
+                acc += x;
                 sg[t * DKP + tid] = acc;
             }
             sbC[tid] = acc;
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(kThreads) simt_pass_kernel(PassArgs a) {
         for (int idx = tid; idx < DK * DV; idx += kThreads) Sout[idx] = sS[idx];
     }
     if (kWritesState && a.logG && tid < DK) a.logG[((long long)bh * a.NP + j) * DK + tid] = logG;
-    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
+    if (range_bad) flag_range(a.flags, (long long)bh * a.NP + j, 1, a.status);
 }
 
 template <typename T, int DK, int DV, int C, int MODE>

@@ -249,42 +249,69 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
     const int i0 = gw * 32 + ig * 8;
     float *ec = reinterpret_cast<float *>(smem + off_ec);
     bool range_bad = false;
+    uint32_t posm = 0x80008000u;  // running int16 max of the log_g bits: > 0 means a positive gate exponent
     for (int it = 0; it < nchunks; ++it) {
         const int s = it % kStages;
         if (!mbar_wait(&b.full[s], (it / kStages) & 1, abort)) break;
         uint8_t *st = smem + s * kStageBytes;
-        float bt[8][8];
+        // The in-chunk cumsum reproduces the dq sweep's bit for bit -- the same sums within
+        // groups of 4 rows and the same Hillis-Steele tree over the 16 group totals (this
+        // thread holds groups 2 tg and 2 tg + 1) -- so that both sweeps form identical bf16
+        // operands Ktil and Qbar' = bf16(q bf16(e^x)); the diagonal term of q . dq and k . dk is
+        // then the same fp32 product in both and cancels exactly in dlog_g.
+        float bt[8][8], tot[2][8];
         {
             uint4 graw[8];
 #pragma unroll
             for (int r = 0; r < 8; ++r)
                 graw[r] = *reinterpret_cast<const uint4 *>(st + off_g + tile_off(tg * 8 + r, i0));
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                float f[8];
-                unpack8(graw[r], f);
+            for (int r = 0; r < 8; ++r) posm = pos_bf16_max(posm, graw[r]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) bt[r][e] = (r ? bt[r - 1][e] : 0.f) + f[e];
+            for (int h = 0; h < 2; ++h) {  // rows 8 tg + 4 h .. + 3
+                float f[4][8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) unpack8(graw[4 * h + k], f[k]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float p01 = f[0][e] + f[1][e], p23 = f[2][e] + f[3][e];
+                    bt[4 * h][e] = f[0][e];
+                    bt[4 * h + 1][e] = p01;
+                    bt[4 * h + 2][e] = f[2][e] + p01;
+                    bt[4 * h + 3][e] = p23 + p01;
+                    tot[h][e] = p01 + p23;
+                }
             }
         }
-        float incl[8];
+        float ia[8], ib[8];  // inclusive scan of the group totals: groups 2 tg, 2 tg + 1
 #pragma unroll
-        for (int e = 0; e < 8; ++e) incl[e] = bt[7][e];
+        for (int e = 0; e < 8; ++e) {  // step 1: group g adds group g - 1
+            const float up = __shfl_up_sync(0xFFFFFFFFu, tot[1][e], 4);
+            ia[e] = tg >= 1 ? tot[0][e] + up : tot[0][e];
+            ib[e] = tot[1][e] + tot[0][e];
+        }
 #pragma unroll
-        for (int d = 1; d < 8; d <<= 1) {
+        for (int dd = 1; dd < 8; dd <<= 1) {  // steps 2, 4, 8: group g adds group g - 2 dd
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float up = __shfl_up_sync(0xFFFFFFFFu, incl[e], 4 * d);
-                if (tg >= d) incl[e] += up;
+                const float ua = __shfl_up_sync(0xFFFFFFFFu, ia[e], 4 * dd);
+                const float ub = __shfl_up_sync(0xFFFFFFFFu, ib[e], 4 * dd);
+                if (tg >= dd) {
+                    ia[e] += ua;
+                    ib[e] += ub;
+                }
             }
         }
         float nbCl[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            const float bC = __shfl_sync(0xFFFFFFFFu, incl[e], 28 + ig);
-            const float off = incl[e] - bt[7][e];
+            const float bC = __shfl_sync(0xFFFFFFFFu, ib[e], 28 + ig);  // group 15
+            const float offa = ia[e] - tot[0][e], offb = ib[e] - tot[1][e];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) bt[r][e] += off;
+            for (int r = 0; r < 4; ++r) {
+                bt[r][e] += offa;
+                bt[4 + r][e] += offb;
+            }
             nbCl[e] = -bC * kLog2e;
             range_bad |= !(fabsf(bC) <= kGateRangeLimit);
         }
@@ -317,7 +344,9 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
                 for (int e = 0; e < 4; ++e) {
                     const float u0 = ex2_approx(x[2 * e]), u1 = ex2_approx(x[2 * e + 1]);
                     const float d0 = ex2_approx(-x[2 * e]), d1 = ex2_approx(-x[2 * e + 1]);
-                    wq[e] = pack_bf16(fq[2 * e] * u0, fq[2 * e + 1] * u1);
+                    const uint32_t fw = pack_bf16(u0, u1);  // F = bf16(e^x), as the dq sweep has it
+                    wq[e] = pack_bf16(fq[2 * e] * __uint_as_float(fw << 16),
+                                      fq[2 * e + 1] * __uint_as_float(fw & 0xFFFF0000u));
                     wk[e] = pack_bf16(fk[2 * e] * d0, fk[2 * e + 1] * d1);
                     wf[e] = pack_bf16(d0, d1);
                 }
@@ -335,7 +364,8 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
     }
     if (!*abort && nchunks > 0)  // dv of the part's first chunk
         dv_readout(b, abort, tmem, lrow, (nchunks - 1) & 1, dv, lane);
-    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
+    if (range_bad || any_pos_bf16(posm))  // this CTA's unit is fine part blockIdx.x = bh * NP + j
+        flag_range(a.flags, (long long)blockIdx.x, 1, a.status);
 }
 
 // Writes a masked (s <= t) bf16 copy of a M=64 TMEM accumulator half into a 64x64 tile.

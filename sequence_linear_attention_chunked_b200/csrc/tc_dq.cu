@@ -8,7 +8,8 @@
 //   M    = dO V^T                    M=64  (t) N=64  (s) K=128 (j)  -> masked s <= t, bf16 tile
 //   S   <- S' + Ktil^T V             M=128 (i) N=128 (j) K=64  (s)  accumulated onto S' in TMEM
 //   dq^T = S' dO^T + Ktil^T M^T      M=128 (i) N=64  (t) K=128 (j) / 64 (s), A = S' from TMEM
-//   dq[t,i] = e^{b_t,i - b_C,i} dq^T[i,t];   q . dq (fp32) for the reverse sweep's dlog_g
+//   dq[t,i] = e^{b_t,i - b_C,i} dq^T[i,t];   q . dq (fp32) for the reverse sweep's dlog_g,
+//   formed as bf16(q F) dq^T with F = bf16(e^{b_t - b_C}) (see the read-out)
 //
 // (the gradient of o_t = q_t S_t with respect to q_t, in the chunk factorisation of the
 // forward).  The sweep also records the state entering each of the segment's `fine` equal
@@ -203,6 +204,7 @@ __device__ __noinline__ void gate_role(uint8_t *smem, const Bars &b, volatile in
 #pragma unroll
     for (int e = 0; e < 8; ++e) logB[e] = 0.f;
     bool range_bad = false;
+    uint32_t posm = 0x80008000u;  // running int16 max of the log_g bits: > 0 means a positive gate exponent
     for (int c = 0; c < w.nchunks; ++c) {
         const int s = c % kStages;
         if (!mbar_wait(b[kFull + s], (c / kStages) & 1, abort)) break;
@@ -214,6 +216,8 @@ __device__ __noinline__ void gate_role(uint8_t *smem, const Bars &b, volatile in
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 graw[k] = *reinterpret_cast<const uint4 *>(st + off_g + tile_off(tg * 4 + (k ^ sw), i0));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) posm = pos_bf16_max(posm, graw[k]);
             float f[4][8];
 #pragma unroll
             for (int k = 0; k < 4; ++k) unpack8(graw[k], f[k]);
@@ -296,7 +300,8 @@ __device__ __noinline__ void gate_role(uint8_t *smem, const Bars &b, volatile in
         __syncwarp();
         if (lane == 0) mbar_arrive(b[kGated + s]);
     }
-    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
+    if (range_bad || any_pos_bf16(posm))  // every fine part of the segment: the state runs through them
+        flag_range(a.flags, ((long long)w.bh * a.NP + w.j) * a.fine, a.fine, a.status);
 }
 
 // ------------------------------------------------------------------ state warps (0-3)
@@ -483,10 +488,17 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
                 const long long t = tok0 + g * 16 + e;
-                const float v0 = __uint_as_float(r16[e]) * __uint_as_float(fq[e] << 16);
-                const float v1 = __uint_as_float(r16[e + 1]) * __uint_as_float(fq[e + 1] << 16);
-                a.dq_ws[t * D + i] = __uint_as_float(fq[e] & 0xFFFF0000u) * v0;
-                a.dq_ws[(t + 1) * D + i] = __uint_as_float(fq[e + 1] & 0xFFFF0000u) * v1;
+                const float F0 = __uint_as_float(fq[e] << 16), F1 = __uint_as_float(fq[e + 1] << 16);
+                const float a0 = __uint_as_float(r16[e]), a1 = __uint_as_float(r16[e + 1]);
+                const float v0 = a0 * F0, v1 = a1 * F1;  // dq
+                // q . dq handed over as Qbar' dq^T, Qbar' = bf16(q F) -- bit for bit the operand
+                // the reverse sweep's MMAs use -- so that the diagonal term (q_t . k_t)(v_t . dO_t)
+                // of q . dq and of k . dk is the same exact fp32 product in both sweeps and
+                // cancels in dlog_g down to fp32 accumulation error
+                const uint32_t qb = pack_bf16(__uint_as_float(fq[e] & 0xFFFF0000u) * F0,
+                                              __uint_as_float(fq[e + 1] & 0xFFFF0000u) * F1);
+                a.dq_ws[t * D + i] = __uint_as_float(qb << 16) * a0;
+                a.dq_ws[(t + 1) * D + i] = __uint_as_float(qb & 0xFFFF0000u) * a1;
                 const uint32_t p = pack_bf16(v0, v1);  // low: token t, high: token t+1
                 unsigned short *h = reinterpret_cast<unsigned short *>(dq + t * D + i);
                 h[0] = (unsigned short)(p & 0xFFFFu);

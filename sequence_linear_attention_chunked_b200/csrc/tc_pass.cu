@@ -264,6 +264,7 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 #pragma unroll
     for (int e = 0; e < 8; ++e) logG[e] = 0.f;
     bool range_bad = false;
+    uint32_t posm = 0x80008000u;  // running int16 max of the log_g bits: > 0 means a positive gate exponent
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % C::stages;
         if (!mbar_wait(&b.full[s], (c / C::stages) & 1, abort)) break;
@@ -275,6 +276,8 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 graw[k] = *reinterpret_cast<const uint4 *>(st + C::off_g + tile_off(tg * 4 + (k ^ sw), i0));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) posm = pos_bf16_max(posm, graw[k]);
             float f[4][8];
 #pragma unroll
             for (int k = 0; k < 4; ++k) unpack8(graw[k], f[k]);
@@ -377,7 +380,7 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
         __syncwarp();
         if (lane == 0) mbar_arrive(lg_full);
     }
-    if (range_bad && a.status) atomicOr(a.status, kStatusGateRange);
+    if (range_bad || any_pos_bf16(posm)) flag_range(a.flags, (long long)bh * a.NP + j, 1, a.status);
 }
 
 // ------------------------------------------------------------------ state warps (0-3)

@@ -26,7 +26,8 @@ EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_s
             "la_seg_state_pass", "la_seg_local_pass", "la_seg_output_pass", "la_seg_correct_pass",
             "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail",
             "la_seg_forward_noalloc", "la_seg_dstate_pass", "la_seg_dq_pass", "la_seg_dkv_pass",
-            "la_seg_backward_parts", "la_seg_chain_pass", "la_seg_chain_reset")
+            "la_seg_backward_parts", "la_seg_chain_pass", "la_seg_chain_reset",
+            "la_seg_noalloc_check_status", "la_seg_gather_states")
 
 _lib = None
 
@@ -71,6 +72,10 @@ def lib():
         L.la_seg_forward_noalloc.argtypes = [P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
                                              i32, P, P, P, i32, P]
         L.la_seg_forward_noalloc.restype = i32
+        L.la_seg_gather_states.argtypes = [P, i32, i32, i32, i32, i32, P, P]
+        L.la_seg_gather_states.restype = i32
+        L.la_seg_noalloc_check_status.argtypes = [P]
+        L.la_seg_noalloc_check_status.restype = i32
         L.la_seg_dstate_pass.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P,
                                          P, P]
         L.la_seg_dstate_pass.restype = i32
@@ -345,6 +350,18 @@ def la_seg_dkv_pass(q, k, v, log_g, dO, S_recv, S_final, dX, qdq, NP, chunk, *, 
                                  _dt(q), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(status),
                                  _stream(stream)), "la_seg_dkv_pass")
     return out
+
+
+def la_seg_gather_states(src, m, *, dst=None, stream=None):
+    """dst[:, :, p] = src[:, :, p * m]: the states at API-segment boundaries (src fp32
+    [B, H, NP, dk, dv], dst [B, H, NP / m, dk, dv])."""
+    B, H, NP, dk, dv = src.shape
+    _need(src, "src", torch.float32, None, src.device)
+    dst = torch.empty((B, H, NP // m, dk, dv), dtype=torch.float32, device=src.device) if dst is None else dst
+    _need(dst, "dst", torch.float32, (B, H, NP // m, dk, dv), src.device)
+    _check(lib().la_seg_gather_states(_ptr(src), B * H, NP, m, dk, dv, _ptr(dst), _stream(stream)),
+           "la_seg_gather_states")
+    return dst
 
 
 def chain_buffers(B, H, dk, dv, device="cuda"):
