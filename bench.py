@@ -3,11 +3,14 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C1] [--schedule auto]
     python bench.py --impl reference ...      # the fp64 CPU oracle on this host's cores
 
-A step is one pass of the whole path over one batch of the workload: every per-segment chunk
-pass, the cross-segment state scan and the output / correction pass (plus the backward
-passes for a fwd+bwd workload), each through the library's C ABI on the current stream.
-Inputs are resident in HBM and L2 is flushed (256 MiB write, untimed) before every step; each
-step is bracketed by CUDA events and its phases by events in between, on the same stream.
+A step is one pass of the whole path over one batch of the workload: la_seg_forward over the
+workload's P segments, saving the states they receive, and for a fwd+bwd workload
+la_seg_backward reusing them -- the calls a user makes, through the library's C ABI on the
+current stream.  Inputs are resident in HBM and L2 is flushed (256 MiB write, untimed) before
+every step; each step is bracketed by CUDA events.  The same kernels are also run through the
+per-step entry points with events between the phases (checked bit for bit against the public
+calls), which gives each kernel's time and roofline.  After the headline workload the forward
+workloads C1-C3 are timed the same way into the line's "configs".
 With N > 1 ranks (torchrun), every rank runs its own replica of the workload on its own GPU:
 the path has no cross-rank exchange, so there is no collective on the data path ("weak"
 scaling); the max over ranks of the device time is reported.
@@ -153,25 +156,84 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- our arm
+def dtype_code(la_seg, w):
+    return la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16
+
+
+class Public:
+    """The calls a user of the library makes for the workload, through the C ABI on the current
+    stream: la_seg_forward saving the received states of its P segments, then (fwd+bwd
+    workloads) la_seg_backward reusing them.  This is what the headline times."""
+
+    def __init__(self, w: Workload, x, schedule: int, device):
+        from sequence_linear_attention_chunked_b200 import la_seg
+        self.la, self.w, self.x, self.schedule = la_seg, w, x, schedule
+        dt = dtype_code(la_seg, w)
+        f32 = dict(dtype=torch.float32, device=device)
+        self.ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device)
+        self.o = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype, device=device)
+        self.S_final = torch.empty((w.B, w.H, w.dk, w.dv), **f32)
+        self.S_save = torch.empty((w.B, w.H, w.P, w.dk, w.dv), **f32) if w.backward else None
+        if w.backward:
+            self.wsb = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, device)
+            self.grads = (torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
+                          torch.empty_like(x["log_g"]), torch.empty_like(self.S_final))
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        # kernels of this library per step: state pass, exact-path states, scan, output pass,
+        # exact-path outputs, state gather; dq sweep, exact-path dq, reverse scan, dk/dv sweep,
+        # exact-path dk/dv (the status / flag memsets are not counted)
+        self.launches_per_step = 5 + (6 if w.backward else 0)
+
+    def run(self, record=True):
+        la, w, x, P = self.la, self.w, self.x, self.la._ptr
+        st = la._stream(None)
+        dt = dtype_code(la, w)
+        if record:
+            self.ev[0].record()
+        la._check(la.lib().la_seg_forward(
+            P(x["q"]), P(x["k"]), P(x["v"]), P(x["log_g"]), None, w.B, w.H, w.L, w.dk, w.dv, w.P,
+            w.chunk, dt, P(self.o), P(self.S_final), P(self.S_save), self.schedule, P(self.ws),
+            self.ws.numel(), st), "la_seg_forward")
+        if w.backward:
+            g = self.grads
+            la._check(la.lib().la_seg_backward(
+                P(x["q"]), P(x["k"]), P(x["v"]), P(x["log_g"]), None, P(self.S_save), P(x["dO"]),
+                None, w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, P(g[0]), P(g[1]), P(g[2]),
+                P(g[3]), P(g[4]), P(self.wsb), self.wsb.numel(), st), "la_seg_backward")
+        if record:
+            self.ev[1].record()
+
+    def ms(self):
+        return self.ev[0].elapsed_time(self.ev[1])
+
+    def check_status(self):
+        self.la.la_seg_check_status(self.ws)
+        if self.w.backward:
+            self.la.la_seg_check_status(self.wsb)
+
+
 class Step:
-    """One pass of the whole path through the C ABI's per-step entry points, with CUDA events
-    between the phases on the launching stream.  Forward: state pass, state scan, output pass
-    (or local pass, scan, correction pass); backward (fwd+bwd workloads): dq pass (which also
-    forms the gradient states), reverse scan, dk/dv/dlog_g pass, reusing the forward's received
-    states."""
+    """The same device work as Public, composed of the C ABI's per-step entry points with CUDA
+    events between the phases on the launching stream, so that each kernel can be timed and
+    set against its roofline.  It reproduces the public calls' splits: the forward's passes over
+    the library's sub-segments (state pass, state scan, output pass -- or the other schedules'
+    passes), the gather of the P received states the forward saves; the backward, which reuses
+    them, over whole segments: dq pass (which also forms the gradient states of the fine parts),
+    reverse scan, dk/dv/dlog_g pass.  bench_ours checks that both give the same bits."""
 
     KERNEL_KEYS = {"chain reset": "chain_reset", "single pass": "chain_kernel",
                    "state pass": "state_pass", "output pass": "output_pass",
                    "local pass": "local_pass", "correction pass": "correct_pass",
-                   "state scan": "scan", "dq pass": "dq_pass", "reverse scan": "scan",
-                   "dkv pass": "dkv_pass"}
+                   "state scan": "scan", "save states": "gather", "dq pass": "dq_pass",
+                   "reverse scan": "scan", "dkv pass": "dkv_pass"}
 
     def __init__(self, w: Workload, x, schedule: str, device):
         from sequence_linear_attention_chunked_b200 import la_seg
         self.la = la_seg
         self.w, self.x, self.dev = w, x, device
-        dt = la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16
+        dt = dtype_code(la_seg, w)
         self.NP = la_seg.la_seg_subsegments(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt)
+        self.m = self.NP // w.P
         self.schedule = schedule
         B, H, L, dk, dv, NP = w.B, w.H, w.L, w.dk, w.dv, self.NP
         f32 = dict(dtype=torch.float32, device=device)
@@ -196,12 +258,14 @@ class Step:
             self.phases = ["state pass", "state scan", "output pass"]
         self.n_fwd = len(self.phases)
         if w.backward:
-            # the backward's fine split (parts of <= 1024 tokens) under the forward's segments
+            # la_seg_backward with saved states: whole API segments, each cut into fine parts
+            self.NPD = w.P
             self.NPF = la_seg.la_seg_backward_parts(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt,
-                                                    False)
-            self.fine = self.NPF // NP
-            self.phases += ["dq pass", "reverse scan", "dkv pass"]
+                                                    True)
+            self.fine = self.NPF // self.NPD
+            self.phases += ["save states", "dq pass", "reverse scan", "dkv pass"]
             NPF = self.NPF
+            self.S_save = torch.empty((B, H, w.P, dk, dv), **f32)
             self.S_fine = torch.empty((B, H, NPF, dk, dv), **f32)
             self.dSloc = torch.empty((B, H, NPF, dk, dv), **f32)
             self.logG_b = torch.empty((B, H, NPF, dk), **f32)
@@ -277,20 +341,22 @@ class Step:
         if not w.backward:
             return
         f = self.n_fwd
-        la.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_recv, NP, self.fine,
-                          w.chunk, dq=self.grads[0], qdq=self.qdq, S_fine=self.S_fine,
-                          dSloc=self.dSloc, log_gamma=self.logG_b, status=self.status)
+        la.la_seg_gather_states(self.S_recv, self.m, dst=self.S_save)
         rec(f + 1)
+        la.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_save, self.NPD,
+                          self.fine, w.chunk, dq=self.grads[0], qdq=self.qdq, S_fine=self.S_fine,
+                          dSloc=self.dSloc, log_gamma=self.logG_b, status=self.status)
+        rec(f + 2)
         NPF = self.NPF
         la._check(la.lib().la_seg_scan(la._ptr(self.dSloc), la._ptr(self.logG_b), None, BH, NPF,
                                        w.dk, w.dv, 1, la._ptr(self.dX), la._ptr(self.dS0),
                                        la._ptr(self.S_fine), None, la._ptr(self.carry),
                                        la._ptr(self.status), la._stream(None)), "la_seg_scan")
-        rec(f + 2)
+        rec(f + 3)
         la.la_seg_dkv_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_fine, None, self.dX,
                            self.qdq, NPF, w.chunk, carry=self.carry, out=self.grads[1:],
                            status=self.status)
-        rec(f + 3)
+        rec(f + 4)
 
     def phase_ms(self):
         ev = self.events
@@ -332,11 +398,13 @@ class Step:
             ab = {"local pass": th * (3 * w.dk + 2 * w.dv) * e + st + lg, "state scan": scan,
                   "correction pass": th * (2 * w.dk + 2 * w.dv) * e + st}
         if w.backward:
+            sts = w.B * w.H * w.P * w.dk * w.dv * 4
             stf = w.B * w.H * self.NPF * w.dk * w.dv * 4
             lgf = w.B * w.H * self.NPF * w.dk * 4
+            ab["save states"] = 2 * sts
             # reads q, k, v, dO, log_g and the received states; writes dq, S_fine, dSloc and
             # log_gamma (the fp32 q . dq hand-over to the dkv pass is not counted)
-            ab["dq pass"] = th * (3 * w.dk + 2 * w.dv + w.dk) * e + st + 2 * stf + lgf
+            ab["dq pass"] = th * (3 * w.dk + 2 * w.dv + w.dk) * e + sts + 2 * stf + lgf
             carry = w.B * w.H * self.NPF * w.dk * 4
             # reverse scan: the parts' gradient states in, their end-state gradients out, and the
             # dlog_g carries (end states read, one float per part and key dim written)
@@ -360,73 +428,73 @@ class Step:
         else:
             fl = {"local pass": th * (intra + 2 * dd), "state scan": 0, "correction pass": th * dd}
         if w.backward:
+            fl["save states"] = 0
             fl["dq pass"] = th * (2 * C * dv + 2 * C * dk + 3 * dd)
             fl["reverse scan"] = 0
             fl["dkv pass"] = th * (3 * dd + 2 * C * (3 * dk + 2 * dv))
         return fl
 
 
-def bench_ours(args, rank, world, device):
-    from sequence_linear_attention_chunked_b200 import la_seg
-    w = WORKLOADS[args.workload]
-    x = make_inputs(w, device)
-    step = Step(w, x, args.schedule, device)
+SCHEDULE_CODES = {"auto": 0, "two": 1, "three": 2, "single": 3, "overlap": 4}
 
-    # The per-step composition must reproduce the public entry point bit for bit.
-    sched = {"auto": la_seg.SCHED_AUTO, "two": la_seg.SCHED_TWO_PASS,
-             "three": la_seg.SCHED_THREE_PHASE, "single": la_seg.SCHED_SINGLE_PASS,
-             "overlap": la_seg.SCHED_OVERLAP}[args.schedule]
-    ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk,
-                          la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16, False, device)
-    o_api, Sf_api, _ = la_seg.la_seg_forward(x["q"], x["k"], x["v"], x["log_g"], None, w.P,
-                                             w.chunk, sched, ws=ws)
-    la_seg.la_seg_check_status(ws)
+
+def check_same_bits(pub: Public, step: Step):
+    """The composition must reproduce the public calls bit for bit."""
+    w = pub.w
+    pairs = [("o", pub.o, step.o), ("S_final", pub.S_final, step.S_final)]
+    if w.backward:
+        pairs += [("S_recv_save", pub.S_save, step.S_save)]
+        pairs += [(n, a, b) for n, a, b in zip(("dq", "dk", "dv", "dlog_g"), pub.grads[:4], step.grads)]
+        pairs += [("dS0", pub.grads[4], step.dS0)]
+    bad = [n for n, a, b in pairs if not torch.equal(a, b)]
+    if bad:
+        raise RuntimeError(f"per-step composition differs from the public calls in {bad}")
+
+
+def time_workload(w: Workload, args, device, world, steps: int, warmup: int):
+    """Times the public calls (the throughput) and the per-step composition (the phases) on
+    the workload, each step after an untimed L2 flush; returns the pieces of the JSON line."""
+    x = make_inputs(w, device)
+    pub = Public(w, x, SCHEDULE_CODES[args.schedule], device)
+    step = Step(w, x, args.schedule, device)
+    pub.run(record=False)
+    pub.check_status()
     step.run(record=False)
     torch.cuda.synchronize()
-    if not (torch.equal(o_api, step.o) and torch.equal(Sf_api, step.S_final)):
-        raise RuntimeError("per-step composition differs from la_seg_forward")
-    del o_api, Sf_api
-    if w.backward:
-        wsb = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk,
-                               la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16, True, device)
-        g_api = la_seg.la_seg_backward(x["q"], x["k"], x["v"], x["log_g"], x["dO"], None, None, None,
-                                       w.P, w.chunk, want_dS0=True, ws=wsb)
-        la_seg.la_seg_check_status(wsb)
-        if not (all(torch.equal(a, b) for a, b in zip(g_api[:4], step.grads))
-                and torch.equal(g_api[4], step.dS0)):
-            raise RuntimeError("per-step composition differs from la_seg_backward")
-        del g_api, wsb
-    torch.cuda.synchronize()
+    check_same_bits(pub, step)
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} after the check run")
-
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
+        flush.zero_()
+        pub.run()
         flush.zero_()
         step.run()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms, phase_ms, overlap = [], [], []
+    pub_ms, step_ms, phase_ms, overlap = [], [], [], []
     sampler = ClockSampler(device.index)
     with sampler:
-        for _ in range(args.steps):
+        for _ in range(steps):
+            flush.zero_()
+            pub.run()
             flush.zero_()
             step.run()
             torch.cuda.synchronize()  # read this step's events before the next one reuses them
-            pm = step.phase_ms()
-            phase_ms.append(pm)
+            pub_ms.append(pub.ms())
+            phase_ms.append(step.phase_ms())
             step_ms.append(step.events[0].elapsed_time(step.events[-1]))
             if args.schedule == "overlap":
                 overlap.append(step.overlap_fraction())
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = max_over_ranks(sum(step_ms), world, device)
-    value = job_throughput(w.B * w.L, world, args.steps, total_ms)
+    total_ms = max_over_ranks(sum(pub_ms), world, device)
+    comp_ms = max_over_ranks(sum(step_ms), world, device)
+    value = job_throughput(w.B * w.L, world, steps, total_ms)
 
-    # phases and the dominant kernel's roofline
     mean_phase = [statistics.fmean(p[i] for p in phase_ms) for i in range(len(step.phases))]
     ab = step.algorithmic_bytes()
     fl = step.flops()
@@ -434,7 +502,6 @@ def bench_ours(args, rank, world, device):
     dom = max(range(len(step.phases)), key=lambda i: mean_phase[i])
     dname = step.phases[dom]
     achieved = ab[dname] / (mean_phase[dom] / 1e3) / 1e9
-    kernel_key = Step.KERNEL_KEYS[dname]
     phases = {}
     for i, name in enumerate(step.phases):
         sec = mean_phase[i] / 1e3
@@ -446,27 +513,65 @@ def bench_ours(args, rank, world, device):
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peak_src} hbm_gbs (burst copy)",
                 "algorithmic_bytes_per_launch": ab[dname],
-                "traffic": ncu_traffic(kernel_key, w.name)}
+                "traffic": ncu_traffic(Step.KERNEL_KEYS[dname], w.name)}
+    out = dict(x=x, pub=pub, step=step, value=value, total_ms=total_ms, comp_ms=comp_ms,
+               pub_ms=pub_ms, phases=phases, roofline=roofline, sampler=sampler,
+               mean_phase=mean_phase)
+    if overlap:  # events on both streams: the scan's window and the local pass's
+        out["overlap"] = {"scan_window_covered": round(statistics.median(overlap), 4),
+                          "min": round(min(overlap), 4),
+                          "scan_ms": round(mean_phase[step.phases.index("state scan")], 5),
+                          "local_pass_ms": round(mean_phase[step.phases.index("local pass")], 5)}
+    return out
 
-    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+
+def bench_ours(args, rank, world, device):
+    w = WORKLOADS[args.workload]
+    r = time_workload(w, args, device, world, args.steps, args.warmup)
+    step, pub = r["step"], r["pub"]
+    line = {"metric": METRIC, "value": round(r["value"], 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(total_ms / args.steps, 5), "ms_per_step_median": round(statistics.median(step_ms), 5),
+            "ms_per_step": round(r["total_ms"] / args.steps, 5),
+            "ms_per_step_median": round(statistics.median(r["pub_ms"]), 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w.describe(), "B": w.B, "H": w.H, "L": w.L, "d": w.dk, "P": w.P,
                        "chunk": w.chunk, "subsegments": step.NP, "schedule": args.schedule,
+                       "timed": "la_seg_forward(P, saving the received states)"
+                                + (" + la_seg_backward(P, reusing them)" if w.backward else ""),
                        "l2": "flushed before every step (256 MiB write, untimed)",
                        "parallelism": f"replicas x{world}"},
-            "phases": phases, "roofline": roofline,
-            "gpu_launches": step.launches_per_step * args.steps,
-            "clocks": sampler.summary()}
-    if overlap:  # events on both streams: the scan's window and the local pass's
-        line["overlap"] = {"scan_window_covered": round(statistics.median(overlap), 4),
-                           "min": round(min(overlap), 4),
-                           "scan_ms": round(mean_phase[step.phases.index("state scan")], 5),
-                           "local_pass_ms": round(mean_phase[step.phases.index("local pass")], 5)}
+            "composed": {"ms_per_step": round(r["comp_ms"] / args.steps, 5),
+                         "vs_public": round(r["comp_ms"] / r["total_ms"], 4),
+                         "what": "the same kernels through the per-step entry points, bit-identical "
+                                 "results; phases and roofline come from it"},
+            "phases": r["phases"], "roofline": r["roofline"],
+            "gpu_launches": pub.launches_per_step * args.steps,
+            "clocks": r["sampler"].summary()}
+    if "overlap" in r:
+        line["overlap"] = r["overlap"]
+    x = r["x"]
     if not args.no_e2e:
         line["e2e"] = bench_e2e(args, w, x, device, world)
+    del r, x, step, pub
+    torch.cuda.empty_cache()
+    configs = [c for c in args.configs.split(",") if c and c != "none" and c != w.name]
+    if configs:
+        line["configs"] = {}
+    for name in configs:
+        cw = WORKLOADS[name]
+        rc = time_workload(cw, args, device, world, args.config_steps, 3)
+        entry = {"workload": cw.describe(), "tokens_per_s": round(rc["value"], 1),
+                 "ms_per_step": round(rc["total_ms"] / args.config_steps, 5),
+                 "composed_ms_per_step": round(rc["comp_ms"] / args.config_steps, 5),
+                 "steps": args.config_steps, "phases": rc["phases"],
+                 "roofline": {k: rc["roofline"][k] for k in ("kernel", "achieved", "frac", "unit")},
+                 "clocks": rc["sampler"].summary()}
+        if "state scan" in rc["phases"]:
+            entry["scan"] = rc["phases"]["state scan"]
+        line["configs"][name] = entry
+        del rc
+        torch.cuda.empty_cache()
     return line
 
 
@@ -632,6 +737,10 @@ def main():
     ap.add_argument("--schedule", default="auto",
                     choices=["auto", "two", "three", "single", "overlap"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--configs", default="C1,C2,C3",
+                    help="forward workloads timed after the headline into the line's 'configs' "
+                         "('none' to skip)")
+    ap.add_argument("--config-steps", type=int, default=10)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
