@@ -104,12 +104,16 @@ FwdLayout fwd_layout(const la::Split &s, int dk, int dv) {
 }
 
 // Fine parts per segment for the backward's reverse sweep: the largest power-of-two split
-// into parts of at most 1024 tokens (whole chunks).  dlog_g is re-anchored on the exact carry
-// rowsum(S_end . dX) at every part boundary, which keeps the bf16 rounding of the per-token
-// terms it sums from accumulating over long segments.
+// into parts of at most kMaxPartTokens tokens (whole chunks).  dlog_g is re-anchored on the
+// exact carry rowsum(S_end . dX) at every part boundary, which keeps the rounding of the
+// per-token terms it sums from accumulating over long segments.  With the sweeps' shared bf16
+// operands the measured dlog_g error is <= 0.67% of max at 1024-token parts, <= 0.86% at 2048
+// and <= 1.06% at 4096 (bound 2%); 2048 halves the reverse scan and the part-boundary state
+// stores of 1024 and keeps a 2.3x margin.
+constexpr long long kMaxPartTokens = 2048;
 int fine_factor(long long T, int chunk) {
     int r = 1;
-    while (T / r > 1024 && T % (2LL * r) == 0 && (T / (2LL * r)) % chunk == 0) r *= 2;
+    while (T / r > kMaxPartTokens && T % (2LL * r) == 0 && (T / (2LL * r)) % chunk == 0) r *= 2;
     return r;
 }
 
