@@ -11,9 +11,11 @@ every step; each step is bracketed by CUDA events.  The same kernels are also ru
 per-step entry points with events between the phases (checked bit for bit against the public
 calls), which gives each kernel's time and roofline.  After the headline workload the forward
 workloads C1-C3 are timed the same way into the line's "configs".
-With N > 1 ranks (torchrun), every rank runs its own replica of the workload on its own GPU:
-the path has no cross-rank exchange, so there is no collective on the data path ("weak"
-scaling); the max over ranks of the device time is reported.
+With N > 1 ranks (torchrun) the default is sequence parallelism across the ranks (sp.py, the
+pages' setting): rank r holds block r of a global sequence of N x L tokens and the ranks
+exchange their (log Gamma, S) pairs over NCCL between the passes ("weak" scaling: the tokens per
+rank are fixed); --mode replicas runs independent copies instead.  The max over ranks of the
+device time is reported.
 """
 from __future__ import annotations
 
@@ -575,6 +577,71 @@ def bench_ours(args, rank, world, device):
     return line
 
 
+def bench_sp(args, rank, world, device):
+    """Sequence parallelism across the ranks (sp.py): rank r holds block r of every sequence of a
+    global sequence of world x L tokens (the workload's L per rank, ZeCO's fixed tokens per
+    device), runs the forward and backward passes on it, and the ranks exchange their (log Gamma,
+    S) pairs over NCCL (all-gather, or the tree All-Scan).  The job time is the slowest rank's."""
+    from sequence_linear_attention_chunked_b200 import sp
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w.with_(seed=w.seed + rank), device)
+    steps = sp.LibrarySteps()
+
+    def one(check=False):
+        o, Sf, saved = sp.sp_forward(x["q"], x["k"], x["v"], x["log_g"], None, w.P, w.chunk,
+                                     method=args.all_scan, steps=steps, check=check)
+        if w.backward:
+            sp.sp_backward(x["q"], x["k"], x["v"], x["log_g"], x["dO"], saved, None, w.P, w.chunk,
+                           method=args.all_scan, steps=steps, check=check)
+
+    one(check=True)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    dist.barrier()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ms = []
+    sampler = ClockSampler(device.index)
+    with sampler:
+        for _ in range(args.steps):
+            flush.zero_()
+            dist.barrier()
+            ev[0].record()
+            one()
+            ev[1].record()
+            torch.cuda.synchronize()
+            ms.append(ev[0].elapsed_time(ev[1]))
+    steps.check()
+    dist.barrier()
+    total_ms = max_over_ranks(sum(ms), world, device)
+    value = job_throughput(w.B * w.L, world, args.steps, total_ms)
+    # the kernels' phases and roofline: the same workload through the per-step entry points on
+    # every rank's own block (one GPU's work)
+    r = time_workload(w, args, device, world, max(3, min(args.steps, 10)), 3)
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+            "ms_per_step_median": round(statistics.median(ms), 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.describe() + f" per rank; global sequence {world} x {w.L}",
+                       "B": w.B, "H": w.H, "L_per_rank": w.L, "L_global": world * w.L, "d": w.dk,
+                       "P_per_rank": w.P, "chunk": w.chunk, "all_scan": args.all_scan,
+                       "timed": "sp_forward" + (" + sp_backward" if w.backward else "") +
+                                " (sequence parallel across the ranks, NCCL)",
+                       "l2": "flushed before every step (256 MiB write, untimed)",
+                       "parallelism": f"sp{world}"},
+            "phases": r["phases"], "roofline": r["roofline"],
+            # per step: state pass, block total (scan, log-decay sum), All-Scan (one rank scan, or
+            # a combine per tree round), the scan from the received state, output pass, state
+            # gather; dq sweep, block total (scan, log-decay sum), All-Scan, reverse scan, dk/dv
+            "gpu_launches": ((7 + (6 if w.backward else 0)) + (0 if args.all_scan == "gather" else
+                             (1 + int(w.backward)) * (max(1, (world - 1).bit_length()) - 1))) * args.steps,
+            "clocks": sampler.summary()}
+    return line
+
+
 def bench_e2e(args, w, x, device, world):
     """Same metric through the public entry points with host buffers: per step, pinned host ->
     device copies of the inputs (q, k, v, log_g, and dO for fwd+bwd), la_seg_forward (saving
@@ -741,6 +808,10 @@ def main():
                     help="forward workloads timed after the headline into the line's 'configs' "
                          "('none' to skip)")
     ap.add_argument("--config-steps", type=int, default=10)
+    ap.add_argument("--mode", choices=["auto", "replicas", "sp"], default="auto",
+                    help="N > 1: sequence parallel across the ranks (sp, the default) or "
+                         "independent replicas")
+    ap.add_argument("--all-scan", choices=["gather", "tree"], default="gather")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -765,14 +836,22 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
+    mode = args.mode if args.mode != "auto" else ("sp" if world > 1 else "replicas")
+    if mode == "sp" and world == 1:  # the orchestration's collectives on a one-rank group
+        import socket
+        with socket.socket() as sock:
+            sock.bind(("127.0.0.1", 0))
+            port = sock.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, device_id=device)
     try:
-        line = bench_ours(args, rank, world, device)
+        line = bench_sp(args, rank, world, device) if mode == "sp" else bench_ours(args, rank, world, device)
         if rank == 0 and world == 1 and not args.no_cpu:
             line["cpu_baseline"] = cpu_sample(w, args.cpu_seconds)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
-        if world > 1:
+        if dist.is_initialized():
             dist.destroy_process_group()
 
 

@@ -276,6 +276,39 @@ LA_API la_status la_seg_dkv_pass(const void *q, const void *k, const void *v, co
 LA_API la_status la_seg_gather_states(const float *src, int BH, int NP, int m, int dk, int dv,
                                       float *dst, void *cuda_stream);
 
+/* ---- The All-Scan between devices ----------------------------------------------------
+ * For a sequence whose consecutive blocks live on N ranks (ZeCO's sequence parallelism; the
+ * review's "key machinery" and the referee's Alg. 2 comment): each rank reduces its block to one
+ * pair (log Gamma_r, S_r) -- la_seg_scan from zero over its sub-segments for S_r and
+ * la_seg_log_gamma_total for log Gamma_r --, the pairs of all ranks are brought into local HBM
+ * (an all-gather, or log2 N point-to-point rounds combined with la_seg_combine), and
+ * la_seg_rank_scan gives the state the rank's block receives.  The backward runs the same steps
+ * with reverse = 1 over the gradient states.  sp.py drives them over torch.distributed. */
+
+/* log_gamma_total[bh][i] = sum over p < NP of log_gamma[bh][p][i] (fp32; [BH, NP, dk] ->
+ * [BH, dk]): the log-decay of NP consecutive segments taken together. */
+LA_API la_status la_seg_log_gamma_total(const float *log_gamma, int BH, int NP, int dk,
+                                        float *log_gamma_total, void *cuda_stream);
+
+/* The exclusive scan across ranks at position `rank`, element-wise over (bh, i, j):
+ *   reverse == 0:  acc = init;  for r = 0 .. rank-1:      acc = exp(log_gamma_ranks[r][bh][i]) acc + S_ranks[r][bh]
+ *   reverse != 0:  acc = init;  for r = N-1 .. rank+1:    (the same update)
+ *   S_in[bh] = acc;  total (nullable) = the update continued over every rank.
+ * S_ranks fp32 [N, BH, dk, dv] and log_gamma_ranks fp32 [N, BH, dk] in rank order (the layout an
+ * all-gather of the ranks' pairs produces); init, S_in, total fp32 [BH, dk, dv], init nullable
+ * (zero).  dv % 4 == 0; 0 <= rank < N. */
+LA_API la_status la_seg_rank_scan(const float *S_ranks, const float *log_gamma_ranks,
+                                  const float *init, int N, int BH, int dk, int dv, int rank,
+                                  int reverse, float *S_in, float *total, void *cuda_stream);
+
+/* Two consecutive spans a then b taken together (one step of a tree All-Scan):
+ * log_gamma_out = log_gamma_a + log_gamma_b (fp32 [BH, dk]) and
+ * S_out = exp(log_gamma_b) S_a + S_b (fp32 [BH, dk, dv], dv % 4 == 0).  S_out may be S_b;
+ * log_gamma_out must differ from both inputs. */
+LA_API la_status la_seg_combine(const float *log_gamma_a, const float *S_a,
+                                const float *log_gamma_b, const float *S_b, int BH, int dk,
+                                int dv, float *log_gamma_out, float *S_out, void *cuda_stream);
+
 /* Number of parts la_seg_backward's gradient-state, reverse-scan and dk/dv steps run over
  * (reuse != 0: the caller passes S_recv_saved and no dS_final), or 0 for rejected sizes. */
 LA_API int la_seg_backward_parts(int B, int H, long long L, int dk, int dv, int P, int chunk,

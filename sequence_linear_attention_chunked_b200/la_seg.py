@@ -27,7 +27,8 @@ EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_s
             "la_seg_subsegments", "la_seg_check_status", "la_last_error_detail",
             "la_seg_forward_noalloc", "la_seg_dstate_pass", "la_seg_dq_pass", "la_seg_dkv_pass",
             "la_seg_backward_parts", "la_seg_chain_pass", "la_seg_chain_reset",
-            "la_seg_noalloc_check_status", "la_seg_gather_states")
+            "la_seg_noalloc_check_status", "la_seg_gather_states", "la_seg_log_gamma_total",
+            "la_seg_rank_scan", "la_seg_combine")
 
 _lib = None
 
@@ -72,6 +73,12 @@ def lib():
         L.la_seg_forward_noalloc.argtypes = [P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
                                              i32, P, P, P, i32, P]
         L.la_seg_forward_noalloc.restype = i32
+        L.la_seg_log_gamma_total.argtypes = [P, i32, i32, i32, P, P]
+        L.la_seg_log_gamma_total.restype = i32
+        L.la_seg_rank_scan.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P, P, P]
+        L.la_seg_rank_scan.restype = i32
+        L.la_seg_combine.argtypes = [P, P, P, P, i32, i32, i32, P, P, P]
+        L.la_seg_combine.restype = i32
         L.la_seg_gather_states.argtypes = [P, i32, i32, i32, i32, i32, P, P]
         L.la_seg_gather_states.restype = i32
         L.la_seg_noalloc_check_status.argtypes = [P]
@@ -362,6 +369,57 @@ def la_seg_gather_states(src, m, *, dst=None, stream=None):
     _check(lib().la_seg_gather_states(_ptr(src), B * H, NP, m, dk, dv, _ptr(dst), _stream(stream)),
            "la_seg_gather_states")
     return dst
+
+
+def la_seg_log_gamma_total(log_gamma, *, out=None, stream=None):
+    """Sum over the segment axis: fp32 [..., NP, dk] -> [..., dk]."""
+    *lead, NP, dk = log_gamma.shape
+    BH = 1
+    for x in lead:
+        BH *= x
+    _need(log_gamma, "log_gamma", torch.float32, None, log_gamma.device)
+    out = torch.empty((*lead, dk), dtype=torch.float32, device=log_gamma.device) if out is None else out
+    _check(lib().la_seg_log_gamma_total(_ptr(log_gamma), BH, NP, dk, _ptr(out), _stream(stream)),
+           "la_seg_log_gamma_total")
+    return out
+
+
+def la_seg_rank_scan(S_ranks, log_gamma_ranks, rank, init=None, reverse=False, *, S_in=None,
+                     total=None, want_total=True, stream=None):
+    """S_in (and the total) of the exclusive scan across ranks: S_ranks fp32 [N, *lead, dk, dv],
+    log_gamma_ranks fp32 [N, *lead, dk] in rank order."""
+    N = S_ranks.shape[0]
+    dk, dv = S_ranks.shape[-2:]
+    lead = S_ranks.shape[1:-2]
+    BH = 1
+    for x in lead:
+        BH *= x
+    dev = S_ranks.device
+    _need(S_ranks, "S_ranks", torch.float32, None, dev)
+    _need(log_gamma_ranks, "log_gamma_ranks", torch.float32, (N, *lead, dk), dev)
+    _need(init, "init", torch.float32, (*lead, dk, dv), dev)
+    S_in = torch.empty((*lead, dk, dv), dtype=torch.float32, device=dev) if S_in is None else S_in
+    if want_total and total is None:
+        total = torch.empty((*lead, dk, dv), dtype=torch.float32, device=dev)
+    _check(lib().la_seg_rank_scan(_ptr(S_ranks), _ptr(log_gamma_ranks), _ptr(init), N, BH, dk, dv,
+                                  int(rank), int(bool(reverse)), _ptr(S_in),
+                                  _ptr(total if want_total else None), _stream(stream)),
+           "la_seg_rank_scan")
+    return S_in, (total if want_total else None)
+
+
+def la_seg_combine(lg_a, S_a, lg_b, S_b, *, lg_out=None, S_out=None, stream=None):
+    """(lg_a, S_a) followed by (lg_b, S_b): (lg_a + lg_b, exp(lg_b) S_a + S_b)."""
+    dk, dv = S_a.shape[-2:]
+    BH = S_a.numel() // (dk * dv)
+    dev = S_a.device
+    for t, n in ((lg_a, "lg_a"), (S_a, "S_a"), (lg_b, "lg_b"), (S_b, "S_b")):
+        _need(t, n, torch.float32, None, dev)
+    lg_out = torch.empty_like(lg_a) if lg_out is None else lg_out
+    S_out = torch.empty_like(S_a) if S_out is None else S_out
+    _check(lib().la_seg_combine(_ptr(lg_a), _ptr(S_a), _ptr(lg_b), _ptr(S_b), BH, dk, dv,
+                                _ptr(lg_out), _ptr(S_out), _stream(stream)), "la_seg_combine")
+    return lg_out, S_out
 
 
 def chain_buffers(B, H, dk, dv, device="cuda"):
