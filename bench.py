@@ -63,13 +63,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def csrc_digest() -> str:
-    """Digest of the kernel sources' code: comments and whitespace are left out, so that a
-    counter recorded for a kernel stays valid across edits of its comments only."""
+# The sources each kernel's code is built from: a counter recorded for a kernel stays valid
+# while these are unchanged (comments and whitespace aside).
+KERNEL_SOURCES = {
+    "dkv_pass": ["tc_bwd.cu"], "dq_pass": ["tc_dq.cu"], "state_pass": ["tc_pass.cu"],
+    "output_pass": ["tc_pass.cu"], "local_pass": ["tc_pass.cu"], "correct_pass": ["tc_pass.cu"],
+    "chain_kernel": ["tc_pass.cu"], "scan": ["scan.cu"],
+}
+SHARED_SOURCES = ["common.cuh", "internal.h", "tc_common.cuh", "sm100.cuh"]
+
+
+def csrc_digest(kernel=None) -> str:
+    """Digest of the code (comments and whitespace left out) of `kernel`'s sources and the
+    headers every kernel shares, or of every source when kernel is None."""
     import re
     d = os.path.join(ROOT, "sequence_linear_attention_chunked_b200", "csrc")
+    names = sorted(os.listdir(d)) if kernel is None else sorted(
+        KERNEL_SOURCES.get(kernel, []) + SHARED_SOURCES)
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
+    for name in names:
         with open(os.path.join(d, name), encoding="utf-8") as f:
             src = f.read()
         code = re.sub(r"//[^\n]*|/\*.*?\*/", " ", src, flags=re.S)
@@ -85,7 +97,7 @@ def ncu_traffic(kernel: str, workload: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{kernel}@{workload}")
-    if not e or e.get("csrc_digest") != csrc_digest():
+    if not e or e.get("csrc_digest") != csrc_digest(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -164,27 +176,33 @@ def dtype_code(la_seg, w):
 
 class Public:
     """The calls a user of the library makes for the workload, through the C ABI on the current
-    stream: la_seg_forward saving the received states of its P segments, then (fwd+bwd
-    workloads) la_seg_backward reusing them.  This is what the headline times."""
+    stream: for a forward-only workload la_seg_forward over its P segments; for fwd+bwd the
+    training pair, la_seg_train_forward over the P segments saving the received states at the
+    library's own split, then la_seg_train_backward reusing them.  This is what the headline
+    times."""
 
     def __init__(self, w: Workload, x, schedule: int, device):
         from sequence_linear_attention_chunked_b200 import la_seg
         self.la, self.w, self.x, self.schedule = la_seg, w, x, schedule
         dt = dtype_code(la_seg, w)
         f32 = dict(dtype=torch.float32, device=device)
-        self.ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device)
         self.o = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype, device=device)
         self.S_final = torch.empty((w.B, w.H, w.dk, w.dv), **f32)
-        self.S_save = torch.empty((w.B, w.H, w.P, w.dk, w.dv), **f32) if w.backward else None
+        self.S_save = None
         if w.backward:
-            self.wsb = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, device)
+            NS = la_seg.lib().la_seg_train_saved_states(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt)
+            self.ws = la_seg.train_workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device)
+            self.wsb = la_seg.train_workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, device)
+            self.S_save = torch.empty((w.B, w.H, NS, w.dk, w.dv), **f32)
             self.grads = (torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
                           torch.empty_like(x["log_g"]), torch.empty_like(self.S_final))
+        else:
+            self.ws = la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device)
         self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         # kernels of this library per step: state pass, exact-path states, scan, output pass,
-        # exact-path outputs, state gather; dq sweep, exact-path dq, reverse scan, dk/dv sweep,
-        # exact-path dk/dv (the status / flag memsets are not counted)
-        self.launches_per_step = 5 + (6 if w.backward else 0)
+        # exact-path outputs; dq sweep, exact-path dq, reverse scan, dk/dv sweep, exact-path
+        # dk/dv (the status / flag memsets are not counted)
+        self.launches_per_step = 5 + (5 if w.backward else 0)
 
     def run(self, record=True):
         la, w, x, P = self.la, self.w, self.x, self.la._ptr
@@ -192,16 +210,17 @@ class Public:
         dt = dtype_code(la, w)
         if record:
             self.ev[0].record()
-        la._check(la.lib().la_seg_forward(
+        fwd = la.lib().la_seg_train_forward if w.backward else la.lib().la_seg_forward
+        la._check(fwd(
             P(x["q"]), P(x["k"]), P(x["v"]), P(x["log_g"]), None, w.B, w.H, w.L, w.dk, w.dv, w.P,
             w.chunk, dt, P(self.o), P(self.S_final), P(self.S_save), self.schedule, P(self.ws),
-            self.ws.numel(), st), "la_seg_forward")
+            self.ws.numel(), st), "forward")
         if w.backward:
             g = self.grads
-            la._check(la.lib().la_seg_backward(
+            la._check(la.lib().la_seg_train_backward(
                 P(x["q"]), P(x["k"]), P(x["v"]), P(x["log_g"]), None, P(self.S_save), P(x["dO"]),
                 None, w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, P(g[0]), P(g[1]), P(g[2]),
-                P(g[3]), P(g[4]), P(self.wsb), self.wsb.numel(), st), "la_seg_backward")
+                P(g[3]), P(g[4]), P(self.wsb), self.wsb.numel(), st), "la_seg_train_backward")
         if record:
             self.ev[1].record()
 
@@ -219,14 +238,14 @@ class Step:
     events between the phases on the launching stream, so that each kernel can be timed and
     set against its roofline.  It reproduces the public calls' splits: the forward's passes over
     the library's sub-segments (state pass, state scan, output pass -- or the other schedules'
-    passes), the gather of the P received states the forward saves; the backward, which reuses
-    them, over whole segments: dq pass (which also forms the gradient states of the fine parts),
-    reverse scan, dk/dv/dlog_g pass.  bench_ours checks that both give the same bits."""
+    passes); the backward, which reuses the received states the training forward saved at the
+    same split: dq pass (which also forms the gradient states of the fine parts), reverse scan,
+    dk/dv/dlog_g pass.  bench_ours checks that both give the same bits."""
 
     KERNEL_KEYS = {"chain reset": "chain_reset", "single pass": "chain_kernel",
                    "state pass": "state_pass", "output pass": "output_pass",
                    "local pass": "local_pass", "correction pass": "correct_pass",
-                   "state scan": "scan", "save states": "gather", "dq pass": "dq_pass",
+                   "state scan": "scan", "dq pass": "dq_pass",
                    "reverse scan": "scan", "dkv pass": "dkv_pass"}
 
     def __init__(self, w: Workload, x, schedule: str, device):
@@ -260,14 +279,13 @@ class Step:
             self.phases = ["state pass", "state scan", "output pass"]
         self.n_fwd = len(self.phases)
         if w.backward:
-            # la_seg_backward with saved states: whole API segments, each cut into fine parts
-            self.NPD = w.P
-            self.NPF = la_seg.la_seg_backward_parts(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt,
+            # la_seg_train_backward: the library's sub-segments, each cut into fine parts
+            self.NPD = NP
+            self.NPF = la_seg.la_seg_backward_parts(w.B, w.H, w.L, w.dk, w.dv, NP, w.chunk, dt,
                                                     True)
             self.fine = self.NPF // self.NPD
-            self.phases += ["save states", "dq pass", "reverse scan", "dkv pass"]
+            self.phases += ["dq pass", "reverse scan", "dkv pass"]
             NPF = self.NPF
-            self.S_save = torch.empty((B, H, w.P, dk, dv), **f32)
             self.S_fine = torch.empty((B, H, NPF, dk, dv), **f32)
             self.dSloc = torch.empty((B, H, NPF, dk, dv), **f32)
             self.logG_b = torch.empty((B, H, NPF, dk), **f32)
@@ -342,10 +360,8 @@ class Step:
             rec(3)
         if not w.backward:
             return
-        f = self.n_fwd
-        la.la_seg_gather_states(self.S_recv, self.m, dst=self.S_save)
-        rec(f + 1)
-        la.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_save, self.NPD,
+        f = self.n_fwd - 1
+        la.la_seg_dq_pass(x["q"], x["k"], x["v"], x["log_g"], x["dO"], self.S_recv, self.NPD,
                           self.fine, w.chunk, dq=self.grads[0], qdq=self.qdq, S_fine=self.S_fine,
                           dSloc=self.dSloc, log_gamma=self.logG_b, status=self.status)
         rec(f + 2)
@@ -400,10 +416,9 @@ class Step:
             ab = {"local pass": th * (3 * w.dk + 2 * w.dv) * e + st + lg, "state scan": scan,
                   "correction pass": th * (2 * w.dk + 2 * w.dv) * e + st}
         if w.backward:
-            sts = w.B * w.H * w.P * w.dk * w.dv * 4
+            sts = st
             stf = w.B * w.H * self.NPF * w.dk * w.dv * 4
             lgf = w.B * w.H * self.NPF * w.dk * 4
-            ab["save states"] = 2 * sts
             # reads q, k, v, dO, log_g and the received states; writes dq, S_fine, dSloc and
             # log_gamma (the fp32 q . dq hand-over to the dkv pass is not counted)
             ab["dq pass"] = th * (3 * w.dk + 2 * w.dv + w.dk) * e + sts + 2 * stf + lgf
@@ -430,7 +445,6 @@ class Step:
         else:
             fl = {"local pass": th * (intra + 2 * dd), "state scan": 0, "correction pass": th * dd}
         if w.backward:
-            fl["save states"] = 0
             fl["dq pass"] = th * (2 * C * dv + 2 * C * dk + 3 * dd)
             fl["reverse scan"] = 0
             fl["dkv pass"] = th * (3 * dd + 2 * C * (3 * dk + 2 * dv))
@@ -445,7 +459,7 @@ def check_same_bits(pub: Public, step: Step):
     w = pub.w
     pairs = [("o", pub.o, step.o), ("S_final", pub.S_final, step.S_final)]
     if w.backward:
-        pairs += [("S_recv_save", pub.S_save, step.S_save)]
+        pairs += [("saved states", pub.S_save, step.S_recv)]
         pairs += [(n, a, b) for n, a, b in zip(("dq", "dk", "dv", "dlog_g"), pub.grads[:4], step.grads)]
         pairs += [("dS0", pub.grads[4], step.dS0)]
     bad = [n for n, a, b in pairs if not torch.equal(a, b)]
@@ -477,15 +491,24 @@ def time_workload(w: Workload, args, device, world, steps: int, warmup: int):
         dist.barrier()
     torch.cuda.synchronize()
     pub_ms, step_ms, phase_ms, overlap = [], [], [], []
+    # the headline steps first, on their own (the composition's extra work would heat the chip
+    # between them), with the SM clock sampled while they run
     sampler = ClockSampler(device.index)
     with sampler:
         for _ in range(steps):
             flush.zero_()
             pub.run()
-            flush.zero_()
-            step.run()
             torch.cuda.synchronize()  # read this step's events before the next one reuses them
             pub_ms.append(pub.ms())
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    comp_sampler = ClockSampler(device.index)
+    with comp_sampler:
+        for _ in range(steps):  # then the composition, for the phases
+            flush.zero_()
+            step.run()
+            torch.cuda.synchronize()
             phase_ms.append(step.phase_ms())
             step_ms.append(step.events[0].elapsed_time(step.events[-1]))
             if args.schedule == "overlap":
@@ -518,13 +541,20 @@ def time_workload(w: Workload, args, device, world, steps: int, warmup: int):
                 "traffic": ncu_traffic(Step.KERNEL_KEYS[dname], w.name)}
     out = dict(x=x, pub=pub, step=step, value=value, total_ms=total_ms, comp_ms=comp_ms,
                pub_ms=pub_ms, phases=phases, roofline=roofline, sampler=sampler,
-               mean_phase=mean_phase)
+               comp_sampler=comp_sampler, mean_phase=mean_phase)
     if overlap:  # events on both streams: the scan's window and the local pass's
         out["overlap"] = {"scan_window_covered": round(statistics.median(overlap), 4),
                           "min": round(min(overlap), 4),
                           "scan_ms": round(mean_phase[step.phases.index("state scan")], 5),
                           "local_pass_ms": round(mean_phase[step.phases.index("local pass")], 5)}
     return out
+
+
+def _clock_ratio(r):
+    a, b = r["comp_sampler"].summary()["sm_mhz"], r["sampler"].summary()["sm_mhz"]
+    if not a or not b:
+        return None
+    return round((r["comp_ms"] * a) / (r["total_ms"] * b), 4)
 
 
 def bench_ours(args, rank, world, device):
@@ -539,12 +569,17 @@ def bench_ours(args, rank, world, device):
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w.describe(), "B": w.B, "H": w.H, "L": w.L, "d": w.dk, "P": w.P,
                        "chunk": w.chunk, "subsegments": step.NP, "schedule": args.schedule,
-                       "timed": "la_seg_forward(P, saving the received states)"
-                                + (" + la_seg_backward(P, reusing them)" if w.backward else ""),
+                       "timed": ("la_seg_train_forward(P, saving the received states at the "
+                                 "library's split) + la_seg_train_backward(P, reusing them)")
+                                if w.backward else "la_seg_forward(P)",
                        "l2": "flushed before every step (256 MiB write, untimed)",
                        "parallelism": f"replicas x{world}"},
             "composed": {"ms_per_step": round(r["comp_ms"] / args.steps, 5),
                          "vs_public": round(r["comp_ms"] / r["total_ms"], 4),
+                         "sm_mhz": r["comp_sampler"].summary()["sm_mhz"],
+                         # time x median SM clock: the two loops run one after the other, and the
+                         # later one under more of the power cap
+                         "vs_public_at_equal_clock": _clock_ratio(r),
                          "what": "the same kernels through the per-step entry points, bit-identical "
                                  "results; phases and roofline come from it"},
             "phases": r["phases"], "roofline": r["roofline"],
@@ -634,9 +669,9 @@ def bench_sp(args, rank, world, device):
                        "parallelism": f"sp{world}"},
             "phases": r["phases"], "roofline": r["roofline"],
             # per step: state pass, block total (scan, log-decay sum), All-Scan (one rank scan, or
-            # a combine per tree round), the scan from the received state, output pass, state
-            # gather; dq sweep, block total (scan, log-decay sum), All-Scan, reverse scan, dk/dv
-            "gpu_launches": ((7 + (6 if w.backward else 0)) + (0 if args.all_scan == "gather" else
+            # a combine per tree round), the scan from the received state, output pass; dq
+            # sweep, block total (scan, log-decay sum), All-Scan, reverse scan, dk/dv sweep
+            "gpu_launches": ((6 + (6 if w.backward else 0)) + (0 if args.all_scan == "gather" else
                              (1 + int(w.backward)) * (max(1, (world - 1).bit_length()) - 1))) * args.steps,
             "clocks": sampler.summary()}
     return line
@@ -644,8 +679,8 @@ def bench_sp(args, rank, world, device):
 
 def bench_e2e(args, w, x, device, world):
     """Same metric through the public entry points with host buffers: per step, pinned host ->
-    device copies of the inputs (q, k, v, log_g, and dO for fwd+bwd), la_seg_forward (saving
-    the received states), la_seg_backward reusing them, and device -> host copies of the
+    device copies of the inputs (q, k, v, log_g, and dO for fwd+bwd), the headline's calls (the
+    training pair for fwd+bwd), and device -> host copies of the
     results (o and S_final; dq, dk, dv, dlog_g and dS0 for fwd+bwd).  Steps are pipelined over
     three streams with two sets of device buffers, as a serving loop would run them: step i's
     inputs are copied in while step i-1 computes and step i-2's results are copied out (PCIe
@@ -656,15 +691,17 @@ def bench_e2e(args, w, x, device, world):
     host = {n: x[n].cpu().pin_memory() for n in names}
     dt = la_seg.LA_F32 if w.dtype == "f32" else la_seg.LA_BF16
     f32 = dict(dtype=torch.float32, device=device)
-    ws = [la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device) for _ in range(2)]
-    wsb = ([la_seg.workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, device)
+    mkws = la_seg.train_workspace if w.backward else la_seg.workspace
+    ws = [mkws(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, False, device) for _ in range(2)]
+    wsb = ([la_seg.train_workspace(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, True, device)
             for _ in range(2)] if w.backward else [None, None])
+    NS = la_seg.lib().la_seg_train_saved_states(w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt)
     bufs = []
     for _ in range(2):  # two sets of device inputs and outputs
         d = {n: torch.empty_like(x[n]) for n in names}
         o_dev = torch.empty((w.B, w.H, w.L, w.dv), dtype=w.torch_dtype, device=device)
         Sf = torch.empty((w.B, w.H, w.dk, w.dv), **f32)
-        Sr = torch.empty((w.B, w.H, w.P, w.dk, w.dv), **f32) if w.backward else None
+        Sr = torch.empty((w.B, w.H, NS, w.dk, w.dv), **f32) if w.backward else None
         outs = [o_dev, Sf]
         grads = None
         if w.backward:
@@ -695,13 +732,14 @@ def bench_e2e(args, w, x, device, world):
             s_comp.wait_event(ev_out[k])  # the step two back's results are copied out
         st = la_seg._stream(s_comp)
         d = bf["inp"]
-        la_seg._check(la_seg.lib().la_seg_forward(
+        fwd = la_seg.lib().la_seg_train_forward if w.backward else la_seg.lib().la_seg_forward
+        la_seg._check(fwd(
             P(d["q"]), P(d["k"]), P(d["v"]), P(d["log_g"]), None, w.B, w.H, w.L, w.dk, w.dv,
             w.P, w.chunk, dt, P(bf["o"]), P(bf["Sf"]), P(bf["Sr"]), 0, P(ws[k]), ws[k].numel(), st),
-            "la_seg_forward")
+            "forward")
         if w.backward:
             g = bf["grads"]
-            la_seg._check(la_seg.lib().la_seg_backward(
+            la_seg._check(la_seg.lib().la_seg_train_backward(
                 P(d["q"]), P(d["k"]), P(d["v"]), P(d["log_g"]), None, P(bf["Sr"]), P(d["dO"]),
                 None, w.B, w.H, w.L, w.dk, w.dv, w.P, w.chunk, dt, P(g[0]), P(g[1]), P(g[2]),
                 P(g[3]), P(g[4]), P(wsb[k]), wsb[k].numel(), st), "la_seg_backward")
@@ -730,7 +768,7 @@ def bench_e2e(args, w, x, device, world):
     ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = sum(v.numel() * v.element_size() for v in bufs[0]["host_out"])
-    api = "la_seg_forward" + (" + la_seg_backward" if w.backward else "")
+    api = "la_seg_train_forward + la_seg_train_backward" if w.backward else "la_seg_forward"
     return {"value": round(job_throughput(w.B * w.L, world, steps, ms), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "api": f"{api} (C ABI) with pinned host buffers, steps pipelined over copy-in, "

@@ -141,6 +141,35 @@ LA_API la_status la_seg_backward(const void *q, const void *k, const void *v, co
                           void *dlog_g, float *dS0, void *workspace, size_t ws_bytes,
                           void *cuda_stream);
 
+/* ---- Training: forward and backward with the states saved at the library's split -----------
+ * la_seg_forward saves the state each of the caller's P segments receives; la_seg_backward,
+ * given those, runs its dq sweep one CTA per saved segment, which for few long segments leaves
+ * part of the GPU idle (C4: B*H*P = 256 CTAs on 148 SMs).  The training pair saves instead the
+ * state every one of the library's sub-segments receives (la_seg_subsegments(P) per (b, h), the
+ * split the forward runs on anyway) and its backward reuses them on that split.  Results are
+ * the same bits as la_seg_forward / la_seg_backward called with P = la_seg_subsegments(P); the
+ * backward's gradients do not depend on P.
+ *  saved       fp32 [B, H, la_seg_train_saved_states(...), dk, dv]: the forward writes it (the
+ *              state of API segment p at index p * (NS / P), NS = la_seg_train_saved_states), the
+ *              backward reads it; for the backward S0 and the loss are as in la_seg_backward.
+ *  workspace   la_seg_train_workspace_bytes (backward = 0 or 1) bytes.
+ * Every other argument as in la_seg_forward / la_seg_backward. */
+LA_API int la_seg_train_saved_states(int B, int H, long long L, int dk, int dv, int P, int chunk,
+                                     la_dtype dt);
+LA_API size_t la_seg_train_workspace_bytes(int B, int H, long long L, int dk, int dv, int P,
+                                           int chunk, la_dtype dt, int backward);
+LA_API la_status la_seg_train_forward(const void *q, const void *k, const void *v,
+                                      const void *log_g, const float *S0, int B, int H, long long L,
+                                      int dk, int dv, int P, int chunk, la_dtype dt, void *o,
+                                      float *S_final, float *saved, int schedule, void *workspace,
+                                      size_t ws_bytes, void *cuda_stream);
+LA_API la_status la_seg_train_backward(const void *q, const void *k, const void *v,
+                                       const void *log_g, const float *S0, const float *saved,
+                                       const void *dO, const float *dS_final, int B, int H,
+                                       long long L, int dk, int dv, int P, int chunk, la_dtype dt,
+                                       void *dq, void *dk_, void *dv_, void *dlog_g, float *dS0,
+                                       void *workspace, size_t ws_bytes, void *cuda_stream);
+
 /* The exclusive decayed scan alone (the All-Scan recurrence of the ZeCO review's "key
  * machinery", run on one device over NP segments; the referee's Alg. 2 comment fixes that
  * the accumulated state is what moves on).  Per (b, h), element-wise over (i, j):

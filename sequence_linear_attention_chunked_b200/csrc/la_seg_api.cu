@@ -682,6 +682,45 @@ la_status la_seg_scan(const float *S_in, const float *log_gamma, const float *in
     return e == cudaSuccess ? LA_OK : cuda_fail(e, "scan");
 }
 
+int la_seg_train_saved_states(int B, int H, long long L, int dk, int dv, int P, int chunk,
+                              la_dtype dt) {
+    return la_seg_subsegments(B, H, L, dk, dv, P, chunk, dt);
+}
+
+// The training pair saves and reuses the states at the library's own split: the same kernels and
+// results as la_seg_forward / la_seg_backward called with P = la_seg_subsegments(P) (the result
+// does not depend on P, and for that P the library keeps the same sub-segments), so the
+// backward's dq sweep runs one CTA per sub-segment rather than per API segment.
+la_status la_seg_train_forward(const void *q, const void *k, const void *v, const void *log_g,
+                               const float *S0, int B, int H, long long L, int dk, int dv, int P,
+                               int chunk, la_dtype dt, void *o, float *S_final, float *saved,
+                               int schedule, void *workspace, size_t ws_bytes, void *cuda_stream) {
+    const int NS = la_seg_subsegments(B, H, L, dk, dv, P, chunk, dt);
+    if (NS == 0)  // rejected sizes: the regular entry point names the reason
+        return la_seg_forward(q, k, v, log_g, S0, B, H, L, dk, dv, P, chunk, dt, o, S_final, saved,
+                              schedule, workspace, ws_bytes, cuda_stream);
+    return la_seg_forward(q, k, v, log_g, S0, B, H, L, dk, dv, NS, chunk, dt, o, S_final, saved,
+                          schedule, workspace, ws_bytes, cuda_stream);
+}
+
+la_status la_seg_train_backward(const void *q, const void *k, const void *v, const void *log_g,
+                                const float *S0, const float *saved, const void *dO,
+                                const float *dS_final, int B, int H, long long L, int dk, int dv,
+                                int P, int chunk, la_dtype dt, void *dq, void *dk_, void *dv_,
+                                void *dlog_g, float *dS0, void *workspace, size_t ws_bytes,
+                                void *cuda_stream) {
+    const int NS = la_seg_subsegments(B, H, L, dk, dv, P, chunk, dt);
+    return la_seg_backward(q, k, v, log_g, S0, saved, dO, dS_final, B, H, L, dk, dv,
+                           NS == 0 ? P : NS, chunk, dt, dq, dk_, dv_, dlog_g, dS0, workspace,
+                           ws_bytes, cuda_stream);
+}
+
+size_t la_seg_train_workspace_bytes(int B, int H, long long L, int dk, int dv, int P, int chunk,
+                                    la_dtype dt, int backward) {
+    const int NS = la_seg_subsegments(B, H, L, dk, dv, P, chunk, dt);
+    return NS == 0 ? 0 : la_seg_workspace_bytes(B, H, L, dk, dv, NS, chunk, dt, backward);
+}
+
 la_status la_seg_gather_states(const float *src, int BH, int NP, int m, int dk, int dv, float *dst,
                                void *cuda_stream) {
     if (BH < 0 || NP < 0 || m < 1 || (NP % m) != 0 || dk < 1 || dv < 4 || dv % 4)

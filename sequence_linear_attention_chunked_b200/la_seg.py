@@ -28,7 +28,8 @@ EXPORTED = ("la_seg_workspace_bytes", "la_seg_forward", "la_seg_backward", "la_s
             "la_seg_forward_noalloc", "la_seg_dstate_pass", "la_seg_dq_pass", "la_seg_dkv_pass",
             "la_seg_backward_parts", "la_seg_chain_pass", "la_seg_chain_reset",
             "la_seg_noalloc_check_status", "la_seg_gather_states", "la_seg_log_gamma_total",
-            "la_seg_rank_scan", "la_seg_combine")
+            "la_seg_rank_scan", "la_seg_combine", "la_seg_train_saved_states",
+            "la_seg_train_workspace_bytes", "la_seg_train_forward", "la_seg_train_backward")
 
 _lib = None
 
@@ -73,6 +74,14 @@ def lib():
         L.la_seg_forward_noalloc.argtypes = [P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32,
                                              i32, P, P, P, i32, P]
         L.la_seg_forward_noalloc.restype = i32
+        L.la_seg_train_saved_states.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32]
+        L.la_seg_train_saved_states.restype = i32
+        L.la_seg_train_workspace_bytes.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32, i32]
+        L.la_seg_train_workspace_bytes.restype = sz
+        L.la_seg_train_forward.argtypes = L.la_seg_forward.argtypes
+        L.la_seg_train_forward.restype = i32
+        L.la_seg_train_backward.argtypes = L.la_seg_backward.argtypes
+        L.la_seg_train_backward.restype = i32
         L.la_seg_log_gamma_total.argtypes = [P, i32, i32, i32, P, P]
         L.la_seg_log_gamma_total.restype = i32
         L.la_seg_rank_scan.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P, P, P]
@@ -217,6 +226,62 @@ def la_seg_backward(q, k, v, log_g, dO, S0=None, S_recv_saved=None, dS_final=Non
                                chunk, dt, _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dS0),
                                _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "la_seg_backward")
+    return dq, dk_, dv_, dg, dS0
+
+
+def train_workspace(B, H, L, dk, dv, P, chunk, dt, backward=False, device="cuda"):
+    n = int(lib().la_seg_train_workspace_bytes(B, H, L, dk, dv, P, chunk, dt, int(bool(backward))))
+    if n == 0:
+        raise LaSegError(-2, "la_seg_train_workspace_bytes", "sizes rejected by the library")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def la_seg_train_forward(q, k, v, log_g, S0=None, P=1, chunk=64, schedule=SCHED_AUTO, *, o=None,
+                         ws=None, stream=None):
+    """o, S_final, saved: the forward of a P-segment caller that will run the backward, with the
+    received states saved at the library's own split (saved: fp32 [B, H, NS, dk, dv])."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    for t, n, shp in ((q, "q", (B, H, L, dk)), (k, "k", (B, H, L, dk)), (v, "v", (B, H, L, dv)),
+                      (log_g, "log_g", (B, H, L, dk))):
+        _need(t, n, q.dtype, shp, dev)
+    _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    dt = _dt(q)
+    NS = int(lib().la_seg_train_saved_states(B, H, L, dk, dv, P, chunk, dt))
+    if NS == 0:
+        raise LaSegError(-2, "la_seg_train_saved_states", "sizes rejected by the library")
+    o = torch.empty((B, H, L, dv), dtype=q.dtype, device=dev) if o is None else o
+    S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    saved = torch.empty((B, H, NS, dk, dv), dtype=torch.float32, device=dev)
+    ws = train_workspace(B, H, L, dk, dv, P, chunk, dt, False, dev) if ws is None else ws
+    _check(lib().la_seg_train_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(S0), B, H, L,
+                                      dk, dv, P, chunk, dt, _ptr(o), _ptr(S_final), _ptr(saved),
+                                      int(schedule), _ptr(ws), ws.numel(), _stream(stream)),
+           "la_seg_train_forward")
+    return o, S_final, saved
+
+
+def la_seg_train_backward(q, k, v, log_g, dO, saved, S0=None, dS_final=None, P=1, chunk=64, *,
+                          want_dS0=False, ws=None, stream=None):
+    """dq, dk, dv, dlog_g, dS0 reusing la_seg_train_forward's saved states."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    dt = _dt(q)
+    NS = int(lib().la_seg_train_saved_states(B, H, L, dk, dv, P, chunk, dt))
+    _need(saved, "saved", torch.float32, (B, H, NS, dk, dv), dev)
+    _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    _need(dS_final, "dS_final", torch.float32, (B, H, dk, dv), dev)
+    dq, dk_, dv_, dg = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                        torch.empty_like(log_g))
+    dS0 = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_dS0 else None
+    ws = train_workspace(B, H, L, dk, dv, P, chunk, dt, True, dev) if ws is None else ws
+    _check(lib().la_seg_train_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(S0),
+                                       _ptr(saved), _ptr(dO), _ptr(dS_final), B, H, L, dk, dv, P,
+                                       chunk, dt, _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg),
+                                       _ptr(dS0), _ptr(ws), ws.numel(), _stream(stream)),
+           "la_seg_train_backward")
     return dq, dk_, dv_, dg, dS0
 
 

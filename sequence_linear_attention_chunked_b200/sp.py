@@ -242,7 +242,8 @@ class _Mirror(Exchange):
 @dataclass
 class Saved:
     """What the backward reuses from the forward on this rank."""
-    S_recv: torch.Tensor   # fp32 [B, H, P, dk, dv]: the state each of the rank's P segments receives
+    S_recv: torch.Tensor   # fp32 [B, H, NS, dk, dv]: the state each of the rank's NS sub-segments
+                           # receives (the library's split of its P segments)
     S_end: torch.Tensor    # fp32 [B, H, dk, dv]: the state after the rank's last token
 
 
@@ -275,10 +276,9 @@ def sp_forward(q, k, v, log_g, S0=None, P=1, chunk=64, *, group=None, method="ga
     if ex.world == 1:
         S_final = S_end
     o = steps.output_pass(q, k, v, log_g, S_recv, NS, chunk)
-    S_save = steps.gather_states(S_recv, NS // P)
     if check:
         steps.check()
-    return o, S_final, Saved(S_save, S_end)
+    return o, S_final, Saved(S_recv, S_end)  # the backward reuses them on the same split
 
 
 def sp_backward(q, k, v, log_g, dO, saved: Saved, dS_final=None, P=1, chunk=64, *, group=None,
@@ -291,9 +291,10 @@ def sp_backward(q, k, v, log_g, dO, saved: Saved, dS_final=None, P=1, chunk=64, 
     ex = Exchange(group)
     B, H, L, dk = q.shape
     dv = v.shape[-1]
-    NPF = steps.backward_parts(B, H, L, dk, dv, P, chunk, _dt(q))
-    fine = NPF // P
-    dq, qdq, S_fine, dSloc, lgf = steps.dq_pass(q, k, v, log_g, dO, saved.S_recv, P, fine, chunk)
+    NS = saved.S_recv.shape[2]
+    NPF = steps.backward_parts(B, H, L, dk, dv, NS, chunk, _dt(q))
+    fine = NPF // NS
+    dq, qdq, S_fine, dSloc, lgf = steps.dq_pass(q, k, v, log_g, dO, saved.S_recv, NS, fine, chunk)
     _, G_r, _ = steps.scan(dSloc, lgf, None, True)          # the block's start, from within it
     lg_r = steps.log_gamma_total(lgf)
     init = dS_final
