@@ -256,6 +256,13 @@ __device__ __forceinline__ float warp_sum(float x) {
 // so the dq sweep hands over qdq'_u = q_u . a_u (S_{u-1} dO_u^T) and the reverse sweep subtracts
 // kdk'_u = k_u . (dS+_u v_u^T): two small terms, no cancellation.
 
+// Element (row r, dim i) of the q . dq hand-over, rows counted from a block start that is a
+// multiple of 4 rows: token-quad interleaved (((r / 4) D + i) 4 + r % 4) when the tensor-core
+// sweeps exchange it, row-major otherwise.
+__device__ __forceinline__ long long qdq_index(long long r, int i, int D, int quad) {
+    return quad ? ((r >> 2) * D + i) * 4 + (r & 3) : r * D + i;
+}
+
 // dq sweep of one segment (bh, j) whose fine parts are marked: from S_recv[j] (or zero), per
 // token dq_t = dO_t S_t^T = a_t (S_{t-1} dO_t^T) + k_t (v_t . dO_t) and qdq'_t; at each fine
 // part's start its entering state (S_fine), and over each fine part its gradient state
@@ -338,9 +345,9 @@ __global__ void __launch_bounds__(kXThreads, 1) exact_dq_kernel(const BwdArgs a)
                 }
                 __syncthreads();
                 for (int idx = threadIdx.x; idx < nb * D; idx += kXThreads) {
-                    const long long e = (b0 + idx / D) * D + idx % D;
-                    dq[e] = from_f32<T>(sdq[idx]);
-                    qdq[e] = sqd[idx];
+                    const long long r = b0 + idx / D;
+                    dq[r * D + idx % D] = from_f32<T>(sdq[idx]);
+                    qdq[qdq_index(r, idx % D, D, a.qdq_quad)] = sqd[idx];
                 }
             }
             if (a.dSloc) store_state_B<D>(R, a.dSloc + uf * D * D);
@@ -393,7 +400,7 @@ __global__ void __launch_bounds__(kXThreads, 1) exact_dkv_kernel(const BwdArgs a
             stage<D>(sd, dO, b0, nb, Id());
             stage<D>(sa, g, b0, nb, Exp());
             for (int idx = threadIdx.x; idx < kTB * D; idx += kXThreads)
-                sqdq[idx] = idx / D < nb ? qdq[(b0 + idx / D) * D + idx % D] : 0.f;
+                sqdq[idx] = idx / D < nb ? qdq[qdq_index(b0 + idx / D, idx % D, D, a.qdq_quad)] : 0.f;
             __syncthreads();
             for (int t = nb - 1; t >= 0; --t) {
                 float vj[CL], dj[CL], pre[RW], pv[CL], vdo = 0.f;
@@ -519,8 +526,10 @@ cudaError_t launch_exact_sequence(const PassArgs &a, const float *S0, float *S_f
     });
 }
 
-cudaError_t launch_exact_dq(const BwdArgs &a, cudaStream_t st) {
-    if (!a.flags || a.dk != a.dv || a.fine < 1) return cudaErrorInvalidValue;
+cudaError_t launch_exact_dq(const BwdArgs &a_in, cudaStream_t st) {
+    if (!a_in.flags || a_in.dk != a_in.dv || a_in.fine < 1) return cudaErrorInvalidValue;
+    BwdArgs a = a_in;
+    a.qdq_quad = tc_bwd_supported(a_in);  // the layout the dq sweep of these arguments writes
     return by_shape(a.dk, a.dt, [&](auto dc, auto tv) {
         constexpr int D = decltype(dc)::value;
         return launch_xb(exact_dq_kernel<D, decltype(tv)>, 8 * kTB * D * sizeof(float),
@@ -528,8 +537,10 @@ cudaError_t launch_exact_dq(const BwdArgs &a, cudaStream_t st) {
     });
 }
 
-cudaError_t launch_exact_dkv(const BwdArgs &a, cudaStream_t st) {
-    if (!a.flags || !a.carry || a.dk != a.dv) return cudaErrorInvalidValue;
+cudaError_t launch_exact_dkv(const BwdArgs &a_in, cudaStream_t st) {
+    if (!a_in.flags || !a_in.carry || a_in.dk != a_in.dv) return cudaErrorInvalidValue;
+    BwdArgs a = a_in;
+    a.qdq_quad = tc_bwd_supported(a_in);
     return by_shape(a.dk, a.dt, [&](auto dc, auto tv) {
         constexpr int D = decltype(dc)::value;
         return launch_xb(exact_dkv_kernel<D, decltype(tv)>,

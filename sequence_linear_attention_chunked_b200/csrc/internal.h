@@ -45,7 +45,9 @@ struct BwdArgs {
     const float *S_end_next;  // reverse sweep: S_end_j = S_end_next[j+1] for j < NP-1 (null: no carry)
     const float *S_fin;       // [BH, dk, dv] state after the last token (null: no carry there)
     const float *dX;          // [BH, NP, dk, dv] gradient of each segment's end state
-    float *dq_ws;             // [BH, L, dk] fp32 q . dq, from the dq sweep to the reverse sweep
+    float *dq_ws;             // [BH, L, dk] fp32 q . dq, from the dq sweep to the reverse sweep:
+                              // token-quad interleaved on the tensor-core path, row-major on
+                              // the SIMT path
     float *dSloc;             // [BH, NP, dk, dv] per-segment gradient states (dstate pass)
     float *logG;              // [BH, NP, dk] per-segment log-decay sums (dstate pass)
     const float *carry;       // reverse sweep: [BH, NP, dk] dlog_g carry per part (null: computed)
@@ -55,6 +57,8 @@ struct BwdArgs {
     long long L, T;
     int BH, NP, dk, dv, chunk, fine;
     la_dtype dt;
+    int qdq_quad;             // exact path only: dq_ws is token-quad interleaved (set by its
+                              // launchers from tc_bwd_supported)
 };
 
 // The single-pass forward's chain through the sub-segments of every (b, h) sequence.

@@ -20,30 +20,37 @@ constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
 // Per chunk, last to first, with dS the gradient of the state at the chunk's end (rows = key
 // dims; starts at dX of the part), Qbar'_t = q_t e^{b_t - b_C}, Ktil_s = k_s e^{b_C - b_s}:
 //
-//   M     = dO V^T,  A = Qbar' Ktil^T   M=64  (t) N=64 (s) K=128          -> masked s <= t, bf16
+//   [M *; * A] = [dO; Qbar'] [V; Ktil]^T  M=128 N=128 K=128: M = dO V^T and A = Qbar' Ktil^T
+//                                       are its diagonal 64 x 64 blocks  -> masked s <= t, bf16
 //   dk^T  = Qbar'^T M + dS V^T          M=128 (i) N=64 (s) K=64 (t) / 128 (j)
 //   dv^T  = dO^T A + dS^T Ktil^T        M=128 (j) N=64 (s) K=64 (t) / 128 (i)
 //   dS   += Qbar'^T dO                  M=128 (i) N=128 (j) K=64 (t), accumulated in TMEM
 //   dk[s,i] = e^{b_C,i - b_s,i} dk^T[i,s];   dS <- diag(e^{b_C}) dS
 //   dlog_g_s = rowsum(S_end . dX) + sum_{u >= s in the part} (q_u dq_u - k_u dk_u)
 //
+// The (dO, Qbar') and (V, Ktil) tiles of a stage sit with their 64-column halves interleaved,
+// [dO h0][Qbar' h0][dO h1][Qbar' h1], so that each pair is also one 128-row K-major operand:
+// M and A come from 8 MMA instructions of full width instead of 16 of half width (the
+// off-diagonal blocks are computed and ignored).
+//
 // Roles (448 threads): warps 0-3 carry dS -- the fp32 dS lives in tensor memory (row i on lane
 // i), they apply the decay, write its bf16 copy into a shared [i][j] tile (read by the MMAs as
 // the K-major A operand of dS V^T and the MN-major A operand of dS^T Ktil^T), turn M and A into
-// masked bf16 tiles (double-buffered); warps 4-7 read dk^T (double-buffered in TMEM) and write
-// dk and dlog_g (thread x owns key dim x for all 64 tokens of the chunk, so the dlog_g suffix
-// sums need no exchange); warps 8-11 gate the chunks and write dv from dv^T; 12 TMA; 13 MMA.  A stage
-// is released once the tensor cores are done with it and the dS and output warps have copied
-// the per-key factors they need into registers or TMEM.
+// masked bf16 tiles (double-buffered) and write dv from dv^T; warps 4-7 read dk^T
+// (double-buffered in TMEM) and write dk and dlog_g (thread x owns key dim x for all 64 tokens
+// of the chunk, so the dlog_g suffix sums need no exchange); warps 8-11 gate the chunks; 12 TMA; 13 MMA.  A stage is
+// released once the tensor cores are done with it and the dS and output warps have copied the
+// per-key factors they need into registers or TMEM.
 namespace dkv {
 
 constexpr int kStateWarps = 4, kOutWarps = 4;
-// Tensor-memory columns: M, A (M=64 layout), dk^T x 2, dv^T, the chunk's (e^{b_C - b_s}, Ktil)
-// pairs for the output warps, dS.
-constexpr uint32_t kColM = 0, kColA = 64, kColDK = 128, kColDV = 256, kColFK = 320, kColDS = 384;
+// Tensor-memory columns: [M *; * A] (128 x 128), dk^T x 2, dv^T, the chunk's
+// (e^{b_C - b_s}, Ktil) pairs for the output warps, dS.
+constexpr uint32_t kColMA = 0, kColDK = 128, kColDV = 256, kColFK = 320, kColDS = 384;
 constexpr int kStages = 2;
-constexpr int off_q = 0, off_k = kTileBytes, off_v = 2 * kTileBytes, off_do = 3 * kTileBytes,
-              off_g = 4 * kTileBytes;
+constexpr int kPairHalf = 2 * kHalfBytes;  // distance between a paired tile's two halves
+constexpr int off_do = 0, off_q = kHalfBytes, off_v = 2 * kTileBytes,
+              off_k = 2 * kTileBytes + kHalfBytes, off_g = 4 * kTileBytes;
 constexpr int kStageBytes = 5 * kTileBytes;
 constexpr int kDsHalf = 128 * 128;            // one 64-column half of the [128 x 128] bf16 dS tile
 constexpr int kMaskBytes = CH * CH * 2;       // one masked 64 x 64 bf16 tile
@@ -58,7 +65,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Bars {
     uint64_t *full, *full_b, *gated, *empty;  // full: log_g, q, k (the gates); full_b: v, dO
-    uint64_t *m_full, *m_free, *a_full, *a_free, *p_full, *dst_full, *dk_full, *dk_free, *dv_full, *dv_free,
+    uint64_t *ma_full, *ma_free, *p_full, *dst_full, *dk_full, *dk_free, *dv_full, *dv_free,
         *dsn_full, *fin, *dx_full;
 };
 
@@ -75,10 +82,10 @@ __device__ __forceinline__ uint32_t ds_off(int row, int col) {
     return (uint32_t)(half * kDsHalf + row * 128 + (((cc >> 3) ^ (row & 7)) << 4) + ((cc & 7) << 1));
 }
 
-__device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const CUtensorMap *tq,
-                         const CUtensorMap *tk, const CUtensorMap *tv, const CUtensorMap *tdo,
-                         const CUtensorMap *tg, const CUtensorMap *tdx, int dx_row,
-                         const float *qdq, long long row0, int nchunks) {
+__device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
+                         const CUtensorMap *tq, const CUtensorMap *tk, const CUtensorMap *tv,
+                         const CUtensorMap *tdo, const CUtensorMap *tg, const CUtensorMap *tdx,
+                         int dx_row, long long row0, int nchunks) {
     mbar_arrive_expect_tx(b.dx_full, 4 * 16384);
     for (int bx = 0; bx < 4; ++bx)
         tma_load_2d(smem + kDxStage + bx * 16384, tdx, 32 * bx, dx_row, b.dx_full);
@@ -86,8 +93,8 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
     for (int it = 0; it < nchunks; ++it) {
         const int s = it % kStages;
         const int c = nchunks - 1 - it;  // last chunk first
-        // the chunk's q . dq rows (read with plain loads by the output warps) on their way to L2
-        bulk_prefetch_l2(qdq + (row0 + (long long)c * CH) * D, CH * D * 4);
+        // the chunk's q . dq block (read with plain loads by the output warps) on its way to L2
+        bulk_prefetch_l2(a.dq_ws + (row0 + (long long)c * CH) * D, CH * D * 4);
         if (it >= kStages && !mbar_wait(&b.empty[s], ((it / kStages) - 1) & 1, abort)) break;
         uint8_t *st = smem + s * kStageBytes;
         const int y = (int)(row0 + (long long)c * CH);
@@ -101,7 +108,7 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
         for (int m = 0; m < 5; ++m) {
             uint64_t *bar = m < 3 ? &b.full[s] : &b.full_b[s];
             tma_load_2d(st + offs[m], maps[m], 0, y, bar);
-            tma_load_2d(st + offs[m] + kHalfBytes, maps[m], 64, y, bar);
+            tma_load_2d(st + offs[m] + (m == 0 ? kHalfBytes : kPairHalf), maps[m], 64, y, bar);
         }
         issued = it + 1;
     }
@@ -116,10 +123,10 @@ __device__ void producer(uint8_t *smem, const Bars &b, volatile int *abort, cons
 
 // The whole warp walks the loop; one elected lane issues.  Per chunk: dk^T and dv^T into
 // buffer it % 2 after the dS update (so that dk_full also frees the q tile), then the next
-// chunk's M and A (so that they are ready when the dS warps finish the decay).
+// chunk's M and A once it is gated (so that they are ready when the dS warps finish the decay).
 __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, uint32_t tmem,
                            int nchunks) {
-    constexpr uint32_t i_sq = idesc_bf16_f32(64, 64, 0, 0);      // M, A
+    constexpr uint32_t i_ma = idesc_bf16_f32(128, 128, 0, 0);    // [M *; * A]
     constexpr uint32_t i_dsn = idesc_bf16_f32(128, 128, 1, 1);   // Qbar'^T dO
     constexpr uint32_t i_dka = idesc_bf16_f32(128, 64, 1, 1);    // Qbar'^T M
     constexpr uint32_t i_dkb = idesc_bf16_f32(128, 64, 0, 0);    // dS V^T
@@ -128,30 +135,19 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
     const uint32_t base = smem_u32(smem);
     const uint32_t ma_addr = base + off_ma, ds_addr = base + off_ds;
     auto stage = [&](int it) { return base + (uint32_t)((it % kStages) * kStageBytes); };
-    // M = dO V^T reads untouched tiles: issued as soon as the chunk lands, so the dS warps mask
-    // it while the gates work; A = Qbar' Ktil^T once the tiles are gated.
+    // [dO; Qbar'] [V; Ktil]^T: both 128-row operands are K-major pairs of interleaved tiles
     auto issue_ma = [&](int it) -> bool {
         const uint32_t st = stage(it);
         if (!warp_wait(&b.full_b[it % kStages], (it / kStages) & 1, abort)) return false;  // v, dO
-        if (it > 0 && !warp_wait(b.m_free, (it - 1) & 1, abort)) return false;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + kColM, desc_kmajor(st + off_do, kk), desc_kmajor(st + off_v, kk), i_sq,
-                       kk > 0);
-            mma_commit(b.m_full);
-        }
-        __syncwarp();
         if (!warp_wait(&b.gated[it % kStages], (it / kStages) & 1, abort)) return false;
-        if (it > 0 && !warp_wait(b.a_free, (it - 1) & 1, abort)) return false;
+        if (it > 0 && !warp_wait(b.ma_free, (it - 1) & 1, abort)) return false;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + kColA, desc_kmajor(st + off_q, kk), desc_kmajor(st + off_k, kk), i_sq,
-                       kk > 0);
-            mma_commit(b.a_full);
+                mma_ss(tmem + kColMA, desc_kmajor(st + off_do, kk, kPairHalf),
+                       desc_kmajor(st + off_v, kk, kPairHalf), i_ma, kk > 0);
+            mma_commit(b.ma_full);
         }
         __syncwarp();
         return true;
@@ -171,24 +167,25 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
             const uint32_t dk_col = tmem + kColDK + bb * 64, dv_col = tmem + kColDV;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dS += Qbar'^T dO  (dk and dv read the old dS tile)
-                mma_ss(tmem + kColDS, desc_mnmajor(qa, kk), desc_mnmajor(da, kk), i_dsn, 1u);
+                mma_ss(tmem + kColDS, desc_mnmajor(qa, kk, kPairHalf), desc_mnmajor(da, kk, kPairHalf),
+                       i_dsn, 1u);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dk^T = Qbar'^T M   (B: M tile read MN-major)
-                mma_ss(dk_col, desc_mnmajor(qa, kk), smem_desc_sw128(mt + kk * 2048, kHalfBytes, 1024),
-                       i_dka, kk > 0);
+                mma_ss(dk_col, desc_mnmajor(qa, kk, kPairHalf),
+                       smem_desc_sw128(mt + kk * 2048, kHalfBytes, 1024), i_dka, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // dk^T += dS V^T   (A: dS tile K-major, 128 rows)
                 mma_ss(dk_col, smem_desc_sw128(ds_addr + (kk >> 2) * kDsHalf + (kk & 3) * 32, 16, 1024),
-                       desc_kmajor(va, kk), i_dkb, 1u);
+                       desc_kmajor(va, kk, kPairHalf), i_dkb, 1u);
             mma_commit(&b.dk_full[bb]);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dv^T = dO^T A   (B: A tile read MN-major)
-                mma_ss(dv_col, desc_mnmajor(da, kk), smem_desc_sw128(at + kk * 2048, kHalfBytes, 1024),
-                       i_dva, kk > 0);
+                mma_ss(dv_col, desc_mnmajor(da, kk, kPairHalf),
+                       smem_desc_sw128(at + kk * 2048, kHalfBytes, 1024), i_dva, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // dv^T += dS^T Ktil^T   (A: dS tile read MN-major)
-                mma_ss(dv_col, smem_desc_sw128(ds_addr + kk * 2048, kDsHalf, 1024), desc_kmajor(ka, kk),
-                       i_dvb, 1u);
+                mma_ss(dv_col, smem_desc_sw128(ds_addr + kk * 2048, kDsHalf, 1024),
+                       desc_kmajor(ka, kk, kPairHalf), i_dvb, 1u);
             mma_commit(b.dv_full);
             mma_commit(b.dsn_full);  // the dS tile is read out as well
             mma_commit(&b.empty[s]);
@@ -201,19 +198,10 @@ __device__ void mma_issuer(uint8_t *smem, const Bars &b, volatile int *abort, ui
     wait_drain(b.fin, 0);
 }
 
-// Stores the bf16 values of tokens t and t+1 of this lane's dim x into a [tokens, 128] bf16
-// tensor (one conversion, two 2-byte stores).  `at` points at element (t, x).
-__device__ __forceinline__ void stg_pair(__nv_bfloat16 *at, float a, float b) {
-    const uint32_t p = pack_bf16(a, b);  // low half: token t, high half: token t+1
-    unsigned short *h = reinterpret_cast<unsigned short *>(at);
-    h[0] = (unsigned short)(p & 0xFFFFu);
-    h[D] = (unsigned short)(p >> 16);
-}
-
-// dv of one chunk from dv^T (thread x = TMEM lane x owns value dim x), straight to HBM;
-// releases the accumulator after the last tensor-memory read.  The gate warps run it right after
-// gating the next chunk, before that chunk's masked A tile (and so its dv^T MMA) can exist, so
-// one dv^T buffer suffices.
+// dv of one chunk from dv^T (thread x = TMEM lane x owns value dim x), straight to HBM (`dvc`
+// points at the chunk's first token, dim 32 w for warp w); releases the accumulator after the
+// last tensor-memory read.  The dS warps run it after the next chunk's decay, while the next
+// chunk's M and A are formed: that chunk's dv^T MMA waits for it (one dv^T buffer).
 __device__ __forceinline__ bool dv_readout(const Bars &b, volatile int *abort, uint32_t tmem,
                                            uint32_t lrow, int parity, __nv_bfloat16 *dvc,
                                            int lane) {
@@ -231,20 +219,17 @@ __device__ __forceinline__ bool dv_readout(const Bars &b, volatile int *abort, u
         }
 #pragma unroll
         for (int t = 0; t < 16; t += 2)
-            stg_pair(dvc + (g * 16 + t) * D, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
+            st_pair_bf16(dvc + (g * 16 + t) * D, lane, __uint_as_float(r[t]), __uint_as_float(r[t + 1]));
     }
     return true;
 }
 
 // Gate warps: Qbar' and Ktil in place of q and k, e^{b_C - b_t} in place of log_g (the dk
-// output factor), e^{b_C} per key dim; then dv of the previous chunk (warp gw reads TMEM lane
-// quarter gw, value dims 32 gw .. 32 gw + 31).
+// output factor), e^{b_C} per key dim.
 __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
-                          uint32_t tmem, long long row0, int nchunks) {
+                          int nchunks) {
     const int gw = (threadIdx.x >> 5) - kEpiWarps;
     const int lane = threadIdx.x & 31;
-    const uint32_t lrow = (uint32_t)(gw * 32) << 16;
-    __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv_out) + row0 * D + gw * 32 + lane;
     const int tg = lane >> 2, ig = lane & 3;
     const int i0 = gw * 32 + ig * 8;
     float *ec = reinterpret_cast<float *>(smem + off_ec);
@@ -327,78 +312,72 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
             uint4 qr[2], kr[2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
+                const uint32_t off = tile_off(tg * 8 + r0 + r, i0, kPairHalf);
                 qr[r] = *reinterpret_cast<const uint4 *>(st + off_q + off);
                 kr[r] = *reinterpret_cast<const uint4 *>(st + off_k + off);
             }
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                const uint32_t off = tile_off(tg * 8 + r0 + r, i0);
-                float x[8], fq[8], fk[8];
+                const uint32_t off = tile_off(tg * 8 + r0 + r, i0, kPairHalf);
+                float x[8], fk[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = fmaf(bt[r0 + r][e], kLog2e, nbCl[e]);
-                unpack8(qr[r], fq);
                 unpack8(kr[r], fk);
+                const uint32_t qw[4] = {qr[r].x, qr[r].y, qr[r].z, qr[r].w};
                 uint32_t wq[4], wk[4], wf[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float u0 = ex2_approx(x[2 * e]), u1 = ex2_approx(x[2 * e + 1]);
                     const float d0 = ex2_approx(-x[2 * e]), d1 = ex2_approx(-x[2 * e + 1]);
                     const uint32_t fw = pack_bf16(u0, u1);  // F = bf16(e^x), as the dq sweep has it
-                    wq[e] = pack_bf16(fq[2 * e] * __uint_as_float(fw << 16),
-                                      fq[2 * e + 1] * __uint_as_float(fw & 0xFFFF0000u));
+                    wq[e] = mul_bf16x2(qw[e], fw);  // bf16(q F): the bf16 product is exact in fp32
                     wk[e] = pack_bf16(fk[2 * e] * d0, fk[2 * e + 1] * d1);
                     wf[e] = pack_bf16(d0, d1);
                 }
                 *reinterpret_cast<uint4 *>(st + off_q + off) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
                 *reinterpret_cast<uint4 *>(st + off_k + off) = make_uint4(wk[0], wk[1], wk[2], wk[3]);
-                *reinterpret_cast<uint4 *>(st + off_g + off) = make_uint4(wf[0], wf[1], wf[2], wf[3]);
+                *reinterpret_cast<uint4 *>(st + off_g + tile_off(tg * 8 + r0 + r, i0)) =
+                    make_uint4(wf[0], wf[1], wf[2], wf[3]);
             }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.gated[s]);
-        if (it > 0 && !dv_readout(b, abort, tmem, lrow, (it - 1) & 1,
-                                  dv + (long long)(nchunks - it) * CH * D, lane))
-            break;
     }
-    if (!*abort && nchunks > 0)  // dv of the part's first chunk
-        dv_readout(b, abort, tmem, lrow, (nchunks - 1) & 1, dv, lane);
     if (range_bad || any_pos_bf16(posm))  // this CTA's unit is fine part blockIdx.x = bh * NP + j
         flag_range(a.flags, (long long)blockIdx.x, 1, a.status);
 }
 
-// Writes a masked (s <= t) bf16 copy of a M=64 TMEM accumulator half into a 64x64 tile.
-__device__ __forceinline__ void masked_tile(uint8_t *tile, const uint32_t (&r)[32], int quarter,
-                                            int h, int lane) {
-    if (lane < 16) {
-        const int t = quarter * 16 + lane;
-        uint8_t *row = tile + t * 128;
+// Writes columns 32 h .. 32 h + 31 of row t of a 64 x 64 tile as its masked (s <= t) bf16 copy.
+__device__ __forceinline__ void masked_row(uint8_t *tile, const uint32_t (&r)[32], int t, int h) {
+    uint8_t *row = tile + t * 128;
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            uint32_t w4[4];
+    for (int jj = 0; jj < 4; ++jj) {
+        uint32_t w4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int sl = jj * 8 + 2 * e, s0 = h * 32 + sl;
-                w4[e] = pack_bf16(s0 <= t ? __uint_as_float(r[sl]) : 0.f,
-                                  s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f);
-            }
-            *reinterpret_cast<uint4 *>(row + (((h * 4 + jj) ^ (t & 7)) << 4)) =
-                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int e = 0; e < 4; ++e) {
+            const int sl = jj * 8 + 2 * e, s0 = h * 32 + sl;
+            w4[e] = pack_bf16(s0 <= t ? __uint_as_float(r[sl]) : 0.f,
+                              s0 + 1 <= t ? __uint_as_float(r[sl + 1]) : 0.f);
         }
+        *reinterpret_cast<uint4 *>(row + (((h * 4 + jj) ^ (t & 7)) << 4)) =
+            make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
 }
 
 // Warps 0-3: thread i owns row i of dS (TMEM lane i).  Per chunk: the decay by the previous
 // chunk's e^{b_C} (S_new = diag(e^{b_C}) (dS + Qbar'^T dO), the sum formed by the MMA), the
-// bf16 copy of row i into the dS tile, the masked M and A tiles; the stage is released as soon
-// as its e^{b_C} is in a register.
+// bf16 copy of row i into the dS tile, dv of the previous chunk (value dim i; M and A of this
+// chunk are formed meanwhile), the masked M and A tiles; the stage is released as soon as its
+// e^{b_C} is in a register.
 __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
                            uint32_t tmem, int bh, int j, int nchunks) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = warp * 32 + lane;
     const uint32_t lrow = (uint32_t)(warp * 32) << 16;
     const float *ec = reinterpret_cast<const float *>(smem + off_ec);
+    __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv_out) +
+                        ((long long)bh * a.L + (long long)j * a.T) * D + warp * 32;
     uint32_t r[32];
     // dS at the part's end: dX, row i from the swizzled staging boxes.  Column groups go last to
     // first: the bf16 copy of group p lands on row i of box 2 + p / 2 (the dS tile's halves
@@ -464,24 +443,30 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(b.dst_full);
-        // (2) masked M and A tiles of this chunk (M=64 layout: lanes 0-15 hold row 16 warp + lane);
-        // M is ready before the gates finish, A only after; dv of the previous chunk in between
-        uint8_t *mt = smem + off_ma + (it & 1) * 2 * kMaskBytes;
+        // dv of the previous chunk: its MMAs completed with dsn_full
+        if (it > 0 && !dv_readout(b, abort, tmem, lrow, (it - 1) & 1,
+                                  dv + (long long)(nchunks - it) * CH * D, lane))
+            break;
+        // (2) masked M and A tiles of this chunk: TMEM lane 32 w + l is row 32 w + l of
+        // [M *; * A], so warps 0-1 hold rows t = 32 w + l of M (columns 0-63) and warps 2-3 rows
+        // t = 32 (w - 2) + l of A (columns 64-127)
+        if (!mbar_wait(b.ma_full, it & 1, abort)) break;
+        tc_fence_after();
+        {
+            const int blk = warp >> 1, t = (warp & 1) * 32 + lane;
+            uint8_t *mt = smem + off_ma + ((it & 1) * 2 + blk) * kMaskBytes;
 #pragma unroll 1
-        for (int t = 0; t < 4; ++t) {  // M half 0, M half 1, A half 0, A half 1
-            if (t == 0 && !mbar_wait(b.m_full, it & 1, abort)) break;
-            if (t == 2 && !mbar_wait(b.a_full, it & 1, abort)) break;
-            if ((t & 1) == 0) tc_fence_after();
-            tmem_ld32(tmem + lrow + (t < 2 ? kColM : kColA) + (t & 1) * 32, r);
-            tmem_wait_ld();
-            if (t & 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(t == 1 ? b.m_free : b.a_free);
+            for (int h = 0; h < 2; ++h) {
+                tmem_ld32(tmem + lrow + kColMA + blk * 64 + h * 32, r);
+                tmem_wait_ld();
+                if (h == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b.ma_free);
+                }
+                masked_row(mt, r, t, h);
             }
-            masked_tile(mt + (t >> 1) * kMaskBytes, r, warp, t & 1, lane);
         }
-        if (*abort) break;
         fence_proxy_async_smem();
         // the chunk's e^{b_C} is this role's last read of the stage
         e2 = (uint64_t)__float_as_uint(ec[(it % kStages) * D + i]) * 0x100000001ull;
@@ -491,13 +476,15 @@ __device__ void state_role(uint8_t *smem, const Bars &b, volatile int *abort, co
             mbar_arrive(&b.empty[it % kStages]);
         }
     }
+    if (!*abort && nchunks > 0)  // dv of the part's first chunk
+        dv_readout(b, abort, tmem, lrow, (nchunks - 1) & 1, dv, lane);
 }
 
 // Warps 4-7: thread x = 32 (warp - 4) + lane owns key dim x of dk and dlog_g for all 64 tokens
 // of the chunk.  As soon as the gates are done with a chunk, each thread copies its dim's 64
 // (e^{b_C - b_s}, Ktil) pairs from the stage into its TMEM lane and releases the stage; the dk
 // loop then reads them back from TMEM beside the dk^T accumulator.  Outputs go straight from
-// registers to HBM.
+// registers to HBM, each lane of a pair writing two dims of one token.
 __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, const BwdArgs &a,
                          uint32_t tmem, int bh, int j, long long row0, int nchunks) {
     const int quarter = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
@@ -535,61 +522,64 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
             carry = part[0];
         }
     }
-    uint32_t r[16], fk[16];
-    float qv[16], qn[16];
+    // q . dq (token-quad interleaved, float4 = 4 tokens of dim x): two buffers of one 16-token
+    // group each; a group's loads go out as soon as the group two before it has been used
+    auto load_qdq = [&](float4 (&dst)[4], long long rq) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) dst[m] = *qdq_quad(a.dq_ws, rq + m, x);
+    };
+    const int dim0 = quarter * 32;
     for (int it = 0; it < nchunks; ++it) {
         const int s = it % kStages, bb = it & 1;
         const int c = nchunks - 1 - it;
-        const float *qdq = a.dq_ws + (row0 + (long long)c * CH) * D + x;
+        const long long tq = (row0 + (long long)c * CH) >> 2;  // the chunk's first token quad
+        float4 qb[2][4];
+        load_qdq(qb[0], tq + 12);  // tokens 48 .. 63, then 32 .. 47 (L2-prefetched with the tiles)
+        load_qdq(qb[1], tq + 8);
         // (1) the chunk's factors and Ktil into this lane of TMEM; then the stage is released
         if (!warp_wait(&b.gated[s], (it / kStages) & 1, abort)) break;
         const uint32_t sa = smem_u32(smem + s * kStageBytes);
-        copy_pairs_to_tmem(sa + off_g, sa + off_k, tmem + kColFK, quarter, lane);
+        copy_pairs_to_tmem(sa + off_g, sa + off_k, tmem + kColFK, quarter, lane, kHalfBytes, kPairHalf);
         tmem_wait_st();
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.empty[s]);
-        // q . dq of the chunk's last 16 tokens (L2-prefetched with the chunk's tiles), in flight
-        // while this thread waits for dk; each later group is loaded one group ahead
-#pragma unroll
-        for (int t = 0; t < 16; ++t) qn[t] = qdq[(48 + t) * D];
         // (2) dk and the dlog_g suffix sums: tokens last to first, 16 at a time
         if (!mbar_wait(&b.dk_full[bb], (it >> 1) & 1, abort)) break;
         tc_fence_after();
 #pragma unroll
         for (int g = 3; g >= 0; --g) {
+            uint32_t r[16], fk[16];
             tmem_ld16(tmem + lrow + kColDK + bb * 64 + g * 16, r);
             tmem_ld16(tmem + lrow + kColFK + g * 16, fk);
-#pragma unroll
-            for (int t = 0; t < 16; ++t) qv[t] = qn[t];
-            if (g > 0) {  // the next group's loads go out before this group's stores
-#pragma unroll
-                for (int t = 0; t < 16; ++t) qn[t] = qdq[((g - 1) * 16 + t) * D];
-            }
             tmem_wait_ld();
             if (g == 0) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&b.dk_free[bb]);
             }
+            const float4 *qv = qb[(3 - g) & 1];
             // dk = e^{b_C - b_s} acc and the contribution q . dq - k . dk (k . dk = Ktil . acc,
             // Ktil = k e^{b_C - b_s} the MMA operand); then the suffix sums
             float fd[16], cg[16];  // dk, then contributions / dlog_g
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
                 const float acc = __uint_as_float(r[t]);
-                fd[t] = __uint_as_float(fk[t] << 16) * acc;                        // dk
-                cg[t] = qv[t] - __uint_as_float(fk[t] & 0xFFFF0000u) * acc;       // contribution
+                const float4 &q4 = qv[t >> 2];
+                const float qq = (t & 3) == 0 ? q4.x : (t & 3) == 1 ? q4.y : (t & 3) == 2 ? q4.z : q4.w;
+                fd[t] = __uint_as_float(fk[t] << 16) * acc;                   // dk
+                cg[t] = qq - __uint_as_float(fk[t] & 0xFFFF0000u) * acc;      // contribution
             }
+            if (g >= 2) load_qdq(qb[(3 - g) & 1], tq + 4 * (g - 2));  // group g - 2
 #pragma unroll
             for (int t = 15; t >= 0; --t) {
                 carry += cg[t];
                 cg[t] = carry;                 // dlog_g
             }
-            const long long e0 = (row0 + (long long)c * CH + g * 16) * D + x;  // element (t0, x)
+            const long long e0 = (row0 + (long long)c * CH + g * 16) * D + dim0;  // (t0, dim0)
 #pragma unroll
             for (int t = 0; t < 16; t += 2) {
-                stg_pair(dk + e0 + t * D, fd[t], fd[t + 1]);
-                stg_pair(dg + e0 + t * D, cg[t], cg[t + 1]);
+                st_pair_bf16(dk + e0 + t * D, lane, fd[t], fd[t + 1]);
+                st_pair_bf16(dg + e0 + t * D, lane, cg[t], cg[t + 1]);
             }
         }
     }
@@ -610,9 +600,9 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     b.empty = bar + 2 * kStages;
     b.full_b = bar + 3 * kStages;
     uint64_t *x = bar + 4 * kStages;
-    b.m_full = x + 0; b.m_free = x + 1; b.p_full = x + 2; b.dst_full = x + 3; b.dk_full = x + 4;
+    b.ma_full = x + 0; b.ma_free = x + 1; b.p_full = x + 2; b.dst_full = x + 3; b.dk_full = x + 4;
     b.dk_free = x + 6; b.dv_full = x + 8; b.dv_free = x + 10; b.dsn_full = x + 12; b.fin = x + 13;
-    b.a_full = x + 14; b.a_free = x + 15; b.dx_full = x + 16;
+    b.dx_full = x + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_misc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + off_misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -626,9 +616,9 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&b.gated[s], kGateWarps);
             mbar_init(&b.empty[s], 1 + kStateWarps + kOutWarps);
         }
-        uint64_t *one[] = {b.m_full, b.a_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dsn_full,
+        uint64_t *one[] = {b.ma_full, b.dk_full, b.dk_full + 1, b.dv_full, b.dsn_full,
                            b.fin, b.dx_full};
-        uint64_t *st4[] = {b.m_free, b.a_free, b.p_full, b.dst_full, b.dv_free};  // dv_free: gates
+        uint64_t *st4[] = {b.ma_free, b.p_full, b.dst_full, b.dv_free};
         uint64_t *out4[] = {b.dk_free, b.dk_free + 1};
         for (uint64_t *p : one) mbar_init(p, 1);
         for (uint64_t *p : st4) mbar_init(p, kStateWarps);
@@ -651,12 +641,12 @@ tc_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
     if (warp == kTmaWarp) {
         if (lane == 0)
-            producer(smem, b, abort, &tm_q, &tm_k, &tm_v, &tm_do, &tm_g, &tm_dx,
-                     (int)(((long long)bh * a.NP + j) * D), a.dq_ws, row0, nchunks);
+            producer(smem, b, abort, a, &tm_q, &tm_k, &tm_v, &tm_do, &tm_g, &tm_dx,
+                     (int)(((long long)bh * a.NP + j) * D), row0, nchunks);
     } else if (warp == kMmaWarp) {
         mma_issuer(smem, b, abort, tmem, nchunks);
     } else if (warp >= kEpiWarps) {
-        gate_role(smem, b, abort, a, tmem, row0, nchunks);
+        gate_role(smem, b, abort, a, nchunks);
     } else if (warp < kStateWarps) {
         state_role(smem, b, abort, a, tmem, bh, j, nchunks);
     } else {

@@ -485,24 +485,29 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
                 __syncwarp();
                 if (lane == 0) mbar_arrive(b[kDqFree]);
             }
+            float dqv[16], qd[16];
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
-                const long long t = tok0 + g * 16 + e;
                 const float F0 = __uint_as_float(fq[e] << 16), F1 = __uint_as_float(fq[e + 1] << 16);
                 const float a0 = __uint_as_float(r16[e]), a1 = __uint_as_float(r16[e + 1]);
-                const float v0 = a0 * F0, v1 = a1 * F1;  // dq
+                dqv[e] = a0 * F0;
+                dqv[e + 1] = a1 * F1;
                 // q . dq handed over as Qbar' dq^T, Qbar' = bf16(q F) -- bit for bit the operand
                 // the reverse sweep's MMAs use -- so that the diagonal term (q_t . k_t)(v_t . dO_t)
                 // of q . dq and of k . dk is the same exact fp32 product in both sweeps and
                 // cancels in dlog_g down to fp32 accumulation error
                 const uint32_t qb = pack_bf16(__uint_as_float(fq[e] & 0xFFFF0000u) * F0,
                                               __uint_as_float(fq[e + 1] & 0xFFFF0000u) * F1);
-                a.dq_ws[t * D + i] = __uint_as_float(qb << 16) * a0;
-                a.dq_ws[(t + 1) * D + i] = __uint_as_float(qb & 0xFFFF0000u) * a1;
-                const uint32_t p = pack_bf16(v0, v1);  // low: token t, high: token t+1
-                unsigned short *h = reinterpret_cast<unsigned short *>(dq + t * D + i);
-                h[0] = (unsigned short)(p & 0xFFFFu);
-                h[D] = (unsigned short)(p >> 16);
+                qd[e] = __uint_as_float(qb << 16) * a0;
+                qd[e + 1] = __uint_as_float(qb & 0xFFFF0000u) * a1;
+            }
+            const long long t0 = tok0 + g * 16;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {  // four tokens per float4 / per quad store
+                *qdq_quad(a.dq_ws, (t0 >> 2) + m, i) =
+                    make_float4(qd[4 * m], qd[4 * m + 1], qd[4 * m + 2], qd[4 * m + 3]);
+                st_quad_bf16(dq + (t0 + 4 * m) * D + quarter * 32, lane, dqv[4 * m],
+                             dqv[4 * m + 1], dqv[4 * m + 2], dqv[4 * m + 3]);
             }
         }
         if (c + 1 < w.nchunks && !make_p(c + 1)) break;
