@@ -270,8 +270,11 @@ LA_API la_status la_seg_dstate_pass(const void *q, const void *dO, const void *l
                                     void *cuda_stream);
 
 /* dq pass (backward step 2): the forward chunk sweep of every segment p from the state it
- * received S_recv[b,h,p] (fp32 [B,H,NP,dk,dv]; null = zero): dq (dtype dt) and q . dq (fp32
- * [B,H,L,dk], read by la_seg_dkv_pass for dlog_g).  S_fine (nullable, fp32
+ * received S_recv[b,h,p] (fp32 [B,H,NP,dk,dv]; null = zero): dq (dtype dt) and q . dq (fp32,
+ * B*H*L*dk values, read by la_seg_dkv_pass for dlog_g; its arrangement is internal: for bf16
+ * with dk = dv = 128 and chunk 64 the tensor-core sweeps keep each four consecutive tokens of a
+ * key dim together, element (row r, dim i) at ((r / 4) * dk + i) * 4 + r % 4 with r counted
+ * over [B,H,L]; row-major [B,H,L,dk] otherwise).  S_fine (nullable, fp32
  * [B,H,NP*fine,dk,dv]) receives the state entering each of the `fine` equal parts of every
  * segment ((L/NP) % fine == 0, parts of whole chunks): the received states of the finer split
  * la_seg_dkv_pass runs on.  dSloc and log_gamma (both or neither; fp32 [B,H,NP*fine,dk,dv] and

@@ -399,7 +399,9 @@ def la_seg_backward_parts(B, H, L, dk, dv, P, chunk, dt=LA_BF16, reuse=True) -> 
 def la_seg_dq_pass(q, k, v, log_g, dO, S_recv, NP, fine, chunk, *, dq=None, qdq=None, S_fine=None,
                    dSloc=None, log_gamma=None, status=None, stream=None):
     """dq and q . dq; optionally (dSloc and log_gamma given, both or neither) the fine parts'
-    gradient states and log-decay sums, as la_seg_dstate_pass over NP * fine parts."""
+    gradient states and log-decay sums, as la_seg_dstate_pass over NP * fine parts.  q . dq is
+    a buffer of B*H*L*dk floats for la_seg_dkv_pass in the library's internal arrangement (see
+    la_seg.h), not a [B, H, L, dk] tensor in general."""
     B, H, L, dk, dv = _seq_shapes(q, v)
     dq = torch.empty_like(q) if dq is None else dq
     qdq = torch.empty((B, H, L, dk), dtype=torch.float32, device=q.device) if qdq is None else qdq
