@@ -258,47 +258,61 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 #pragma unroll
                 for (int k = 0; k < 4; ++k) unpack8(graw[4 * h + k], f[k]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float p01 = f[0][e] + f[1][e], p23 = f[2][e] + f[3][e];
+                for (int e = 0; e < 8; e += 2) {  // two key dims per f32x2 instruction
+                    float p01[2], p23[2];
+                    add_x2(p01[0], p01[1], f[0][e], f[0][e + 1], f[1][e], f[1][e + 1]);
+                    add_x2(p23[0], p23[1], f[2][e], f[2][e + 1], f[3][e], f[3][e + 1]);
                     bt[4 * h][e] = f[0][e];
-                    bt[4 * h + 1][e] = p01;
-                    bt[4 * h + 2][e] = f[2][e] + p01;
-                    bt[4 * h + 3][e] = p23 + p01;
-                    tot[h][e] = p01 + p23;
+                    bt[4 * h][e + 1] = f[0][e + 1];
+                    bt[4 * h + 1][e] = p01[0];
+                    bt[4 * h + 1][e + 1] = p01[1];
+                    add_x2(bt[4 * h + 2][e], bt[4 * h + 2][e + 1], f[2][e], f[2][e + 1], p01[0], p01[1]);
+                    add_x2(bt[4 * h + 3][e], bt[4 * h + 3][e + 1], p23[0], p23[1], p01[0], p01[1]);
+                    add_x2(tot[h][e], tot[h][e + 1], p01[0], p01[1], p23[0], p23[1]);
                 }
             }
         }
         float ia[8], ib[8];  // inclusive scan of the group totals: groups 2 tg, 2 tg + 1
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {  // step 1: group g adds group g - 1
-            const float up = __shfl_up_sync(0xFFFFFFFFu, tot[1][e], 4);
-            ia[e] = tg >= 1 ? tot[0][e] + up : tot[0][e];
-            ib[e] = tot[1][e] + tot[0][e];
+        for (int e = 0; e < 8; e += 2) {  // step 1: group g adds group g - 1
+            const float u0 = __shfl_up_sync(0xFFFFFFFFu, tot[1][e], 4);
+            const float u1 = __shfl_up_sync(0xFFFFFFFFu, tot[1][e + 1], 4);
+            add_x2(ia[e], ia[e + 1], tot[0][e], tot[0][e + 1], u0, u1);
+            if (tg < 1) {
+                ia[e] = tot[0][e];
+                ia[e + 1] = tot[0][e + 1];
+            }
+            add_x2(ib[e], ib[e + 1], tot[1][e], tot[1][e + 1], tot[0][e], tot[0][e + 1]);
         }
 #pragma unroll
         for (int dd = 1; dd < 8; dd <<= 1) {  // steps 2, 4, 8: group g adds group g - 2 dd
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float ua = __shfl_up_sync(0xFFFFFFFFu, ia[e], 4 * dd);
-                const float ub = __shfl_up_sync(0xFFFFFFFFu, ib[e], 4 * dd);
+            for (int e = 0; e < 8; e += 2) {
+                const float a0 = __shfl_up_sync(0xFFFFFFFFu, ia[e], 4 * dd);
+                const float a1 = __shfl_up_sync(0xFFFFFFFFu, ia[e + 1], 4 * dd);
+                const float b0 = __shfl_up_sync(0xFFFFFFFFu, ib[e], 4 * dd);
+                const float b1 = __shfl_up_sync(0xFFFFFFFFu, ib[e + 1], 4 * dd);
                 if (tg >= dd) {
-                    ia[e] += ua;
-                    ib[e] += ub;
+                    add_x2(ia[e], ia[e + 1], ia[e], ia[e + 1], a0, a1);
+                    add_x2(ib[e], ib[e + 1], ib[e], ib[e + 1], b0, b1);
                 }
             }
         }
         float nbCl[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float bC = __shfl_sync(0xFFFFFFFFu, ib[e], 28 + ig);  // group 15
-            const float offa = ia[e] - tot[0][e], offb = ib[e] - tot[1][e];
+        for (int e = 0; e < 8; e += 2) {
+            const float bC0 = __shfl_sync(0xFFFFFFFFu, ib[e], 28 + ig);  // group 15
+            const float bC1 = __shfl_sync(0xFFFFFFFFu, ib[e + 1], 28 + ig);
+            float offa[2], offb[2];
+            sub_x2(offa[0], offa[1], ia[e], ia[e + 1], tot[0][e], tot[0][e + 1]);
+            sub_x2(offb[0], offb[1], ib[e], ib[e + 1], tot[1][e], tot[1][e + 1]);
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                bt[r][e] += offa;
-                bt[4 + r][e] += offb;
+                add_x2(bt[r][e], bt[r][e + 1], bt[r][e], bt[r][e + 1], offa[0], offa[1]);
+                add_x2(bt[4 + r][e], bt[4 + r][e + 1], bt[4 + r][e], bt[4 + r][e + 1], offb[0], offb[1]);
             }
-            nbCl[e] = -bC * kLog2e;
-            range_bad |= !(fabsf(bC) <= kGateRangeLimit);
+            mul_x2(nbCl[e], nbCl[e + 1], -bC0, -bC1, kLog2e, kLog2e);
+            range_bad |= !(fabsf(bC0) <= kGateRangeLimit) || !(fabsf(bC1) <= kGateRangeLimit);
         }
         if (tg == 0) {
             float4 *e4 = reinterpret_cast<float4 *>(ec + s * D + i0);
@@ -321,7 +335,9 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
                 const uint32_t off = tile_off(tg * 8 + r0 + r, i0, kPairHalf);
                 float x[8], fk[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = fmaf(bt[r0 + r][e], kLog2e, nbCl[e]);
+                for (int e = 0; e < 8; e += 2)
+                    fma_x2(x[e], x[e + 1], bt[r0 + r][e], bt[r0 + r][e + 1], kLog2e, kLog2e, nbCl[e],
+                           nbCl[e + 1]);
                 unpack8(kr[r], fk);
                 const uint32_t qw[4] = {qr[r].x, qr[r].y, qr[r].z, qr[r].w};
                 uint32_t wq[4], wk[4], wf[4];
@@ -331,7 +347,9 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
                     const float d0 = ex2_approx(-x[2 * e]), d1 = ex2_approx(-x[2 * e + 1]);
                     const uint32_t fw = pack_bf16(u0, u1);  // F = bf16(e^x), as the dq sweep has it
                     wq[e] = mul_bf16x2(qw[e], fw);  // bf16(q F): the bf16 product is exact in fp32
-                    wk[e] = pack_bf16(fk[2 * e] * d0, fk[2 * e + 1] * d1);
+                    float k0, k1;
+                    mul_x2(k0, k1, fk[2 * e], fk[2 * e + 1], d0, d1);
+                    wk[e] = pack_bf16(k0, k1);
                     wf[e] = pack_bf16(d0, d1);
                 }
                 *reinterpret_cast<uint4 *>(st + off_q + off) = make_uint4(wq[0], wq[1], wq[2], wq[3]);

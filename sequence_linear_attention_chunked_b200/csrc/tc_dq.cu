@@ -222,16 +222,19 @@ __device__ __noinline__ void gate_role(uint8_t *smem, const Bars &b, volatile in
 #pragma unroll
             for (int k = 0; k < 4; ++k) unpack8(graw[k], f[k]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < 8; e += 2) {  // two key dims per f32x2 instruction
                 // steps (0,1) and (2,3) each visit one row pair in order; the pair of rows
                 // 4tg, 4tg+1 is at steps 0,1 when sw == 0, at steps 2,3 otherwise
-                const float p01 = f[0][e] + f[1][e], p23 = f[2][e] + f[3][e];
-                const float o01 = sw ? p23 : 0.f, o23 = sw ? 0.f : p01;
-                bk[0][e] = f[0][e] + o01;
-                bk[1][e] = p01 + o01;
-                bk[2][e] = f[2][e] + o23;
-                bk[3][e] = p23 + o23;
-                tot[e] = p01 + p23;
+                float p01[2], p23[2];
+                add_x2(p01[0], p01[1], f[0][e], f[0][e + 1], f[1][e], f[1][e + 1]);
+                add_x2(p23[0], p23[1], f[2][e], f[2][e + 1], f[3][e], f[3][e + 1]);
+                const float o01a = sw ? p23[0] : 0.f, o01b = sw ? p23[1] : 0.f;
+                const float o23a = sw ? 0.f : p01[0], o23b = sw ? 0.f : p01[1];
+                add_x2(bk[0][e], bk[0][e + 1], f[0][e], f[0][e + 1], o01a, o01b);
+                add_x2(bk[1][e], bk[1][e + 1], p01[0], p01[1], o01a, o01b);
+                add_x2(bk[2][e], bk[2][e + 1], f[2][e], f[2][e + 1], o23a, o23b);
+                add_x2(bk[3][e], bk[3][e + 1], p23[0], p23[1], o23a, o23b);
+                add_x2(tot[e], tot[e + 1], p01[0], p01[1], p23[0], p23[1]);
             }
         }
         float incl[8];  // inclusive scan of the group totals across tg (lanes ig, ig+2, ...)
@@ -239,24 +242,32 @@ __device__ __noinline__ void gate_role(uint8_t *smem, const Bars &b, volatile in
         for (int e = 0; e < 8; ++e) incl[e] = tot[e];
 #pragma unroll
         for (int d = 1; d < 16; d <<= 1) {
+            float up[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float up = __shfl_up_sync(0xFFFFFFFFu, incl[e], 2 * d);
-                if (tg >= d) incl[e] += up;
+            for (int e = 0; e < 8; ++e) up[e] = __shfl_up_sync(0xFFFFFFFFu, incl[e], 2 * d);
+            if (tg >= d) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2)
+                    add_x2(incl[e], incl[e + 1], incl[e], incl[e + 1], up[e], up[e + 1]);
             }
         }
         float nbCl[8], eB[8];
         const bool part_start = c % w.cpf == 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float bC = __shfl_sync(0xFFFFFFFFu, incl[e], 30 + ig);
-            const float off = incl[e] - tot[e];  // exclusive prefix of this token group
+        for (int e = 0; e < 8; e += 2) {
+            const float bC0 = __shfl_sync(0xFFFFFFFFu, incl[e], 30 + ig);
+            const float bC1 = __shfl_sync(0xFFFFFFFFu, incl[e + 1], 30 + ig);
+            float off[2];  // exclusive prefix of this token group
+            sub_x2(off[0], off[1], incl[e], incl[e + 1], tot[e], tot[e + 1]);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) bk[k][e] += off;
-            nbCl[e] = -bC * kLog2e;
-            range_bad |= !(fabsf(bC) <= kGateRangeLimit);
-            logB[e] = (part_start ? 0.f : logB[e]) + bC;
+            for (int k = 0; k < 4; ++k)
+                add_x2(bk[k][e], bk[k][e + 1], bk[k][e], bk[k][e + 1], off[0], off[1]);
+            mul_x2(nbCl[e], nbCl[e + 1], -bC0, -bC1, kLog2e, kLog2e);
+            range_bad |= !(fabsf(bC0) <= kGateRangeLimit) || !(fabsf(bC1) <= kGateRangeLimit);
+            logB[e] = (part_start ? 0.f : logB[e]) + bC0;
+            logB[e + 1] = (part_start ? 0.f : logB[e + 1]) + bC1;
             eB[e] = w.dstate ? ex2_approx(logB[e] * kLog2e) : 0.f;
+            eB[e + 1] = w.dstate ? ex2_approx(logB[e + 1] * kLog2e) : 0.f;
         }
         if (tg == 0) {
             float4 *e4 = reinterpret_cast<float4 *>(ec + s * D + i0);
@@ -282,11 +293,13 @@ __device__ __noinline__ void gate_role(uint8_t *smem, const Bars &b, volatile in
             uint32_t wk[4], wf[4], wq[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float x0 = fmaf(bk[k][2 * e], kLog2e, nbCl[2 * e]);
-                const float x1 = fmaf(bk[k][2 * e + 1], kLog2e, nbCl[2 * e + 1]);
+                float x0, x1, k0, k1;
+                fma_x2(x0, x1, bk[k][2 * e], bk[k][2 * e + 1], kLog2e, kLog2e, nbCl[2 * e],
+                       nbCl[2 * e + 1]);
                 const float u0 = ex2_approx(x0), u1 = ex2_approx(x1);
-                wk[e] = pack_bf16(__uint_as_float(kw[e] << 16) * ex2_approx(-x0),
-                                  __uint_as_float(kw[e] & 0xFFFF0000u) * ex2_approx(-x1));
+                mul_x2(k0, k1, __uint_as_float(kw[e] << 16), __uint_as_float(kw[e] & 0xFFFF0000u),
+                       ex2_approx(-x0), ex2_approx(-x1));
+                wk[e] = pack_bf16(k0, k1);
                 wf[e] = pack_bf16(u0, u1);
                 wq[e] = pack_bf16(__uint_as_float(qw[e] << 16) * u0 * eB[2 * e],
                                   __uint_as_float(qw[e] & 0xFFFF0000u) * u1 * eB[2 * e + 1]);

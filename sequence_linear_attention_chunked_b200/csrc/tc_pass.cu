@@ -282,16 +282,19 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
 #pragma unroll
             for (int k = 0; k < 4; ++k) unpack8(graw[k], f[k]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < 8; e += 2) {  // two key dims per f32x2 instruction
                 // steps (0,1) and (2,3) each visit one row pair in order; the pair visited
                 // first (rows 4tg, 4tg+1) is at steps 0,1 when sw == 0, at steps 2,3 otherwise
-                const float p01 = f[0][e] + f[1][e], p23 = f[2][e] + f[3][e];
-                const float o01 = sw ? p23 : 0.f, o23 = sw ? 0.f : p01;
-                bk[0][e] = f[0][e] + o01;
-                bk[1][e] = p01 + o01;
-                bk[2][e] = f[2][e] + o23;
-                bk[3][e] = p23 + o23;
-                tot[e] = p01 + p23;
+                float p01[2], p23[2];
+                add_x2(p01[0], p01[1], f[0][e], f[0][e + 1], f[1][e], f[1][e + 1]);
+                add_x2(p23[0], p23[1], f[2][e], f[2][e + 1], f[3][e], f[3][e + 1]);
+                const float o01a = sw ? p23[0] : 0.f, o01b = sw ? p23[1] : 0.f;
+                const float o23a = sw ? 0.f : p01[0], o23b = sw ? 0.f : p01[1];
+                add_x2(bk[0][e], bk[0][e + 1], f[0][e], f[0][e + 1], o01a, o01b);
+                add_x2(bk[1][e], bk[1][e + 1], p01[0], p01[1], o01a, o01b);
+                add_x2(bk[2][e], bk[2][e + 1], f[2][e], f[2][e + 1], o23a, o23b);
+                add_x2(bk[3][e], bk[3][e + 1], p23[0], p23[1], o23a, o23b);
+                add_x2(tot[e], tot[e + 1], p01[0], p01[1], p23[0], p23[1]);
             }
         }
         // inclusive scan of the group totals across tg (lanes ig, ig+2, ..., ig+30)
@@ -300,23 +303,31 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
         for (int e = 0; e < 8; ++e) incl[e] = tot[e];
 #pragma unroll
         for (int d = 1; d < 16; d <<= 1) {
+            float up[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float up = __shfl_up_sync(0xFFFFFFFFu, incl[e], 2 * d);
-                if (tg >= d) incl[e] += up;
+            for (int e = 0; e < 8; ++e) up[e] = __shfl_up_sync(0xFFFFFFFFu, incl[e], 2 * d);
+            if (tg >= d) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2)
+                    add_x2(incl[e], incl[e + 1], incl[e], incl[e + 1], up[e], up[e + 1]);
             }
         }
         float bC[8], nbCl[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            bC[e] = __shfl_sync(0xFFFFFFFFu, incl[e], 30 + ig);
-            const float off = incl[e] - tot[e];  // exclusive prefix of this token group
+        for (int e = 0; e < 8; ++e) bC[e] = __shfl_sync(0xFFFFFFFFu, incl[e], 30 + ig);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) bk[k][e] += off;
+        for (int e = 0; e < 8; e += 2) {
+            float off[2];  // exclusive prefix of this token group
+            sub_x2(off[0], off[1], incl[e], incl[e + 1], tot[e], tot[e + 1]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                add_x2(bk[k][e], bk[k][e + 1], bk[k][e], bk[k][e + 1], off[0], off[1]);
             // exponent offset of q's factor: e^{b_t - b_C}, or e^{B_start + b_t} for Qhat
-            nbCl[e] = (C::dstate ? logG[e] : -bC[e]) * kLog2e;
-            range_bad |= !(fabsf(bC[e]) <= kGateRangeLimit);
+            mul_x2(nbCl[e], nbCl[e + 1], C::dstate ? logG[e] : -bC[e],
+                   C::dstate ? logG[e + 1] : -bC[e + 1], kLog2e, kLog2e);
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) range_bad |= !(fabsf(bC[e]) <= kGateRangeLimit);
         if (tg == 0) {
             float4 *e4 = reinterpret_cast<float4 *>(ec + s * D + i0);
             e4[0] = make_float4(ex2_approx(bC[0] * kLog2e), ex2_approx(bC[1] * kLog2e),
@@ -343,15 +354,19 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
                 const uint32_t off = tile_off(tg * 4 + ((k0 + r) ^ sw), i0);
                 float x[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = fmaf(bk[k0 + r][e], kLog2e, nbCl[e]);
+                for (int e = 0; e < 8; e += 2)
+                    fma_x2(x[e], x[e + 1], bk[k0 + r][e], bk[k0 + r][e + 1], kLog2e, kLog2e, nbCl[e],
+                           nbCl[e + 1]);
                 if (C::q) {
                     float f[8];
                     unpack8(qr[r], f);
                     uint32_t w[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w[e] = pack_bf16(f[2 * e] * ex2_approx(x[2 * e]),
-                                         f[2 * e + 1] * ex2_approx(x[2 * e + 1]));
+                    for (int e = 0; e < 4; ++e) {
+                        float p0, p1;
+                        mul_x2(p0, p1, f[2 * e], f[2 * e + 1], ex2_approx(x[2 * e]), ex2_approx(x[2 * e + 1]));
+                        w[e] = pack_bf16(p0, p1);
+                    }
                     *reinterpret_cast<uint4 *>(st + C::off_q + off) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
                 if (C::k) {
@@ -359,9 +374,11 @@ __device__ void gate_role(uint8_t *smem, const Bars &b, volatile int *abort, con
                     unpack8(kr[r], f);
                     uint32_t w[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w[e] = pack_bf16(f[2 * e] * ex2_approx(-x[2 * e]),
-                                         f[2 * e + 1] * ex2_approx(-x[2 * e + 1]));
+                    for (int e = 0; e < 4; ++e) {
+                        float p0, p1;
+                        mul_x2(p0, p1, f[2 * e], f[2 * e + 1], ex2_approx(-x[2 * e]), ex2_approx(-x[2 * e + 1]));
+                        w[e] = pack_bf16(p0, p1);
+                    }
                     *reinterpret_cast<uint4 *>(st + C::off_k + off) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
