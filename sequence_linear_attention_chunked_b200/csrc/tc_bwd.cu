@@ -580,12 +580,14 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
             // Ktil = k e^{b_C - b_s} the MMA operand); then the suffix sums
             float fd[16], cg[16];  // dk, then contributions / dlog_g
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const float acc = __uint_as_float(r[t]);
+            for (int t = 0; t < 16; t += 2) {  // two tokens per f32x2 instruction
+                const float a0 = __uint_as_float(r[t]), a1 = __uint_as_float(r[t + 1]);
                 const float4 &q4 = qv[t >> 2];
-                const float qq = (t & 3) == 0 ? q4.x : (t & 3) == 1 ? q4.y : (t & 3) == 2 ? q4.z : q4.w;
-                fd[t] = __uint_as_float(fk[t] << 16) * acc;                   // dk
-                cg[t] = qq - __uint_as_float(fk[t] & 0xFFFF0000u) * acc;      // contribution
+                const float q0 = (t & 3) == 0 ? q4.x : q4.z, q1 = (t & 3) == 0 ? q4.y : q4.w;
+                mul_x2(fd[t], fd[t + 1], __uint_as_float(fk[t] << 16), __uint_as_float(fk[t + 1] << 16),
+                       a0, a1);  // dk
+                fma_x2(cg[t], cg[t + 1], -__uint_as_float(fk[t] & 0xFFFF0000u),
+                       -__uint_as_float(fk[t + 1] & 0xFFFF0000u), a0, a1, q0, q1);  // contribution
             }
             if (g >= 2) load_qdq(qb[(3 - g) & 1], tq + 4 * (g - 2));  // group g - 2
 #pragma unroll

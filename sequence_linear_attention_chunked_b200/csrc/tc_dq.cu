@@ -503,16 +503,15 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
             for (int e = 0; e < 16; e += 2) {
                 const float F0 = __uint_as_float(fq[e] << 16), F1 = __uint_as_float(fq[e + 1] << 16);
                 const float a0 = __uint_as_float(r16[e]), a1 = __uint_as_float(r16[e + 1]);
-                dqv[e] = a0 * F0;
-                dqv[e + 1] = a1 * F1;
+                mul_x2(dqv[e], dqv[e + 1], a0, a1, F0, F1);
                 // q . dq handed over as Qbar' dq^T, Qbar' = bf16(q F) -- bit for bit the operand
                 // the reverse sweep's MMAs use -- so that the diagonal term (q_t . k_t)(v_t . dO_t)
                 // of q . dq and of k . dk is the same exact fp32 product in both sweeps and
                 // cancels in dlog_g down to fp32 accumulation error
-                const uint32_t qb = pack_bf16(__uint_as_float(fq[e] & 0xFFFF0000u) * F0,
-                                              __uint_as_float(fq[e + 1] & 0xFFFF0000u) * F1);
-                qd[e] = __uint_as_float(qb << 16) * a0;
-                qd[e + 1] = __uint_as_float(qb & 0xFFFF0000u) * a1;
+                const uint32_t qb = mul_bf16x2(__byte_perm(fq[e], fq[e + 1], 0x7632),
+                                               __byte_perm(fq[e], fq[e + 1], 0x5410));
+                mul_x2(qd[e], qd[e + 1], __uint_as_float(qb << 16), __uint_as_float(qb & 0xFFFF0000u),
+                       a0, a1);
             }
             const long long t0 = tok0 + g * 16;
 #pragma unroll
