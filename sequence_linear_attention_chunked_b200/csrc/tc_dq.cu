@@ -301,8 +301,10 @@ __device__ __noinline__ void gate_role(uint8_t *smem, const Bars &b, volatile in
                        ex2_approx(-x0), ex2_approx(-x1));
                 wk[e] = pack_bf16(k0, k1);
                 wf[e] = pack_bf16(u0, u1);
-                wq[e] = pack_bf16(__uint_as_float(qw[e] << 16) * u0 * eB[2 * e],
-                                  __uint_as_float(qw[e] & 0xFFFF0000u) * u1 * eB[2 * e + 1]);
+                float h0, h1;  // Qhat = (q u) e^B
+                mul_x2(h0, h1, __uint_as_float(qw[e] << 16), __uint_as_float(qw[e] & 0xFFFF0000u), u0, u1);
+                mul_x2(h0, h1, h0, h1, eB[2 * e], eB[2 * e + 1]);
+                wq[e] = pack_bf16(h0, h1);
             }
             *reinterpret_cast<uint4 *>(st + off_k + off) = make_uint4(wk[0], wk[1], wk[2], wk[3]);
             *reinterpret_cast<uint4 *>(st + off_g + off) = make_uint4(wf[0], wf[1], wf[2], wf[3]);
