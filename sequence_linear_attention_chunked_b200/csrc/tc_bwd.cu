@@ -38,9 +38,9 @@ constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
 // the K-major A operand of dS V^T and the MN-major A operand of dS^T Ktil^T), turn M and A into
 // masked bf16 tiles (double-buffered) and write dv from dv^T; warps 4-7 read dk^T
 // (double-buffered in TMEM) and write dk and dlog_g (thread x owns key dim x for all 64 tokens
-// of the chunk, so the dlog_g suffix sums need no exchange); warps 8-11 gate the chunks; 12 TMA; 13 MMA.  A stage is
-// released once the tensor cores are done with it and the dS and output warps have copied the
-// per-key factors they need into registers or TMEM.
+// of the chunk, so the dlog_g suffix sums need no exchange); warps 8-11 gate the chunks; 12 TMA;
+// 13 MMA.  A stage is released once the tensor cores are done with it and the dS and output
+// warps have copied the per-key factors they need into registers or TMEM.
 namespace dkv {
 
 constexpr int kStateWarps = 4, kOutWarps = 4;
