@@ -1,7 +1,8 @@
 // tc_common.cuh -- pieces shared by the tcgen05 chunk kernels (forward and backward):
 // tile geometry, swizzled-tile addressing, UMMA descriptors for the two operand majors,
-// bf16 packing, the fast exp2, the copy of interleaved token pairs into tensor memory, and the
-// TMA tensor-map encoder.
+// bf16 packing and products, the fast exp2, the lane-pair output store, the layout of the q . dq
+// hand-over, the copy of interleaved token pairs into tensor memory, and the TMA tensor-map
+// encoder.
 #pragma once
 
 #include <cuda.h>
@@ -92,27 +93,6 @@ __device__ __forceinline__ void st_pair_bf16(__nv_bfloat16 *row0, int lane, floa
     // even: (own t0, partner t0) = dims l, l+1 of t0; odd: (partner t0+1, own t0+1)
     const uint32_t w = __byte_perm(p, got, odd ? 0x3276u : 0x5410u);
     *reinterpret_cast<uint32_t *>(row0 + (lane & 1) * D + (lane & ~1)) = w;
-}
-
-// Tokens t0 .. t0+3 of this lane's dim (a warp's 32 lanes hold 32 consecutive dims, lane l dim
-// dim0 + l) into a row-major [tokens][128] bf16 tensor with one 8-byte store per lane: the
-// lanes of each quad trade halves in two shuffle steps so that lane 4a + j writes dims
-// dim0 + 4a .. + 3 of token t0 + j.  `row0` points at element (t0, dim0).  The values are
-// rounded once, as by pack_bf16.  Called by all 32 lanes.
-__device__ __forceinline__ void st_quad_bf16(__nv_bfloat16 *row0, int lane, float v0, float v1,
-                                             float v2, float v3) {
-    const uint32_t p01 = pack_bf16(v0, v1), p23 = pack_bf16(v2, v3);  // low half: even token
-    const bool odd = lane & 1, hi = lane & 2;
-    // step 1 (lanes l, l ^ 1): the even lane keeps tokens t0, t0+2 of dims l, l+1; the odd lane
-    // tokens t0+1, t0+3 of dims l-1, l
-    const uint32_t send = __byte_perm(p01, p23, odd ? 0x5410u : 0x7632u);
-    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-    const uint32_t w0 = __byte_perm(p01, recv, odd ? 0x3254u : 0x5410u);  // token t0 (+1 if odd)
-    const uint32_t w1 = __byte_perm(p23, recv, odd ? 0x3276u : 0x7610u);  // token t0+2 (+1 if odd)
-    // step 2 (lanes j, j ^ 2 of the quad): lane j ends with token t0 + j, dims 4a .. 4a+3
-    const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, hi ? w0 : w1, 2);
-    const uint2 out = hi ? make_uint2(got, w1) : make_uint2(w0, got);
-    *reinterpret_cast<uint2 *>(row0 + (lane & 3) * D + (lane & ~3)) = out;
 }
 
 // The fp32 q . dq hand-over between the dq sweep and the reverse sweep is kept token-quad

@@ -517,11 +517,12 @@ __device__ void out_role(uint8_t *smem, const Bars &b, volatile int *abort, cons
             }
             const long long t0 = tok0 + g * 16;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {  // four tokens per float4 / per quad store
+            for (int m = 0; m < 4; ++m) {  // four tokens per float4, two per pair store
                 *qdq_quad(a.dq_ws, (t0 >> 2) + m, i) =
                     make_float4(qd[4 * m], qd[4 * m + 1], qd[4 * m + 2], qd[4 * m + 3]);
-                st_quad_bf16(dq + (t0 + 4 * m) * D + quarter * 32, lane, dqv[4 * m],
-                             dqv[4 * m + 1], dqv[4 * m + 2], dqv[4 * m + 3]);
+                st_pair_bf16(dq + (t0 + 4 * m) * D + quarter * 32, lane, dqv[4 * m], dqv[4 * m + 1]);
+                st_pair_bf16(dq + (t0 + 4 * m + 2) * D + quarter * 32, lane, dqv[4 * m + 2],
+                             dqv[4 * m + 3]);
             }
         }
         if (c + 1 < w.nchunks && !make_p(c + 1)) break;
